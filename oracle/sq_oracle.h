@@ -1,0 +1,103 @@
+/*
+ * sq_oracle.h -- plain CPU oracle for the SmoothQuant W8A8 linear layer.
+ *
+ * TEST INFRASTRUCTURE, NOT PRODUCT CODE. Only the tests, the smoke check in
+ * __graft_entry__.py and the CPU-baseline leg of bench.py may load it. The CUDA
+ * path never includes this header and this library never includes the CUDA
+ * path's headers: the two share no code, constants or helpers.
+ *
+ * Conventions
+ *   - Every floating-point step is one IEEE-754 binary32 operation rounded to
+ *     nearest-even, compiled with -ffp-contract=off (no fused multiply-add),
+ *     except where a function says it works in binary64.
+ *   - Matrices are dense row-major. X is [M,K] (tokens x input channels),
+ *     W is [K,N] (input channels x output channels), Y = X W is [M,N].
+ *   - Quantized weights are stored transposed, Wq[n][k] ([N,K], K contiguous).
+ *   - "bf16" arguments are raw bfloat16 bit patterns (uint16).
+ *   - dtype codes: 0 = fp32, 1 = bf16 (raw uint16).
+ *   - qtype codes: 0 = symmetric INT8 (scale amax/127, clamp to +-127),
+ *                  1 = FP8 E4M3 (scale amax/448, round-to-nearest-even,
+ *                      saturating to +-448).
+ */
+#ifndef SQ_ORACLE_H
+#define SQ_ORACLE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* bfloat16 <-> binary32 (definition of the format; widening is exact). */
+float    sqo_bf16_to_f32(uint16_t h);
+uint16_t sqo_f32_to_bf16_rne(float f);
+
+/* FP8 E4M3: value of a code, and round-to-nearest-even saturating encode. */
+double   sqo_e4m3_decode(uint8_t code);
+uint8_t  sqo_e4m3_encode_rn_sat(float x);
+
+/* a1/a2 calibration: out[c] = max_r |x[r*cols + c]| (per column) when
+ * per_column != 0, else out[r] = max_c |x[r*cols + c]| (per row). */
+void sqo_amax(const void* x, int dtype, int64_t rows, int64_t cols,
+              int per_column, float* out);
+
+/* a3 smoothing factors, computed in binary64 and rounded once to binary32:
+ * s[k] = max(ax,eps)^alpha / max(aw,eps)^(1-alpha), eps = 1e-5. */
+void sqo_smooth_factors(const float* amax_x, const float* amax_w, int64_t K,
+                        double alpha, float* s);
+
+/* The smoothing transform alone, before any quantization:
+ * X~[m][k] = X[m][k] / s[k] and W~[k][n] = s[k] * W[k][n]. */
+void sqo_smooth_act(const void* x, int dtype, int64_t M, int64_t K,
+                    const float* s, float* out);
+void sqo_smooth_weight(const void* w, int dtype, int64_t K, int64_t N,
+                       const float* s, float* out);
+
+/* a4 offline weight smoothing + per-output-channel quantization.
+ * w: [K,N] (dtype), s: [K] or NULL (no smoothing).
+ * wq: [N,K] int8 or E4M3 codes, sw: [N] binary32 scales. */
+void sqo_quantize_weight(const void* w, int dtype, int64_t K, int64_t N,
+                         const float* s, int qtype, void* wq, float* sw);
+
+/* a5 runtime activation smoothing + per-token quantization.
+ * x: [M,K] (dtype), s: [K] or NULL. xq: [M,K] codes, sx: [M] scales. */
+void sqo_quantize_act(const void* x, int dtype, int64_t M, int64_t K,
+                      const float* s, int qtype, void* xq, float* sx);
+
+/* a6 INT8 x INT8 -> int32 accumulators, acc[m][n] = sum_k xq[m][k]*wq[n][k]. */
+void sqo_gemm_i8(const int8_t* xq, const int8_t* wq, int64_t M, int64_t N,
+                 int64_t K, int32_t* acc);
+
+/* a7 E4M3 x E4M3 products summed exactly in binary64 (see the .c file). */
+void sqo_gemm_e4m3(const uint8_t* xq, const uint8_t* wq, int64_t M, int64_t N,
+                   int64_t K, double* acc);
+
+/* Dequantization epilogue for one accumulator value (already widened to
+ * binary32 by the caller's rule): t = a*sx; t = t*sw; t = t + bias. */
+float sqo_dequant(float acc_f32, float sx_m, float sw_n, int has_bias,
+                  uint16_t bias_bf16);
+
+/* Full epilogue over [M,N]. acc_kind 0: int32 accumulators (acc_i32),
+ * 1: binary64 accumulators (acc_f64, rounded once to binary32).
+ * bias: [N] bf16 or NULL. y_f32 (may be NULL) gets the binary32 value before
+ * the bf16 cast, y_bf16 (may be NULL) the bf16 result. */
+void sqo_epilogue(const int32_t* acc_i32, const double* acc_f64, int acc_kind,
+                  const float* sx, const float* sw, const uint16_t* bias,
+                  int64_t M, int64_t N, float* y_f32, uint16_t* y_bf16);
+
+/* One output element computed from scratch (for sampled checks at full size):
+ * the dot product over K followed by the epilogue. qtype as above. */
+void sqo_linear_at(const void* xq, const float* sx, const void* wq,
+                   const float* sw, const uint16_t* bias, int qtype,
+                   int64_t K, const int64_t* rows, const int64_t* cols,
+                   int64_t count, double* acc_out, float* y_f32,
+                   uint16_t* y_bf16);
+
+/* Threads OpenMP will use (1 when built without OpenMP). */
+int sqo_num_threads(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SQ_ORACLE_H */

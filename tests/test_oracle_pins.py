@@ -1,0 +1,443 @@
+"""Pins for the CPU oracle: checks against what the pages print and what the
+mathematics fixes, never against the oracle's own formulas retyped.
+
+Pages: "Weight-Activation Quantization" (infra.bea.ai) §2 (per-tensor scale
+80/127), §3 (worked smoothing example, smoothing-factor formula), §4 (E4M3
+range and scaling).
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from w8a8_smoothquant_int8_02_b200 import synth, workloads
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _fixture(name):
+    out = {}
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            k, v = line.split(":", 1)
+            out[k.strip()] = v.split()
+    return out
+
+
+def _f32_dot(a, b):
+    """Sequential binary32 dot product."""
+    acc = np.float32(0.0)
+    for x, y in zip(np.asarray(a, np.float32), np.asarray(b, np.float32)):
+        acc = np.float32(acc + np.float32(x * y))
+    return acc
+
+
+# ---------------------------------------------------------------------------
+# §3 worked example: smoothing preserves the inner product.
+# ---------------------------------------------------------------------------
+
+def test_worked_example_smoothing_values():
+    fx = _fixture("worked_example.txt")
+    x = np.array([fx["x"]], np.float32)
+    w = np.array(fx["w"], np.float32).reshape(3, 1)
+    s = np.array(fx["s"], np.float32)
+    xs = oracle.smooth_act(x, s)[0]
+    ws = oracle.smooth_weight(w, s)[:, 0]
+    np.testing.assert_array_equal(xs, np.array(fx["x_smoothed"], np.float32))
+    np.testing.assert_array_equal(ws, np.array(fx["w_smoothed"], np.float32))
+
+
+def test_worked_example_inner_product_preserved():
+    fx = _fixture("worked_example.txt")
+    x = np.array([fx["x"]], np.float32)
+    w = np.array(fx["w"], np.float32).reshape(3, 1)
+    s = np.array(fx["s"], np.float32)
+    xs = oracle.smooth_act(x, s)[0]
+    ws = oracle.smooth_weight(w, s)[:, 0]
+    target = float(fx["inner_product"][0])
+    before = _f32_dot(x[0], w[:, 0])
+    after = _f32_dot(xs, ws)
+    assert abs(float(before) - target) < 1e-5
+    # s is a power of two, so every product is unchanged and the binary32
+    # sums agree bit for bit.
+    assert before == after
+
+
+def test_power_of_two_smoothing_is_exact_on_random_rows():
+    rng = np.random.default_rng(5)
+    K = 97
+    x = rng.standard_normal((3, K)).astype(np.float32)
+    w = rng.standard_normal((K, 4)).astype(np.float32)
+    s = (2.0 ** rng.integers(-6, 7, size=K)).astype(np.float32)
+    xs = oracle.smooth_act(x, s)
+    ws = oracle.smooth_weight(w, s)
+    for m in range(3):
+        for n in range(4):
+            assert _f32_dot(x[m], w[:, n]) == _f32_dot(xs[m], ws[:, n])
+
+
+def test_general_smoothing_preserves_product_within_rounding():
+    rng = np.random.default_rng(6)
+    K = 256
+    x = rng.standard_normal((4, K)).astype(np.float32)
+    w = rng.standard_normal((K, 5)).astype(np.float32)
+    s = rng.uniform(0.05, 20.0, size=K).astype(np.float32)
+    xs = oracle.smooth_act(x, s).astype(np.float64)
+    ws = oracle.smooth_weight(w, s).astype(np.float64)
+    exact = x.astype(np.float64) @ w.astype(np.float64)
+    smoothed = xs @ ws
+    # each smoothed product carries two binary32 roundings
+    bound = 2.5 * 2.0 ** -24 * (np.abs(x.astype(np.float64)) @ np.abs(w.astype(np.float64)))
+    assert np.all(np.abs(smoothed - exact) <= bound)
+
+
+# ---------------------------------------------------------------------------
+# §2 per-tensor scale set by the outlier: 80/127 = 0.63.
+# ---------------------------------------------------------------------------
+
+def test_per_tensor_scale_example():
+    fx = _fixture("per_tensor_scale.txt")
+    row = np.array([fx["row"]], np.float32)
+    xq, sx = oracle.quantize_act(row, None)
+    assert abs(float(sx[0]) - float(fx["scale_approx"][0])) <= \
+        float(fx["scale_rel_tol"][0]) * float(fx["scale_approx"][0])
+    np.testing.assert_array_equal(xq[0], np.array(fx["codes"], np.int8))
+
+
+def test_round_half_even_ties():
+    fx = _fixture("rounding_ties.txt")
+    row = np.array([fx["row"]], np.float32)
+    xq, sx = oracle.quantize_act(row, None)
+    assert sx[0] == np.float32(1.0)
+    np.testing.assert_array_equal(xq[0], np.array(fx["codes"], np.int8))
+
+
+# ---------------------------------------------------------------------------
+# §4 E4M3 format.
+# ---------------------------------------------------------------------------
+
+def test_e4m3_fixture_points():
+    with open(os.path.join(GOLDEN, "e4m3_points.txt")) as f:
+        pts = [l.split() for l in f if l.strip() and not l.startswith("#")]
+    vals = np.array([float(v) for v, _ in pts], np.float32)
+    codes = oracle.e4m3_encode(vals)
+    assert [int(c) for c in codes] == [int(c, 16) for _, c in pts]
+
+
+def test_e4m3_decode_matches_torch_and_format():
+    codes = np.arange(256, dtype=np.uint8)
+    dec = oracle.e4m3_decode(codes)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    nan = np.isnan(ref)
+    assert list(np.nonzero(nan)[0]) == [0x7F, 0xFF]
+    np.testing.assert_array_equal(np.isnan(dec), nan)
+    np.testing.assert_array_equal(dec[~nan], ref[~nan])
+    assert np.nanmax(dec) == 448.0 and np.nanmin(dec) == -448.0
+
+
+def test_e4m3_roundtrip_all_finite_codes():
+    codes = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], np.uint8)
+    vals = oracle.e4m3_decode(codes).astype(np.float32)
+    np.testing.assert_array_equal(oracle.e4m3_encode(vals), codes)
+
+
+def test_e4m3_encode_matches_torch_in_range():
+    rng = np.random.default_rng(7)
+    finite = oracle.e4m3_decode(np.arange(0, 0x7F, dtype=np.uint8))
+    mids = ((finite[1:] + finite[:-1]) / 2).astype(np.float32)  # exact ties
+    x = np.concatenate([
+        rng.uniform(-448, 448, 20000).astype(np.float32),
+        (rng.standard_normal(20000) * 0.01).astype(np.float32),
+        mids, -mids,
+        np.nextafter(mids, np.float32(np.inf)), np.nextafter(mids, np.float32(0)),
+    ]).astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    np.testing.assert_array_equal(oracle.e4m3_encode(x), ref)
+
+
+def test_e4m3_saturates_above_range():
+    x = np.array([448.0, 449.0, 463.9, 464.0, 480.0, 1e30, -600.0], np.float32)
+    np.testing.assert_array_equal(oracle.e4m3_encode(x),
+                                  np.array([0x7E] * 6 + [0xFE], np.uint8))
+
+
+# ---------------------------------------------------------------------------
+# bfloat16 rounding (the output format) against torch's conversion.
+# ---------------------------------------------------------------------------
+
+def test_bf16_rounding_matches_torch():
+    rng = np.random.default_rng(8)
+    bits = rng.integers(0, 2 ** 32, size=30000, dtype=np.uint64).astype(np.uint32)
+    x = bits.view(np.float32)
+    x = x[np.isfinite(x)]
+    # exact ties: low 16 bits = 0x8000
+    ties = ((rng.integers(0, 2 ** 16, 2000).astype(np.uint32) << 16) | 0x8000).view(np.float32)
+    ties = ties[np.isfinite(ties)]
+    x = np.concatenate([x, ties, np.float32([0.0, -0.0, 3.4e38, -3.4e38, 1e-45])])
+    ref = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    np.testing.assert_array_equal(oracle.f32_to_bf16(x), ref)
+
+
+def test_bf16_widening_exact():
+    h = np.arange(0, 2 ** 16, 97, dtype=np.uint16)
+    ref = torch.from_numpy(h.view(np.int16)).view(torch.bfloat16).float().numpy()
+    got = oracle.bf16_to_f32(h)
+    finite = np.isfinite(ref)
+    np.testing.assert_array_equal(got[finite], ref[finite])
+
+
+# ---------------------------------------------------------------------------
+# §3 "Choosing the Smoothing Factor": s_j = max|X_j|^a / max|W_j|^(1-a).
+# ---------------------------------------------------------------------------
+
+def test_smooth_factor_hand_values():
+    ax = np.float32([16.0, 16.0, 16.0, 16.0, 9.0])
+    aw = np.float32([4.0, 4.0, 4.0, 4.0, 1.0])
+    assert oracle.smooth_factors(ax, aw, 0.5)[0] == np.float32(2.0)
+    assert oracle.smooth_factors(ax, aw, 1.0)[0] == np.float32(16.0)
+    assert oracle.smooth_factors(ax, aw, 0.0)[0] == np.float32(0.25)
+    # 16^0.75 / 4^0.25 = 8 / sqrt(2) = 4 sqrt(2); swapping alpha and 1-alpha
+    # would give 16^0.25 / 4^0.75 = sqrt(2)/2 instead.
+    got = oracle.smooth_factors(ax, aw, 0.75)[0]
+    assert got == np.float32(4.0 * math.sqrt(2.0))
+    assert oracle.smooth_factors(ax, aw, 0.5)[4] == np.float32(3.0)
+
+
+def test_smooth_factor_zero_amax_is_clamped():
+    s = oracle.smooth_factors(np.float32([0.0, 1.0]), np.float32([1.0, 0.0]), 0.5)
+    assert np.isfinite(s).all() and (s > 0).all()
+    assert abs(float(s[0]) - math.sqrt(1e-5)) <= 1e-7 * math.sqrt(1e-5) + 1e-12
+    assert abs(float(s[1]) - 1.0 / math.sqrt(1e-5)) <= 1e-6 / math.sqrt(1e-5)
+
+
+def test_alpha_half_balances_ranges():
+    rng = np.random.default_rng(9)
+    ax = rng.uniform(0.1, 100.0, 512).astype(np.float32)
+    aw = rng.uniform(0.001, 0.5, 512).astype(np.float32)
+    s = oracle.smooth_factors(ax, aw, 0.5).astype(np.float64)
+    # after smoothing both channel ranges equal sqrt(ax*aw)
+    lhs = ax / s
+    rhs = aw * s
+    g = np.sqrt(ax.astype(np.float64) * aw.astype(np.float64))
+    assert np.all(np.abs(lhs - g) <= 4e-7 * g)
+    assert np.all(np.abs(rhs - g) <= 4e-7 * g)
+
+
+def test_alpha_one_normalizes_calibration_channels():
+    case = workloads.TINY
+    d = synth.generate(case)
+    ax = oracle.amax(d["x_cal"], per_column=True)
+    aw = oracle.amax(d["w"], per_column=False)
+    s = oracle.smooth_factors(ax, aw, 1.0)
+    np.testing.assert_array_equal(s, ax)
+    xs = oracle.smooth_act(d["x_cal"], s)
+    np.testing.assert_array_equal(np.abs(xs).max(axis=0), np.ones(case.K, np.float32))
+
+
+def test_alpha_zero_normalizes_weight_rows():
+    rng = np.random.default_rng(10)
+    w = (rng.standard_normal((40, 24)) * 0.02).astype(np.float32)
+    aw = oracle.amax(w, per_column=False)
+    s = oracle.smooth_factors(np.ones(40, np.float32), aw, 0.0)
+    ws = oracle.smooth_weight(w, s)
+    rowmax = np.abs(ws).max(axis=1)
+    assert np.all(np.abs(rowmax - 1.0) <= 2.0 ** -22)
+
+
+# ---------------------------------------------------------------------------
+# Calibration amax along each axis, and quantization of weights / activations.
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_amax_axes(dtype):
+    rng = np.random.default_rng(11)
+    x = rng.standard_normal((37, 53)).astype(np.float32) * 3
+    if dtype == "bf16":
+        xb = synth.to_bf16_bits(x)
+        xf = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).float().numpy()
+        src = xb
+    else:
+        xf = x
+        src = x
+    np.testing.assert_array_equal(oracle.amax(src, True), np.abs(xf).max(axis=0))
+    np.testing.assert_array_equal(oracle.amax(src, False), np.abs(xf).max(axis=1))
+
+
+def test_quantize_weight_layout_and_scale():
+    K, N = 48, 40
+    w = np.full((K, N), 0.001, np.float32)
+    w[7, 29] = -3.0
+    w[:, 5] = 0.0
+    wq, sw = oracle.quantize_weight(w, None)
+    assert wq.shape == (N, K)
+    assert wq[29, 7] == -127
+    assert abs(float(sw[29]) - 3.0 / 127) <= 1e-7
+    assert sw[5] == 0 and not wq[5].any()
+    # every other entry of column 29 is tiny
+    assert np.abs(wq[29].astype(int)).sum() == 127
+
+
+@pytest.mark.parametrize("smooth", [False, True])
+def test_weight_quant_error_bound(smooth):
+    rng = np.random.default_rng(12)
+    K, N = 64, 48
+    w = (rng.standard_normal((K, N)) * 0.02).astype(np.float32)
+    s = rng.uniform(0.2, 5.0, K).astype(np.float32) if smooth else None
+    wq, sw = oracle.quantize_weight(w, s)
+    wt = oracle.smooth_weight(w, s) if smooth else w
+    deq = wq.T.astype(np.float64) * sw.astype(np.float64)[None, :]
+    err = np.abs(wt.astype(np.float64) - deq)
+    assert np.all(err <= sw.astype(np.float64)[None, :] / 2 * (1 + 2.0 ** -20))
+    # the largest element of each column lands on +-127
+    assert np.all(np.abs(wq.astype(int)).max(axis=1) == 127)
+
+
+def test_act_quant_error_bound_and_extremes():
+    case = workloads.TINY
+    d = synth.generate(case)
+    x = d["x"]
+    s = synth.random_floats(case.K, seed=3, lo=0.5, hi=8.0)
+    xq, sx = oracle.quantize_act(x, s)
+    xs = oracle.smooth_act(x, s).astype(np.float64)
+    deq = xq.astype(np.float64) * sx.astype(np.float64)[:, None]
+    assert np.all(np.abs(xs - deq) <= sx.astype(np.float64)[:, None] / 2 * (1 + 2.0 ** -20))
+    assert np.all(np.abs(xq.astype(int)).max(axis=1) == 127)
+    assert xq.min() >= -127
+
+
+def test_act_quant_zero_row_and_no_smoothing():
+    x = np.zeros((3, 16), np.float32)
+    x[1] = np.linspace(-2, 2, 16, dtype=np.float32)
+    xq, sx = oracle.quantize_act(x, None)
+    assert sx[0] == 0 and sx[2] == 0 and not xq[0].any() and not xq[2].any()
+    xq1, sx1 = oracle.quantize_act(x, np.ones(16, np.float32))
+    np.testing.assert_array_equal(xq, xq1)
+    np.testing.assert_array_equal(sx, sx1)
+
+
+def test_act_quant_e4m3_bound():
+    rng = np.random.default_rng(13)
+    x = (rng.standard_normal((8, 64)) * 5).astype(np.float32)
+    xq, sx = oracle.quantize_act(x, None, oracle.E4M3)
+    dec = oracle.e4m3_decode(xq) * sx.astype(np.float64)[:, None]
+    xd = x.astype(np.float64)
+    # 3 mantissa bits: half-ulp relative error 2^-4 for normals, plus the
+    # half subnormal step 2^-10 in units of the scale
+    assert np.all(np.abs(xd - dec) <= 2.0 ** -4 * np.abs(xd) + 2.0 ** -10 * sx[:, None] * 1.0001)
+    absmax_codes = xq[np.arange(8), np.abs(x).argmax(axis=1)]
+    assert np.all((absmax_codes & 0x7F) == 0x7E)
+
+
+# ---------------------------------------------------------------------------
+# 8-bit GEMMs against independent brute force.
+# ---------------------------------------------------------------------------
+
+def test_gemm_i8_brute_force_nonsquare():
+    xq = synth.random_matrix((7, 48), np.int8, seed=1)
+    wq = synth.random_matrix((5, 48), np.int8, seed=2)
+    acc = oracle.gemm_i8(xq, wq)
+    ref = xq.astype(np.int64) @ wq.astype(np.int64).T
+    np.testing.assert_array_equal(acc, ref)
+
+
+def test_gemm_i8_extremes():
+    K = 4096
+    xq = np.full((2, K), 127, np.int8)
+    xq[1] = -127
+    wq = np.full((3, K), 127, np.int8)
+    wq[2] = 0
+    wq[2, 17] = 1
+    acc = oracle.gemm_i8(xq, wq)
+    assert acc[0, 0] == K * 127 * 127 and acc[1, 1] == -K * 127 * 127
+    assert acc[0, 2] == 127 and acc[1, 2] == -127
+
+
+def test_gemm_e4m3_exact():
+    rng = np.random.default_rng(14)
+    codes = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], np.uint8)
+    xq = rng.choice(codes, size=(6, 160)).astype(np.uint8)
+    wq = rng.choice(codes, size=(9, 160)).astype(np.uint8)
+    acc = oracle.gemm_e4m3(xq, wq)
+    # all partial sums are exact in binary64, so any summation order gives the
+    # same value; numpy's matmul of the decoded values is an independent sum
+    ref = oracle.e4m3_decode(xq) @ oracle.e4m3_decode(wq).T
+    np.testing.assert_array_equal(acc, ref)
+
+
+# ---------------------------------------------------------------------------
+# Dequantization epilogue.
+# ---------------------------------------------------------------------------
+
+def test_epilogue_power_of_two_scales_exact():
+    acc = np.array([[3, -1000, 12345], [0, 7, -8]], np.int32)
+    sx = np.float32([2.0 ** -7, 0.5])
+    sw = np.float32([0.25, 2.0 ** -10, 8.0])
+    yf, yb = oracle.epilogue(acc, sx, sw, None)
+    exact = acc.astype(np.float64) * sx[:, None].astype(np.float64) * sw[None, :].astype(np.float64)
+    np.testing.assert_array_equal(yf.astype(np.float64), exact)
+    ref = torch.from_numpy(yf).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    np.testing.assert_array_equal(yb, ref)
+
+
+def test_epilogue_bias_added():
+    acc = np.array([[4, 0]], np.int32)
+    bias = synth.to_bf16_bits(np.float32([0.5, -1.25]))
+    yf, _ = oracle.epilogue(acc, np.float32([0.25]), np.float32([1.0, 1.0]), bias)
+    np.testing.assert_array_equal(yf, np.float32([[1.5, -1.25]]))
+
+
+def test_epilogue_relative_error_bound():
+    rng = np.random.default_rng(15)
+    acc = rng.integers(-2 ** 28, 2 ** 28, size=(16, 32)).astype(np.int32)
+    sx = rng.uniform(0.01, 1, 16).astype(np.float32)
+    sw = rng.uniform(1e-4, 1e-2, 32).astype(np.float32)
+    yf, _ = oracle.epilogue(acc, sx, sw, None)
+    exact = acc.astype(np.float64) * sx[:, None] * sw[None, :]
+    # int->float rounding plus two products: below 3 units of 2^-24
+    assert np.all(np.abs(yf - exact) <= 3.01 * 2.0 ** -24 * np.abs(exact))
+
+
+def test_linear_at_matches_full_path():
+    case = workloads.TINY
+    d = synth.generate(case)
+    ax = oracle.amax(d["x_cal"], True)
+    aw = oracle.amax(d["w"], False)
+    s = oracle.smooth_factors(ax, aw, case.alpha)
+    wq, sw = oracle.quantize_weight(d["w"], s)
+    bias = synth.to_bf16_bits(synth.random_floats(case.N, seed=4, std=0.1))
+    full = oracle.linear(d["x"], s, wq, sw, bias)
+    rows = np.array([0, 3, 15, 8], np.int64)
+    cols = np.array([0, 63, 41, 7], np.int64)
+    acc, yf, yb = oracle.linear_at(full["xq"], full["sx"], wq, sw, bias, rows, cols)
+    np.testing.assert_array_equal(acc, full["acc"][rows, cols].astype(np.float64))
+    np.testing.assert_array_equal(yf, full["y_f32"][rows, cols])
+    np.testing.assert_array_equal(yb, full["y_bf16"][rows, cols])
+
+
+# ---------------------------------------------------------------------------
+# §3: quantization after smoothing gives a smaller error than without.
+# ---------------------------------------------------------------------------
+
+def test_smoothing_reduces_quantization_error_on_outlier_data():
+    case = workloads.TINY
+    d = synth.generate(case)
+    x, w = d["x"], d["w"]
+    exact = x.astype(np.float64) @ w.astype(np.float64)
+
+    def err(s):
+        wq, sw = oracle.quantize_weight(w, s)
+        y = oracle.linear(x, s, wq, sw)["y_f32"].astype(np.float64)
+        return np.linalg.norm(y - exact) / np.linalg.norm(exact)
+
+    ax = oracle.amax(x, True)
+    aw = oracle.amax(w, False)
+    s = oracle.smooth_factors(ax, aw, 0.5)
+    e_smooth, e_plain = err(s), err(None)
+    assert e_smooth < 0.5 * e_plain, (e_smooth, e_plain)
+    assert e_smooth < 0.05

@@ -1,0 +1,48 @@
+"""The five SmoothQuant linear-layer workloads this library is measured on.
+
+Shapes follow transformer linear layers: Y[M,N] = X[M,K] W[K,N], M tokens,
+K input channels, N output channels.  Prefill / MLP shapes are compute-bound
+and run on the 8-bit tensor cores; the 16-token decode shape is bound by the
+weight read from HBM ("W8A8 vs W4A16": prefill is compute-bound, decode is
+memory-bound).
+"""
+from __future__ import annotations
+
+from .synth import LinearCase
+
+TINY = LinearCase(
+    name="tiny_16x64x64", M=16, K=64, N=64, x_dtype="f32", alpha=0.5,
+    qtype="i8", w_std=0.02, outlier_channels=(3, 41), outlier_factor=60.0,
+    cal_tokens=0,
+    note="X fp32 [16,64] N(0,1), channels 3 and 41 x60; W fp32 [64,64] "
+         "N(0,0.02); calibrated on X itself")
+
+PREFILL = LinearCase(
+    name="prefill_512x4096x4096", M=512, K=4096, N=4096, x_dtype="bf16",
+    alpha=0.5, qtype="i8", w_std=0.02, outlier_frac=0.01, outlier_lo=20.0,
+    outlier_hi=100.0, cal_tokens=512,
+    note="X bf16 [512,4096], 1% outlier channels x U(20,100); W bf16 "
+         "[4096,4096] N(0,0.02); 512 calibration tokens")
+
+MLP_UP = LinearCase(
+    name="mlp_up_4096x4096x14336", M=4096, K=4096, N=14336, x_dtype="bf16",
+    alpha=0.5, qtype="i8", w_std=0.02, outlier_frac=0.01, outlier_lo=20.0,
+    outlier_hi=100.0, bias_std=0.01, cal_tokens=512,
+    note="X bf16 [4096,4096], 1% outlier channels x U(20,100); W bf16 "
+         "[4096,14336] N(0,0.02); bias bf16 N(0,0.01); 512 calibration tokens")
+
+FP8_DOWN = LinearCase(
+    name="fp8_down_4096x14336x4096", M=4096, K=14336, N=4096, x_dtype="bf16",
+    alpha=0.85, qtype="e4m3", w_std=0.015, outlier_frac=0.005,
+    outlier_lo=10.0, outlier_hi=80.0, cal_tokens=512,
+    note="X bf16 [4096,14336], 0.5% outlier channels x U(10,80); W bf16 "
+         "[14336,4096] N(0,0.015); alpha 0.85; E4M3 with amax/448 scales")
+
+DECODE = LinearCase(
+    name="decode_16x8192x28672", M=16, K=8192, N=28672, x_dtype="bf16",
+    alpha=0.5, qtype="i8", w_std=0.02, outlier_frac=0.01, outlier_lo=20.0,
+    outlier_hi=100.0, cal_tokens=512,
+    note="X bf16 [16,8192], 1% outlier channels x U(20,100); W bf16 "
+         "[8192,28672] N(0,0.02) quantized offline; HBM-bound")
+
+ALL = {c.name: c for c in (TINY, PREFILL, MLP_UP, FP8_DOWN, DECODE)}
