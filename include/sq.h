@@ -1,0 +1,203 @@
+/*
+ * sq.h -- C ABI of libsq.so, the B200 (sm_100a) SmoothQuant W8A8 linear layer
+ *
+ *     Y = X W = (X diag(s)^-1) (diag(s) W)
+ *
+ * as described by "Weight-Activation Quantization" (infra.bea.ai), §3
+ * "SmoothQuant: The Smoothing Trick" (equivalence, two-step pipeline,
+ * "Choosing the Smoothing Factor") and §4 "FP8 W8A8 (Native on Hopper+)".
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Matrices are dense and row-major. X is [M,K] (M tokens, K input
+ *    channels), W is [K,N] (N output channels), Y is [M,N]. Quantized weights
+ *    are stored transposed as Wq [N,K] (K contiguous); quantized activations
+ *    as Xq [M,K]. Both 8-bit operands are therefore "K-major".
+ *  - Every pointer argument is a DEVICE pointer owned by the caller (the
+ *    library never frees or keeps it). Large tensors (x, w, xq, wq, y, acc)
+ *    must be 16-byte aligned; vectors (s, sx, sw, amax) 4-byte aligned; bias
+ *    2-byte aligned. Inputs and outputs must not alias.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream). Every call is asynchronous on that stream: argument checks run
+ *    synchronously on the host and launch nothing when they fail; a failed
+ *    launch returns SQ_ERR_CUDA. A device-side wait that gives up (see
+ *    sq_get_device_status) is reported through the device status word.
+ *  - K must be a positive multiple of 16 (16-byte rows of 8-bit data for the
+ *    tensor-memory-accelerator copies); N a positive multiple of 8 (16-byte
+ *    rows of bf16 output). M may be any value >= 0; M == 0 is a no-op that
+ *    returns SQ_OK after the size checks (the M-sized pointers may then be
+ *    NULL, as they are for empty torch tensors).
+ *  - Floating-point arithmetic is IEEE binary32 with round-to-nearest-even
+ *    and no contraction into fused multiply-adds, so results are
+ *    reproducible bit for bit against a plain CPU implementation (see
+ *    each function for the exact operation order).
+ *  - The library allocates no device memory of its own except a 4-byte
+ *    device status word.
+ */
+#ifndef SQ_H
+#define SQ_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SQ_ABI_VERSION 1
+
+typedef enum {
+    SQ_OK = 0,
+    SQ_ERR_INVALID_ARG = 1,  /* null pointer, bad size, bad alpha, bad enum   */
+    SQ_ERR_MISALIGNED = 2,   /* pointer or leading dimension misaligned       */
+    SQ_ERR_UNSUPPORTED = 3,  /* valid but not implemented combination         */
+    SQ_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed           */
+    SQ_ERR_TIMEOUT = 5       /* a bounded device-side wait gave up             */
+} sq_status;
+
+typedef enum {
+    SQ_F32 = 0,   /* IEEE binary32                                           */
+    SQ_BF16 = 1,  /* bfloat16 (raw 16-bit patterns)                          */
+    SQ_I8 = 2,    /* signed 8-bit integer code                               */
+    SQ_E4M3 = 3,  /* FP8 E4M3 code: bias 7, no infinity, max finite 448      */
+    SQ_I32 = 4    /* signed 32-bit integer                                   */
+} sq_dtype;
+
+typedef enum {
+    SQ_AMAX_PER_COLUMN = 0,  /* amax[c] = max_r |x[r,c]|  (reduce over rows)  */
+    SQ_AMAX_PER_ROW = 1      /* amax[r] = max_c |x[r,c]|  (reduce over cols)  */
+} sq_axis;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* sq_status_string(sq_status st);
+
+/* SQ_ABI_VERSION of the loaded library. */
+int sq_abi_version(void);
+
+/*
+ * Synchronizes `stream`, then reads and clears the device status word.
+ * Returns SQ_OK if no kernel reported a problem since the last call, or
+ * SQ_ERR_TIMEOUT if a bounded wait inside a kernel gave up (the kernel then
+ * skipped the rest of its work and released its tensor memory, so the
+ * context stays usable but its outputs are undefined). SQ_ERR_CUDA if the
+ * synchronization itself failed.
+ */
+sq_status sq_get_device_status(void* stream);
+
+/*
+ * a1 / a2 -- calibration amax.
+ * Source: "Weight-Activation Quantization" §3 "Choosing the Smoothing
+ * Factor" (max|X_j| and max|W_j|); the zenaique flashcard "Define activation
+ * quantization ..." (calibration on a small held-out corpus).
+ *   x      : [rows, cols] row-major, dtype xt (SQ_F32 or SQ_BF16)
+ *   axis   : SQ_AMAX_PER_COLUMN -> amax has `cols` entries (calibration of
+ *            activations: one value per input channel over the tokens);
+ *            SQ_AMAX_PER_ROW    -> amax has `rows` entries (weights W [K,N]:
+ *            one value per input channel over the output channels).
+ *   accumulate : 0 -> amax is overwritten; 1 -> amax = max(amax, new), so a
+ *            calibration corpus can be streamed batch by batch.
+ *   cols must be a multiple of 8; rows >= 1.
+ */
+sq_status sq_calibrate_amax(const void* x, sq_dtype xt, int64_t rows,
+                            int64_t cols, sq_axis axis, float* amax,
+                            int accumulate, void* stream);
+
+/*
+ * a3 -- smoothing factors, "Choosing the Smoothing Factor":
+ *   s[k] = max(amax_x[k], 1e-5)^alpha / max(amax_w[k], 1e-5)^(1-alpha)
+ * evaluated in binary64 and rounded once to binary32. 0 <= alpha <= 1
+ * (SQ_ERR_INVALID_ARG otherwise). K >= 1.
+ */
+sq_status sq_smooth_factors(const float* amax_x, const float* amax_w,
+                            int64_t K, double alpha, float* s, void* stream);
+
+/*
+ * a4 -- offline weight smoothing and per-output-channel quantization.
+ * Source: §3 "Step 1" (W_tilde = diag(s) W) and "Step 2" (W_int8 =
+ * quantize(W_tilde)); §4 "Per-Tensor Scaling for FP8" for qt = SQ_E4M3.
+ *   w  : [K,N] row-major, dtype wt (SQ_F32 or SQ_BF16)
+ *   s  : [K] smoothing factors, or NULL for no smoothing
+ *   qt : SQ_I8 or SQ_E4M3
+ *   wq : [N,K] output codes (transposed, K contiguous)
+ *   sw : [N] output scales
+ * For each n: wt[k] = s[k]*w[k,n]; sw[n] = max_k|wt[k]| / Q (Q = 127 for
+ * INT8, 448 for E4M3); wq[n,k] = clamp(rne(wt[k]/sw[n]), -127, 127) for INT8,
+ * or the E4M3 code of wt[k]/sw[n] (nearest-even, saturating to +-448). A
+ * column with sw[n] == 0 gets all-zero codes.
+ */
+sq_status sq_quantize_weight(const void* w, sq_dtype wt, int64_t K, int64_t N,
+                             const float* s, sq_dtype qt, void* wq, float* sw,
+                             void* stream);
+
+/*
+ * a5 -- fused runtime activation smoothing + per-token quantization (one
+ * kernel, one read of X). Source: §3 "divide each activation channel by
+ * s_j" and "Step 2" (X_int8 = quantize(X_tilde) at inference time); §2
+ * scale = max|x|/127; §4 q = cast_fp8(x/s) with s = max|x|/448.
+ *   x  : [M,K] row-major, SQ_F32 or SQ_BF16
+ *   s  : [K] smoothing factors, or NULL for no smoothing
+ *   qt : SQ_I8 or SQ_E4M3
+ *   xq : [M,K] output codes; sx : [M] output per-token scales
+ * For each row m: xs[k] = x[m,k] / s[k] (IEEE division); sx[m] =
+ * max_k|xs[k]| / Q; codes as in sq_quantize_weight with xs and sx[m].
+ * Rows with sx[m] == 0 get all-zero codes. K <= 65536.
+ */
+sq_status sq_quantize_act(const void* x, sq_dtype xt, int64_t M, int64_t K,
+                          const float* s, sq_dtype qt, void* xq, float* sx,
+                          void* stream);
+
+/*
+ * a6 -- INT8 x INT8 tensor-core GEMM with int32 accumulation and a fused
+ * dequantization epilogue. Source: §3 "Step 2" (Y = dequantize(X_int8 @
+ * W_int8), "INT8 Tensor Core GEMM"); §1 table (INT8 x INT8 row).
+ *   xq : [M,K] int8, sx : [M];  wq : [N,K] int8, sw : [N]
+ *   bias : [N] bf16 or NULL
+ *   y  : [M,N], yt = SQ_BF16 or SQ_F32
+ *   acc: [M,N] int32 accumulators or NULL (written when non-NULL)
+ * acc[m,n] = sum_k xq[m,k]*wq[n,k] (exact in int32 for K < 133144);
+ * t = float(acc) (nearest-even); t = t*sx[m]; t = t*sw[n]; t = t + bias[n];
+ * y = t (SQ_F32) or bf16(t) rounded to nearest-even (SQ_BF16).
+ */
+sq_status sq_gemm_w8a8(const int8_t* xq, const float* sx, const int8_t* wq,
+                       const float* sw, const uint16_t* bias, int64_t M,
+                       int64_t N, int64_t K, void* y, sq_dtype yt,
+                       int32_t* acc, void* stream);
+
+/*
+ * a7 -- FP8 E4M3 x E4M3 tensor-core GEMM, binary32 accumulation in tensor
+ * memory, same epilogue. Source: §4 "FP8 W8A8 (Native on Hopper+)"; §1
+ * table (FP8 x FP8 row). xq / wq hold E4M3 codes; other arguments as in
+ * sq_gemm_w8a8. The tensor cores' summation order is not specified, so the
+ * result differs from an exact sum by accumulated binary32 rounding.
+ */
+sq_status sq_gemm_fp8(const uint8_t* xq, const float* sx, const uint8_t* wq,
+                      const float* sw, const uint16_t* bias, int64_t M,
+                      int64_t N, int64_t K, void* y, sq_dtype yt,
+                      void* stream);
+
+/*
+ * Runtime forward of one SmoothQuant linear layer: sq_quantize_act followed
+ * by sq_gemm_w8a8 (qt = SQ_I8) or sq_gemm_fp8 (qt = SQ_E4M3) on the same
+ * stream. xq_buf [M,K] (8-bit codes) and sx_buf [M] are caller-owned
+ * buffers that receive the quantized activations.
+ */
+sq_status sq_linear(const void* x, sq_dtype xt, const float* s,
+                    const void* wq, const float* sw, const uint16_t* bias,
+                    sq_dtype qt, int64_t M, int64_t N, int64_t K,
+                    void* xq_buf, float* sx_buf, void* y, sq_dtype yt,
+                    void* stream);
+
+/*
+ * Diagnostic: launches one block whose single thread waits on a shared-memory
+ * barrier that nothing ever completes, through the same bounded wait the GEMM
+ * kernels use, with a limit of `timeout_ns` nanoseconds (1e6 .. 1e10). The
+ * wait gives up, the kernel records SQ_ERR_TIMEOUT in the device status word
+ * and returns; sq_get_device_status then reports it. Used to test the
+ * failure path without faulting or hanging the GPU.
+ */
+sq_status sq_probe_wait_timeout(int64_t timeout_ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SQ_H */

@@ -1,0 +1,139 @@
+"""The C-ABI library loads, exports every entry point include/sq.h declares,
+and rejects bad arguments on the host without launching anything.
+
+No GPU needed: every call here fails validation (or is the M == 0 no-op)
+before the library touches the CUDA runtime, so the fake device addresses
+are never dereferenced.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from w8a8_smoothquant_int8_02_b200 import ops
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sq.h")
+
+A = 0x7F0000000000  # 16-byte aligned fake device address (never dereferenced)
+MIS = A + 1
+NUL = None
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:sq_status|const char\s*\*|int)\s+(sq_\w+)\s*\(",
+                                 text, flags=re.M)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return ops.load()
+
+
+def test_header_declares_the_expected_entry_points():
+    assert set(declared_symbols()) == set(ops.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+        assert ctypes.cast(getattr(lib, name), ctypes.c_void_p).value
+
+
+def test_exported_symbols_are_visible_to_the_dynamic_linker():
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", ops.library_path()],
+                         capture_output=True, text=True, check=True).stdout
+    syms = {l.split()[-1] for l in out.splitlines() if l.strip()}
+    for name in declared_symbols():
+        assert name in syms, name
+
+
+def test_abi_version_and_status_strings(lib):
+    assert lib.sq_abi_version() == 1
+    for st in range(6):
+        assert ops.status_string(st).startswith("SQ_")
+    assert "TIMEOUT" in ops.status_string(ops.SQ_ERR_TIMEOUT)
+
+
+def c(v):
+    return ctypes.c_void_p(v) if v is not None else None
+
+
+def test_quantize_act_validation(lib):
+    f = lib.sq_quantize_act
+    ok = dict(x=A, xt=ops.SQ_BF16, M=4, K=64, s=A, qt=ops.SQ_I8, xq=A, sx=A)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return f(c(a["x"]), a["xt"], a["M"], a["K"], c(a["s"]), a["qt"], c(a["xq"]), c(a["sx"]), None)
+
+    assert call(x=NUL) == ops.SQ_ERR_INVALID_ARG
+    assert call(xq=NUL) == ops.SQ_ERR_INVALID_ARG
+    assert call(sx=NUL) == ops.SQ_ERR_INVALID_ARG
+    assert call(K=0) == ops.SQ_ERR_INVALID_ARG
+    assert call(K=24) == ops.SQ_ERR_INVALID_ARG       # not a multiple of 16
+    assert call(K=65536 + 16) == ops.SQ_ERR_INVALID_ARG
+    assert call(M=-1) == ops.SQ_ERR_INVALID_ARG
+    assert call(xt=ops.SQ_I8) == ops.SQ_ERR_INVALID_ARG
+    assert call(qt=ops.SQ_BF16) == ops.SQ_ERR_INVALID_ARG
+    assert call(x=MIS) == ops.SQ_ERR_MISALIGNED
+    assert call(xq=A + 8) == ops.SQ_ERR_MISALIGNED
+    assert call(s=A + 4) == ops.SQ_ERR_MISALIGNED
+    assert call(M=0) == ops.SQ_OK                      # empty input: no-op
+
+
+def test_gemm_validation(lib):
+    f = lib.sq_gemm_w8a8
+    ok = dict(xq=A, sx=A, wq=A, sw=A, bias=None, M=16, N=64, K=64, y=A, yt=ops.SQ_BF16, acc=None)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return f(c(a["xq"]), c(a["sx"]), c(a["wq"]), c(a["sw"]), c(a["bias"]), a["M"], a["N"],
+                 a["K"], c(a["y"]), a["yt"], c(a["acc"]), None)
+
+    assert call(xq=NUL) == ops.SQ_ERR_INVALID_ARG
+    assert call(wq=NUL) == ops.SQ_ERR_INVALID_ARG
+    assert call(y=NUL) == ops.SQ_ERR_INVALID_ARG
+    assert call(N=0) == ops.SQ_ERR_INVALID_ARG
+    assert call(N=12) == ops.SQ_ERR_INVALID_ARG        # not a multiple of 8
+    assert call(K=40) == ops.SQ_ERR_INVALID_ARG        # not a multiple of 16
+    assert call(K=133152) == ops.SQ_ERR_UNSUPPORTED    # int32 accumulator could overflow
+    assert call(yt=ops.SQ_I8) == ops.SQ_ERR_INVALID_ARG
+    assert call(wq=A + 2) == ops.SQ_ERR_MISALIGNED
+    assert call(y=A + 8) == ops.SQ_ERR_MISALIGNED
+    assert call(bias=A + 1) == ops.SQ_ERR_MISALIGNED
+    assert call(acc=A + 4) == ops.SQ_ERR_MISALIGNED
+    assert call(M=0) == ops.SQ_OK
+    g = lib.sq_gemm_fp8
+    assert g(c(A), c(A), c(A), c(A), None, 16, 64, 40, c(A), ops.SQ_BF16, None) == ops.SQ_ERR_INVALID_ARG
+    assert g(c(A), c(A), c(A), c(A), None, 0, 64, 64, c(A), ops.SQ_BF16, None) == ops.SQ_OK
+
+
+def test_smooth_factor_and_calibration_validation(lib):
+    sf = lib.sq_smooth_factors
+    assert sf(c(A), c(A), 64, 1.5, c(A), None) == ops.SQ_ERR_INVALID_ARG
+    assert sf(c(A), c(A), 64, -0.1, c(A), None) == ops.SQ_ERR_INVALID_ARG
+    assert sf(c(A), c(A), 64, float("nan"), c(A), None) == ops.SQ_ERR_INVALID_ARG
+    assert sf(c(A), c(A), 0, 0.5, c(A), None) == ops.SQ_ERR_INVALID_ARG
+    assert sf(c(A), None, 64, 0.5, c(A), None) == ops.SQ_ERR_INVALID_ARG
+    assert sf(c(A + 2), c(A), 64, 0.5, c(A), None) == ops.SQ_ERR_MISALIGNED
+    ca = lib.sq_calibrate_amax
+    assert ca(c(A), ops.SQ_BF16, 0, 64, 0, c(A), 0, None) == ops.SQ_ERR_INVALID_ARG
+    assert ca(c(A), ops.SQ_BF16, 8, 60, 0, c(A), 0, None) == ops.SQ_ERR_INVALID_ARG
+    assert ca(c(A), ops.SQ_BF16, 8, 64, 7, c(A), 0, None) == ops.SQ_ERR_INVALID_ARG
+    assert ca(c(A), ops.SQ_E4M3, 8, 64, 0, c(A), 0, None) == ops.SQ_ERR_INVALID_ARG
+    assert ca(c(MIS), ops.SQ_BF16, 8, 64, 0, c(A), 0, None) == ops.SQ_ERR_MISALIGNED
+    qw = lib.sq_quantize_weight
+    assert qw(c(A), ops.SQ_BF16, 64, 60, None, ops.SQ_I8, c(A), c(A), None) == ops.SQ_ERR_INVALID_ARG
+    assert qw(c(A), ops.SQ_BF16, 64, 64, None, ops.SQ_I32, c(A), c(A), None) == ops.SQ_ERR_INVALID_ARG
+    assert qw(c(A), ops.SQ_BF16, 64, 64, None, ops.SQ_I8, c(A), c(A + 4), None) == ops.SQ_ERR_MISALIGNED
+    lin = lib.sq_linear
+    assert lin(c(A), ops.SQ_BF16, None, c(A), c(A), None, ops.SQ_I32, 4, 64, 64, c(A), c(A), c(A),
+               ops.SQ_BF16, None) == ops.SQ_ERR_INVALID_ARG
+    assert lin(c(A), ops.SQ_BF16, None, c(A), c(A), None, ops.SQ_I8, 0, 64, 64, c(A), c(A), c(A),
+               ops.SQ_BF16, None) == ops.SQ_OK
+    assert lib.sq_probe_wait_timeout(10, None) == ops.SQ_ERR_INVALID_ARG

@@ -1,0 +1,254 @@
+"""Stage-by-stage parity of the CUDA path against the CPU oracle.
+
+Each GPU stage gets exactly the inputs the oracle gets (seeded synthetic
+data, or the oracle's own outputs of the previous stage), so a one-ulp
+difference upstream cannot cascade. The bar: bit-exact INT8 / E4M3 codes,
+scales, int32 accumulators and INT8-path outputs; smoothing factors within
+2 ulp; the FP8 GEMM within 1e-3 of the exact sum on the normalized metric.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from w8a8_smoothquant_int8_02_b200 import ops, synth
+
+from _gpu_util import dev, fp8_normalized_error, host, ulp_distance
+
+pytestmark = pytest.mark.gpu
+
+E4M3_FINITE = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], np.uint8)
+
+
+def _x(shape, seed, dtype, outliers=True):
+    x = synth.random_floats(shape, seed=seed, std=1.0)
+    if outliers:
+        g = np.random.default_rng(seed + 1000)
+        ch = g.choice(shape[1], size=max(1, shape[1] // 64), replace=False)
+        x[:, ch] *= g.uniform(20, 100, ch.size).astype(np.float32)
+    return synth.to_bf16_bits(x) if dtype == "bf16" else x
+
+
+# ------------------------------------------------------------------ a1 / a2 --
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("rows,cols", [(1, 64), (37, 200), (512, 4096), (3000, 8)])
+def test_calibrate_amax(dtype, rows, cols):
+    x = _x((rows, cols), seed=rows + cols, dtype=dtype)
+    xd = dev(x)
+    np.testing.assert_array_equal(host(ops.calibrate_amax(xd, "column")), oracle.amax(x, True))
+    np.testing.assert_array_equal(host(ops.calibrate_amax(xd, "row")), oracle.amax(x, False))
+
+
+def test_calibrate_amax_accumulates_over_batches():
+    a = _x((64, 128), seed=1, dtype="bf16")
+    b = _x((40, 128), seed=2, dtype="bf16")
+    out = ops.calibrate_amax(dev(a), "column")
+    ops.calibrate_amax(dev(b), "column", out=out, accumulate=True)
+    ref = np.maximum(oracle.amax(a, True), oracle.amax(b, True))
+    np.testing.assert_array_equal(host(out), ref)
+    assert ops.device_status() == ops.SQ_OK
+
+
+# ----------------------------------------------------------------------- a3 --
+
+@pytest.mark.parametrize("alpha", [0.0, 0.5, 0.85, 1.0])
+def test_smooth_factors(alpha):
+    g = np.random.default_rng(3)
+    ax = g.uniform(0.01, 100, 4096).astype(np.float32)
+    aw = g.uniform(1e-4, 0.2, 4096).astype(np.float32)
+    ax[:3] = 0.0
+    aw[3:6] = 0.0
+    got = host(ops.smooth_factors(dev(ax), dev(aw), alpha))
+    ref = oracle.smooth_factors(ax, aw, alpha)
+    d = ulp_distance(got, ref)
+    assert d.max() <= 2, d.max()
+    assert (d == 0).mean() >= 0.99
+
+
+# ----------------------------------------------------------------------- a4 --
+
+@pytest.mark.parametrize("qtype", ["i8", "e4m3"])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("smooth", [True, False])
+@pytest.mark.parametrize("K,N", [(64, 64), (208, 200), (4096, 256), (96, 8)])
+def test_quantize_weight(qtype, dtype, smooth, K, N):
+    w = synth.random_floats((K, N), seed=K * 7 + N, std=0.02)
+    w[:, 0] = 0.0  # an all-zero output channel
+    w = synth.to_bf16_bits(w) if dtype == "bf16" else w
+    s = synth.random_floats(K, seed=K, lo=0.05, hi=20.0) if smooth else None
+    qt = oracle.E4M3 if qtype == "e4m3" else oracle.INT8
+    wq_ref, sw_ref = oracle.quantize_weight(w, s, qt)
+    wq, sw = ops.quantize_weight(dev(w), None if s is None else dev(s), qtype)
+    np.testing.assert_array_equal(host(sw), sw_ref)
+    np.testing.assert_array_equal(host(wq).view(np.uint8), wq_ref.view(np.uint8))
+
+
+# ----------------------------------------------------------------------- a5 --
+
+@pytest.mark.parametrize("qtype", ["i8", "e4m3"])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("smooth", [True, False])
+@pytest.mark.parametrize("M,K", [(1, 64), (17, 96), (129, 4096), (16, 8192), (3, 14336), (5, 16),
+                                 (2, 20000)])
+def test_quantize_act(qtype, dtype, smooth, M, K):
+    x = _x((M, K), seed=M * 31 + K, dtype=dtype)
+    s = synth.random_floats(K, seed=K + 1, lo=0.05, hi=20.0) if smooth else None
+    qt = oracle.E4M3 if qtype == "e4m3" else oracle.INT8
+    xq_ref, sx_ref = oracle.quantize_act(x, s, qt)
+    xq, sx = ops.quantize_act(dev(x), None if s is None else dev(s), qtype)
+    np.testing.assert_array_equal(host(sx), sx_ref)
+    np.testing.assert_array_equal(host(xq).view(np.uint8), xq_ref.view(np.uint8))
+
+
+def test_quantize_act_zero_rows_and_ties():
+    x = np.zeros((4, 32), np.float32)
+    x[1, :10] = [2.5, 3.5, -2.5, 126.5, 127.0, -126.5, 0.5, -0.5, 1.5, 0.49999997]
+    x[3] = np.linspace(-1e-3, 1e-3, 32, dtype=np.float32)
+    for qtype, qt in (("i8", oracle.INT8), ("e4m3", oracle.E4M3)):
+        xq_ref, sx_ref = oracle.quantize_act(x, None, qt)
+        xq, sx = ops.quantize_act(dev(x), None, qtype)
+        np.testing.assert_array_equal(host(sx), sx_ref)
+        np.testing.assert_array_equal(host(xq).view(np.uint8), xq_ref.view(np.uint8))
+
+
+def test_quantize_act_empty_is_noop():
+    x = torch.empty((0, 64), dtype=torch.bfloat16, device="cuda")
+    xq, sx = ops.quantize_act(x, None, "i8")
+    assert xq.shape == (0, 64) and sx.shape == (0,)
+    assert ops.device_status() == ops.SQ_OK
+
+
+# ------------------------------------------------------------------ a6 INT8 --
+
+GEMM_SHAPES = [(1, 16, 32), (17, 64, 64), (129, 200, 96), (128, 128, 128), (300, 392, 4096),
+               (256, 256, 208), (7, 8, 16), (640, 136, 1040)]
+
+
+@pytest.mark.parametrize("M,N,K", GEMM_SHAPES)
+@pytest.mark.parametrize("with_bias", [False, True])
+def test_gemm_w8a8(M, N, K, with_bias):
+    xq = synth.random_matrix((M, K), np.int8, seed=M + K)
+    wq = synth.random_matrix((N, K), np.int8, seed=N + 2 * K)
+    sx = synth.random_floats(M, seed=5, lo=1e-3, hi=0.5)
+    sw = synth.random_floats(N, seed=6, lo=1e-4, hi=1e-2)
+    bias = synth.to_bf16_bits(synth.random_floats(N, seed=7, std=0.1)) if with_bias else None
+    acc_ref = oracle.gemm_i8(xq, wq)
+    yf_ref, yb_ref = oracle.epilogue(acc_ref, sx, sw, bias)
+    d = [dev(a) for a in (xq, sx, wq, sw)]
+    b = None if bias is None else dev(bias)
+    acc = torch.empty((M, N), dtype=torch.int32, device="cuda")
+    yf = ops.gemm_w8a8(*d, bias=b, out_dtype=torch.float32, acc=acc)
+    yb = ops.gemm_w8a8(*d, bias=b, out_dtype=torch.bfloat16)
+    assert ops.device_status() == ops.SQ_OK
+    np.testing.assert_array_equal(host(acc), acc_ref)
+    np.testing.assert_array_equal(host(yf), yf_ref)
+    np.testing.assert_array_equal(host(yb), yb_ref)
+
+
+def test_gemm_w8a8_extreme_accumulators():
+    M, N, K = 130, 136, 16384
+    xq = np.full((M, K), 127, np.int8)
+    xq[1::2] = -127
+    wq = np.full((N, K), 127, np.int8)
+    wq[5] = -127
+    wq[7] = 0
+    wq[7, 1234] = 1
+    sx = np.ones(M, np.float32)
+    sw = np.ones(N, np.float32)
+    acc = torch.empty((M, N), dtype=torch.int32, device="cuda")
+    ops.gemm_w8a8(dev(xq), dev(sx), dev(wq), dev(sw), out_dtype=torch.float32, acc=acc)
+    a = host(acc)
+    assert a[0, 0] == K * 127 * 127 and a[1, 0] == -K * 127 * 127 and a[1, 5] == K * 127 * 127
+    assert a[0, 7] == 127 and a[1, 7] == -127
+    np.testing.assert_array_equal(a, oracle.gemm_i8(xq, wq))
+
+
+def test_gemm_does_not_write_outside_output():
+    M, N, K = 100, 72, 64
+    xq = synth.random_matrix((M, K), np.int8, seed=11)
+    wq = synth.random_matrix((N, K), np.int8, seed=12)
+    sx = synth.random_floats(M, seed=13, lo=0.01, hi=0.1)
+    sw = synth.random_floats(N, seed=14, lo=0.01, hi=0.1)
+    guard = 4096
+    buf = torch.full((M * N + 2 * guard,), -7777.0, dtype=torch.float32, device="cuda")
+    out = buf[guard:guard + M * N].view(M, N)
+    ops.gemm_w8a8(dev(xq), dev(sx), dev(wq), dev(sw), out=out)
+    h = host(buf)
+    assert (h[:guard] == -7777.0).all() and (h[guard + M * N:] == -7777.0).all()
+    np.testing.assert_array_equal(host(out), oracle.epilogue(oracle.gemm_i8(xq, wq), sx, sw)[0])
+
+
+# ------------------------------------------------------------------ a7 FP8 --
+
+@pytest.mark.parametrize("M,N,K", [(1, 16, 32), (17, 64, 64), (129, 200, 96), (300, 392, 4096),
+                                   (256, 256, 14336)])
+@pytest.mark.parametrize("with_bias", [False, True])
+def test_gemm_fp8(M, N, K, with_bias):
+    g = np.random.default_rng(M * N + K)
+    mag = np.abs(oracle.e4m3_decode(E4M3_FINITE))
+    codes = E4M3_FINITE[(mag <= 64.0)]
+    xq = g.choice(codes, size=(M, K)).astype(np.uint8)
+    wq = g.choice(codes, size=(N, K)).astype(np.uint8)
+    sx = synth.random_floats(M, seed=21, lo=1e-3, hi=0.5)
+    sw = synth.random_floats(N, seed=22, lo=1e-4, hi=1e-2)
+    bias = synth.to_bf16_bits(synth.random_floats(N, seed=23, std=0.1)) if with_bias else None
+    acc_ref = oracle.gemm_e4m3(xq, wq)
+    yf_ref, _ = oracle.epilogue(acc_ref, sx, sw, bias)
+    yf = ops.gemm_fp8(dev(xq), dev(sx), dev(wq), dev(sw), bias=None if bias is None else dev(bias),
+                      out_dtype=torch.float32)
+    yb = ops.gemm_fp8(dev(xq), dev(sx), dev(wq), dev(sw), bias=None if bias is None else dev(bias))
+    assert ops.device_status() == ops.SQ_OK
+    rows, cols = np.divmod(np.arange(M * N, dtype=np.int64), N)
+    e = fp8_normalized_error(host(yf).reshape(-1), yf_ref.reshape(-1), xq, wq, sx, sw, bias, rows, cols)
+    assert e.max() <= 1e-3, e.max()
+    # the bf16 output is the nearest-even rounding of the same binary32 values
+    # (the tensor-core summation order is fixed for a given launch shape)
+    np.testing.assert_array_equal(host(yb), oracle.f32_to_bf16(host(yf)))
+
+
+# --------------------------------------------------------- the whole layer --
+
+@pytest.mark.parametrize("qtype", ["i8", "e4m3"])
+def test_linear_matches_oracle(qtype):
+    M, K, N = 77, 320, 136
+    x = _x((M, K), seed=99, dtype="bf16")
+    w = synth.to_bf16_bits(synth.random_floats((K, N), seed=98, std=0.02))
+    bias = synth.to_bf16_bits(synth.random_floats(N, seed=97, std=0.01))
+    qt = oracle.E4M3 if qtype == "e4m3" else oracle.INT8
+    s = oracle.smooth_factors(oracle.amax(x, True), oracle.amax(w, False), 0.5)
+    wq, sw = oracle.quantize_weight(w, s, qt)
+    ref = oracle.linear(x, s, wq, sw, bias, qt)
+    y = ops.linear(dev(x), dev(s), dev(wq), dev(sw), dev(bias), qtype, out_dtype=torch.float32)
+    assert ops.device_status() == ops.SQ_OK
+    if qtype == "i8":
+        np.testing.assert_array_equal(host(y), ref["y_f32"])
+    else:
+        rows, cols = np.divmod(np.arange(M * N, dtype=np.int64), N)
+        e = fp8_normalized_error(host(y).reshape(-1), ref["y_f32"].reshape(-1), ref["xq"], wq,
+                                 ref["sx"], sw, bias, rows, cols)
+        assert e.max() <= 1e-3
+
+
+def test_prepare_pipeline_matches_oracle():
+    x_cal = _x((64, 256), seed=5, dtype="bf16")
+    w = synth.to_bf16_bits(synth.random_floats((256, 64), seed=6, std=0.02))
+    p = ops.prepare(dev(w), dev(x_cal), alpha=0.5, qtype="i8")
+    ax, aw = oracle.amax(x_cal, True), oracle.amax(w, False)
+    np.testing.assert_array_equal(host(p["amax_x"]), ax)
+    np.testing.assert_array_equal(host(p["amax_w"]), aw)
+    s = oracle.smooth_factors(ax, aw, 0.5)
+    assert ulp_distance(host(p["s"]), s).max() <= 2
+
+
+# ---------------------------------------------------------- failure path --
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    assert ops.device_status() == ops.SQ_OK
+    ops.probe_wait_timeout(20_000_000)  # 20 ms
+    assert ops.device_status() == ops.SQ_ERR_TIMEOUT
+    assert ops.device_status() == ops.SQ_OK  # read-and-clear
+    # the context is still usable
+    x = _x((4, 64), seed=1, dtype="bf16")
+    xq, sx = ops.quantize_act(dev(x), None, "i8")
+    np.testing.assert_array_equal(host(xq), oracle.quantize_act(x, None)[0])

@@ -1,0 +1,190 @@
+// sq_api.cu -- the C ABI of libsq.so (declared in include/sq.h).
+//
+// Argument validation happens here, synchronously, before anything is
+// launched; the launchers in sq_quant.cu / sq_gemm.cu assume valid input.
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "sq.h"
+#include "sq_common.cuh"
+#include "sq_internal.h"
+
+// The library's only device allocation: one status word per device that a
+// kernel sets when a bounded wait gives up.
+static __device__ int g_sq_status = 0;
+
+namespace sqh {
+
+int* status_ptr() {
+  // One lookup per device (the symbol has a different address per device).
+  static int* ptrs[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_sq_status) != cudaSuccess) return nullptr;
+    ptrs[dev] = static_cast<int*>(p);
+  }
+  return ptrs[dev];
+}
+
+}  // namespace sqh
+
+namespace {
+
+__global__ void probe_wait_kernel(int64_t timeout_ns, int* status) {
+  __shared__ __align__(8) uint64_t bar;
+  const uint32_t b = sqk::smem_u32(&bar);
+  if (threadIdx.x == 0) {
+    sqk::mbar_init(b, 1);
+    sqk::fence_barrier_init();
+    // Nothing ever arrives on `bar`, so phase 0 never completes.
+    if (!sqk::mbar_wait(b, 0, uint64_t(timeout_ns))) sqk::record_status(status, sqk::kStatusTimeout);
+  }
+}
+
+inline bool al(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+inline cudaStream_t S(void* st) { return static_cast<cudaStream_t>(st); }
+inline sq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? SQ_OK : SQ_ERR_CUDA; }
+
+// Common checks for the 8-bit GEMMs.
+sq_status check_gemm(const void* xq, const float* sx, const void* wq, const float* sw,
+                     const uint16_t* bias, int64_t M, int64_t N, int64_t K, const void* y,
+                     sq_dtype yt, const int32_t* acc) {
+  if (M < 0 || N <= 0 || K <= 0 || K % 16 != 0 || N % 8 != 0) return SQ_ERR_INVALID_ARG;
+  if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return SQ_ERR_INVALID_ARG;
+  if (K >= 133144) return SQ_ERR_UNSUPPORTED;  // int32 accumulator bound K*127^2 < 2^31
+  if (yt != SQ_BF16 && yt != SQ_F32) return SQ_ERR_INVALID_ARG;
+  if (M == 0) return SQ_OK;  // empty batch: pointers may be NULL
+  if (!xq || !sx || !wq || !sw || !y) return SQ_ERR_INVALID_ARG;
+  if (!al(xq, 16) || !al(wq, 16) || !al(y, 16) || !al(sx, 4) || !al(sw, 4)) return SQ_ERR_MISALIGNED;
+  if (bias && !al(bias, 2)) return SQ_ERR_MISALIGNED;
+  if (acc && !al(acc, 16)) return SQ_ERR_MISALIGNED;
+  return SQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* sq_status_string(sq_status st) {
+  switch (st) {
+    case SQ_OK: return "SQ_OK";
+    case SQ_ERR_INVALID_ARG: return "SQ_ERR_INVALID_ARG: invalid argument";
+    case SQ_ERR_MISALIGNED: return "SQ_ERR_MISALIGNED: pointer not aligned as required";
+    case SQ_ERR_UNSUPPORTED: return "SQ_ERR_UNSUPPORTED: unsupported combination";
+    case SQ_ERR_CUDA: return "SQ_ERR_CUDA: CUDA runtime error";
+    case SQ_ERR_TIMEOUT: return "SQ_ERR_TIMEOUT: a bounded device wait gave up";
+  }
+  return "SQ_ERR_UNKNOWN";
+}
+
+int sq_abi_version(void) { return SQ_ABI_VERSION; }
+
+sq_status sq_get_device_status(void* stream) {
+  if (cudaStreamSynchronize(S(stream)) != cudaSuccess) return SQ_ERR_CUDA;
+  int* p = sqh::status_ptr();
+  if (!p) return SQ_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, p, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return SQ_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpy(p, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return SQ_ERR_CUDA;
+  }
+  return v == 0 ? SQ_OK : static_cast<sq_status>(v);
+}
+
+sq_status sq_calibrate_amax(const void* x, sq_dtype xt, int64_t rows, int64_t cols, sq_axis axis,
+                            float* amax, int accumulate, void* stream) {
+  if (!x || !amax) return SQ_ERR_INVALID_ARG;
+  if (xt != SQ_F32 && xt != SQ_BF16) return SQ_ERR_INVALID_ARG;
+  if (axis != SQ_AMAX_PER_COLUMN && axis != SQ_AMAX_PER_ROW) return SQ_ERR_INVALID_ARG;
+  if (rows <= 0 || cols <= 0 || cols % 8 != 0 || rows > INT32_MAX) return SQ_ERR_INVALID_ARG;
+  if (!al(x, 16) || !al(amax, 4)) return SQ_ERR_MISALIGNED;
+  const bool bf = xt == SQ_BF16;
+  if (axis == SQ_AMAX_PER_COLUMN)
+    return from_cuda(sqh::launch_amax_cols(x, bf, rows, cols, amax, accumulate != 0, S(stream)));
+  return from_cuda(sqh::launch_amax_rows(x, bf, rows, cols, amax, accumulate != 0, S(stream)));
+}
+
+sq_status sq_smooth_factors(const float* amax_x, const float* amax_w, int64_t K, double alpha,
+                            float* s, void* stream) {
+  if (!amax_x || !amax_w || !s || K <= 0) return SQ_ERR_INVALID_ARG;
+  if (!(alpha >= 0.0 && alpha <= 1.0)) return SQ_ERR_INVALID_ARG;  // also rejects NaN
+  if (!al(amax_x, 4) || !al(amax_w, 4) || !al(s, 4)) return SQ_ERR_MISALIGNED;
+  return from_cuda(sqh::launch_smooth_factors(amax_x, amax_w, K, alpha, s, S(stream)));
+}
+
+sq_status sq_quantize_weight(const void* w, sq_dtype wt, int64_t K, int64_t N, const float* s,
+                             sq_dtype qt, void* wq, float* sw, void* stream) {
+  if (!w || !wq || !sw) return SQ_ERR_INVALID_ARG;
+  if (wt != SQ_F32 && wt != SQ_BF16) return SQ_ERR_INVALID_ARG;
+  if (qt != SQ_I8 && qt != SQ_E4M3) return SQ_ERR_INVALID_ARG;
+  if (K <= 0 || N <= 0 || K % 16 != 0 || N % 8 != 0 || K > INT32_MAX || N > INT32_MAX)
+    return SQ_ERR_INVALID_ARG;
+  if (!al(w, 16) || !al(wq, 16) || !al(sw, 16)) return SQ_ERR_MISALIGNED;
+  if (s && !al(s, 4)) return SQ_ERR_MISALIGNED;
+  return from_cuda(sqh::launch_quantize_weight(w, wt == SQ_BF16, K, N, s, qt == SQ_E4M3,
+                                               static_cast<uint8_t*>(wq), sw, S(stream)));
+}
+
+sq_status sq_quantize_act(const void* x, sq_dtype xt, int64_t M, int64_t K, const float* s,
+                          sq_dtype qt, void* xq, float* sx, void* stream) {
+  if (xt != SQ_F32 && xt != SQ_BF16) return SQ_ERR_INVALID_ARG;
+  if (qt != SQ_I8 && qt != SQ_E4M3) return SQ_ERR_INVALID_ARG;
+  if (M < 0 || K <= 0 || K % 16 != 0 || K > 65536 || M > INT32_MAX) return SQ_ERR_INVALID_ARG;
+  if (M == 0) return SQ_OK;  // empty batch: pointers may be NULL
+  if (!x || !xq || !sx) return SQ_ERR_INVALID_ARG;
+  if (!al(x, 16) || !al(xq, 16) || !al(sx, 4)) return SQ_ERR_MISALIGNED;
+  if (s && !al(s, 16)) return SQ_ERR_MISALIGNED;
+  return from_cuda(sqh::launch_quantize_act(x, xt == SQ_BF16, M, K, s, qt == SQ_E4M3,
+                                            static_cast<uint8_t*>(xq), sx, S(stream)));
+}
+
+sq_status sq_gemm_w8a8(const int8_t* xq, const float* sx, const int8_t* wq, const float* sw,
+                       const uint16_t* bias, int64_t M, int64_t N, int64_t K, void* y, sq_dtype yt,
+                       int32_t* acc, void* stream) {
+  sq_status c = check_gemm(xq, sx, wq, sw, bias, M, N, K, y, yt, acc);
+  if (c != SQ_OK) return c;
+  if (M == 0) return SQ_OK;
+  return from_cuda(sqh::launch_gemm(false, reinterpret_cast<const uint8_t*>(xq), sx,
+                                    reinterpret_cast<const uint8_t*>(wq), sw, bias, M, N, K, y,
+                                    yt == SQ_BF16 ? sqh::OutKind::BF16 : sqh::OutKind::F32, acc,
+                                    S(stream)));
+}
+
+sq_status sq_gemm_fp8(const uint8_t* xq, const float* sx, const uint8_t* wq, const float* sw,
+                      const uint16_t* bias, int64_t M, int64_t N, int64_t K, void* y, sq_dtype yt,
+                      void* stream) {
+  sq_status c = check_gemm(xq, sx, wq, sw, bias, M, N, K, y, yt, nullptr);
+  if (c != SQ_OK) return c;
+  if (M == 0) return SQ_OK;
+  return from_cuda(sqh::launch_gemm(true, xq, sx, wq, sw, bias, M, N, K, y,
+                                    yt == SQ_BF16 ? sqh::OutKind::BF16 : sqh::OutKind::F32, nullptr,
+                                    S(stream)));
+}
+
+sq_status sq_linear(const void* x, sq_dtype xt, const float* s, const void* wq, const float* sw,
+                    const uint16_t* bias, sq_dtype qt, int64_t M, int64_t N, int64_t K,
+                    void* xq_buf, float* sx_buf, void* y, sq_dtype yt, void* stream) {
+  if (qt != SQ_I8 && qt != SQ_E4M3) return SQ_ERR_INVALID_ARG;
+  sq_status c = check_gemm(xq_buf, sx_buf, wq, sw, bias, M, N, K, y, yt, nullptr);
+  if (c != SQ_OK || M == 0) return c;
+  c = sq_quantize_act(x, xt, M, K, s, qt, xq_buf, sx_buf, stream);
+  if (c != SQ_OK) return c;
+  if (qt == SQ_I8)
+    return sq_gemm_w8a8(static_cast<const int8_t*>(xq_buf), sx_buf, static_cast<const int8_t*>(wq),
+                        sw, bias, M, N, K, y, yt, nullptr, stream);
+  return sq_gemm_fp8(static_cast<const uint8_t*>(xq_buf), sx_buf, static_cast<const uint8_t*>(wq),
+                     sw, bias, M, N, K, y, yt, stream);
+}
+
+sq_status sq_probe_wait_timeout(int64_t timeout_ns, void* stream) {
+  if (timeout_ns < 1000000 || timeout_ns > 10000000000LL) return SQ_ERR_INVALID_ARG;
+  int* st = sqh::status_ptr();
+  if (!st) return SQ_ERR_CUDA;
+  probe_wait_kernel<<<1, 32, 0, S(stream)>>>(timeout_ns, st);
+  return from_cuda(cudaGetLastError());
+}
+
+}  // extern "C"

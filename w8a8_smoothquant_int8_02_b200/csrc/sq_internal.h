@@ -1,0 +1,34 @@
+// sq_internal.h -- host-side launchers shared between the libsq translation
+// units. Arguments are already validated by the C-ABI layer (sq_api.cu).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace sqh {
+
+// Device address of the library's status word (see sq_get_device_status).
+int* status_ptr();
+
+// a1 / a2
+cudaError_t launch_amax_cols(const void* x, bool bf16, int64_t rows, int64_t cols, float* amax,
+                             bool accumulate, cudaStream_t st);
+cudaError_t launch_amax_rows(const void* x, bool bf16, int64_t rows, int64_t cols, float* amax,
+                             bool accumulate, cudaStream_t st);
+// a3
+cudaError_t launch_smooth_factors(const float* ax, const float* aw, int64_t K, double alpha,
+                                  float* s, cudaStream_t st);
+// a4
+cudaError_t launch_quantize_weight(const void* w, bool bf16, int64_t K, int64_t N, const float* s,
+                                   bool e4m3, uint8_t* wq, float* sw, cudaStream_t st);
+// a5
+cudaError_t launch_quantize_act(const void* x, bool bf16, int64_t M, int64_t K, const float* s,
+                                bool e4m3, uint8_t* xq, float* sx, cudaStream_t st);
+// a6 / a7
+enum class OutKind { BF16, F32 };
+cudaError_t launch_gemm(bool e4m3, const uint8_t* xq, const float* sx, const uint8_t* wq,
+                        const float* sw, const uint16_t* bias, int64_t M, int64_t N, int64_t K,
+                        void* y, OutKind yk, int32_t* acc, cudaStream_t st);
+
+
+}  // namespace sqh

@@ -1,0 +1,251 @@
+"""Python binding of libsq.so (the C ABI in include/sq.h).
+
+Argument marshalling only: every step of the layer runs in the CUDA library.
+torch supplies device memory and the current stream. If the library cannot
+be built or loaded, every call raises -- there is no CPU fallback.
+
+Layouts follow include/sq.h: X [M,K], W [K,N], Wq [N,K] (K contiguous),
+Y [M,N], all row-major; bf16 tensors are passed as torch.bfloat16, E4M3 codes
+as torch.uint8 or torch.float8_e4m3fn.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+from . import build as _build
+
+SQ_OK, SQ_ERR_INVALID_ARG, SQ_ERR_MISALIGNED, SQ_ERR_UNSUPPORTED, SQ_ERR_CUDA, SQ_ERR_TIMEOUT = range(6)
+SQ_F32, SQ_BF16, SQ_I8, SQ_E4M3, SQ_I32 = range(5)
+SQ_AMAX_PER_COLUMN, SQ_AMAX_PER_ROW = 0, 1
+
+EXPORTED = (
+    "sq_status_string", "sq_abi_version", "sq_get_device_status", "sq_calibrate_amax",
+    "sq_smooth_factors", "sq_quantize_weight", "sq_quantize_act", "sq_gemm_w8a8",
+    "sq_gemm_fp8", "sq_linear", "sq_probe_wait_timeout",
+)
+
+_lock = threading.Lock()
+_lib = None
+
+
+class SQError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)}")
+
+
+def library_path() -> str:
+    return _build.LIB
+
+
+def load(build_if_needed: bool = True) -> ctypes.CDLL:
+    """Load libsq.so (building it first with nvcc if it is missing or stale)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if build_if_needed and _build.is_stale():
+                _build.build()
+            if not os.path.exists(_build.LIB):
+                raise RuntimeError(f"libsq.so not found at {_build.LIB}; build it with "
+                                   "`python -m w8a8_smoothquant_int8_02_b200.build`")
+            lib = ctypes.CDLL(_build.LIB)
+            P, I64, I, D = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_double
+            lib.sq_status_string.argtypes = [I]
+            lib.sq_status_string.restype = ctypes.c_char_p
+            lib.sq_abi_version.restype = I
+            lib.sq_get_device_status.argtypes = [P]
+            lib.sq_calibrate_amax.argtypes = [P, I, I64, I64, I, P, I, P]
+            lib.sq_smooth_factors.argtypes = [P, P, I64, D, P, P]
+            lib.sq_quantize_weight.argtypes = [P, I, I64, I64, P, I, P, P, P]
+            lib.sq_quantize_act.argtypes = [P, I, I64, I64, P, I, P, P, P]
+            lib.sq_gemm_w8a8.argtypes = [P, P, P, P, P, I64, I64, I64, P, I, P, P]
+            lib.sq_gemm_fp8.argtypes = [P, P, P, P, P, I64, I64, I64, P, I, P]
+            lib.sq_linear.argtypes = [P, I, P, P, P, P, I, I64, I64, I64, P, P, P, I, P]
+            lib.sq_probe_wait_timeout.argtypes = [I64, P]
+            for name in EXPORTED:
+                if name not in ("sq_status_string", "sq_abi_version"):
+                    getattr(lib, name).restype = I
+            _lib = lib
+    return _lib
+
+
+def status_string(st: int) -> str:
+    return load().sq_status_string(int(st)).decode()
+
+
+def _check(st: int, what: str):
+    if st != SQ_OK:
+        raise SQError(st, what)
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device=None):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _fdtype(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return SQ_BF16
+    if t.dtype == torch.float32:
+        return SQ_F32
+    raise TypeError(f"expected a bfloat16 or float32 tensor, got {t.dtype}")
+
+
+def _qtype(q: str) -> int:
+    if q in ("i8", "int8"):
+        return SQ_I8
+    if q in ("e4m3", "fp8"):
+        return SQ_E4M3
+    raise ValueError(f"qtype must be 'i8' or 'e4m3', got {q!r}")
+
+
+def _cuda(*ts):
+    for t in ts:
+        if t is not None:
+            if not t.is_cuda:
+                raise ValueError("all tensors must be CUDA tensors")
+            if not t.is_contiguous():
+                raise ValueError("all tensors must be contiguous")
+
+
+def _codes(t: torch.Tensor) -> torch.Tensor:
+    return t.view(torch.uint8) if t.dtype == torch.float8_e4m3fn else t
+
+
+# ---------------------------------------------------------------- stages --
+
+def calibrate_amax(x: torch.Tensor, axis: str = "column", out: torch.Tensor | None = None,
+                   accumulate: bool = False) -> torch.Tensor:
+    """a1/a2: per-column ("column", over rows) or per-row ("row") max |x|."""
+    _cuda(x, out)
+    rows, cols = x.shape
+    ax = SQ_AMAX_PER_COLUMN if axis == "column" else SQ_AMAX_PER_ROW
+    n = cols if ax == SQ_AMAX_PER_COLUMN else rows
+    if out is None:
+        out = torch.empty(n, dtype=torch.float32, device=x.device)
+    _check(load().sq_calibrate_amax(_p(x), _fdtype(x), rows, cols, ax, _p(out), int(accumulate),
+                                    _stream(x.device)), "sq_calibrate_amax")
+    return out
+
+
+def smooth_factors(amax_x: torch.Tensor, amax_w: torch.Tensor, alpha: float) -> torch.Tensor:
+    """a3: s = max(ax,1e-5)^alpha / max(aw,1e-5)^(1-alpha) (binary64 -> binary32)."""
+    _cuda(amax_x, amax_w)
+    s = torch.empty_like(amax_x)
+    _check(load().sq_smooth_factors(_p(amax_x), _p(amax_w), amax_x.numel(), float(alpha), _p(s),
+                                    _stream(amax_x.device)), "sq_smooth_factors")
+    return s
+
+
+def quantize_weight(w: torch.Tensor, s: torch.Tensor | None, qtype: str = "i8"):
+    """a4: returns (wq [N,K] int8 / uint8-E4M3, sw [N] float32)."""
+    _cuda(w, s)
+    K, N = w.shape
+    qt = _qtype(qtype)
+    wq = torch.empty((N, K), dtype=torch.int8 if qt == SQ_I8 else torch.uint8, device=w.device)
+    sw = torch.empty(N, dtype=torch.float32, device=w.device)
+    _check(load().sq_quantize_weight(_p(w), _fdtype(w), K, N, _p(s), qt, _p(wq), _p(sw),
+                                     _stream(w.device)), "sq_quantize_weight")
+    return wq, sw
+
+
+def quantize_act(x: torch.Tensor, s: torch.Tensor | None, qtype: str = "i8", xq=None, sx=None):
+    """a5: fused smoothing + per-token quantization; returns (xq [M,K], sx [M])."""
+    _cuda(x, s, xq, sx)
+    M, K = x.shape
+    qt = _qtype(qtype)
+    if xq is None:
+        xq = torch.empty((M, K), dtype=torch.int8 if qt == SQ_I8 else torch.uint8, device=x.device)
+    if sx is None:
+        sx = torch.empty(M, dtype=torch.float32, device=x.device)
+    _check(load().sq_quantize_act(_p(x), _fdtype(x), M, K, _p(s), qt, _p(xq), _p(sx),
+                                  _stream(x.device)), "sq_quantize_act")
+    return xq, sx
+
+
+def gemm_w8a8(xq, sx, wq, sw, bias=None, out_dtype=torch.bfloat16, out=None, acc=None):
+    """a6: INT8 tensor-core GEMM + dequant epilogue. Returns y (and fills acc if given)."""
+    _cuda(xq, sx, wq, sw, bias, out, acc)
+    M, K = xq.shape
+    N = wq.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=xq.device)
+    _check(load().sq_gemm_w8a8(_p(xq), _p(sx), _p(wq), _p(sw), _p(bias), M, N, K, _p(out),
+                               _fdtype(out), _p(acc), _stream(xq.device)), "sq_gemm_w8a8")
+    return out
+
+
+def gemm_fp8(xq, sx, wq, sw, bias=None, out_dtype=torch.bfloat16, out=None):
+    """a7: FP8 E4M3 tensor-core GEMM + dequant epilogue."""
+    xq, wq = _codes(xq), _codes(wq)
+    _cuda(xq, sx, wq, sw, bias, out)
+    M, K = xq.shape
+    N = wq.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=xq.device)
+    _check(load().sq_gemm_fp8(_p(xq), _p(sx), _p(wq), _p(sw), _p(bias), M, N, K, _p(out),
+                              _fdtype(out), _stream(xq.device)), "sq_gemm_fp8")
+    return out
+
+
+def linear(x, s, wq, sw, bias=None, qtype="i8", out_dtype=torch.bfloat16, out=None,
+           xq_buf=None, sx_buf=None):
+    """Runtime forward: quantize_act then the 8-bit GEMM, one C call."""
+    wq = _codes(wq)
+    _cuda(x, s, wq, sw, bias, out, xq_buf, sx_buf)
+    M, K = x.shape
+    N = wq.shape[0]
+    qt = _qtype(qtype)
+    if xq_buf is None:
+        xq_buf = torch.empty((M, K), dtype=torch.int8 if qt == SQ_I8 else torch.uint8,
+                             device=x.device)
+    if sx_buf is None:
+        sx_buf = torch.empty(M, dtype=torch.float32, device=x.device)
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=x.device)
+    _check(load().sq_linear(_p(x), _fdtype(x), _p(s), _p(wq), _p(sw), _p(bias), qt, M, N, K,
+                            _p(xq_buf), _p(sx_buf), _p(out), _fdtype(out), _stream(x.device)),
+           "sq_linear")
+    return out
+
+
+def device_status(device=None) -> int:
+    """Synchronize the current stream and return (and clear) the status word."""
+    return int(load().sq_get_device_status(_stream(device)))
+
+
+def probe_wait_timeout(timeout_ns: int, device=None):
+    _check(load().sq_probe_wait_timeout(int(timeout_ns), _stream(device)), "sq_probe_wait_timeout")
+
+
+# ------------------------------------------------------------ a layer API --
+
+def prepare(w: torch.Tensor, x_cal: torch.Tensor, alpha: float = 0.5, qtype: str = "i8"):
+    """Offline preparation of one layer: calibrate, smoothing factors, quantized weights."""
+    ax = calibrate_amax(x_cal, "column")
+    aw = calibrate_amax(w, "row")
+    s = smooth_factors(ax, aw, alpha)
+    wq, sw = quantize_weight(w, s, qtype)
+    return dict(s=s, wq=wq, sw=sw, amax_x=ax, amax_w=aw)
+
+
+class SmoothQuantLinear:
+    """A prepared SmoothQuant W8A8 linear layer: y = x @ W (+ bias)."""
+
+    def __init__(self, w: torch.Tensor, x_cal: torch.Tensor, alpha: float = 0.5,
+                 qtype: str = "i8", bias: torch.Tensor | None = None):
+        p = prepare(w, x_cal, alpha, qtype)
+        self.s, self.wq, self.sw = p["s"], p["wq"], p["sw"]
+        self.qtype = qtype
+        self.bias = bias
+        self.in_features, self.out_features = w.shape
+
+    def __call__(self, x: torch.Tensor, out_dtype=torch.bfloat16) -> torch.Tensor:
+        return linear(x, self.s, self.wq, self.sw, self.bias, self.qtype, out_dtype)
