@@ -37,7 +37,24 @@ sys.path.insert(0, ROOT)
 
 METRIC = "W8A8 smooth+quant+GEMM TOPS and % of INT8 TC peak at M4096 K4096 N14336"
 UNIT = "TOPS"
-ROTATE = 3
+L2_BYTES = 126 * 2 ** 20
+
+
+def metric_for(case):
+    if case.name.startswith("mlp_up"):
+        return METRIC
+    kind = "FP8" if case.qtype == "e4m3" else "INT8"
+    return (f"W8A8 smooth+quant+GEMM TOPS and % of {kind} TC peak at "
+            f"M{case.M} K{case.K} N{case.N}")
+
+
+def rotate_count(case):
+    """Input sets to rotate through so that the inputs of one step are not
+    left in L2 by the previous steps (X and Wq of all sets > 1.5 x L2)."""
+    per_set = case.M * case.K * 2 + case.N * case.K
+    if per_set >= 1.5 * L2_BYTES:
+        return 1
+    return max(2, -(-int(1.5 * L2_BYTES) // per_set))
 
 
 def _peaks():
@@ -151,23 +168,29 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
-def cpu_baseline(case, d, s, wq, sw, budget_s: float):
-    """Oracle throughput on a bounded sample of the workload (rank 0, N=1 only)."""
+def cpu_baseline(case, d, budget_s: float):
+    """Oracle throughput on a bounded sample of the workload (rank 0, N=1 only).
+    The oracle prepares its own weights (untimed), then runs the runtime path
+    (activation quant + 8-bit GEMM + epilogue) on as many token rows as fit
+    in about `budget_s` seconds."""
     import oracle
+    qt = oracle.E4M3 if case.qtype == "e4m3" else oracle.INT8
+    s = oracle.smooth_factors(oracle.amax(d["x_cal"], True), oracle.amax(d["w"], False), case.alpha)
+    wq, sw = oracle.quantize_weight(d["w"], s, qt)
     rows = 2
     xs = np.ascontiguousarray(d["x"][:rows])
     t0 = time.perf_counter()
-    oracle.linear(xs, s, wq, sw, d["bias"])
+    oracle.linear(xs, s, wq, sw, d["bias"], qt)
     dt = time.perf_counter() - t0
     rows2 = int(max(2, min(case.M, rows * budget_s / max(dt, 1e-3))))
     xs = np.ascontiguousarray(d["x"][:rows2])
     t0 = time.perf_counter()
-    oracle.linear(xs, s, wq, sw, d["bias"])
+    oracle.linear(xs, s, wq, sw, d["bias"], qt)
     dt = time.perf_counter() - t0
     return {"value": 2.0 * rows2 * case.N * case.K / dt / 1e12, "unit": UNIT,
             "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": f"{rows2} of {case.M} token rows through the whole layer (act quant + "
-                      f"INT8 GEMM + epilogue), full K={case.K} and N={case.N}; {dt:.1f} s"}
+            "sample": f"{rows2} of {case.M} token rows through the runtime path (act quant + "
+                      f"8-bit GEMM + epilogue), full K={case.K} and N={case.N}; {dt:.1f} s"}
 
 
 def run_ours(args):
@@ -177,14 +200,18 @@ def run_ours(args):
     from w8a8_smoothquant_int8_02_b200 import ops, synth, workloads
 
     ws, rank, local = _dist()
+    if args.tile:
+        os.environ["SQ_GEMM_TILE"] = args.tile
     torch.cuda.set_device(local)
     if ws > 1:
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
     ops.load()
-    case = workloads.MLP_UP
+    case = workloads.ALL[args.workload]
     M, K, N = case.M, case.K, case.N
+    qt = case.qtype
+    ROTATE = rotate_count(case)
     dev = torch.device("cuda", local)
     d = synth.generate(case)
 
@@ -196,24 +223,25 @@ def run_ours(args):
 
     # ---- offline preparation (untimed) ----
     w = to_dev(d["w"])
-    p = ops.prepare(w, to_dev(d["x_cal"]), alpha=case.alpha, qtype="i8")
+    p = ops.prepare(w, to_dev(d["x_cal"]), alpha=case.alpha, qtype=qt)
     s, wq0, sw = p["s"], p["wq"], p["sw"]
-    bias = to_dev(d["bias"])
+    bias = to_dev(d["bias"]) if d["bias"] is not None else None
+    gemm = ops.gemm_w8a8 if qt == "i8" else ops.gemm_fp8
     del w
     xs = [to_dev(d["x"])] + [None] * (ROTATE - 1)
     wqs = [wq0] + [None] * (ROTATE - 1)
     for r in range(1, ROTATE):
         xs[r] = xs[0].clone()
         wqs[r] = wq0.clone()
-    xq = torch.empty((M, K), dtype=torch.int8, device=dev)
+    xq = torch.empty((M, K), dtype=torch.int8 if qt == "i8" else torch.uint8, device=dev)
     sx = torch.empty(M, dtype=torch.float32, device=dev)
     y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream()
 
     def step(i):
         r = i % ROTATE
-        ops.quantize_act(xs[r], s, "i8", xq=xq, sx=sx)
-        ops.gemm_w8a8(xq, sx, wqs[r], sw, bias, out=y)
+        ops.quantize_act(xs[r], s, qt, xq=xq, sx=sx)
+        gemm(xq, sx, wqs[r], sw, bias, out=y)
 
     for i in range(max(3, args.warmup)):
         step(i)
@@ -238,9 +266,9 @@ def run_ours(args):
     for i in range(K_steps):
         r = i % ROTATE
         ev[i][0].record(stream)
-        ops.quantize_act(xs[r], s, "i8", xq=xq, sx=sx)
+        ops.quantize_act(xs[r], s, qt, xq=xq, sx=sx)
         ev[i][1].record(stream)
-        ops.gemm_w8a8(xq, sx, wqs[r], sw, bias, out=y)
+        gemm(xq, sx, wqs[r], sw, bias, out=y)
         ev[i][2].record(stream)
     end.record(stream)
     torch.cuda.synchronize()
@@ -270,7 +298,7 @@ def run_ours(args):
 
         def e2e_step():
             x_dev.copy_(x_host, non_blocking=True)
-            ops.linear(x_dev, s, wq0, sw, bias, "i8", out=y, xq_buf=xq, sx_buf=sx)
+            ops.linear(x_dev, s, wq0, sw, bias, qt, out=y, xq_buf=xq, sx_buf=sx)
             y_host.copy_(y, non_blocking=True)
 
         for _ in range(3):
@@ -296,32 +324,33 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        import oracle
-        s_h = s.cpu().numpy()
-        wq_h = wq0.cpu().numpy()
-        sw_h = sw.cpu().numpy()
-        cpu = cpu_baseline(case, d, s_h, wq_h, sw_h, args.cpu_budget)
+        cpu = cpu_baseline(case, d, args.cpu_budget)
 
     if rank == 0:
         pk = _peaks()
-        int8_peak = 2.0 * pk["bf16"]        # dense INT8 = 2x dense bf16 (nominal 4.5 vs 2.25 POPS)
+        int8_peak = 2.0 * pk["bf16"]        # dense INT8 / FP8 = 2x dense bf16 (4.5 vs 2.25 P)
         int8_peak_sus = 2.0 * pk["bf16_sus"]
         gemm_tops = case.ops / (t_gemm * 1e-3) / 1e12
         value = ws * case.ops * K_steps / (elapsed_ms * 1e-3) / 1e12
         q_bytes = M * K * 2 + M * K + M * 4 + K * 4   # read X (bf16) + s, write Xq + sx
+        g_bytes = M * K + N * K + M * N * 2 + 4 * (M + N) + (2 * N if bias is not None else 0)
         line = {
-            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": K_steps,
-            "warmup": args.warmup, "ms_per_step": elapsed_ms / K_steps,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "i8",
+            "metric": metric_for(case), "value": value, "unit": UNIT, "n_gpus": ws,
+            "steps": K_steps, "warmup": args.warmup, "ms_per_step": elapsed_ms / K_steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "i8" if qt == "i8" else "e4m3",
             "data": "synthetic (seeded N(0,1) activations with 1% outlier channels x U(20,100), "
                     "N(0,0.02) weights)",
             "config": {"workload": case.name, "M": M, "K": K, "N": N, "alpha": case.alpha,
-                       "bias": True, "out": "bf16",
-                       "l2": f"{ROTATE} rotating input sets (X + Wq, 277 MB) > 126 MB L2",
-                       "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU"},
+                       "bias": bias is not None, "out": "bf16",
+                       "l2": (f"{ROTATE} rotating input sets (X + Wq, "
+                              f"{ROTATE * (M * K * 2 + N * K) / 2 ** 20:.0f} MiB) > 126 MiB L2"),
+                       "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU",
+                       "gemm_tile": os.environ.get("SQ_GEMM_TILE", "auto")},
             "frac_of_int8_peak": value / ws / int8_peak,
             "int8_peak_tops": int8_peak,
             "int8_peak_source": f"2 x {pk['src']} bf16 dense ({pk['bf16']} TFLOP/s burst)",
+            "gemm_hbm_gbs": g_bytes / (t_gemm * 1e-3) / 1e9,
             "roofline": {"bound": "tensor", "kernel": "gemm_w8a8_kernel", "achieved": gemm_tops,
                          "peak": int8_peak, "unit": "TFLOP/s", "frac": gemm_tops / int8_peak,
                          "frac_of_sustained": gemm_tops / int8_peak_sus,
@@ -355,6 +384,10 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--workload", default="mlp_up_4096x4096x14336",
+                    help="one of the five workloads (default: the MLP up-projection)")
+    ap.add_argument("--tile", default=None, help="force a GEMM tile shape (c1n128, c1n256, "
+                    "c2n224, c2n256); default: chosen by problem size")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -15,8 +15,9 @@
  *    as Xq [M,K]. Both 8-bit operands are therefore "K-major".
  *  - Every pointer argument is a DEVICE pointer owned by the caller (the
  *    library never frees or keeps it). Large tensors (x, w, xq, wq, y, acc)
- *    must be 16-byte aligned; vectors (s, sx, sw, amax) 4-byte aligned; bias
- *    2-byte aligned. Inputs and outputs must not alias.
+ *    and the per-channel vectors of the GEMMs (sw, bias) must be 16-byte
+ *    aligned, as must s in sq_quantize_act; other vectors (s elsewhere, sx,
+ *    amax) 4-byte aligned. Inputs and outputs must not alias.
  *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *    stream). Every call is asynchronous on that stream: argument checks run
  *    synchronously on the host and launch nothing when they fail; a failed

@@ -105,7 +105,8 @@ def test_gemm_validation(lib):
     assert call(yt=ops.SQ_I8) == ops.SQ_ERR_INVALID_ARG
     assert call(wq=A + 2) == ops.SQ_ERR_MISALIGNED
     assert call(y=A + 8) == ops.SQ_ERR_MISALIGNED
-    assert call(bias=A + 1) == ops.SQ_ERR_MISALIGNED
+    assert call(bias=A + 2) == ops.SQ_ERR_MISALIGNED
+    assert call(sw=A + 4) == ops.SQ_ERR_MISALIGNED
     assert call(acc=A + 4) == ops.SQ_ERR_MISALIGNED
     assert call(M=0) == ops.SQ_OK
     g = lib.sq_gemm_fp8

@@ -146,6 +146,48 @@ def test_gemm_w8a8(M, N, K, with_bias):
     np.testing.assert_array_equal(host(yb), yb_ref)
 
 
+@pytest.mark.parametrize("tile", ops.GEMM_TILES)
+@pytest.mark.parametrize("M,N,K", [(300, 392, 4096), (129, 200, 96), (513, 520, 208),
+                                   (1, 16, 32), (256, 448, 1024), (1100, 904, 272)])
+@pytest.mark.parametrize("qtype", ["i8", "e4m3"])
+def test_gemm_every_tile_shape(tile, M, N, K, qtype):
+    """Every compiled tile shape (1-CTA and SM-pair) on ragged sizes."""
+    g = np.random.default_rng(M + N + K)
+    if qtype == "i8":
+        xq = synth.random_matrix((M, K), np.int8, seed=M * 3 + K)
+        wq = synth.random_matrix((N, K), np.int8, seed=N * 5 + K)
+    else:
+        codes = E4M3_FINITE[np.abs(oracle.e4m3_decode(E4M3_FINITE)) <= 64.0]
+        xq = g.choice(codes, size=(M, K)).astype(np.uint8)
+        wq = g.choice(codes, size=(N, K)).astype(np.uint8)
+    sx = synth.random_floats(M, seed=31, lo=1e-3, hi=0.5)
+    sw = synth.random_floats(N, seed=32, lo=1e-4, hi=1e-2)
+    bias = synth.to_bf16_bits(synth.random_floats(N, seed=33, std=0.1))
+    d = [dev(a) for a in (xq, sx, wq, sw)]
+    with ops.gemm_tile(tile):
+        if qtype == "i8":
+            acc = torch.empty((M, N), dtype=torch.int32, device="cuda")
+            yf = ops.gemm_w8a8(*d, bias=dev(bias), out_dtype=torch.float32, acc=acc)
+            yb = ops.gemm_w8a8(*d, bias=dev(bias))
+        else:
+            yf = ops.gemm_fp8(*d, bias=dev(bias), out_dtype=torch.float32)
+            yb = ops.gemm_fp8(*d, bias=dev(bias))
+    assert ops.device_status() == ops.SQ_OK
+    if qtype == "i8":
+        acc_ref = oracle.gemm_i8(xq, wq)
+        yf_ref, yb_ref = oracle.epilogue(acc_ref, sx, sw, bias)
+        np.testing.assert_array_equal(host(acc), acc_ref)
+        np.testing.assert_array_equal(host(yf), yf_ref)
+        np.testing.assert_array_equal(host(yb), yb_ref)
+    else:
+        yf_ref, _ = oracle.epilogue(oracle.gemm_e4m3(xq, wq), sx, sw, bias)
+        rows, cols = np.divmod(np.arange(M * N, dtype=np.int64), N)
+        e = fp8_normalized_error(host(yf).reshape(-1), yf_ref.reshape(-1), xq, wq, sx, sw, bias,
+                                 rows, cols)
+        assert e.max() <= 1e-3, e.max()
+        np.testing.assert_array_equal(host(yb), oracle.f32_to_bf16(host(yf)))
+
+
 def test_gemm_w8a8_extreme_accumulators():
     M, N, K = 130, 136, 16384
     xq = np.full((M, K), 127, np.int8)

@@ -57,8 +57,8 @@ sq_status check_gemm(const void* xq, const float* sx, const void* wq, const floa
   if (yt != SQ_BF16 && yt != SQ_F32) return SQ_ERR_INVALID_ARG;
   if (M == 0) return SQ_OK;  // empty batch: pointers may be NULL
   if (!xq || !sx || !wq || !sw || !y) return SQ_ERR_INVALID_ARG;
-  if (!al(xq, 16) || !al(wq, 16) || !al(y, 16) || !al(sx, 4) || !al(sw, 4)) return SQ_ERR_MISALIGNED;
-  if (bias && !al(bias, 2)) return SQ_ERR_MISALIGNED;
+  if (!al(xq, 16) || !al(wq, 16) || !al(y, 16) || !al(sx, 4) || !al(sw, 16)) return SQ_ERR_MISALIGNED;
+  if (bias && !al(bias, 16)) return SQ_ERR_MISALIGNED;
   if (acc && !al(acc, 16)) return SQ_ERR_MISALIGNED;
   return SQ_OK;
 }

@@ -9,19 +9,29 @@
 // (Y = dequantize(X_int8 @ W_int8) on INT8 tensor cores), §1 table
 // (INT8 x INT8 and FP8 x FP8 GEMM rows), §4 (FP8 E4M3 operands).
 //
-// Kernel structure (one CTA computes one BM x BN output tile, BM = 128):
-//   warp 0      : TMA producer -- streams 128-byte-wide K slices of the Xq
-//                 and Wq tiles into a STAGES-deep shared-memory ring
-//                 (128-byte swizzle), one mbarrier pair per slot.
-//   warp 1      : allocates the tensor-memory accumulator, and one elected
-//                 thread issues tcgen05.mma (M=128, N=BN, K=32 per
-//                 instruction) and frees ring slots with tcgen05.commit.
-//   warps 2..5  : epilogue -- tcgen05.ld the accumulator rows (warp w reads
-//                 TMEM lanes 32*(w%4)..+31), dequantize with per-token and
-//                 per-channel scales (+bias), round to bf16, store.
-// Every barrier wait is bounded (sq_common.cuh); a wait that gives up sets
-// the status word, skips the remaining work and still frees tensor memory.
+// Persistent, warp-specialized kernel. CG = 1: one CTA computes 128 x BN
+// output tiles; CG = 2: a cluster of two CTAs on neighbouring SMs computes
+// 256 x BN tiles with tcgen05.mma.cta_group::2 -- each CTA loads its own 128
+// rows of Xq and its own BN/2 rows of Wq (no multicast), and the pair's MMA
+// reads both halves, which halves the operand bytes each SM stages per MAC.
+//   warp 0     : TMA producer -- 128-byte-wide K slices of the Xq / Wq tiles
+//                into a STAGES-deep ring (128-byte swizzle); in a pair both
+//                CTAs' copies complete on the leader CTA's "full" barrier.
+//   warp 1     : allocates tensor memory (two BN-column accumulators); in the
+//                leader CTA one thread issues the MMAs (K = 32 per
+//                instruction) and frees ring slots / publishes finished
+//                accumulators with tcgen05.commit.
+//   warps 2..5 : epilogue -- tcgen05.ld of accumulator rows (warp w reads
+//                TMEM lanes 32*(w%4)..+31), dequantize, bf16, store; then
+//                hand the accumulator buffer back to the MMA thread. Two
+//                buffers let the epilogue of tile i overlap the MMAs of i+1.
+// Tiles are walked in groups of kGroupM M-tiles so that the CTAs working at
+// the same time share Wq tiles in L2. Every barrier wait is bounded: a wait
+// that gives up records SQ_ERR_TIMEOUT, the CTA skips its remaining work,
+// drains its MMAs and still frees tensor memory.
 #include <cstdint>
+#include <cstdlib>
+#include <cstring>
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -30,159 +40,247 @@
 
 namespace sqk {
 
-constexpr int kBM = 128;
 constexpr int kBK = 128;  // bytes of K per pipeline stage (one swizzle row)
 constexpr int kThreads = 192;
+constexpr int kGroupM = 16;
 
-template <int BN, int STAGES>
-struct GemmSmem {
-  static constexpr uint32_t kABytes = kBM * kBK;
-  static constexpr uint32_t kBBytes = BN * kBK;
+template <int CG, int BN, int STAGES>
+struct GemmCfg {
+  static constexpr int kTileM = 128 * CG;  // output rows per tile
+  static constexpr int kBRows = BN / CG;   // Wq rows staged per CTA
+  static constexpr uint32_t kABytes = 128 * kBK;
+  static constexpr uint32_t kBBytes = kBRows * kBK;
   static constexpr uint32_t kStageBytes = kABytes + kBBytes;
-  static constexpr uint32_t kRing = STAGES * kStageBytes;
-  // barriers: full[STAGES], empty[STAGES], tmem_full
-  static constexpr uint32_t kBarOff = kRing;
-  static constexpr uint32_t kMiscOff = kBarOff + (2 * STAGES + 1) * 8;  // tmem slot, abort
-  static constexpr uint32_t kScaleOff = (kMiscOff + 16 + 15) & ~15u;    // sw[BN], bias[BN]
-  static constexpr uint32_t kTotal = kScaleOff + 2 * BN * 4;
+  static constexpr uint32_t kTxBytes = kStageBytes * CG;  // landing on one "full" barrier
+  static constexpr uint32_t kAccStride = BN <= 128 ? 128 : 256;  // TMEM columns per buffer
+  static constexpr uint32_t kTmemCols = 2 * kAccStride;
+  static constexpr uint32_t kRingA = 0;
+  static constexpr uint32_t kRingB = STAGES * kABytes;
+  static constexpr uint32_t kBarOff = STAGES * kStageBytes;
+  // barriers: full[S], empty[S], tfull[2], tempty[2], drain
+  static constexpr uint32_t kMiscOff = kBarOff + (2 * STAGES + 5) * 8;  // tmem slot, abort flag
+  static constexpr uint32_t kTotal = kMiscOff + 16;
   static constexpr uint32_t kDynamic = kTotal + 1024;  // slack for 1024-B alignment
-  static constexpr uint32_t kTmemCols = BN <= 32 ? 32 : BN <= 64 ? 64 : BN <= 128 ? 128 : 256;
+  static_assert(BN % 32 == 0 && BN <= 256, "BN must be a multiple of 32, at most 256");
+  static_assert(kBRows % 8 == 0, "staged Wq rows must be whole 8-row swizzle atoms");
+  static_assert(kDynamic <= 232448, "shared memory budget exceeded");
 };
 
-template <int BN, int STAGES, bool E4M3, bool OUT_BF16, bool HAS_BIAS, bool WRITE_ACC>
+__device__ __forceinline__ void tile_coords(int tile, int num_mt, int num_nt, int& mt, int& nt) {
+  const int per_group = kGroupM * num_nt;
+  const int g = tile / per_group, r = tile - g * per_group;
+  const int first = g * kGroupM;
+  const int gm = min(kGroupM, num_mt - first);
+  mt = first + r % gm;
+  nt = r / gm;
+}
+
+template <int CG, int BN, int STAGES, bool E4M3, bool OUT_BF16, bool HAS_BIAS, bool WRITE_ACC>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                      const float* __restrict__ sx, const float* __restrict__ sw,
                      const uint16_t* __restrict__ bias, void* __restrict__ y,
                      int32_t* __restrict__ acc_out, int M, int N, int K, int* status) {
-  using L = GemmSmem<BN, STAGES>;
+  using C = GemmCfg<CG, BN, STAGES>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const uint32_t s_base = smem_u32(smem);
-  const uint32_t s_a = s_base;
-  const uint32_t s_b = s_base + STAGES * L::kABytes;
-  const uint32_t bar_full = s_base + L::kBarOff;
+  const uint32_t s_a = s_base + C::kRingA;
+  const uint32_t s_b = s_base + C::kRingB;
+  const uint32_t bar_full = s_base + C::kBarOff;
   const uint32_t bar_empty = bar_full + STAGES * 8;
-  const uint32_t bar_tmem_full = bar_empty + STAGES * 8;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
-  float* s_sw = reinterpret_cast<float*>(smem + L::kScaleOff);
-  float* s_bias = s_sw + BN;
+  const uint32_t bar_tfull = bar_empty + STAGES * 8;
+  const uint32_t bar_tempty = bar_tfull + 2 * 8;
+  const uint32_t bar_drain = bar_tempty + 2 * 8;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.y * kBM, n0 = blockIdx.x * BN;
-  const int nk = (K + kBK - 1) / kBK;
+  const uint32_t rank = CG == 2 ? cluster_ctarank() : 0u;
+  const bool leader = rank == 0;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < STAGES; ++i) {
       mbar_init(bar_full + 8 * i, 1);
       mbar_init(bar_empty + 8 * i, 1);
     }
-    mbar_init(bar_tmem_full, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar_tfull + 8 * b, 1);
+      mbar_init(bar_tempty + 8 * b, 4 * CG);
+    }
+    mbar_init(bar_drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_map(&tm_a);
     tma_prefetch_map(&tm_b);
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), L::kTmemCols);
-    tmem_relinquish();
+    if constexpr (CG == 2) {
+      tmem_alloc_pair(smem_u32(tmem_slot), C::kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  if constexpr (CG == 2) cluster_sync_all(); else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
+  const int num_mt = (M + C::kTileM - 1) / C::kTileM;
+  const int num_nt = (N + BN - 1) / BN;
+  const int num_tiles = num_mt * num_nt;
+  const int unit = blockIdx.x / CG, num_units = gridDim.x / CG;
+  const int nk = (K + kBK - 1) / kBK;
+
   if (warp == 0) {
+    // ------------------------------------------------------------ producer --
     if (lane == 0) {
+      uint32_t it = 0;
+      bool ok = true;
 #pragma unroll 1
-      for (int kb = 0; kb < nk; ++kb) {
-        const int st = kb % STAGES;
-        const uint32_t ph = (kb / STAGES) & 1;
-        if (!mbar_wait(bar_empty + 8 * st, ph ^ 1)) {
-          record_status(status, kStatusTimeout);
-          *abort_flag = 1;
-          break;
+      for (int tile = unit; tile < num_tiles && ok; tile += num_units) {
+        int mt, nt;
+        tile_coords(tile, num_mt, num_nt, mt, nt);
+        const int a_row = mt * C::kTileM + int(rank) * 128;
+        const int b_row = nt * BN + int(rank) * C::kBRows;
+#pragma unroll 1
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const uint32_t st = it % STAGES, ph = (it / STAGES) & 1u;
+          if (!mbar_wait(bar_empty + 8 * st, ph ^ 1u) || *abort_flag) {
+            record_status(status, kStatusTimeout);
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          if constexpr (CG == 2) {
+            if (leader) mbar_arrive_expect_tx(bar_full + 8 * st, C::kTxBytes);
+            const uint32_t full_leader = map_to_rank(bar_full + 8 * st, 0);
+            tma_load_2d_pair(s_a + st * C::kABytes, &tm_a, full_leader, kb * kBK, a_row);
+            tma_load_2d_pair(s_b + st * C::kBBytes, &tm_b, full_leader, kb * kBK, b_row);
+          } else {
+            mbar_arrive_expect_tx(bar_full + 8 * st, C::kTxBytes);
+            tma_load_2d(s_a + st * C::kABytes, &tm_a, bar_full + 8 * st, kb * kBK, a_row);
+            tma_load_2d(s_b + st * C::kBBytes, &tm_b, bar_full + 8 * st, kb * kBK, b_row);
+          }
         }
-        if (*abort_flag) break;
-        mbar_arrive_expect_tx(bar_full + 8 * st, L::kStageBytes);
-        tma_load_2d(s_a + st * L::kABytes, &tm_a, bar_full + 8 * st, kb * kBK, m0);
-        tma_load_2d(s_b + st * L::kBBytes, &tm_b, bar_full + 8 * st, kb * kBK, n0);
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      constexpr uint32_t idesc = E4M3 ? idesc_e4m3_f32(kBM, BN) : idesc_s8_s32(kBM, BN);
+    // ----------------------------------------------------------------- MMA --
+    if (lane == 0 && leader) {
+      constexpr uint32_t idesc = E4M3 ? idesc_e4m3_f32(C::kTileM, BN) : idesc_s8_s32(C::kTileM, BN);
+      uint32_t it = 0, tc = 0;
       bool ok = true;
 #pragma unroll 1
-      for (int kb = 0; kb < nk; ++kb) {
-        const int st = kb % STAGES;
-        const uint32_t ph = (kb / STAGES) & 1;
-        if (!mbar_wait(bar_full + 8 * st, ph)) {
+      for (int tile = unit; tile < num_tiles && ok; tile += num_units, ++tc) {
+        const uint32_t buf = tc & 1u, use = tc >> 1;
+        if (!mbar_wait(bar_tempty + 8 * buf, (use & 1u) ^ 1u)) {
           record_status(status, kStatusTimeout);
           *abort_flag = 1;
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t a_addr = s_a + st * L::kABytes;
-        const uint32_t b_addr = s_b + st * L::kBBytes;
+        const uint32_t d = tmem_base + buf * C::kAccStride;
+#pragma unroll 1
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const uint32_t st = it % STAGES, ph = (it / STAGES) & 1u;
+          if (!mbar_wait(bar_full + 8 * st, ph)) {
+            record_status(status, kStatusTimeout);
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = s_a + st * C::kABytes;
+          const uint32_t b_addr = s_b + st * C::kBBytes;
 #pragma unroll
-        for (int kk = 0; kk < kBK / 32; ++kk) {
-          const uint64_t ad = sw128_desc(a_addr + kk * 32);
-          const uint64_t bd = sw128_desc(b_addr + kk * 32);
-          const uint32_t accum = (kb > 0 || kk > 0) ? 1u : 0u;
-          if constexpr (E4M3) mma_f8(tmem_base, ad, bd, idesc, accum);
-          else mma_i8(tmem_base, ad, bd, idesc, accum);
+          for (int kk = 0; kk < kBK / 32; ++kk) {
+            const uint64_t ad = sw128_desc(a_addr + kk * 32);
+            const uint64_t bd = sw128_desc(b_addr + kk * 32);
+            const uint32_t accum = (kb > 0 || kk > 0) ? 1u : 0u;
+            if constexpr (CG == 2) {
+              if constexpr (E4M3) mma_f8_pair(d, ad, bd, idesc, accum);
+              else mma_i8_pair(d, ad, bd, idesc, accum);
+            } else {
+              if constexpr (E4M3) mma_f8(d, ad, bd, idesc, accum);
+              else mma_i8(d, ad, bd, idesc, accum);
+            }
+          }
+          if constexpr (CG == 2) {
+            tc_commit_pair(bar_empty + 8 * st);
+            tc_commit_pair(map_to_rank(bar_empty + 8 * st, 1));
+          } else {
+            tc_commit(bar_empty + 8 * st);
+          }
         }
-        tc_commit(bar_empty + 8 * st);
+        if (!ok) break;
+        if constexpr (CG == 2) {
+          tc_commit_pair(bar_tfull + 8 * buf);
+          tc_commit_pair(map_to_rank(bar_tfull + 8 * buf, 1));
+        } else {
+          tc_commit(bar_tfull + 8 * buf);
+        }
       }
-      // Signals the epilogue even after an abort so that it does not wait
-      // for the full timeout a second time (the abort flag tells it to skip).
-      tc_commit(bar_tmem_full);
-      // After an abort nobody else consumes that signal: wait here (bounded)
-      // for the MMAs already issued, so tensor memory is idle when freed.
-      if (!ok) (void)mbar_wait(bar_tmem_full, 0);
+      // Make sure every MMA issued has completed before tensor memory can be
+      // freed (matters only on the abort path; normally the epilogue has
+      // already observed the last accumulator).
+      if constexpr (CG == 2) tc_commit_pair(bar_drain); else tc_commit(bar_drain);
+      (void)mbar_wait(bar_drain, 0);
     }
   } else {
-    // ---------------------------------------------------------- epilogue --
-    const int et = threadIdx.x - 64;  // 0..127
-    for (int j = et; j < BN; j += 128) {
-      const int n = n0 + j;
-      s_sw[j] = n < N ? __ldg(sw + n) : 0.0f;
-      if constexpr (HAS_BIAS) s_bias[j] = n < N ? __uint_as_float(uint32_t(__ldg(bias + n)) << 16) : 0.0f;
-    }
-    named_barrier_sync(1, 128);
-    const bool ready = mbar_wait(bar_tmem_full, 0);
-    if (!ready) {
-      record_status(status, kStatusTimeout);
-      *abort_flag = 1;
-    }
-    tc_fence_after();
-    if (ready && !*abort_flag) {
-      const int sub = warp & 3;
-      const int row = sub * 32 + lane;
-      const int m = m0 + row;
+    // ------------------------------------------------------------ epilogue --
+    const int sub = warp & 3;
+    const int row_in_tile = int(rank) * 128 + sub * 32 + lane;
+    const uint32_t tempty_leader = CG == 2 ? map_to_rank(bar_tempty, 0) : bar_tempty;
+    uint32_t tc = 0;
+#pragma unroll 1
+    for (int tile = unit; tile < num_tiles; tile += num_units, ++tc) {
+      const uint32_t buf = tc & 1u, use = tc >> 1;
+      if (!mbar_wait(bar_tfull + 8 * buf, use & 1u) || *abort_flag) {
+        record_status(status, kStatusTimeout);
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      int mt, nt;
+      tile_coords(tile, num_mt, num_nt, mt, nt);
+      const int m = mt * C::kTileM + row_in_tile;
+      const int n_base = nt * BN;
       const float sxm = m < M ? __ldg(sx + m) : 0.0f;
+      const uint32_t t_addr = tmem_base + buf * C::kAccStride + (uint32_t(sub * 32) << 16);
 #pragma unroll 1
       for (int c0 = 0; c0 < BN; c0 += 32) {
         uint32_t r[32];
-        tmem_ld32(tmem_base + (uint32_t(sub * 32) << 16) + uint32_t(c0), r);
+        tmem_ld32(t_addr + uint32_t(c0), r);
         tmem_wait_ld(r);
         if (m < M) {
 #pragma unroll
           for (int g = 0; g < 4; ++g) {
-            const int n = n0 + c0 + g * 8;
+            const int n = n_base + c0 + g * 8;
             if (n < N) {
+              const float4 w0 = __ldg(reinterpret_cast<const float4*>(sw + n));
+              const float4 w1 = __ldg(reinterpret_cast<const float4*>(sw + n) + 1);
+              const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+              float bv[8];
+              if constexpr (HAS_BIAS) {
+                const uint4 b = __ldg(reinterpret_cast<const uint4*>(bias + n));
+                bv[0] = bf16_lo(b.x); bv[1] = bf16_hi(b.x);
+                bv[2] = bf16_lo(b.y); bv[3] = bf16_hi(b.y);
+                bv[4] = bf16_lo(b.z); bv[5] = bf16_hi(b.z);
+                bv[6] = bf16_lo(b.w); bv[7] = bf16_hi(b.w);
+              }
               float t[8];
 #pragma unroll
               for (int i = 0; i < 8; ++i) {
                 const uint32_t raw = r[g * 8 + i];
                 float a = E4M3 ? __uint_as_float(raw) : __int2float_rn(int32_t(raw));
                 a = __fmul_rn(a, sxm);
-                a = __fmul_rn(a, s_sw[c0 + g * 8 + i]);
-                if constexpr (HAS_BIAS) a = __fadd_rn(a, s_bias[c0 + g * 8 + i]);
+                a = __fmul_rn(a, wv[i]);
+                if constexpr (HAS_BIAS) a = __fadd_rn(a, bv[i]);
                 t[i] = a;
               }
               const int64_t off = int64_t(m) * N + n;
@@ -207,13 +305,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
+      // hand the accumulator buffer back to the MMA thread
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if constexpr (CG == 2) mbar_arrive_cluster(tempty_leader + 8 * buf);
+        else mbar_arrive(bar_tempty + 8 * buf);
+      }
     }
   }
+  __syncwarp();
   tc_fence_before();
-  __syncthreads();
+  if constexpr (CG == 2) cluster_sync_all(); else __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, L::kTmemCols);
+    if constexpr (CG == 2) tmem_dealloc_pair(tmem_base, C::kTmemCols);
+    else tmem_dealloc(tmem_base, C::kTmemCols);
   }
 }
 
@@ -255,56 +362,160 @@ static bool make_map_k_major(CUtensorMap* map, const void* base, int64_t rows, i
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BN, int STAGES, bool E4M3, bool OUT_BF16, bool HAS_BIAS, bool WRITE_ACC>
-static cudaError_t run_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const float* sx,
-                            const float* sw, const uint16_t* bias, void* y, int32_t* acc, int M,
-                            int N, int K, cudaStream_t st) {
-  using L = GemmSmem<BN, STAGES>;
-  auto kern = gemm_w8a8_kernel<BN, STAGES, E4M3, OUT_BF16, HAS_BIAS, WRITE_ACC>;
-  static uint64_t attr_set_mask = 0;  // one bit per device ordinal
+static int device_sms() {
+  static int n[64] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev >= 64 || !((attr_set_mask >> dev) & 1u)) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         int(L::kDynamic));
-    if (e != cudaSuccess) return e;
-    if (dev < 64) attr_set_mask |= uint64_t(1) << dev;
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (n[dev] == 0) {
+    int v = 0;
+    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    n[dev] = v > 0 ? v : 148;
   }
-  dim3 grid(unsigned((N + BN - 1) / BN), unsigned((M + kBM - 1) / kBM));
-  kern<<<grid, kThreads, L::kDynamic, st>>>(ta, tb, sx, sw, bias, y, acc, M, N, K, status_ptr());
-  return cudaGetLastError();
+  return n[dev];
 }
 
-template <int BN, int STAGES, bool E4M3>
-static cudaError_t dispatch_epilogue(const CUtensorMap& ta, const CUtensorMap& tb, const float* sx,
+template <int CG, int BN, int STAGES, bool E4M3, bool OUT_BF16, bool HAS_BIAS, bool WRITE_ACC>
+static cudaError_t run_gemm(const void* xq, const void* wq, const float* sx, const float* sw,
+                            const uint16_t* bias, void* y, int32_t* acc, int M, int N, int K,
+                            cudaStream_t st) {
+  using C = GemmCfg<CG, BN, STAGES>;
+  auto kern = gemm_w8a8_kernel<CG, BN, STAGES, E4M3, OUT_BF16, HAS_BIAS, WRITE_ACC>;
+  CUtensorMap ta, tb;
+  if (!make_map_k_major(&ta, xq, M, K, 128) || !make_map_k_major(&tb, wq, N, K, C::kBRows))
+    return cudaErrorInvalidValue;
+  static uint64_t attr_set_mask = 0;  // one bit per device ordinal
+  static int max_units[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const bool cached = dev < 64 && ((attr_set_mask >> dev) & 1u);
+  if (!cached) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         int(C::kDynamic));
+    if (e != cudaSuccess) return e;
+    int units = device_sms() / CG;
+    if (CG == 2) {
+      cudaLaunchConfig_t q = {};
+      cudaLaunchAttribute a[1];
+      a[0].id = cudaLaunchAttributeClusterDimension;
+      a[0].val.clusterDim.x = 2;
+      a[0].val.clusterDim.y = 1;
+      a[0].val.clusterDim.z = 1;
+      q.gridDim = dim3(2 * units);
+      q.blockDim = dim3(kThreads);
+      q.dynamicSmemBytes = C::kDynamic;
+      q.attrs = a;
+      q.numAttrs = 1;
+      int clusters = 0;
+      if (cudaOccupancyMaxActiveClusters(&clusters, kern, &q) == cudaSuccess && clusters > 0)
+        units = clusters < units ? clusters : units;
+      cudaGetLastError();
+    }
+    if (dev < 64) {
+      max_units[dev] = units;
+      attr_set_mask |= uint64_t(1) << dev;
+    }
+  }
+  const int units_max = dev < 64 ? max_units[dev] : device_sms() / CG;
+  const int tiles = ((M + C::kTileM - 1) / C::kTileM) * ((N + BN - 1) / BN);
+  const int units = tiles < units_max ? tiles : units_max;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attrs[1];
+  cfg.gridDim = dim3(unsigned(units * CG));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = C::kDynamic;
+  cfg.stream = st;
+  if (CG == 2) {
+    attrs[0].id = cudaLaunchAttributeClusterDimension;
+    attrs[0].val.clusterDim.x = 2;
+    attrs[0].val.clusterDim.y = 1;
+    attrs[0].val.clusterDim.z = 1;
+    cfg.attrs = attrs;
+    cfg.numAttrs = 1;
+  }
+  int* status = status_ptr();
+  return cudaLaunchKernelEx(&cfg, kern, ta, tb, sx, sw, bias, y, acc, M, N, K, status);
+}
+
+template <int CG, int BN, int STAGES, bool E4M3>
+static cudaError_t dispatch_epilogue(const void* xq, const void* wq, const float* sx,
                                      const float* sw, const uint16_t* bias, void* y, OutKind yk,
                                      int32_t* acc, int M, int N, int K, cudaStream_t st) {
   const bool bf = yk == OutKind::BF16, hb = bias != nullptr, wa = acc != nullptr;
   const int key = (bf ? 4 : 0) | (hb ? 2 : 0) | (wa ? 1 : 0);
+#define SQ_RUN(B, H, W) \
+  run_gemm<CG, BN, STAGES, E4M3, B, H, W>(xq, wq, sx, sw, bias, y, acc, M, N, K, st)
   switch (key) {
-    case 0: return run_gemm<BN, STAGES, E4M3, false, false, false>(ta, tb, sx, sw, bias, y, acc, M, N, K, st);
-    case 1: return run_gemm<BN, STAGES, E4M3, false, false, true>(ta, tb, sx, sw, bias, y, acc, M, N, K, st);
-    case 2: return run_gemm<BN, STAGES, E4M3, false, true, false>(ta, tb, sx, sw, bias, y, acc, M, N, K, st);
-    case 3: return run_gemm<BN, STAGES, E4M3, false, true, true>(ta, tb, sx, sw, bias, y, acc, M, N, K, st);
-    case 4: return run_gemm<BN, STAGES, E4M3, true, false, false>(ta, tb, sx, sw, bias, y, acc, M, N, K, st);
-    case 5: return run_gemm<BN, STAGES, E4M3, true, false, true>(ta, tb, sx, sw, bias, y, acc, M, N, K, st);
-    case 6: return run_gemm<BN, STAGES, E4M3, true, true, false>(ta, tb, sx, sw, bias, y, acc, M, N, K, st);
-    default: return run_gemm<BN, STAGES, E4M3, true, true, true>(ta, tb, sx, sw, bias, y, acc, M, N, K, st);
+    case 0: return SQ_RUN(false, false, false);
+    case 1: return SQ_RUN(false, false, true);
+    case 2: return SQ_RUN(false, true, false);
+    case 3: return SQ_RUN(false, true, true);
+    case 4: return SQ_RUN(true, false, false);
+    case 5: return SQ_RUN(true, false, true);
+    case 6: return SQ_RUN(true, true, false);
+    default: return SQ_RUN(true, true, true);
   }
+#undef SQ_RUN
+}
+
+// Tile shapes compiled in. Each entry: CTAs per tile (1 or 2), N per tile,
+// pipeline depth.
+enum class TileCfg { C1_N128, C1_N256, C2_N224, C2_N256 };
+
+static TileCfg choose_tile(int64_t M, int64_t N) {
+  // Estimated time ~ (number of rounds of tiles over the SMs) x (work per
+  // tile); pick the cheapest, preferring SM pairs on ties (less operand
+  // traffic per MAC).
+  const int sms = device_sms();
+  struct Cand { TileCfg c; int cg, bm, bn; double eff; };
+  const Cand cands[] = {{TileCfg::C2_N256, 2, 256, 256, 1.0},
+                        {TileCfg::C2_N224, 2, 256, 224, 1.0},
+                        {TileCfg::C1_N256, 1, 128, 256, 0.9},
+                        {TileCfg::C1_N128, 1, 128, 128, 0.8}};
+  double best = 1e30;
+  TileCfg pick = TileCfg::C1_N128;
+  for (const Cand& c : cands) {
+    const int64_t tiles = ((M + c.bm - 1) / c.bm) * ((N + c.bn - 1) / c.bn);
+    const int64_t units = sms / c.cg;
+    const int64_t rounds = (tiles + units - 1) / units;
+    const double t = double(rounds) * double(c.bm) * double(c.bn) / (double(c.cg) * c.eff);
+    if (t < best * 0.999) {
+      best = t;
+      pick = c.c;
+    }
+  }
+  return pick;
+}
+
+// SQ_GEMM_TILE = c1n128 | c1n256 | c2n224 | c2n256 forces one tile shape
+// (used to test every shape and to compare them); unset or anything else
+// selects by problem size.
+static bool forced_tile(TileCfg* out) {
+  const char* e = getenv("SQ_GEMM_TILE");
+  if (!e) return false;
+  if (!strcmp(e, "c1n128")) { *out = TileCfg::C1_N128; return true; }
+  if (!strcmp(e, "c1n256")) { *out = TileCfg::C1_N256; return true; }
+  if (!strcmp(e, "c2n224")) { *out = TileCfg::C2_N224; return true; }
+  if (!strcmp(e, "c2n256")) { *out = TileCfg::C2_N256; return true; }
+  return false;
 }
 
 cudaError_t launch_gemm(bool e4m3, const uint8_t* xq, const float* sx, const uint8_t* wq,
                         const float* sw, const uint16_t* bias, int64_t M, int64_t N, int64_t K,
                         void* y, OutKind yk, int32_t* acc, cudaStream_t st) {
-  constexpr int BN = 128, STAGES = 6;
-  CUtensorMap ta, tb;
-  if (!make_map_k_major(&ta, xq, M, K, kBM) || !make_map_k_major(&tb, wq, N, K, BN))
-    return cudaErrorInvalidValue;
-  if (e4m3)
-    return dispatch_epilogue<BN, STAGES, true>(ta, tb, sx, sw, bias, y, yk, acc, int(M), int(N),
-                                               int(K), st);
-  return dispatch_epilogue<BN, STAGES, false>(ta, tb, sx, sw, bias, y, yk, acc, int(M), int(N),
-                                              int(K), st);
+  const int m = int(M), n = int(N), k = int(K);
+  TileCfg c;
+  if (!forced_tile(&c)) c = choose_tile(M, N);
+#define SQ_CASE(CG, BN, S)                                                                     \
+  return e4m3 ? dispatch_epilogue<CG, BN, S, true>(xq, wq, sx, sw, bias, y, yk, acc, m, n, k, st) \
+              : dispatch_epilogue<CG, BN, S, false>(xq, wq, sx, sw, bias, y, yk, acc, m, n, k, st)
+  switch (c) {
+    case TileCfg::C2_N256: SQ_CASE(2, 256, 6);
+    case TileCfg::C2_N224: SQ_CASE(2, 224, 7);
+    case TileCfg::C1_N256: SQ_CASE(1, 256, 4);
+    default: SQ_CASE(1, 128, 6);
+  }
+#undef SQ_CASE
 }
 
 }  // namespace sqh

@@ -225,6 +225,34 @@ def probe_wait_timeout(timeout_ns: int, device=None):
     _check(load().sq_probe_wait_timeout(int(timeout_ns), _stream(device)), "sq_probe_wait_timeout")
 
 
+# GEMM tile shapes compiled into libsq.so (CTAs per tile x N per tile).
+GEMM_TILES = ("c1n128", "c1n256", "c2n224", "c2n256")
+
+
+class gemm_tile:
+    """Context manager forcing one GEMM tile shape (testing / tuning); the
+    library otherwise picks the shape from the problem size."""
+
+    def __init__(self, name: str | None):
+        if name is not None and name not in GEMM_TILES:
+            raise ValueError(f"unknown tile {name!r}; choose from {GEMM_TILES}")
+        self.name = name
+
+    def __enter__(self):
+        self.prev = os.environ.get("SQ_GEMM_TILE")
+        if self.name is None:
+            os.environ.pop("SQ_GEMM_TILE", None)
+        else:
+            os.environ["SQ_GEMM_TILE"] = self.name
+        return self
+
+    def __exit__(self, *exc):
+        if self.prev is None:
+            os.environ.pop("SQ_GEMM_TILE", None)
+        else:
+            os.environ["SQ_GEMM_TILE"] = self.prev
+
+
 # ------------------------------------------------------------ a layer API --
 
 def prepare(w: torch.Tensor, x_cal: torch.Tensor, alpha: float = 0.5, qtype: str = "i8"):
