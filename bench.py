@@ -224,7 +224,7 @@ def run_ours(args):
     # ---- offline preparation (untimed) ----
     w = to_dev(d["w"])
     p = ops.prepare(w, to_dev(d["x_cal"]), alpha=case.alpha, qtype=qt)
-    s, wq0, sw = p["s"], p["wq"], p["sw"]
+    s, s_inv, wq0, sw = p["s"], p["s_inv"], p["wq"], p["sw"]
     bias = to_dev(d["bias"]) if d["bias"] is not None else None
     gemm = ops.gemm_w8a8 if qt == "i8" else ops.gemm_fp8
     del w
@@ -240,7 +240,7 @@ def run_ours(args):
 
     def step(i):
         r = i % ROTATE
-        ops.quantize_act(xs[r], s, qt, xq=xq, sx=sx)
+        ops.quantize_act(xs[r], s, qt, xq=xq, sx=sx, s_inv=s_inv)
         gemm(xq, sx, wqs[r], sw, bias, out=y)
 
     for i in range(max(3, args.warmup)):
@@ -266,7 +266,7 @@ def run_ours(args):
     for i in range(K_steps):
         r = i % ROTATE
         ev[i][0].record(stream)
-        ops.quantize_act(xs[r], s, qt, xq=xq, sx=sx)
+        ops.quantize_act(xs[r], s, qt, xq=xq, sx=sx, s_inv=s_inv)
         ev[i][1].record(stream)
         gemm(xq, sx, wqs[r], sw, bias, out=y)
         ev[i][2].record(stream)
@@ -298,7 +298,7 @@ def run_ours(args):
 
         def e2e_step():
             x_dev.copy_(x_host, non_blocking=True)
-            ops.linear(x_dev, s, wq0, sw, bias, qt, out=y, xq_buf=xq, sx_buf=sx)
+            ops.linear(x_dev, s, wq0, sw, bias, qt, out=y, xq_buf=xq, sx_buf=sx, s_inv=s_inv)
             y_host.copy_(y, non_blocking=True)
 
         for _ in range(3):

@@ -33,7 +33,7 @@
  *    reproducible bit for bit against a plain CPU implementation (see
  *    each function for the exact operation order).
  *  - The library allocates no device memory of its own except a 4-byte
- *    device status word.
+ *    device status word and the 8-byte counter of sq_selftest_fast_division.
  */
 #ifndef SQ_H
 #define SQ_H
@@ -44,7 +44,7 @@
 extern "C" {
 #endif
 
-#define SQ_ABI_VERSION 1
+#define SQ_ABI_VERSION 2
 
 typedef enum {
     SQ_OK = 0,
@@ -107,9 +107,15 @@ sq_status sq_calibrate_amax(const void* x, sq_dtype xt, int64_t rows,
  *   s[k] = max(amax_x[k], 1e-5)^alpha / max(amax_w[k], 1e-5)^(1-alpha)
  * evaluated in binary64 and rounded once to binary32. 0 <= alpha <= 1
  * (SQ_ERR_INVALID_ARG otherwise). K >= 1.
+ *   s_inv : [K] or NULL. When given, also receives the reciprocals the
+ *           runtime kernel uses to divide by s quickly ("X_tilde = X @
+ *           diag(1/s)", §3 Step 1): s_inv[k] = RN(1/s[k]) when
+ *           2^-20 <= s[k] <= 2^20, NaN otherwise (NaN sends that channel to
+ *           the exact division path). Pass it to sq_quantize_act/sq_linear.
  */
 sq_status sq_smooth_factors(const float* amax_x, const float* amax_w,
-                            int64_t K, double alpha, float* s, void* stream);
+                            int64_t K, double alpha, float* s, float* s_inv,
+                            void* stream);
 
 /*
  * a4 -- offline weight smoothing and per-output-channel quantization.
@@ -141,10 +147,16 @@ sq_status sq_quantize_weight(const void* w, sq_dtype wt, int64_t K, int64_t N,
  * For each row m: xs[k] = x[m,k] / s[k] (IEEE division); sx[m] =
  * max_k|xs[k]| / Q; codes as in sq_quantize_weight with xs and sx[m].
  * Rows with sx[m] == 0 get all-zero codes. K <= 65536.
+ *   s_inv : [K] or NULL (16-byte aligned) -- the reciprocals written by
+ *           sq_smooth_factors for this s. They only speed the kernel up: the
+ *           result is the IEEE quotient x/s either way (bf16 input divides
+ *           by a reciprocal product with one exact correction step and falls
+ *           back to the IEEE division wherever that is not provably exact).
+ *           Results are undefined if s_inv does not come from s.
  */
 sq_status sq_quantize_act(const void* x, sq_dtype xt, int64_t M, int64_t K,
-                          const float* s, sq_dtype qt, void* xq, float* sx,
-                          void* stream);
+                          const float* s, const float* s_inv, sq_dtype qt,
+                          void* xq, float* sx, void* stream);
 
 /*
  * a6 -- INT8 x INT8 tensor-core GEMM with int32 accumulation and a fused
@@ -179,13 +191,25 @@ sq_status sq_gemm_fp8(const uint8_t* xq, const float* sx, const uint8_t* wq,
  * Runtime forward of one SmoothQuant linear layer: sq_quantize_act followed
  * by sq_gemm_w8a8 (qt = SQ_I8) or sq_gemm_fp8 (qt = SQ_E4M3) on the same
  * stream. xq_buf [M,K] (8-bit codes) and sx_buf [M] are caller-owned
- * buffers that receive the quantized activations.
+ * buffers that receive the quantized activations; s_inv as in
+ * sq_quantize_act.
  */
 sq_status sq_linear(const void* x, sq_dtype xt, const float* s,
-                    const void* wq, const float* sw, const uint16_t* bias,
+                    const float* s_inv, const void* wq, const float* sw, const uint16_t* bias,
                     sq_dtype qt, int64_t M, int64_t N, int64_t K,
                     void* xq_buf, float* sx_buf, void* y, sq_dtype yt,
                     void* stream);
+
+/*
+ * Self-test of the division shortcut used by sq_quantize_act for bf16 input
+ * (an IEEE division x / s_k computed as a reciprocal product corrected with
+ * one fused multiply-add residual, after Markstein): runs every bf16
+ * significand of x against every binary32 significand of s (2^30 pairs, both
+ * signs) and counts results that differ from the IEEE division. Synchronous
+ * (waits for `stream`). *mismatches receives the count; 0 means the shortcut
+ * is exact wherever sq_quantize_act uses it.
+ */
+sq_status sq_selftest_fast_division(int64_t* mismatches, void* stream);
 
 /*
  * Diagnostic: launches one block whose single thread waits on a shared-memory

@@ -205,29 +205,42 @@ void sqo_smooth_factors(const float* amax_x, const float* amax_w, int64_t K,
 void sqo_quantize_weight(const void* w, int dtype, int64_t K, int64_t N,
                          const float* s, int qtype, void* wq, float* sw) {
     const float qmax = (qtype == 1) ? 448.0f : 127.0f;
-    #pragma omp parallel for schedule(static)
-    for (int64_t n = 0; n < N; ++n) {
-        /* column n of W~ */
-        float amax = 0.0f;
-        for (int64_t k = 0; k < K; ++k) {
-            float v = load_elem(w, dtype, k * N + n);
-            float wt = s ? smooth_w(v, s[k]) : v;
-            float a = fabsf(wt);
-            if (a > amax) amax = a;
-        }
-        float scale = amax / qmax;
-        sw[n] = scale;
-        for (int64_t k = 0; k < K; ++k) {
-            float v = load_elem(w, dtype, k * N + n);
-            float wt = s ? smooth_w(v, s[k]) : v;
-            if (qtype == 1) {
-                ((uint8_t*)wq)[n * K + k] =
-                    (scale == 0.0f) ? 0 : sqo_e4m3_encode_rn_sat(wt / scale);
-            } else {
-                ((int8_t*)wq)[n * K + k] =
-                    (scale == 0.0f) ? 0 : quant_i8(wt, scale);
+    /* Each thread owns a block of output channels (columns of W) and walks
+     * the rows of W in order; every element's value is computed exactly as
+     * written in the page: wt = s_k * w[k][n]. */
+    #pragma omp parallel
+    {
+#ifdef _OPENMP
+        int nt = omp_get_num_threads(), t = omp_get_thread_num();
+#else
+        int nt = 1, t = 0;
+#endif
+        int64_t n0 = N * t / nt, n1 = N * (t + 1) / nt;
+        /* pass 1: amax of column n of W~ */
+        for (int64_t n = n0; n < n1; ++n) sw[n] = 0.0f;
+        for (int64_t k = 0; k < K; ++k)
+            for (int64_t n = n0; n < n1; ++n) {
+                float v = load_elem(w, dtype, k * N + n);
+                float wt = s ? smooth_w(v, s[k]) : v;
+                float a = fabsf(wt);
+                if (a > sw[n]) sw[n] = a;
             }
-        }
+        /* scale = amax / Q */
+        for (int64_t n = n0; n < n1; ++n) sw[n] = sw[n] / qmax;
+        /* pass 2: codes, stored transposed as wq[n][k] */
+        for (int64_t k = 0; k < K; ++k)
+            for (int64_t n = n0; n < n1; ++n) {
+                float v = load_elem(w, dtype, k * N + n);
+                float wt = s ? smooth_w(v, s[k]) : v;
+                float scale = sw[n];
+                if (qtype == 1) {
+                    ((uint8_t*)wq)[n * K + k] =
+                        (scale == 0.0f) ? 0 : sqo_e4m3_encode_rn_sat(wt / scale);
+                } else {
+                    ((int8_t*)wq)[n * K + k] =
+                        (scale == 0.0f) ? 0 : quant_i8(wt, scale);
+                }
+            }
     }
 }
 

@@ -53,7 +53,7 @@ def test_exported_symbols_are_visible_to_the_dynamic_linker():
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.sq_abi_version() == 1
+    assert lib.sq_abi_version() == 2
     for st in range(6):
         assert ops.status_string(st).startswith("SQ_")
     assert "TIMEOUT" in ops.status_string(ops.SQ_ERR_TIMEOUT)
@@ -69,7 +69,8 @@ def test_quantize_act_validation(lib):
 
     def call(**kw):
         a = dict(ok, **kw)
-        return f(c(a["x"]), a["xt"], a["M"], a["K"], c(a["s"]), a["qt"], c(a["xq"]), c(a["sx"]), None)
+        return f(c(a["x"]), a["xt"], a["M"], a["K"], c(a["s"]), c(a.get("s_inv")), a["qt"], c(a["xq"]),
+                 c(a["sx"]), None)
 
     assert call(x=NUL) == ops.SQ_ERR_INVALID_ARG
     assert call(xq=NUL) == ops.SQ_ERR_INVALID_ARG
@@ -83,6 +84,7 @@ def test_quantize_act_validation(lib):
     assert call(x=MIS) == ops.SQ_ERR_MISALIGNED
     assert call(xq=A + 8) == ops.SQ_ERR_MISALIGNED
     assert call(s=A + 4) == ops.SQ_ERR_MISALIGNED
+    assert call(s_inv=A + 4) == ops.SQ_ERR_MISALIGNED
     assert call(M=0) == ops.SQ_OK                      # empty input: no-op
 
 
@@ -116,12 +118,13 @@ def test_gemm_validation(lib):
 
 def test_smooth_factor_and_calibration_validation(lib):
     sf = lib.sq_smooth_factors
-    assert sf(c(A), c(A), 64, 1.5, c(A), None) == ops.SQ_ERR_INVALID_ARG
-    assert sf(c(A), c(A), 64, -0.1, c(A), None) == ops.SQ_ERR_INVALID_ARG
-    assert sf(c(A), c(A), 64, float("nan"), c(A), None) == ops.SQ_ERR_INVALID_ARG
-    assert sf(c(A), c(A), 0, 0.5, c(A), None) == ops.SQ_ERR_INVALID_ARG
-    assert sf(c(A), None, 64, 0.5, c(A), None) == ops.SQ_ERR_INVALID_ARG
-    assert sf(c(A + 2), c(A), 64, 0.5, c(A), None) == ops.SQ_ERR_MISALIGNED
+    assert sf(c(A), c(A), 64, 1.5, c(A), None, None) == ops.SQ_ERR_INVALID_ARG
+    assert sf(c(A), c(A), 64, -0.1, c(A), None, None) == ops.SQ_ERR_INVALID_ARG
+    assert sf(c(A), c(A), 64, float("nan"), c(A), None, None) == ops.SQ_ERR_INVALID_ARG
+    assert sf(c(A), c(A), 0, 0.5, c(A), None, None) == ops.SQ_ERR_INVALID_ARG
+    assert sf(c(A), None, 64, 0.5, c(A), None, None) == ops.SQ_ERR_INVALID_ARG
+    assert sf(c(A + 2), c(A), 64, 0.5, c(A), None, None) == ops.SQ_ERR_MISALIGNED
+    assert sf(c(A), c(A), 64, 0.5, c(A), c(A + 2), None) == ops.SQ_ERR_MISALIGNED
     ca = lib.sq_calibrate_amax
     assert ca(c(A), ops.SQ_BF16, 0, 64, 0, c(A), 0, None) == ops.SQ_ERR_INVALID_ARG
     assert ca(c(A), ops.SQ_BF16, 8, 60, 0, c(A), 0, None) == ops.SQ_ERR_INVALID_ARG
@@ -133,8 +136,8 @@ def test_smooth_factor_and_calibration_validation(lib):
     assert qw(c(A), ops.SQ_BF16, 64, 64, None, ops.SQ_I32, c(A), c(A), None) == ops.SQ_ERR_INVALID_ARG
     assert qw(c(A), ops.SQ_BF16, 64, 64, None, ops.SQ_I8, c(A), c(A + 4), None) == ops.SQ_ERR_MISALIGNED
     lin = lib.sq_linear
-    assert lin(c(A), ops.SQ_BF16, None, c(A), c(A), None, ops.SQ_I32, 4, 64, 64, c(A), c(A), c(A),
-               ops.SQ_BF16, None) == ops.SQ_ERR_INVALID_ARG
-    assert lin(c(A), ops.SQ_BF16, None, c(A), c(A), None, ops.SQ_I8, 0, 64, 64, c(A), c(A), c(A),
-               ops.SQ_BF16, None) == ops.SQ_OK
+    assert lin(c(A), ops.SQ_BF16, None, None, c(A), c(A), None, ops.SQ_I32, 4, 64, 64, c(A), c(A),
+               c(A), ops.SQ_BF16, None) == ops.SQ_ERR_INVALID_ARG
+    assert lin(c(A), ops.SQ_BF16, None, None, c(A), c(A), None, ops.SQ_I8, 0, 64, 64, c(A), c(A),
+               c(A), ops.SQ_BF16, None) == ops.SQ_OK
     assert lib.sq_probe_wait_timeout(10, None) == ops.SQ_ERR_INVALID_ARG

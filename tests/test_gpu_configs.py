@@ -1,0 +1,86 @@
+"""The five workloads at full size, in the launch configuration bench.py
+times (tile shape chosen by problem size), against the CPU oracle.
+
+Per workload: calibration amaxes bit-exact, smoothing factors within 2 ulp,
+weight codes / scales and activation codes / scales bit-exact (each GPU
+stage fed the oracle's inputs), and the GEMM output on sampled elements
+(complete rows and columns through every tile edge plus random points):
+bit-exact for INT8, within 1e-3 of the exact sum (normalized) for FP8.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from w8a8_smoothquant_int8_02_b200 import ops, synth, workloads
+
+from _gpu_util import dev, fp8_normalized_error, host, sample_points, ulp_distance
+
+pytestmark = pytest.mark.gpu
+
+
+def _reciprocals(s):
+    s = np.asarray(s, np.float32)
+    inside = (s >= np.float32(2.0 ** -20)) & (s <= np.float32(2.0 ** 20))
+    return np.where(inside, np.float32(1.0) / np.where(inside, s, 1), np.float32(np.nan)).astype(np.float32)
+
+
+@pytest.mark.parametrize("name", list(workloads.ALL))
+def test_workload_end_to_end(name):
+    case = workloads.ALL[name]
+    qt = oracle.E4M3 if case.qtype == "e4m3" else oracle.INT8
+    d = synth.generate(case)
+    x, x_cal, w, bias = d["x"], d["x_cal"], d["w"], d["bias"]
+    M, K, N = case.M, case.K, case.N
+
+    # ---- offline preparation ----
+    ax = oracle.amax(x_cal, True)
+    aw = oracle.amax(w, False)
+    s = oracle.smooth_factors(ax, aw, case.alpha)
+    w_d = dev(w)
+    p = ops.prepare(w_d, dev(x_cal), alpha=case.alpha, qtype=case.qtype)
+    np.testing.assert_array_equal(host(p["amax_x"]), ax)
+    np.testing.assert_array_equal(host(p["amax_w"]), aw)
+    assert ulp_distance(host(p["s"]), s).max() <= 2
+
+    wq_ref, sw_ref = oracle.quantize_weight(w, s, qt)
+    wq_d, sw_d = ops.quantize_weight(w_d, dev(s), case.qtype)
+    del w_d
+    np.testing.assert_array_equal(host(sw_d), sw_ref)
+    np.testing.assert_array_equal(host(wq_d).view(np.uint8), wq_ref.view(np.uint8))
+
+    # ---- runtime: activation smoothing + per-token quantization ----
+    xq_ref, sx_ref = oracle.quantize_act(x, s, qt)
+    xq_d, sx_d = ops.quantize_act(dev(x), dev(s), case.qtype, s_inv=dev(_reciprocals(s)))
+    np.testing.assert_array_equal(host(sx_d), sx_ref)
+    np.testing.assert_array_equal(host(xq_d).view(np.uint8), xq_ref.view(np.uint8))
+
+    # ---- runtime: 8-bit GEMM + epilogue, on the oracle's operands ----
+    bias_d = None if bias is None else dev(bias)
+    gemm = ops.gemm_w8a8 if case.qtype == "i8" else ops.gemm_fp8
+    ops_x, ops_w = dev(xq_ref), dev(wq_ref)
+    yf = gemm(ops_x, dev(sx_ref), ops_w, dev(sw_ref), bias_d, out_dtype=torch.float32)
+    yb = gemm(ops_x, dev(sx_ref), ops_w, dev(sw_ref), bias_d)
+    assert ops.device_status() == ops.SQ_OK
+    full = M * N <= 1 << 20
+    if full:
+        rows, cols = np.divmod(np.arange(M * N, dtype=np.int64), N)
+    else:
+        rows, cols = sample_points(M, N, seed=hash(name) % 1000,
+                                   full_rows=2 if N > 20000 else 4, full_cols=4)
+    acc, yf_ref, yb_ref = oracle.linear_at(xq_ref, sx_ref, wq_ref, sw_ref, bias, rows, cols, qt)
+    yf_got = host(yf)[rows, cols]
+    yb_got = host(yb)[rows, cols]
+    if case.qtype == "i8":
+        np.testing.assert_array_equal(yf_got, yf_ref)
+        np.testing.assert_array_equal(yb_got, yb_ref)
+    else:
+        e = fp8_normalized_error(yf_got, yf_ref, xq_ref, wq_ref, sx_ref, sw_ref, bias, rows, cols)
+        assert e.max() <= 1e-3, e.max()
+        np.testing.assert_array_equal(yb_got, oracle.f32_to_bf16(yf_got))
+
+    # ---- the fused forward through one C call (same operands) ----
+    y2 = ops.linear(dev(x), dev(s), ops_w, dev(sw_ref), bias_d, case.qtype,
+                    out_dtype=torch.float32, s_inv=dev(_reciprocals(s)))
+    assert ops.device_status() == ops.SQ_OK
+    np.testing.assert_array_equal(host(y2)[rows, cols], yf_got)

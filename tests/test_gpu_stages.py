@@ -52,6 +52,14 @@ def test_calibrate_amax_accumulates_over_batches():
 
 # ----------------------------------------------------------------------- a3 --
 
+def reciprocals(s):
+    """The documented content of s_inv: the IEEE binary32 reciprocal inside
+    [2^-20, 2^20], NaN outside."""
+    s = np.asarray(s, np.float32)
+    inside = (s >= np.float32(2.0 ** -20)) & (s <= np.float32(2.0 ** 20))
+    return np.where(inside, np.float32(1.0) / np.where(inside, s, 1), np.float32(np.nan)).astype(np.float32)
+
+
 @pytest.mark.parametrize("alpha", [0.0, 0.5, 0.85, 1.0])
 def test_smooth_factors(alpha):
     g = np.random.default_rng(3)
@@ -59,11 +67,13 @@ def test_smooth_factors(alpha):
     aw = g.uniform(1e-4, 0.2, 4096).astype(np.float32)
     ax[:3] = 0.0
     aw[3:6] = 0.0
-    got = host(ops.smooth_factors(dev(ax), dev(aw), alpha))
+    s_d, inv_d = ops.smooth_factors(dev(ax), dev(aw), alpha, with_inverse=True)
+    got = host(s_d)
     ref = oracle.smooth_factors(ax, aw, alpha)
     d = ulp_distance(got, ref)
     assert d.max() <= 2, d.max()
     assert (d == 0).mean() >= 0.99
+    np.testing.assert_array_equal(host(inv_d), reciprocals(got))
 
 
 # ----------------------------------------------------------------------- a4 --
@@ -96,9 +106,12 @@ def test_quantize_act(qtype, dtype, smooth, M, K):
     s = synth.random_floats(K, seed=K + 1, lo=0.05, hi=20.0) if smooth else None
     qt = oracle.E4M3 if qtype == "e4m3" else oracle.INT8
     xq_ref, sx_ref = oracle.quantize_act(x, s, qt)
-    xq, sx = ops.quantize_act(dev(x), None if s is None else dev(s), qtype)
-    np.testing.assert_array_equal(host(sx), sx_ref)
-    np.testing.assert_array_equal(host(xq).view(np.uint8), xq_ref.view(np.uint8))
+    variants = [None] if s is None else [None, reciprocals(s)]
+    for s_inv in variants:
+        xq, sx = ops.quantize_act(dev(x), None if s is None else dev(s), qtype,
+                                  s_inv=None if s_inv is None else dev(s_inv))
+        np.testing.assert_array_equal(host(sx), sx_ref)
+        np.testing.assert_array_equal(host(xq).view(np.uint8), xq_ref.view(np.uint8))
 
 
 def test_quantize_act_zero_rows_and_ties():
@@ -261,7 +274,8 @@ def test_linear_matches_oracle(qtype):
     s = oracle.smooth_factors(oracle.amax(x, True), oracle.amax(w, False), 0.5)
     wq, sw = oracle.quantize_weight(w, s, qt)
     ref = oracle.linear(x, s, wq, sw, bias, qt)
-    y = ops.linear(dev(x), dev(s), dev(wq), dev(sw), dev(bias), qtype, out_dtype=torch.float32)
+    y = ops.linear(dev(x), dev(s), dev(wq), dev(sw), dev(bias), qtype, out_dtype=torch.float32,
+                   s_inv=dev(reciprocals(s)))
     assert ops.device_status() == ops.SQ_OK
     if qtype == "i8":
         np.testing.assert_array_equal(host(y), ref["y_f32"])
@@ -281,6 +295,39 @@ def test_prepare_pipeline_matches_oracle():
     np.testing.assert_array_equal(host(p["amax_w"]), aw)
     s = oracle.smooth_factors(ax, aw, 0.5)
     assert ulp_distance(host(p["s"]), s).max() <= 2
+    np.testing.assert_array_equal(host(p["s_inv"]), reciprocals(host(p["s"])))
+
+
+def test_fast_division_is_exact_on_every_bf16_significand():
+    """The reciprocal-product division used for bf16 activations equals the
+    IEEE division on all 2^30 (x, s) significand pairs, both signs."""
+    assert ops.selftest_fast_division() == 0
+
+
+@pytest.mark.parametrize("qtype", ["i8", "e4m3"])
+def test_quantize_act_fast_path_edge_values(qtype):
+    """bf16 rows with zeros of both signs, subnormals, huge values, exact
+    ties after smoothing, and smoothing factors outside the fast window."""
+    K = 256
+    g = np.random.default_rng(77)
+    x = (g.standard_normal((6, K)) * 3).astype(np.float32)
+    x[0, :8] = [0.0, -0.0, 1e-40, -1e-40, 3e38, -3e38, 2.0 ** -130, 1.0]
+    x[1] = np.float32(2.0) ** g.integers(-20, 20, K).astype(np.float32)
+    x[2] = 0.0
+    x[3, :4] = [127.0, 63.5, -0.5, 1.5]
+    x[4] *= 1e-38
+    s = synth.random_floats(K, seed=78, lo=0.05, hi=20.0)
+    # channels 1..3 lie outside the fast-division window; no quotient overflows
+    s[:4] = [1.0, 2.0 ** -30, 2.0 ** 30, 2.0 ** -25]
+    s[4:8] = 2.0 ** g.integers(0, 5, 4).astype(np.float32)
+    xb = synth.to_bf16_bits(x)
+    qt = oracle.E4M3 if qtype == "e4m3" else oracle.INT8
+    for smooth, inv in ((s, reciprocals(s)), (s, None), (None, None)):
+        xq_ref, sx_ref = oracle.quantize_act(xb, smooth, qt)
+        xq, sx = ops.quantize_act(dev(xb), None if smooth is None else dev(smooth), qtype,
+                                  s_inv=None if inv is None else dev(inv))
+        np.testing.assert_array_equal(host(sx), sx_ref)
+        np.testing.assert_array_equal(host(xq).view(np.uint8), xq_ref.view(np.uint8))
 
 
 # ---------------------------------------------------------- failure path --

@@ -9,9 +9,11 @@
 #include "sq_common.cuh"
 #include "sq_internal.h"
 
-// The library's only device allocation: one status word per device that a
-// kernel sets when a bounded wait gives up.
+// The library's only device allocations: one status word per device that a
+// kernel sets when a bounded wait gives up, and the mismatch counter of the
+// arithmetic self-test.
 static __device__ int g_sq_status = 0;
+static __device__ unsigned long long g_sq_selftest_count = 0;
 
 namespace sqh {
 
@@ -108,11 +110,12 @@ sq_status sq_calibrate_amax(const void* x, sq_dtype xt, int64_t rows, int64_t co
 }
 
 sq_status sq_smooth_factors(const float* amax_x, const float* amax_w, int64_t K, double alpha,
-                            float* s, void* stream) {
+                            float* s, float* s_inv, void* stream) {
   if (!amax_x || !amax_w || !s || K <= 0) return SQ_ERR_INVALID_ARG;
   if (!(alpha >= 0.0 && alpha <= 1.0)) return SQ_ERR_INVALID_ARG;  // also rejects NaN
   if (!al(amax_x, 4) || !al(amax_w, 4) || !al(s, 4)) return SQ_ERR_MISALIGNED;
-  return from_cuda(sqh::launch_smooth_factors(amax_x, amax_w, K, alpha, s, S(stream)));
+  if (s_inv && !al(s_inv, 4)) return SQ_ERR_MISALIGNED;
+  return from_cuda(sqh::launch_smooth_factors(amax_x, amax_w, K, alpha, s, s_inv, S(stream)));
 }
 
 sq_status sq_quantize_weight(const void* w, sq_dtype wt, int64_t K, int64_t N, const float* s,
@@ -129,7 +132,7 @@ sq_status sq_quantize_weight(const void* w, sq_dtype wt, int64_t K, int64_t N, c
 }
 
 sq_status sq_quantize_act(const void* x, sq_dtype xt, int64_t M, int64_t K, const float* s,
-                          sq_dtype qt, void* xq, float* sx, void* stream) {
+                          const float* s_inv, sq_dtype qt, void* xq, float* sx, void* stream) {
   if (xt != SQ_F32 && xt != SQ_BF16) return SQ_ERR_INVALID_ARG;
   if (qt != SQ_I8 && qt != SQ_E4M3) return SQ_ERR_INVALID_ARG;
   if (M < 0 || K <= 0 || K % 16 != 0 || K > 65536 || M > INT32_MAX) return SQ_ERR_INVALID_ARG;
@@ -137,8 +140,10 @@ sq_status sq_quantize_act(const void* x, sq_dtype xt, int64_t M, int64_t K, cons
   if (!x || !xq || !sx) return SQ_ERR_INVALID_ARG;
   if (!al(x, 16) || !al(xq, 16) || !al(sx, 4)) return SQ_ERR_MISALIGNED;
   if (s && !al(s, 16)) return SQ_ERR_MISALIGNED;
-  return from_cuda(sqh::launch_quantize_act(x, xt == SQ_BF16, M, K, s, qt == SQ_E4M3,
-                                            static_cast<uint8_t*>(xq), sx, S(stream)));
+  if (s_inv && !al(s_inv, 16)) return SQ_ERR_MISALIGNED;
+  return from_cuda(sqh::launch_quantize_act(x, xt == SQ_BF16, M, K, s, s ? s_inv : nullptr,
+                                            qt == SQ_E4M3, static_cast<uint8_t*>(xq), sx,
+                                            S(stream)));
 }
 
 sq_status sq_gemm_w8a8(const int8_t* xq, const float* sx, const int8_t* wq, const float* sw,
@@ -164,19 +169,35 @@ sq_status sq_gemm_fp8(const uint8_t* xq, const float* sx, const uint8_t* wq, con
                                     S(stream)));
 }
 
-sq_status sq_linear(const void* x, sq_dtype xt, const float* s, const void* wq, const float* sw,
+sq_status sq_linear(const void* x, sq_dtype xt, const float* s, const float* s_inv,
+                    const void* wq, const float* sw,
                     const uint16_t* bias, sq_dtype qt, int64_t M, int64_t N, int64_t K,
                     void* xq_buf, float* sx_buf, void* y, sq_dtype yt, void* stream) {
   if (qt != SQ_I8 && qt != SQ_E4M3) return SQ_ERR_INVALID_ARG;
   sq_status c = check_gemm(xq_buf, sx_buf, wq, sw, bias, M, N, K, y, yt, nullptr);
   if (c != SQ_OK || M == 0) return c;
-  c = sq_quantize_act(x, xt, M, K, s, qt, xq_buf, sx_buf, stream);
+  c = sq_quantize_act(x, xt, M, K, s, s_inv, qt, xq_buf, sx_buf, stream);
   if (c != SQ_OK) return c;
   if (qt == SQ_I8)
     return sq_gemm_w8a8(static_cast<const int8_t*>(xq_buf), sx_buf, static_cast<const int8_t*>(wq),
                         sw, bias, M, N, K, y, yt, nullptr, stream);
   return sq_gemm_fp8(static_cast<const uint8_t*>(xq_buf), sx_buf, static_cast<const uint8_t*>(wq),
                      sw, bias, M, N, K, y, yt, stream);
+}
+
+sq_status sq_selftest_fast_division(int64_t* mismatches, void* stream) {
+  if (!mismatches) return SQ_ERR_INVALID_ARG;
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_sq_selftest_count) != cudaSuccess) return SQ_ERR_CUDA;
+  if (cudaMemsetAsync(p, 0, sizeof(unsigned long long), S(stream)) != cudaSuccess) return SQ_ERR_CUDA;
+  if (sqh::launch_selftest_fast_division(static_cast<unsigned long long*>(p), S(stream)) != cudaSuccess)
+    return SQ_ERR_CUDA;
+  unsigned long long v = 0;
+  if (cudaMemcpyAsync(&v, p, sizeof(v), cudaMemcpyDeviceToHost, S(stream)) != cudaSuccess ||
+      cudaStreamSynchronize(S(stream)) != cudaSuccess)
+    return SQ_ERR_CUDA;
+  *mismatches = static_cast<int64_t>(v);
+  return SQ_OK;
 }
 
 sq_status sq_probe_wait_timeout(int64_t timeout_ns, void* stream) {

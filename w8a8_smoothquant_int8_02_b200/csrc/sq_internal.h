@@ -17,13 +17,15 @@ cudaError_t launch_amax_rows(const void* x, bool bf16, int64_t rows, int64_t col
                              bool accumulate, cudaStream_t st);
 // a3
 cudaError_t launch_smooth_factors(const float* ax, const float* aw, int64_t K, double alpha,
-                                  float* s, cudaStream_t st);
+                                  float* s, float* s_inv, cudaStream_t st);
 // a4
 cudaError_t launch_quantize_weight(const void* w, bool bf16, int64_t K, int64_t N, const float* s,
                                    bool e4m3, uint8_t* wq, float* sw, cudaStream_t st);
 // a5
 cudaError_t launch_quantize_act(const void* x, bool bf16, int64_t M, int64_t K, const float* s,
-                                bool e4m3, uint8_t* xq, float* sx, cudaStream_t st);
+                                const float* s_inv, bool e4m3, uint8_t* xq, float* sx,
+                                cudaStream_t st);
+cudaError_t launch_selftest_fast_division(unsigned long long* mismatches, cudaStream_t st);
 // a6 / a7
 enum class OutKind { BF16, F32 };
 cudaError_t launch_gemm(bool e4m3, const uint8_t* xq, const float* sx, const uint8_t* wq,

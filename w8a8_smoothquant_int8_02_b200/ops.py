@@ -25,7 +25,7 @@ SQ_AMAX_PER_COLUMN, SQ_AMAX_PER_ROW = 0, 1
 EXPORTED = (
     "sq_status_string", "sq_abi_version", "sq_get_device_status", "sq_calibrate_amax",
     "sq_smooth_factors", "sq_quantize_weight", "sq_quantize_act", "sq_gemm_w8a8",
-    "sq_gemm_fp8", "sq_linear", "sq_probe_wait_timeout",
+    "sq_gemm_fp8", "sq_linear", "sq_probe_wait_timeout", "sq_selftest_fast_division",
 )
 
 _lock = threading.Lock()
@@ -59,13 +59,14 @@ def load(build_if_needed: bool = True) -> ctypes.CDLL:
             lib.sq_abi_version.restype = I
             lib.sq_get_device_status.argtypes = [P]
             lib.sq_calibrate_amax.argtypes = [P, I, I64, I64, I, P, I, P]
-            lib.sq_smooth_factors.argtypes = [P, P, I64, D, P, P]
+            lib.sq_smooth_factors.argtypes = [P, P, I64, D, P, P, P]
             lib.sq_quantize_weight.argtypes = [P, I, I64, I64, P, I, P, P, P]
-            lib.sq_quantize_act.argtypes = [P, I, I64, I64, P, I, P, P, P]
+            lib.sq_quantize_act.argtypes = [P, I, I64, I64, P, P, I, P, P, P]
             lib.sq_gemm_w8a8.argtypes = [P, P, P, P, P, I64, I64, I64, P, I, P, P]
             lib.sq_gemm_fp8.argtypes = [P, P, P, P, P, I64, I64, I64, P, I, P]
-            lib.sq_linear.argtypes = [P, I, P, P, P, P, I, I64, I64, I64, P, P, P, I, P]
+            lib.sq_linear.argtypes = [P, I, P, P, P, P, P, I, I64, I64, I64, P, P, P, I, P]
             lib.sq_probe_wait_timeout.argtypes = [I64, P]
+            lib.sq_selftest_fast_division.argtypes = [ctypes.POINTER(ctypes.c_int64), P]
             for name in EXPORTED:
                 if name not in ("sq_status_string", "sq_abi_version"):
                     getattr(lib, name).restype = I
@@ -135,13 +136,16 @@ def calibrate_amax(x: torch.Tensor, axis: str = "column", out: torch.Tensor | No
     return out
 
 
-def smooth_factors(amax_x: torch.Tensor, amax_w: torch.Tensor, alpha: float) -> torch.Tensor:
-    """a3: s = max(ax,1e-5)^alpha / max(aw,1e-5)^(1-alpha) (binary64 -> binary32)."""
+def smooth_factors(amax_x: torch.Tensor, amax_w: torch.Tensor, alpha: float,
+                   with_inverse: bool = False):
+    """a3: s = max(ax,1e-5)^alpha / max(aw,1e-5)^(1-alpha) (binary64 -> binary32).
+    with_inverse=True also returns s_inv (the reciprocals sq_quantize_act uses)."""
     _cuda(amax_x, amax_w)
     s = torch.empty_like(amax_x)
+    s_inv = torch.empty_like(amax_x) if with_inverse else None
     _check(load().sq_smooth_factors(_p(amax_x), _p(amax_w), amax_x.numel(), float(alpha), _p(s),
-                                    _stream(amax_x.device)), "sq_smooth_factors")
-    return s
+                                    _p(s_inv), _stream(amax_x.device)), "sq_smooth_factors")
+    return (s, s_inv) if with_inverse else s
 
 
 def quantize_weight(w: torch.Tensor, s: torch.Tensor | None, qtype: str = "i8"):
@@ -156,16 +160,18 @@ def quantize_weight(w: torch.Tensor, s: torch.Tensor | None, qtype: str = "i8"):
     return wq, sw
 
 
-def quantize_act(x: torch.Tensor, s: torch.Tensor | None, qtype: str = "i8", xq=None, sx=None):
-    """a5: fused smoothing + per-token quantization; returns (xq [M,K], sx [M])."""
-    _cuda(x, s, xq, sx)
+def quantize_act(x: torch.Tensor, s: torch.Tensor | None, qtype: str = "i8", xq=None, sx=None,
+                 s_inv: torch.Tensor | None = None):
+    """a5: fused smoothing + per-token quantization; returns (xq [M,K], sx [M]).
+    s_inv (from smooth_factors(..., with_inverse=True)) only makes it faster."""
+    _cuda(x, s, xq, sx, s_inv)
     M, K = x.shape
     qt = _qtype(qtype)
     if xq is None:
         xq = torch.empty((M, K), dtype=torch.int8 if qt == SQ_I8 else torch.uint8, device=x.device)
     if sx is None:
         sx = torch.empty(M, dtype=torch.float32, device=x.device)
-    _check(load().sq_quantize_act(_p(x), _fdtype(x), M, K, _p(s), qt, _p(xq), _p(sx),
+    _check(load().sq_quantize_act(_p(x), _fdtype(x), M, K, _p(s), _p(s_inv), qt, _p(xq), _p(sx),
                                   _stream(x.device)), "sq_quantize_act")
     return xq, sx
 
@@ -196,10 +202,10 @@ def gemm_fp8(xq, sx, wq, sw, bias=None, out_dtype=torch.bfloat16, out=None):
 
 
 def linear(x, s, wq, sw, bias=None, qtype="i8", out_dtype=torch.bfloat16, out=None,
-           xq_buf=None, sx_buf=None):
+           xq_buf=None, sx_buf=None, s_inv=None):
     """Runtime forward: quantize_act then the 8-bit GEMM, one C call."""
     wq = _codes(wq)
-    _cuda(x, s, wq, sw, bias, out, xq_buf, sx_buf)
+    _cuda(x, s, wq, sw, bias, out, xq_buf, sx_buf, s_inv)
     M, K = x.shape
     N = wq.shape[0]
     qt = _qtype(qtype)
@@ -210,7 +216,8 @@ def linear(x, s, wq, sw, bias=None, qtype="i8", out_dtype=torch.bfloat16, out=No
         sx_buf = torch.empty(M, dtype=torch.float32, device=x.device)
     if out is None:
         out = torch.empty((M, N), dtype=out_dtype, device=x.device)
-    _check(load().sq_linear(_p(x), _fdtype(x), _p(s), _p(wq), _p(sw), _p(bias), qt, M, N, K,
+    _check(load().sq_linear(_p(x), _fdtype(x), _p(s), _p(s_inv), _p(wq), _p(sw), _p(bias), qt,
+                            M, N, K,
                             _p(xq_buf), _p(sx_buf), _p(out), _fdtype(out), _stream(x.device)),
            "sq_linear")
     return out
@@ -219,6 +226,15 @@ def linear(x, s, wq, sw, bias=None, qtype="i8", out_dtype=torch.bfloat16, out=No
 def device_status(device=None) -> int:
     """Synchronize the current stream and return (and clear) the status word."""
     return int(load().sq_get_device_status(_stream(device)))
+
+
+def selftest_fast_division(device=None) -> int:
+    """Exhaustive check of the activation-smoothing division shortcut; returns
+    the number of (x, s) significand pairs where it differs from IEEE division."""
+    n = ctypes.c_int64(-1)
+    _check(load().sq_selftest_fast_division(ctypes.byref(n), _stream(device)),
+           "sq_selftest_fast_division")
+    return int(n.value)
 
 
 def probe_wait_timeout(timeout_ns: int, device=None):
@@ -259,9 +275,9 @@ def prepare(w: torch.Tensor, x_cal: torch.Tensor, alpha: float = 0.5, qtype: str
     """Offline preparation of one layer: calibrate, smoothing factors, quantized weights."""
     ax = calibrate_amax(x_cal, "column")
     aw = calibrate_amax(w, "row")
-    s = smooth_factors(ax, aw, alpha)
+    s, s_inv = smooth_factors(ax, aw, alpha, with_inverse=True)
     wq, sw = quantize_weight(w, s, qtype)
-    return dict(s=s, wq=wq, sw=sw, amax_x=ax, amax_w=aw)
+    return dict(s=s, s_inv=s_inv, wq=wq, sw=sw, amax_x=ax, amax_w=aw)
 
 
 class SmoothQuantLinear:
@@ -270,10 +286,11 @@ class SmoothQuantLinear:
     def __init__(self, w: torch.Tensor, x_cal: torch.Tensor, alpha: float = 0.5,
                  qtype: str = "i8", bias: torch.Tensor | None = None):
         p = prepare(w, x_cal, alpha, qtype)
-        self.s, self.wq, self.sw = p["s"], p["wq"], p["sw"]
+        self.s, self.s_inv, self.wq, self.sw = p["s"], p["s_inv"], p["wq"], p["sw"]
         self.qtype = qtype
         self.bias = bias
         self.in_features, self.out_features = w.shape
 
     def __call__(self, x: torch.Tensor, out_dtype=torch.bfloat16) -> torch.Tensor:
-        return linear(x, self.s, self.wq, self.sw, self.bias, self.qtype, out_dtype)
+        return linear(x, self.s, self.wq, self.sw, self.bias, self.qtype, out_dtype,
+                      s_inv=self.s_inv)
