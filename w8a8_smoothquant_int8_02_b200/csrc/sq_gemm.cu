@@ -21,9 +21,12 @@
 //                leader CTA one thread issues the MMAs (K = 32 per
 //                instruction) and frees ring slots / publishes finished
 //                accumulators with tcgen05.commit.
-//   warps 2..5 : epilogue -- tcgen05.ld of accumulator rows (warp w reads
-//                TMEM lanes 32*(w%4)..+31), dequantize, bf16, store; then
-//                hand the accumulator buffer back to the MMA thread. Two
+//   warps 2..9 : epilogue -- two warps per TMEM lane quarter (warp w reads
+//                lanes 32*(w%4)..+31, the two warps of a quarter take
+//                alternate 32-column chunks): tcgen05.ld, dequantize with the
+//                per-token scale and the per-channel scales / bias that the
+//                producer staged in shared memory by bulk copy, bf16, store;
+//                then hand the accumulator buffer back to the MMA thread. Two
 //                buffers let the epilogue of tile i overlap the MMAs of i+1.
 // Tiles are walked in groups of kGroupM M-tiles so that the CTAs working at
 // the same time share Wq tiles in L2. Every barrier wait is bounded: a wait
@@ -41,10 +44,11 @@
 namespace sqk {
 
 constexpr int kBK = 128;  // bytes of K per pipeline stage (one swizzle row)
-constexpr int kThreads = 192;
+constexpr int kEpiWarps = 8;  // 4 or 8 (one or two per TMEM lane quarter)
+constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int kGroupM = 16;
 
-template <int CG, int BN, int STAGES>
+template <int CG, int BN, int MAXST, bool OUT_BF16>
 struct GemmCfg {
   static constexpr int kTileM = 128 * CG;  // output rows per tile
   static constexpr int kBRows = BN / CG;   // Wq rows staged per CTA
@@ -54,15 +58,30 @@ struct GemmCfg {
   static constexpr uint32_t kTxBytes = kStageBytes * CG;  // landing on one "full" barrier
   static constexpr uint32_t kAccStride = BN <= 128 ? 128 : 256;  // TMEM columns per buffer
   static constexpr uint32_t kTmemCols = 2 * kAccStride;
+  // output staging: per epilogue warp two boxes of 32 rows x 32 columns,
+  // written swizzled (64-byte rows for bf16, 128-byte rows for binary32) and
+  // stored by TMA
+  static constexpr uint32_t kOutRow = OUT_BF16 ? 64 : 128;
+  static constexpr uint32_t kOutBox = 32 * kOutRow;
+  static constexpr uint32_t kOutBytes = kEpiWarps * 2 * kOutBox;
+  static constexpr uint32_t kFixed = kOutBytes + 2048 + 2 * (BN * 6) + 1024;
+  static constexpr int kFit = int((232448 - kFixed) / kStageBytes);
+  static constexpr int STAGES = kFit < MAXST ? kFit : MAXST;
   static constexpr uint32_t kRingA = 0;
   static constexpr uint32_t kRingB = STAGES * kABytes;
-  static constexpr uint32_t kBarOff = STAGES * kStageBytes;
-  // barriers: full[S], empty[S], tfull[2], tempty[2], drain
-  static constexpr uint32_t kMiscOff = kBarOff + (2 * STAGES + 5) * 8;  // tmem slot, abort flag
-  static constexpr uint32_t kTotal = kMiscOff + 16;
+  static constexpr uint32_t kOutOff = STAGES * kStageBytes;  // 1024-aligned
+  static constexpr uint32_t kBarOff = kOutOff + kOutBytes;
+  // barriers: full[S], empty[S], tfull[2], tempty[2], sfull[2], sempty[2], drain
+  static constexpr uint32_t kMiscOff = kBarOff + (2 * STAGES + 9) * 8;  // tmem slot, abort flag
+  // per-tile per-channel scales (binary32) and bias (bf16), one slot per
+  // accumulator buffer
+  static constexpr uint32_t kScaleSlot = BN * 4 + BN * 2;
+  static constexpr uint32_t kScaleOff = (kMiscOff + 16 + 127) & ~127u;
+  static constexpr uint32_t kTotal = kScaleOff + 2 * kScaleSlot;
   static constexpr uint32_t kDynamic = kTotal + 1024;  // slack for 1024-B alignment
   static_assert(BN % 32 == 0 && BN <= 256, "BN must be a multiple of 32, at most 256");
   static_assert(kBRows % 8 == 0, "staged Wq rows must be whole 8-row swizzle atoms");
+  static_assert(STAGES >= 3, "too few pipeline stages fit");
   static_assert(kDynamic <= 232448, "shared memory budget exceeded");
 };
 
@@ -75,13 +94,14 @@ __device__ __forceinline__ void tile_coords(int tile, int num_mt, int num_nt, in
   nt = r / gm;
 }
 
-template <int CG, int BN, int STAGES, bool E4M3, bool OUT_BF16, bool HAS_BIAS, bool WRITE_ACC>
+template <int CG, int BN, int MAXST, bool E4M3, bool OUT_BF16, bool HAS_BIAS, bool WRITE_ACC>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-                     const float* __restrict__ sx, const float* __restrict__ sw,
-                     const uint16_t* __restrict__ bias, void* __restrict__ y,
+                     const __grid_constant__ CUtensorMap tm_y, const float* __restrict__ sx,
+                     const float* __restrict__ sw, const uint16_t* __restrict__ bias,
                      int32_t* __restrict__ acc_out, int M, int N, int K, int* status) {
-  using C = GemmCfg<CG, BN, STAGES>;
+  using C = GemmCfg<CG, BN, MAXST, OUT_BF16>;
+  constexpr int STAGES = C::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -92,7 +112,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t bar_empty = bar_full + STAGES * 8;
   const uint32_t bar_tfull = bar_empty + STAGES * 8;
   const uint32_t bar_tempty = bar_tfull + 2 * 8;
-  const uint32_t bar_drain = bar_tempty + 2 * 8;
+  const uint32_t bar_sfull = bar_tempty + 2 * 8;
+  const uint32_t bar_sempty = bar_sfull + 2 * 8;
+  const uint32_t bar_drain = bar_sempty + 2 * 8;
+  const uint32_t s_scale = s_base + C::kScaleOff;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
 
@@ -107,13 +130,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar_tfull + 8 * b, 1);
-      mbar_init(bar_tempty + 8 * b, 4 * CG);
+      mbar_init(bar_tempty + 8 * b, kEpiWarps * CG);
+      mbar_init(bar_sfull + 8 * b, 1);
+      mbar_init(bar_sempty + 8 * b, kEpiWarps);
     }
     mbar_init(bar_drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_map(&tm_a);
     tma_prefetch_map(&tm_b);
+    tma_prefetch_map(&tm_y);
   }
   if (warp == 1) {
     if constexpr (CG == 2) {
@@ -138,14 +164,31 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer --
     if (lane == 0) {
-      uint32_t it = 0;
+      uint32_t it = 0, tc = 0;
       bool ok = true;
 #pragma unroll 1
-      for (int tile = unit; tile < num_tiles && ok; tile += num_units) {
+      for (int tile = unit; tile < num_tiles && ok; tile += num_units, ++tc) {
         int mt, nt;
         tile_coords(tile, num_mt, num_nt, mt, nt);
         const int a_row = mt * C::kTileM + int(rank) * 128;
         const int b_row = nt * BN + int(rank) * C::kBRows;
+        {
+          // stage this tile's per-channel scales (and bias) for the epilogue
+          const uint32_t buf = tc & 1u;
+          if (!mbar_wait(bar_sempty + 8 * buf, ((tc >> 1) & 1u) ^ 1u) || *abort_flag) {
+            record_status(status, kStatusTimeout);
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          const int n0 = nt * BN;
+          const int cols = N - n0 < BN ? N - n0 : BN;
+          const uint32_t sw_bytes = uint32_t(cols) * 4, b_bytes = HAS_BIAS ? uint32_t(cols) * 2 : 0;
+          const uint32_t slot = s_scale + buf * C::kScaleSlot;
+          mbar_arrive_expect_tx(bar_sfull + 8 * buf, sw_bytes + b_bytes);
+          bulk_load(slot, sw + n0, sw_bytes, bar_sfull + 8 * buf);
+          if constexpr (HAS_BIAS) bulk_load(slot + BN * 4, bias + n0, b_bytes, bar_sfull + 8 * buf);
+        }
 #pragma unroll 1
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const uint32_t st = it % STAGES, ph = (it / STAGES) & 1u;
@@ -233,14 +276,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue --
+    constexpr int NCH = BN / 32;  // 32-column chunks per tile
     const int sub = warp & 3;
+    constexpr int WPQ = kEpiWarps / 4;  // epilogue warps per TMEM lane quarter
+    const int half = (warp - 2) >> 2;   // which warp of this lane quarter
     const int row_in_tile = int(rank) * 128 + sub * 32 + lane;
     const uint32_t tempty_leader = CG == 2 ? map_to_rank(bar_tempty, 0) : bar_tempty;
     uint32_t tc = 0;
+    uint32_t emitted = 0;  // chunks this warp has handed to TMA stores
 #pragma unroll 1
     for (int tile = unit; tile < num_tiles; tile += num_units, ++tc) {
       const uint32_t buf = tc & 1u, use = tc >> 1;
-      if (!mbar_wait(bar_tfull + 8 * buf, use & 1u) || *abort_flag) {
+      if (!mbar_wait(bar_tfull + 8 * buf, use & 1u) || !mbar_wait(bar_sfull + 8 * buf, use & 1u) ||
+          *abort_flag) {
         record_status(status, kStatusTimeout);
         *abort_flag = 1;
         break;
@@ -252,67 +300,111 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int n_base = nt * BN;
       const float sxm = m < M ? __ldg(sx + m) : 0.0f;
       const uint32_t t_addr = tmem_base + buf * C::kAccStride + (uint32_t(sub * 32) << 16);
-#pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 32) {
-        uint32_t r[32];
-        tmem_ld32(t_addr + uint32_t(c0), r);
-        tmem_wait_ld(r);
-        if (m < M) {
+      const float* s_sw = reinterpret_cast<const float*>(smem + C::kScaleOff + buf * C::kScaleSlot);
+      const uint16_t* s_b = reinterpret_cast<const uint16_t*>(smem + C::kScaleOff +
+                                                                buf * C::kScaleSlot + BN * 4);
+
+      // dequantize one 32-column chunk held in r[] into a staging box and
+      // store it with TMA (the box's rows / columns outside Y are clipped)
+      const int e = warp - 2;
+      const int box_row = mt * C::kTileM + int(rank) * 128 + sub * 32;
+      auto emit = [&](const uint32_t (&r)[32], int chunk) {
+        const uint32_t sbuf = s_base + C::kOutOff + uint32_t(e * 2 + (emitted & 1)) * C::kOutBox;
+        if (emitted >= 2) {
+          // the bulk store that last read this buffer must be done reading
+          if (lane == 0) bulk_wait_read<1>();
+          __syncwarp();
+        }
 #pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            const int n = n_base + c0 + g * 8;
-            if (n < N) {
-              const float4 w0 = __ldg(reinterpret_cast<const float4*>(sw + n));
-              const float4 w1 = __ldg(reinterpret_cast<const float4*>(sw + n) + 1);
-              const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-              float bv[8];
-              if constexpr (HAS_BIAS) {
-                const uint4 b = __ldg(reinterpret_cast<const uint4*>(bias + n));
-                bv[0] = bf16_lo(b.x); bv[1] = bf16_hi(b.x);
-                bv[2] = bf16_lo(b.y); bv[3] = bf16_hi(b.y);
-                bv[4] = bf16_lo(b.z); bv[5] = bf16_hi(b.z);
-                bv[6] = bf16_lo(b.w); bv[7] = bf16_hi(b.w);
-              }
-              float t[8];
+        for (int g = 0; g < 4; ++g) {
+          const int nl = chunk * 32 + g * 8;
+          const float4 w0 = *reinterpret_cast<const float4*>(s_sw + nl);
+          const float4 w1 = *reinterpret_cast<const float4*>(s_sw + nl + 4);
+          const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+          float bv[8];
+          if constexpr (HAS_BIAS) {
+            const uint4 b = *reinterpret_cast<const uint4*>(s_b + nl);
+            bv[0] = bf16_lo(b.x); bv[1] = bf16_hi(b.x);
+            bv[2] = bf16_lo(b.y); bv[3] = bf16_hi(b.y);
+            bv[4] = bf16_lo(b.z); bv[5] = bf16_hi(b.z);
+            bv[6] = bf16_lo(b.w); bv[7] = bf16_hi(b.w);
+          }
+          float t[8];
 #pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                const uint32_t raw = r[g * 8 + i];
-                float a = E4M3 ? __uint_as_float(raw) : __int2float_rn(int32_t(raw));
-                a = __fmul_rn(a, sxm);
-                a = __fmul_rn(a, wv[i]);
-                if constexpr (HAS_BIAS) a = __fadd_rn(a, bv[i]);
-                t[i] = a;
-              }
-              const int64_t off = int64_t(m) * N + n;
-              if constexpr (OUT_BF16) {
-                uint4 u;
-                u.x = pack_bf16x2(t[0], t[1]);
-                u.y = pack_bf16x2(t[2], t[3]);
-                u.z = pack_bf16x2(t[4], t[5]);
-                u.w = pack_bf16x2(t[6], t[7]);
-                *reinterpret_cast<uint4*>(static_cast<uint16_t*>(y) + off) = u;
-              } else {
-                float4* p = reinterpret_cast<float4*>(static_cast<float*>(y) + off);
-                p[0] = make_float4(t[0], t[1], t[2], t[3]);
-                p[1] = make_float4(t[4], t[5], t[6], t[7]);
-              }
-              if constexpr (WRITE_ACC) {
-                int4* q = reinterpret_cast<int4*>(acc_out + off);
-                q[0] = make_int4(int(r[g * 8 + 0]), int(r[g * 8 + 1]), int(r[g * 8 + 2]), int(r[g * 8 + 3]));
-                q[1] = make_int4(int(r[g * 8 + 4]), int(r[g * 8 + 5]), int(r[g * 8 + 6]), int(r[g * 8 + 7]));
-              }
+          for (int i = 0; i < 8; ++i) {
+            const uint32_t raw = r[g * 8 + i];
+            float a = E4M3 ? __uint_as_float(raw) : __int2float_rn(int32_t(raw));
+            a = __fmul_rn(a, sxm);
+            a = __fmul_rn(a, wv[i]);
+            if constexpr (HAS_BIAS) a = __fadd_rn(a, bv[i]);
+            t[i] = a;
+          }
+          if constexpr (OUT_BF16) {
+            // row = lane (64 B); 16-byte unit g, 64-byte swizzle
+            const uint32_t unit = uint32_t(g) ^ ((uint32_t(lane) >> 1) & 3u);
+            const uint32_t addr = sbuf + uint32_t(lane) * 64 + unit * 16;
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
+                         "r"(pack_bf16x2(t[0], t[1])), "r"(pack_bf16x2(t[2], t[3])),
+                         "r"(pack_bf16x2(t[4], t[5])), "r"(pack_bf16x2(t[6], t[7]))
+                         : "memory");
+          } else {
+            // row = lane (128 B); 16-byte units 2g, 2g+1, 128-byte swizzle
+            const uint32_t u0 = (uint32_t(2 * g) ^ (uint32_t(lane) & 7u));
+            const uint32_t u1 = (uint32_t(2 * g + 1) ^ (uint32_t(lane) & 7u));
+            const uint32_t base = sbuf + uint32_t(lane) * 128;
+            asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(base + u0 * 16),
+                         "f"(t[0]), "f"(t[1]), "f"(t[2]), "f"(t[3])
+                         : "memory");
+            asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(base + u1 * 16),
+                         "f"(t[4]), "f"(t[5]), "f"(t[6]), "f"(t[7])
+                         : "memory");
+          }
+          if constexpr (WRITE_ACC) {
+            const int n = n_base + nl;
+            if (m < M && n < N) {
+              int4* q = reinterpret_cast<int4*>(acc_out + int64_t(m) * N + n);
+              q[0] = make_int4(int(r[g * 8 + 0]), int(r[g * 8 + 1]), int(r[g * 8 + 2]), int(r[g * 8 + 3]));
+              q[1] = make_int4(int(r[g * 8 + 4]), int(r[g * 8 + 5]), int(r[g * 8 + 6]), int(r[g * 8 + 7]));
             }
           }
         }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tm_y, sbuf, n_base + chunk * 32, box_row);
+          bulk_commit_group();
+        }
+        ++emitted;
+      };
+
+      // this warp's chunks are half, half+WPQ, half+2*WPQ, ...; two loads in
+      // flight at a time
+#pragma unroll 1
+      for (int c = half; c < NCH; c += 2 * WPQ) {
+        uint32_t r0[32], r1[32];
+        const bool two = c + WPQ < NCH;  // warp-uniform
+        tmem_ld32(t_addr + uint32_t(c * 32), r0);
+        if (two) {
+          tmem_ld32(t_addr + uint32_t((c + WPQ) * 32), r1);
+          tmem_wait_ld2(r0, r1);
+        } else {
+          tmem_wait_ld(r0);
+        }
+        emit(r0, c);
+        if (two) emit(r1, c + WPQ);
       }
-      // hand the accumulator buffer back to the MMA thread
+      // hand the accumulator buffer and the scale slot back
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
         if constexpr (CG == 2) mbar_arrive_cluster(tempty_leader + 8 * buf);
         else mbar_arrive(bar_tempty + 8 * buf);
+        mbar_arrive(bar_sempty + 8 * buf);
       }
     }
+    // the staging buffers must outlive the bulk stores reading them
+    if (lane == 0) bulk_wait_all<0>();
+    __syncwarp();
   }
   __syncwarp();
   tc_fence_before();
@@ -362,6 +454,23 @@ static bool make_map_k_major(CUtensorMap* map, const void* base, int64_t rows, i
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Tensor map of the row-major [M, N] output (bf16 or binary32) for the
+// epilogue's TMA stores: box = 32 rows x 32 columns, swizzled like the
+// staging buffers (64-byte rows for bf16, 128-byte rows for binary32).
+static bool make_map_out(CUtensorMap* map, void* y, int64_t M, int64_t N, bool bf16) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t es = bf16 ? 2 : 4;
+  cuuint64_t dims[2] = {cuuint64_t(N), cuuint64_t(M)};
+  cuuint64_t strides[1] = {cuuint64_t(N) * es};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, y,
+             dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             bf16 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 static int device_sms() {
   static int n[64] = {0};
   int dev = 0;
@@ -379,10 +488,11 @@ template <int CG, int BN, int STAGES, bool E4M3, bool OUT_BF16, bool HAS_BIAS, b
 static cudaError_t run_gemm(const void* xq, const void* wq, const float* sx, const float* sw,
                             const uint16_t* bias, void* y, int32_t* acc, int M, int N, int K,
                             cudaStream_t st) {
-  using C = GemmCfg<CG, BN, STAGES>;
+  using C = GemmCfg<CG, BN, STAGES, OUT_BF16>;
   auto kern = gemm_w8a8_kernel<CG, BN, STAGES, E4M3, OUT_BF16, HAS_BIAS, WRITE_ACC>;
-  CUtensorMap ta, tb;
-  if (!make_map_k_major(&ta, xq, M, K, 128) || !make_map_k_major(&tb, wq, N, K, C::kBRows))
+  CUtensorMap ta, tb, ty;
+  if (!make_map_k_major(&ta, xq, M, K, 128) || !make_map_k_major(&tb, wq, N, K, C::kBRows) ||
+      !make_map_out(&ty, y, M, N, OUT_BF16))
     return cudaErrorInvalidValue;
   static uint64_t attr_set_mask = 0;  // one bit per device ordinal
   static int max_units[64] = {0};
@@ -434,7 +544,7 @@ static cudaError_t run_gemm(const void* xq, const void* wq, const float* sx, con
     cfg.numAttrs = 1;
   }
   int* status = status_ptr();
-  return cudaLaunchKernelEx(&cfg, kern, ta, tb, sx, sw, bias, y, acc, M, N, K, status);
+  return cudaLaunchKernelEx(&cfg, kern, ta, tb, ty, sx, sw, bias, acc, M, N, K, status);
 }
 
 template <int CG, int BN, int STAGES, bool E4M3>
@@ -464,14 +574,15 @@ enum class TileCfg { C1_N128, C1_N256, C2_N224, C2_N256 };
 
 static TileCfg choose_tile(int64_t M, int64_t N) {
   // Estimated time ~ (number of rounds of tiles over the SMs) x (work per
-  // tile); pick the cheapest, preferring SM pairs on ties (less operand
-  // traffic per MAC).
+  // tile) / (relative MAC throughput of the tile shape, measured on B200 at
+  // 4096 x 4096 x 14336: 256x256 pairs 1.0, 256x224 pairs 0.89, 128x256
+  // single CTAs 0.90, 128x128 single CTAs 0.62).
   const int sms = device_sms();
   struct Cand { TileCfg c; int cg, bm, bn; double eff; };
   const Cand cands[] = {{TileCfg::C2_N256, 2, 256, 256, 1.0},
-                        {TileCfg::C2_N224, 2, 256, 224, 1.0},
-                        {TileCfg::C1_N256, 1, 128, 256, 0.9},
-                        {TileCfg::C1_N128, 1, 128, 128, 0.8}};
+                        {TileCfg::C2_N224, 2, 256, 224, 0.89},
+                        {TileCfg::C1_N256, 1, 128, 256, 0.90},
+                        {TileCfg::C1_N128, 1, 128, 128, 0.62}};
   double best = 1e30;
   TileCfg pick = TileCfg::C1_N128;
   for (const Cand& c : cands) {
