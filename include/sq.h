@@ -34,17 +34,20 @@
  *    each function for the exact operation order).
  *  - The library allocates no device memory of its own except a 4-byte
  *    device status word and the 8-byte counter of sq_selftest_fast_division.
+ *    Scratch memory for the GEMMs is passed in by the caller (see
+ *    sq_gemm_workspace_bytes).
  */
 #ifndef SQ_H
 #define SQ_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
 extern "C" {
 #endif
 
-#define SQ_ABI_VERSION 2
+#define SQ_ABI_VERSION 3
 
 typedef enum {
     SQ_OK = 0,
@@ -159,6 +162,20 @@ sq_status sq_quantize_act(const void* x, sq_dtype xt, int64_t M, int64_t K,
                           void* xq, float* sx, void* stream);
 
 /*
+ * Size in bytes of the GEMM workspace for the current device (its SM count
+ * sets the size; the same workspace serves calls of every shape). The
+ * workspace lets the last, partial wave of output tiles be split along K
+ * across all SMs ("stream-K"): SMs that finish part of a tile leave its raw
+ * partial accumulators there, and the SM that owns the tile adds them (in a
+ * fixed order; exact for INT8) before the epilogue. Contract: 256-byte
+ * aligned, zero-filled by the caller before its first use (the GEMMs leave
+ * it zeroed again), not shared by GEMMs that may run concurrently, and
+ * re-zeroed by the caller after a call reported SQ_ERR_TIMEOUT. Passing NULL
+ * (or fewer bytes) is always valid and only disables the split.
+ */
+size_t sq_gemm_workspace_bytes(void);
+
+/*
  * a6 -- INT8 x INT8 tensor-core GEMM with int32 accumulation and a fused
  * dequantization epilogue. Source: §3 "Step 2" (Y = dequantize(X_int8 @
  * W_int8), "INT8 Tensor Core GEMM"); §1 table (INT8 x INT8 row).
@@ -166,6 +183,7 @@ sq_status sq_quantize_act(const void* x, sq_dtype xt, int64_t M, int64_t K,
  *   bias : [N] bf16 or NULL
  *   y  : [M,N], yt = SQ_BF16 or SQ_F32
  *   acc: [M,N] int32 accumulators or NULL (written when non-NULL)
+ *   workspace, workspace_bytes: see sq_gemm_workspace_bytes (NULL, 0 allowed)
  * acc[m,n] = sum_k xq[m,k]*wq[n,k] (exact in int32 for K < 133144);
  * t = float(acc) (nearest-even); t = t*sx[m]; t = t*sw[n]; t = t + bias[n];
  * y = t (SQ_F32) or bf16(t) rounded to nearest-even (SQ_BF16).
@@ -173,7 +191,8 @@ sq_status sq_quantize_act(const void* x, sq_dtype xt, int64_t M, int64_t K,
 sq_status sq_gemm_w8a8(const int8_t* xq, const float* sx, const int8_t* wq,
                        const float* sw, const uint16_t* bias, int64_t M,
                        int64_t N, int64_t K, void* y, sq_dtype yt,
-                       int32_t* acc, void* stream);
+                       int32_t* acc, void* workspace, size_t workspace_bytes,
+                       void* stream);
 
 /*
  * a7 -- FP8 E4M3 x E4M3 tensor-core GEMM, binary32 accumulation in tensor
@@ -185,7 +204,7 @@ sq_status sq_gemm_w8a8(const int8_t* xq, const float* sx, const int8_t* wq,
 sq_status sq_gemm_fp8(const uint8_t* xq, const float* sx, const uint8_t* wq,
                       const float* sw, const uint16_t* bias, int64_t M,
                       int64_t N, int64_t K, void* y, sq_dtype yt,
-                      void* stream);
+                      void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * Runtime forward of one SmoothQuant linear layer: sq_quantize_act followed
@@ -198,7 +217,7 @@ sq_status sq_linear(const void* x, sq_dtype xt, const float* s,
                     const float* s_inv, const void* wq, const float* sw, const uint16_t* bias,
                     sq_dtype qt, int64_t M, int64_t N, int64_t K,
                     void* xq_buf, float* sx_buf, void* y, sq_dtype yt,
-                    void* stream);
+                    void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * Self-test of the division shortcut used by sq_quantize_act for bf16 input

@@ -24,7 +24,7 @@ NUL = None
 def declared_symbols():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"^\s*(?:sq_status|const char\s*\*|int)\s+(sq_\w+)\s*\(",
+    return sorted(set(re.findall(r"^\s*(?:sq_status|const char\s*\*|int|size_t)\s+(sq_\w+)\s*\(",
                                  text, flags=re.M)))
 
 
@@ -53,7 +53,7 @@ def test_exported_symbols_are_visible_to_the_dynamic_linker():
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.sq_abi_version() == 2
+    assert lib.sq_abi_version() == 3
     for st in range(6):
         assert ops.status_string(st).startswith("SQ_")
     assert "TIMEOUT" in ops.status_string(ops.SQ_ERR_TIMEOUT)
@@ -90,12 +90,13 @@ def test_quantize_act_validation(lib):
 
 def test_gemm_validation(lib):
     f = lib.sq_gemm_w8a8
-    ok = dict(xq=A, sx=A, wq=A, sw=A, bias=None, M=16, N=64, K=64, y=A, yt=ops.SQ_BF16, acc=None)
+    ok = dict(xq=A, sx=A, wq=A, sw=A, bias=None, M=16, N=64, K=64, y=A, yt=ops.SQ_BF16, acc=None,
+              ws=None, wsn=0)
 
     def call(**kw):
         a = dict(ok, **kw)
         return f(c(a["xq"]), c(a["sx"]), c(a["wq"]), c(a["sw"]), c(a["bias"]), a["M"], a["N"],
-                 a["K"], c(a["y"]), a["yt"], c(a["acc"]), None)
+                 a["K"], c(a["y"]), a["yt"], c(a["acc"]), c(a["ws"]), a["wsn"], None)
 
     assert call(xq=NUL) == ops.SQ_ERR_INVALID_ARG
     assert call(wq=NUL) == ops.SQ_ERR_INVALID_ARG
@@ -110,10 +111,11 @@ def test_gemm_validation(lib):
     assert call(bias=A + 2) == ops.SQ_ERR_MISALIGNED
     assert call(sw=A + 4) == ops.SQ_ERR_MISALIGNED
     assert call(acc=A + 4) == ops.SQ_ERR_MISALIGNED
+    assert call(ws=A + 16, wsn=1 << 20) == ops.SQ_ERR_MISALIGNED
     assert call(M=0) == ops.SQ_OK
     g = lib.sq_gemm_fp8
-    assert g(c(A), c(A), c(A), c(A), None, 16, 64, 40, c(A), ops.SQ_BF16, None) == ops.SQ_ERR_INVALID_ARG
-    assert g(c(A), c(A), c(A), c(A), None, 0, 64, 64, c(A), ops.SQ_BF16, None) == ops.SQ_OK
+    assert g(c(A), c(A), c(A), c(A), None, 16, 64, 40, c(A), ops.SQ_BF16, None, 0, None) == ops.SQ_ERR_INVALID_ARG
+    assert g(c(A), c(A), c(A), c(A), None, 0, 64, 64, c(A), ops.SQ_BF16, None, 0, None) == ops.SQ_OK
 
 
 def test_smooth_factor_and_calibration_validation(lib):
@@ -137,7 +139,7 @@ def test_smooth_factor_and_calibration_validation(lib):
     assert qw(c(A), ops.SQ_BF16, 64, 64, None, ops.SQ_I8, c(A), c(A + 4), None) == ops.SQ_ERR_MISALIGNED
     lin = lib.sq_linear
     assert lin(c(A), ops.SQ_BF16, None, None, c(A), c(A), None, ops.SQ_I32, 4, 64, 64, c(A), c(A),
-               c(A), ops.SQ_BF16, None) == ops.SQ_ERR_INVALID_ARG
+               c(A), ops.SQ_BF16, None, 0, None) == ops.SQ_ERR_INVALID_ARG
     assert lin(c(A), ops.SQ_BF16, None, None, c(A), c(A), None, ops.SQ_I8, 0, 64, 64, c(A), c(A),
-               c(A), ops.SQ_BF16, None) == ops.SQ_OK
+               c(A), ops.SQ_BF16, None, 0, None) == ops.SQ_OK
     assert lib.sq_probe_wait_timeout(10, None) == ops.SQ_ERR_INVALID_ARG

@@ -159,11 +159,12 @@ def test_gemm_w8a8(M, N, K, with_bias):
     np.testing.assert_array_equal(host(yb), yb_ref)
 
 
+@pytest.mark.parametrize("split", [True, False])
 @pytest.mark.parametrize("tile", ops.GEMM_TILES)
 @pytest.mark.parametrize("M,N,K", [(300, 392, 4096), (129, 200, 96), (513, 520, 208),
                                    (1, 16, 32), (256, 448, 1024), (1100, 904, 272)])
 @pytest.mark.parametrize("qtype", ["i8", "e4m3"])
-def test_gemm_every_tile_shape(tile, M, N, K, qtype):
+def test_gemm_every_tile_shape(tile, M, N, K, qtype, split):
     """Every compiled tile shape (1-CTA and SM-pair) on ragged sizes."""
     g = np.random.default_rng(M + N + K)
     if qtype == "i8":
@@ -180,11 +181,11 @@ def test_gemm_every_tile_shape(tile, M, N, K, qtype):
     with ops.gemm_tile(tile):
         if qtype == "i8":
             acc = torch.empty((M, N), dtype=torch.int32, device="cuda")
-            yf = ops.gemm_w8a8(*d, bias=dev(bias), out_dtype=torch.float32, acc=acc)
-            yb = ops.gemm_w8a8(*d, bias=dev(bias))
+            yf = ops.gemm_w8a8(*d, bias=dev(bias), out_dtype=torch.float32, acc=acc, split=split)
+            yb = ops.gemm_w8a8(*d, bias=dev(bias), split=split)
         else:
-            yf = ops.gemm_fp8(*d, bias=dev(bias), out_dtype=torch.float32)
-            yb = ops.gemm_fp8(*d, bias=dev(bias))
+            yf = ops.gemm_fp8(*d, bias=dev(bias), out_dtype=torch.float32, split=split)
+            yb = ops.gemm_fp8(*d, bias=dev(bias), split=split)
     assert ops.device_status() == ops.SQ_OK
     if qtype == "i8":
         acc_ref = oracle.gemm_i8(xq, wq)
@@ -199,6 +200,26 @@ def test_gemm_every_tile_shape(tile, M, N, K, qtype):
                                  rows, cols)
         assert e.max() <= 1e-3, e.max()
         np.testing.assert_array_equal(host(yb), oracle.f32_to_bf16(host(yf)))
+
+
+def test_split_tiles_leave_workspace_clean_and_match_whole_tiles():
+    """Stream-K split tiles give the same bits as whole tiles (INT8 partial
+    sums are exact) and the workspace counters are zero again afterwards."""
+    M, N, K = 1000, 2056, 2048
+    xq = synth.random_matrix((M, K), np.int8, seed=41)
+    wq = synth.random_matrix((N, K), np.int8, seed=42)
+    sx = synth.random_floats(M, seed=43, lo=1e-3, hi=0.5)
+    sw = synth.random_floats(N, seed=44, lo=1e-4, hi=1e-2)
+    d = [dev(a) for a in (xq, sx, wq, sw)]
+    ref = oracle.epilogue(oracle.gemm_i8(xq, wq), sx, sw)[0]
+    for tile in ops.GEMM_TILES:
+        with ops.gemm_tile(tile):
+            for _ in range(3):
+                y = ops.gemm_w8a8(*d, out_dtype=torch.float32, split=True)
+                np.testing.assert_array_equal(host(y), ref)
+        assert ops.device_status() == ops.SQ_OK
+        counters = host(ops.workspace()[:4096])
+        assert not counters.any(), tile
 
 
 def test_gemm_w8a8_extreme_accumulators():

@@ -146,33 +146,38 @@ sq_status sq_quantize_act(const void* x, sq_dtype xt, int64_t M, int64_t K, cons
                                             S(stream)));
 }
 
+size_t sq_gemm_workspace_bytes(void) { return sqh::gemm_workspace_bytes(); }
+
 sq_status sq_gemm_w8a8(const int8_t* xq, const float* sx, const int8_t* wq, const float* sw,
                        const uint16_t* bias, int64_t M, int64_t N, int64_t K, void* y, sq_dtype yt,
-                       int32_t* acc, void* stream) {
+                       int32_t* acc, void* workspace, size_t workspace_bytes, void* stream) {
   sq_status c = check_gemm(xq, sx, wq, sw, bias, M, N, K, y, yt, acc);
   if (c != SQ_OK) return c;
   if (M == 0) return SQ_OK;
+  if (workspace && !al(workspace, 256)) return SQ_ERR_MISALIGNED;
   return from_cuda(sqh::launch_gemm(false, reinterpret_cast<const uint8_t*>(xq), sx,
                                     reinterpret_cast<const uint8_t*>(wq), sw, bias, M, N, K, y,
                                     yt == SQ_BF16 ? sqh::OutKind::BF16 : sqh::OutKind::F32, acc,
-                                    S(stream)));
+                                    workspace, workspace_bytes, S(stream)));
 }
 
 sq_status sq_gemm_fp8(const uint8_t* xq, const float* sx, const uint8_t* wq, const float* sw,
                       const uint16_t* bias, int64_t M, int64_t N, int64_t K, void* y, sq_dtype yt,
-                      void* stream) {
+                      void* workspace, size_t workspace_bytes, void* stream) {
   sq_status c = check_gemm(xq, sx, wq, sw, bias, M, N, K, y, yt, nullptr);
   if (c != SQ_OK) return c;
   if (M == 0) return SQ_OK;
+  if (workspace && !al(workspace, 256)) return SQ_ERR_MISALIGNED;
   return from_cuda(sqh::launch_gemm(true, xq, sx, wq, sw, bias, M, N, K, y,
                                     yt == SQ_BF16 ? sqh::OutKind::BF16 : sqh::OutKind::F32, nullptr,
-                                    S(stream)));
+                                    workspace, workspace_bytes, S(stream)));
 }
 
 sq_status sq_linear(const void* x, sq_dtype xt, const float* s, const float* s_inv,
                     const void* wq, const float* sw,
                     const uint16_t* bias, sq_dtype qt, int64_t M, int64_t N, int64_t K,
-                    void* xq_buf, float* sx_buf, void* y, sq_dtype yt, void* stream) {
+                    void* xq_buf, float* sx_buf, void* y, sq_dtype yt, void* workspace,
+                    size_t workspace_bytes, void* stream) {
   if (qt != SQ_I8 && qt != SQ_E4M3) return SQ_ERR_INVALID_ARG;
   sq_status c = check_gemm(xq_buf, sx_buf, wq, sw, bias, M, N, K, y, yt, nullptr);
   if (c != SQ_OK || M == 0) return c;
@@ -180,9 +185,9 @@ sq_status sq_linear(const void* x, sq_dtype xt, const float* s, const float* s_i
   if (c != SQ_OK) return c;
   if (qt == SQ_I8)
     return sq_gemm_w8a8(static_cast<const int8_t*>(xq_buf), sx_buf, static_cast<const int8_t*>(wq),
-                        sw, bias, M, N, K, y, yt, nullptr, stream);
+                        sw, bias, M, N, K, y, yt, nullptr, workspace, workspace_bytes, stream);
   return sq_gemm_fp8(static_cast<const uint8_t*>(xq_buf), sx_buf, static_cast<const uint8_t*>(wq),
-                     sw, bias, M, N, K, y, yt, stream);
+                     sw, bias, M, N, K, y, yt, workspace, workspace_bytes, stream);
 }
 
 sq_status sq_selftest_fast_division(int64_t* mismatches, void* stream) {

@@ -94,12 +94,75 @@ __device__ __forceinline__ void tile_coords(int tile, int num_mt, int num_nt, in
   nt = r / gm;
 }
 
+// ---------------------------------------------------------------------------
+// Work schedule (identical in every role of every CTA). With U units (CTAs,
+// or CTA pairs), the first dp_rounds rounds are whole tiles (tile = unit +
+// r*U). The remaining sk_tiles tiles form a "stream-K" region: their
+// sk_tiles * nk k-blocks are cut into U contiguous ranges, one per unit, so
+// the last partial wave is shared by every unit. A tile cut by range
+// boundaries is finished by the unit holding its k-block 0 (the "owner",
+// whose range ends there, so it waits last); the others ("contributors",
+// whose ranges start there, so they contribute first) leave their raw
+// accumulators in the caller's workspace. Nothing ever waits in a cycle.
+// ---------------------------------------------------------------------------
+struct WorkItem {
+  int tile;      // tile index in the raster order
+  int kb0, kb1;  // k-blocks [kb0, kb1)
+  int kind;      // 0 whole tile, 1 owner of a split tile, 2 contributor
+  int sk;        // index of the tile inside the stream-K region (kinds 1, 2)
+};
+
+struct Schedule {
+  int unit, U, nk, dp_limit, dp_tiles, sk_tiles;
+  int64_t S, it, it_end;
+  int next_dp;
+  __device__ void init(int unit_, int U_, int nk_, int num_tiles, int dp_rounds, int sk_tiles_) {
+    unit = unit_; U = U_; nk = nk_; sk_tiles = sk_tiles_;
+    dp_tiles = dp_rounds * U;
+    dp_limit = min(num_tiles, dp_tiles);
+    next_dp = unit;
+    S = int64_t(sk_tiles) * nk;
+    it = S ? int64_t(unit) * S / U : 0;
+    it_end = S ? int64_t(unit + 1) * S / U : 0;
+  }
+  __device__ bool next(WorkItem& w) {
+    if (next_dp < dp_limit) {
+      w.tile = next_dp; w.kb0 = 0; w.kb1 = nk; w.kind = 0; w.sk = -1;
+      next_dp += U;
+      return true;
+    }
+    if (it < it_end) {
+      const int64_t t = it / nk;
+      const int kb0 = int(it - t * nk);
+      const int64_t e = min((t + 1) * int64_t(nk), it_end);
+      w.tile = dp_tiles + int(t); w.kb0 = kb0; w.kb1 = int(e - t * nk); w.sk = int(t);
+      w.kind = (w.kb0 == 0 && w.kb1 == nk) ? 0 : (w.kb0 == 0 ? 1 : 2);
+      it = e;
+      return true;
+    }
+    return false;
+  }
+  // unit whose range holds stream-K iteration i
+  __device__ int unit_of(int64_t i) const { return int(((i + 1) * U - 1) / S); }
+  __device__ int contributors(int t) const {
+    return unit_of((int64_t(t) + 1) * nk - 1) - unit_of(int64_t(t) * nk);
+  }
+};
+
+// Workspace layout: arrived[kMaxSkTiles], done[kMaxSkTiles] (uint32), then
+// one partial-accumulator slot per CTA (128 rows x BN x 4 bytes). The
+// counters sit at fixed offsets so that calls of any shape can share one
+// workspace; every call leaves them zero.
+constexpr int kMaxSkTiles = 512;
+__host__ __device__ inline size_t ws_slot_offset(int) { return size_t(kMaxSkTiles) * 8; }
+
 template <int CG, int BN, int MAXST, bool E4M3, bool OUT_BF16, bool HAS_BIAS, bool WRITE_ACC>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                      const __grid_constant__ CUtensorMap tm_y, const float* __restrict__ sx,
                      const float* __restrict__ sw, const uint16_t* __restrict__ bias,
-                     int32_t* __restrict__ acc_out, int M, int N, int K, int* status) {
+                     int32_t* __restrict__ acc_out, int M, int N, int K, int dp_rounds,
+                     int sk_tiles, uint8_t* __restrict__ ws, int* status) {
   using C = GemmCfg<CG, BN, MAXST, OUT_BF16>;
   constexpr int STAGES = C::STAGES;
   extern __shared__ uint8_t smem_raw[];
@@ -166,10 +229,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       uint32_t it = 0, tc = 0;
       bool ok = true;
+      Schedule sch;
+      sch.init(unit, num_units, nk, num_tiles, dp_rounds, sk_tiles);
+      WorkItem wi;
 #pragma unroll 1
-      for (int tile = unit; tile < num_tiles && ok; tile += num_units, ++tc) {
+      for (; ok && sch.next(wi); ++tc) {
         int mt, nt;
-        tile_coords(tile, num_mt, num_nt, mt, nt);
+        tile_coords(wi.tile, num_mt, num_nt, mt, nt);
         const int a_row = mt * C::kTileM + int(rank) * 128;
         const int b_row = nt * BN + int(rank) * C::kBRows;
         {
@@ -190,7 +256,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if constexpr (HAS_BIAS) bulk_load(slot + BN * 4, bias + n0, b_bytes, bar_sfull + 8 * buf);
         }
 #pragma unroll 1
-        for (int kb = 0; kb < nk; ++kb, ++it) {
+        for (int kb = wi.kb0; kb < wi.kb1; ++kb, ++it) {
           const uint32_t st = it % STAGES, ph = (it / STAGES) & 1u;
           if (!mbar_wait(bar_empty + 8 * st, ph ^ 1u) || *abort_flag) {
             record_status(status, kStatusTimeout);
@@ -217,8 +283,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc = E4M3 ? idesc_e4m3_f32(C::kTileM, BN) : idesc_s8_s32(C::kTileM, BN);
       uint32_t it = 0, tc = 0;
       bool ok = true;
+      Schedule sch;
+      sch.init(unit, num_units, nk, num_tiles, dp_rounds, sk_tiles);
+      WorkItem wi;
 #pragma unroll 1
-      for (int tile = unit; tile < num_tiles && ok; tile += num_units, ++tc) {
+      for (; ok && sch.next(wi); ++tc) {
         const uint32_t buf = tc & 1u, use = tc >> 1;
         if (!mbar_wait(bar_tempty + 8 * buf, (use & 1u) ^ 1u)) {
           record_status(status, kStatusTimeout);
@@ -229,7 +298,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t d = tmem_base + buf * C::kAccStride;
 #pragma unroll 1
-        for (int kb = 0; kb < nk; ++kb, ++it) {
+        for (int kb = wi.kb0; kb < wi.kb1; ++kb, ++it) {
           const uint32_t st = it % STAGES, ph = (it / STAGES) & 1u;
           if (!mbar_wait(bar_full + 8 * st, ph)) {
             record_status(status, kStatusTimeout);
@@ -244,7 +313,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int kk = 0; kk < kBK / 32; ++kk) {
             const uint64_t ad = sw128_desc(a_addr + kk * 32);
             const uint64_t bd = sw128_desc(b_addr + kk * 32);
-            const uint32_t accum = (kb > 0 || kk > 0) ? 1u : 0u;
+            const uint32_t accum = (kb > wi.kb0 || kk > 0) ? 1u : 0u;
             if constexpr (CG == 2) {
               if constexpr (E4M3) mma_f8_pair(d, ad, bd, idesc, accum);
               else mma_i8_pair(d, ad, bd, idesc, accum);
@@ -284,8 +353,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tempty_leader = CG == 2 ? map_to_rank(bar_tempty, 0) : bar_tempty;
     uint32_t tc = 0;
     uint32_t emitted = 0;  // chunks this warp has handed to TMA stores
+    Schedule sch;
+    sch.init(unit, num_units, nk, num_tiles, dp_rounds, sk_tiles);
+    WorkItem wi;
+    uint32_t* arrived = reinterpret_cast<uint32_t*>(ws);
+    uint32_t* done = arrived + sk_tiles;
+    int32_t* slots = reinterpret_cast<int32_t*>(ws + ws_slot_offset(sk_tiles));
+    constexpr int kSlotWords = 128 * BN;
+    const int row_in_cta = sub * 32 + lane;
 #pragma unroll 1
-    for (int tile = unit; tile < num_tiles; tile += num_units, ++tc) {
+    for (; sch.next(wi); ++tc) {
       const uint32_t buf = tc & 1u, use = tc >> 1;
       if (!mbar_wait(bar_tfull + 8 * buf, use & 1u) || !mbar_wait(bar_sfull + 8 * buf, use & 1u) ||
           *abort_flag) {
@@ -295,7 +372,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       int mt, nt;
-      tile_coords(tile, num_mt, num_nt, mt, nt);
+      tile_coords(wi.tile, num_mt, num_nt, mt, nt);
       const int m = mt * C::kTileM + row_in_tile;
       const int n_base = nt * BN;
       const float sxm = m < M ? __ldg(sx + m) : 0.0f;
@@ -377,10 +454,62 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++emitted;
       };
 
+      // partial accumulators of a split tile: one slot per CTA, laid out
+      // [chunk][column][row] (raw int32 for INT8, binary32 bits for FP8) so
+      // that a warp's 32 rows of one column are one coalesced 128-byte line
+      auto slot_col = [&](int u, int chunk) {
+        return slots + size_t(u * CG + int(rank)) * kSlotWords + size_t(chunk) * 32 * 128 +
+               size_t(sub * 32 + lane);
+      };
+      int n_contrib = 0;
+      bool give_up = false;
+      if (wi.kind == 1) {
+        // owner: wait until every contributing warp has published its part
+        n_contrib = sch.contributors(wi.sk);
+        const uint32_t target = uint32_t(n_contrib * kEpiWarps * CG);
+        if (lane == 0) {
+          const uint64_t t0 = globaltimer_ns();
+          uint32_t polls = 0;
+          while (ld_acquire_gpu(arrived + wi.sk) < target) {
+            __nanosleep(128);
+            if ((++polls & 255u) == 0u && globaltimer_ns() - t0 > kWaitTimeoutNs) {
+              record_status(status, kStatusTimeout);
+              *abort_flag = 1;
+              break;
+            }
+          }
+          __threadfence();
+        }
+        __syncwarp();
+        give_up = *abort_flag != 0;
+      }
+      const int first_contrib = wi.kind == 1 ? sch.unit_of(int64_t(wi.sk) * nk) + 1 : 0;
+      // add the contributors' partial sums to this warp's accumulator chunk
+      auto add_partials = [&](uint32_t (&r)[32], int chunk) {
+        for (int cu = 0; cu < n_contrib; ++cu) {
+          const int32_t* src = slot_col(first_contrib + cu, chunk);
+          int32_t pw[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) pw[j] = __ldcg(src + j * 128);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            if constexpr (E4M3)
+              r[j] = __float_as_uint(__fadd_rn(__uint_as_float(r[j]), __int_as_float(pw[j])));
+            else
+              r[j] = uint32_t(int32_t(r[j]) + pw[j]);
+          }
+        }
+      };
+      auto publish = [&](const uint32_t (&r)[32], int chunk) {
+        int32_t* dst = slot_col(unit, chunk);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) __stcg(dst + j * 128, int32_t(r[j]));
+      };
+
       // this warp's chunks are half, half+WPQ, half+2*WPQ, ...; two loads in
       // flight at a time
 #pragma unroll 1
-      for (int c = half; c < NCH; c += 2 * WPQ) {
+      for (int c = half; c < NCH && !give_up; c += 2 * WPQ) {
         uint32_t r0[32], r1[32];
         const bool two = c + WPQ < NCH;  // warp-uniform
         tmem_ld32(t_addr + uint32_t(c * 32), r0);
@@ -390,8 +519,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
           tmem_wait_ld(r0);
         }
+        if (wi.kind == 2) {
+          publish(r0, c);
+          if (two) publish(r1, c + WPQ);
+          continue;
+        }
+        if (wi.kind == 1) {
+          add_partials(r0, c);
+          if (two) add_partials(r1, c + WPQ);
+        }
         emit(r0, c);
         if (two) emit(r1, c + WPQ);
+      }
+      if (wi.kind == 2) {
+        // contributor: make the slot visible, then count this warp in
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) atomicAdd(arrived + wi.sk, 1u);
+      } else if (wi.kind == 1 && !give_up) {
+        // owner: the last of its warps to finish resets the counters, so the
+        // workspace is clean for the next launch
+        __syncwarp();
+        if (lane == 0) {
+          if (atomicAdd(done + wi.sk, 1u) == uint32_t(kEpiWarps * CG - 1)) {
+            atomicExch(arrived + wi.sk, 0u);
+            atomicExch(done + wi.sk, 0u);
+          }
+        }
       }
       // hand the accumulator buffer and the scale slot back
       tc_fence_before();
@@ -484,10 +638,25 @@ static int device_sms() {
   return n[dev];
 }
 
+// Whole-tile rounds first; when the last round would leave units idle, the
+// last one or two rounds' worth of tiles become a stream-K region shared by
+// all units (needs a workspace).
+static void plan_schedule(int num_tiles, int units, bool can_split, int* dp_rounds, int* sk_tiles) {
+  const int full = num_tiles / units, rem = num_tiles % units;
+  const bool split = can_split && rem != 0 && (full == 0 || rem < units * 85 / 100);
+  if (!split) {
+    *dp_rounds = (num_tiles + units - 1) / units;
+    *sk_tiles = 0;
+    return;
+  }
+  *dp_rounds = full > 0 ? full - 1 : 0;
+  *sk_tiles = num_tiles - *dp_rounds * units;
+}
+
 template <int CG, int BN, int STAGES, bool E4M3, bool OUT_BF16, bool HAS_BIAS, bool WRITE_ACC>
 static cudaError_t run_gemm(const void* xq, const void* wq, const float* sx, const float* sw,
                             const uint16_t* bias, void* y, int32_t* acc, int M, int N, int K,
-                            cudaStream_t st) {
+                            void* ws, size_t ws_bytes, cudaStream_t st) {
   using C = GemmCfg<CG, BN, STAGES, OUT_BF16>;
   auto kern = gemm_w8a8_kernel<CG, BN, STAGES, E4M3, OUT_BF16, HAS_BIAS, WRITE_ACC>;
   CUtensorMap ta, tb, ty;
@@ -528,7 +697,19 @@ static cudaError_t run_gemm(const void* xq, const void* wq, const float* sx, con
   }
   const int units_max = dev < 64 ? max_units[dev] : device_sms() / CG;
   const int tiles = ((M + C::kTileM - 1) / C::kTileM) * ((N + BN - 1) / BN);
-  const int units = tiles < units_max ? tiles : units_max;
+  // stream-K needs every unit resident at once: units never exceeds what the
+  // occupancy query says fits. With a workspace every unit gets work even
+  // when there are fewer tiles than units.
+  const size_t need = ws_slot_offset(0) + size_t(units_max) * CG * 128 * BN * 4;
+  const bool can_split = ws != nullptr && ws_bytes >= need && !getenv("SQ_GEMM_NO_SPLIT");
+  int units = tiles < units_max ? tiles : units_max;
+  if (can_split && tiles > 0 && int64_t(tiles) * ((K + kBK - 1) / kBK) >= units_max) units = units_max;
+  int dp_rounds = 0, sk_tiles = 0;
+  plan_schedule(tiles, units, can_split, &dp_rounds, &sk_tiles);
+  if (sk_tiles > kMaxSkTiles) {
+    dp_rounds = (tiles + units - 1) / units;
+    sk_tiles = 0;
+  }
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attrs[1];
   cfg.gridDim = dim3(unsigned(units * CG));
@@ -544,17 +725,19 @@ static cudaError_t run_gemm(const void* xq, const void* wq, const float* sx, con
     cfg.numAttrs = 1;
   }
   int* status = status_ptr();
-  return cudaLaunchKernelEx(&cfg, kern, ta, tb, ty, sx, sw, bias, acc, M, N, K, status);
+  return cudaLaunchKernelEx(&cfg, kern, ta, tb, ty, sx, sw, bias, acc, M, N, K, dp_rounds,
+                            sk_tiles, static_cast<uint8_t*>(ws), status);
 }
 
 template <int CG, int BN, int STAGES, bool E4M3>
 static cudaError_t dispatch_epilogue(const void* xq, const void* wq, const float* sx,
                                      const float* sw, const uint16_t* bias, void* y, OutKind yk,
-                                     int32_t* acc, int M, int N, int K, cudaStream_t st) {
+                                     int32_t* acc, int M, int N, int K, void* ws, size_t ws_bytes,
+                                     cudaStream_t st) {
   const bool bf = yk == OutKind::BF16, hb = bias != nullptr, wa = acc != nullptr;
   const int key = (bf ? 4 : 0) | (hb ? 2 : 0) | (wa ? 1 : 0);
 #define SQ_RUN(B, H, W) \
-  run_gemm<CG, BN, STAGES, E4M3, B, H, W>(xq, wq, sx, sw, bias, y, acc, M, N, K, st)
+  run_gemm<CG, BN, STAGES, E4M3, B, H, W>(xq, wq, sx, sw, bias, y, acc, M, N, K, ws, ws_bytes, st)
   switch (key) {
     case 0: return SQ_RUN(false, false, false);
     case 1: return SQ_RUN(false, false, true);
@@ -572,7 +755,7 @@ static cudaError_t dispatch_epilogue(const void* xq, const void* wq, const float
 // pipeline depth.
 enum class TileCfg { C1_N128, C1_N256, C2_N224, C2_N256 };
 
-static TileCfg choose_tile(int64_t M, int64_t N) {
+static TileCfg choose_tile(int64_t M, int64_t N, bool can_split) {
   // Estimated time ~ (number of rounds of tiles over the SMs) x (work per
   // tile) / (relative MAC throughput of the tile shape, measured on B200 at
   // 4096 x 4096 x 14336: 256x256 pairs 1.0, 256x224 pairs 0.89, 128x256
@@ -588,8 +771,11 @@ static TileCfg choose_tile(int64_t M, int64_t N) {
   for (const Cand& c : cands) {
     const int64_t tiles = ((M + c.bm - 1) / c.bm) * ((N + c.bn - 1) / c.bn);
     const int64_t units = sms / c.cg;
-    const int64_t rounds = (tiles + units - 1) / units;
-    const double t = double(rounds) * double(c.bm) * double(c.bn) / (double(c.cg) * c.eff);
+    // with split tiles the last wave is shared (fractional rounds, plus a
+    // small cost for the partial sums); without, whole rounds
+    const double rounds = can_split ? double(tiles) / double(units) + (tiles % units ? 0.1 : 0.0)
+                                    : double((tiles + units - 1) / units);
+    const double t = rounds * double(c.bm) * double(c.bn) / (double(c.cg) * c.eff);
     if (t < best * 0.999) {
       best = t;
       pick = c.c;
@@ -611,15 +797,21 @@ static bool forced_tile(TileCfg* out) {
   return false;
 }
 
+size_t gemm_workspace_bytes() {
+  // the largest need of any tile shape: one 128 x 256 binary32 slot per SM
+  return ws_slot_offset(0) + size_t(device_sms()) * 128 * 256 * 4;
+}
+
 cudaError_t launch_gemm(bool e4m3, const uint8_t* xq, const float* sx, const uint8_t* wq,
                         const float* sw, const uint16_t* bias, int64_t M, int64_t N, int64_t K,
-                        void* y, OutKind yk, int32_t* acc, cudaStream_t st) {
+                        void* y, OutKind yk, int32_t* acc, void* ws, size_t ws_bytes,
+                        cudaStream_t st) {
   const int m = int(M), n = int(N), k = int(K);
   TileCfg c;
-  if (!forced_tile(&c)) c = choose_tile(M, N);
+  if (!forced_tile(&c)) c = choose_tile(M, N, ws != nullptr && ws_bytes >= gemm_workspace_bytes());
 #define SQ_CASE(CG, BN, S)                                                                     \
-  return e4m3 ? dispatch_epilogue<CG, BN, S, true>(xq, wq, sx, sw, bias, y, yk, acc, m, n, k, st) \
-              : dispatch_epilogue<CG, BN, S, false>(xq, wq, sx, sw, bias, y, yk, acc, m, n, k, st)
+  return e4m3 ? dispatch_epilogue<CG, BN, S, true>(xq, wq, sx, sw, bias, y, yk, acc, m, n, k, ws, ws_bytes, st) \
+              : dispatch_epilogue<CG, BN, S, false>(xq, wq, sx, sw, bias, y, yk, acc, m, n, k, ws, ws_bytes, st)
   switch (c) {
     case TileCfg::C2_N256: SQ_CASE(2, 256, 6);
     case TileCfg::C2_N224: SQ_CASE(2, 224, 7);

@@ -30,7 +30,9 @@ cudaError_t launch_selftest_fast_division(unsigned long long* mismatches, cudaSt
 enum class OutKind { BF16, F32 };
 cudaError_t launch_gemm(bool e4m3, const uint8_t* xq, const float* sx, const uint8_t* wq,
                         const float* sw, const uint16_t* bias, int64_t M, int64_t N, int64_t K,
-                        void* y, OutKind yk, int32_t* acc, cudaStream_t st);
+                        void* y, OutKind yk, int32_t* acc, void* ws, size_t ws_bytes,
+                        cudaStream_t st);
+size_t gemm_workspace_bytes();
 
 
 }  // namespace sqh

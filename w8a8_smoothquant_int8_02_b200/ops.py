@@ -26,6 +26,7 @@ EXPORTED = (
     "sq_status_string", "sq_abi_version", "sq_get_device_status", "sq_calibrate_amax",
     "sq_smooth_factors", "sq_quantize_weight", "sq_quantize_act", "sq_gemm_w8a8",
     "sq_gemm_fp8", "sq_linear", "sq_probe_wait_timeout", "sq_selftest_fast_division",
+    "sq_gemm_workspace_bytes",
 )
 
 _lock = threading.Lock()
@@ -62,13 +63,16 @@ def load(build_if_needed: bool = True) -> ctypes.CDLL:
             lib.sq_smooth_factors.argtypes = [P, P, I64, D, P, P, P]
             lib.sq_quantize_weight.argtypes = [P, I, I64, I64, P, I, P, P, P]
             lib.sq_quantize_act.argtypes = [P, I, I64, I64, P, P, I, P, P, P]
-            lib.sq_gemm_w8a8.argtypes = [P, P, P, P, P, I64, I64, I64, P, I, P, P]
-            lib.sq_gemm_fp8.argtypes = [P, P, P, P, P, I64, I64, I64, P, I, P]
-            lib.sq_linear.argtypes = [P, I, P, P, P, P, P, I, I64, I64, I64, P, P, P, I, P]
+            SZ = ctypes.c_size_t
+            lib.sq_gemm_w8a8.argtypes = [P, P, P, P, P, I64, I64, I64, P, I, P, P, SZ, P]
+            lib.sq_gemm_fp8.argtypes = [P, P, P, P, P, I64, I64, I64, P, I, P, SZ, P]
+            lib.sq_linear.argtypes = [P, I, P, P, P, P, P, I, I64, I64, I64, P, P, P, I, P, SZ, P]
+            lib.sq_gemm_workspace_bytes.argtypes = []
+            lib.sq_gemm_workspace_bytes.restype = SZ
             lib.sq_probe_wait_timeout.argtypes = [I64, P]
             lib.sq_selftest_fast_division.argtypes = [ctypes.POINTER(ctypes.c_int64), P]
             for name in EXPORTED:
-                if name not in ("sq_status_string", "sq_abi_version"):
+                if name not in ("sq_status_string", "sq_abi_version", "sq_gemm_workspace_bytes"):
                     getattr(lib, name).restype = I
             _lib = lib
     return _lib
@@ -176,19 +180,51 @@ def quantize_act(x: torch.Tensor, s: torch.Tensor | None, qtype: str = "i8", xq=
     return xq, sx
 
 
-def gemm_w8a8(xq, sx, wq, sw, bias=None, out_dtype=torch.bfloat16, out=None, acc=None):
-    """a6: INT8 tensor-core GEMM + dequant epilogue. Returns y (and fills acc if given)."""
+_workspaces: dict = {}
+
+
+def workspace(device=None) -> torch.Tensor:
+    """The per-device GEMM workspace (zero-filled once; the GEMMs keep it
+    zeroed). Calls on one device share it, so they must not run
+    concurrently on different streams."""
+    dev = torch.device("cuda", torch.cuda.current_device() if device is None else
+                       torch.device(device).index or 0)
+    ws = _workspaces.get(dev)
+    if ws is None:
+        with torch.cuda.device(dev):
+            n = int(load().sq_gemm_workspace_bytes())
+        ws = torch.zeros(n, dtype=torch.uint8, device=dev)
+        _workspaces[dev] = ws
+    return ws
+
+
+def _ws_args(use_split, device):
+    """(pointer, bytes) of the workspace, or (None, 0) to run without split tiles."""
+    if not use_split:
+        return None, 0
+    ws = workspace(device)
+    return _p(ws), ws.numel()
+
+
+def gemm_w8a8(xq, sx, wq, sw, bias=None, out_dtype=torch.bfloat16, out=None, acc=None,
+              split=False):
+    """a6: INT8 tensor-core GEMM + dequant epilogue. Returns y (and fills acc if given).
+    split=True passes the workspace so the last partial wave of tiles may be
+    split along K over all SMs (same results; opt-in: on B200 it has not yet
+    beaten whole tiles on the measured shapes)."""
     _cuda(xq, sx, wq, sw, bias, out, acc)
     M, K = xq.shape
     N = wq.shape[0]
     if out is None:
         out = torch.empty((M, N), dtype=out_dtype, device=xq.device)
+    wsp, wsn = _ws_args(split, xq.device)
     _check(load().sq_gemm_w8a8(_p(xq), _p(sx), _p(wq), _p(sw), _p(bias), M, N, K, _p(out),
-                               _fdtype(out), _p(acc), _stream(xq.device)), "sq_gemm_w8a8")
+                               _fdtype(out), _p(acc), wsp, wsn, _stream(xq.device)),
+           "sq_gemm_w8a8")
     return out
 
 
-def gemm_fp8(xq, sx, wq, sw, bias=None, out_dtype=torch.bfloat16, out=None):
+def gemm_fp8(xq, sx, wq, sw, bias=None, out_dtype=torch.bfloat16, out=None, split=False):
     """a7: FP8 E4M3 tensor-core GEMM + dequant epilogue."""
     xq, wq = _codes(xq), _codes(wq)
     _cuda(xq, sx, wq, sw, bias, out)
@@ -196,13 +232,14 @@ def gemm_fp8(xq, sx, wq, sw, bias=None, out_dtype=torch.bfloat16, out=None):
     N = wq.shape[0]
     if out is None:
         out = torch.empty((M, N), dtype=out_dtype, device=xq.device)
+    wsp, wsn = _ws_args(split, xq.device)
     _check(load().sq_gemm_fp8(_p(xq), _p(sx), _p(wq), _p(sw), _p(bias), M, N, K, _p(out),
-                              _fdtype(out), _stream(xq.device)), "sq_gemm_fp8")
+                              _fdtype(out), wsp, wsn, _stream(xq.device)), "sq_gemm_fp8")
     return out
 
 
 def linear(x, s, wq, sw, bias=None, qtype="i8", out_dtype=torch.bfloat16, out=None,
-           xq_buf=None, sx_buf=None, s_inv=None):
+           xq_buf=None, sx_buf=None, s_inv=None, split=False):
     """Runtime forward: quantize_act then the 8-bit GEMM, one C call."""
     wq = _codes(wq)
     _cuda(x, s, wq, sw, bias, out, xq_buf, sx_buf, s_inv)
@@ -216,16 +253,24 @@ def linear(x, s, wq, sw, bias=None, qtype="i8", out_dtype=torch.bfloat16, out=No
         sx_buf = torch.empty(M, dtype=torch.float32, device=x.device)
     if out is None:
         out = torch.empty((M, N), dtype=out_dtype, device=x.device)
+    wsp, wsn = _ws_args(split, x.device)
     _check(load().sq_linear(_p(x), _fdtype(x), _p(s), _p(s_inv), _p(wq), _p(sw), _p(bias), qt,
-                            M, N, K,
-                            _p(xq_buf), _p(sx_buf), _p(out), _fdtype(out), _stream(x.device)),
+                            M, N, K, _p(xq_buf), _p(sx_buf), _p(out), _fdtype(out), wsp, wsn,
+                            _stream(x.device)),
            "sq_linear")
     return out
 
 
 def device_status(device=None) -> int:
-    """Synchronize the current stream and return (and clear) the status word."""
-    return int(load().sq_get_device_status(_stream(device)))
+    """Synchronize the current stream and return (and clear) the status word.
+    After a timeout the GEMM workspace may hold partial counters: it is
+    zero-filled again here, as its contract requires."""
+    st = int(load().sq_get_device_status(_stream(device)))
+    if st == SQ_ERR_TIMEOUT:
+        for ws in _workspaces.values():
+            ws.zero_()
+        torch.cuda.synchronize()
+    return st
 
 
 def selftest_fast_division(device=None) -> int:
