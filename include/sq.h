@@ -55,7 +55,8 @@ typedef enum {
     SQ_ERR_MISALIGNED = 2,   /* pointer or leading dimension misaligned       */
     SQ_ERR_UNSUPPORTED = 3,  /* valid but not implemented combination         */
     SQ_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed           */
-    SQ_ERR_TIMEOUT = 5       /* a bounded device-side wait gave up             */
+    SQ_ERR_TIMEOUT = 5,      /* a bounded device-side wait gave up             */
+    SQ_ERR_SCRATCH_TOO_SMALL = 6  /* sq_gemm_w8a8_noalloc: fixed scratch too small */
 } sq_status;
 
 typedef enum {
@@ -218,6 +219,37 @@ sq_status sq_linear(const void* x, sq_dtype xt, const float* s,
                     sq_dtype qt, int64_t M, int64_t N, int64_t K,
                     void* xq_buf, float* sx_buf, void* y, sq_dtype yt,
                     void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Allocation-free variant of sq_gemm_w8a8 (no counterpart in the pages: it
+ * exists for callers, not for the method). Some callers cannot allocate
+ * device memory while they run -- for example an inference runtime that
+ * reserves all device memory up front for its own pool, so a foreign
+ * cudaMalloc would fail or fragment it, or latency-critical code that cannot
+ * afford the device-wide synchronization cudaMalloc / cudaFree may imply --
+ * and so cannot provide the workspace the split-tile GEMM needs. This entry
+ * point takes the same inputs and outputs as sq_gemm_w8a8 (without acc and
+ * without a workspace) and uses a fixed 20 MiB array inside the library's
+ * device image as its scratch instead. It calls no cudaMalloc / cudaFree or
+ * other allocating routine.
+ *  - Limit: the scratch this call needs (see sq_gemm_workspace_bytes; it
+ *    depends on the GPU's SM count, not on M, N, K) must fit 20 MiB,
+ *    otherwise SQ_ERR_SCRATCH_TOO_SMALL and nothing is launched. Every GPU
+ *    that loads the library holds the 20 MiB array until the process exits.
+ *  - Set-up: the first call on each device looks up the array's device
+ *    address (cudaGetSymbolAddress) with that device current; make that first
+ *    call before any stream capture.
+ *  - Every call shares the one array, which keeps the last call's contents;
+ *    each call first clears the part that must start at zero (an async
+ *    memset on `stream`). Calls that overlap on the GPU (different streams,
+ *    or the same device from several host threads without ordering) race on
+ *    the array and may produce wrong results.
+ * Results are identical to sq_gemm_w8a8 with a workspace (INT8 sums exact).
+ */
+sq_status sq_gemm_w8a8_noalloc(const int8_t* xq, const float* sx,
+                               const int8_t* wq, const float* sw,
+                               const uint16_t* bias, int64_t M, int64_t N,
+                               int64_t K, void* y, sq_dtype yt, void* stream);
 
 /*
  * Self-test of the division shortcut used by sq_quantize_act for bf16 input

@@ -65,6 +65,32 @@ sq_status check_gemm(const void* xq, const float* sx, const void* wq, const floa
   return SQ_OK;
 }
 
+// ---------------------------------------------------------------------------
+// Scratch of the allocation-free GEMM entry point (sq_gemm_w8a8_noalloc):
+// a fixed array in the library's own device image, so the call allocates
+// nothing. 20 MiB holds the split-tile workspace of every tile shape on a GPU
+// with up to 160 SMs (4 KiB of counters + one 128 x 256 x 4-byte slot per SM).
+// Every GPU that loads the library keeps this array until the process exits.
+// ---------------------------------------------------------------------------
+constexpr size_t kNoAllocScratchBytes = size_t(20) << 20;
+static __device__ __align__(256) unsigned char g_sq_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of the array for the current device. Host code must not use
+// the array's name as a pointer (it is a host-side stand-in); the runtime
+// gives the device address, looked up once per device and cached.
+void* noalloc_scratch_ptr() {
+  static void* ptrs[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_sq_noalloc_scratch) != cudaSuccess || p == nullptr)
+      return nullptr;
+    ptrs[dev] = p;
+  }
+  return ptrs[dev];
+}
+
 }  // namespace
 
 extern "C" {
@@ -77,6 +103,9 @@ const char* sq_status_string(sq_status st) {
     case SQ_ERR_UNSUPPORTED: return "SQ_ERR_UNSUPPORTED: unsupported combination";
     case SQ_ERR_CUDA: return "SQ_ERR_CUDA: CUDA runtime error";
     case SQ_ERR_TIMEOUT: return "SQ_ERR_TIMEOUT: a bounded device wait gave up";
+    case SQ_ERR_SCRATCH_TOO_SMALL:
+      return "SQ_ERR_SCRATCH_TOO_SMALL: this call needs more scratch than the fixed 20 MiB array "
+             "of the allocation-free entry point";
   }
   return "SQ_ERR_UNKNOWN";
 }
@@ -188,6 +217,26 @@ sq_status sq_linear(const void* x, sq_dtype xt, const float* s, const float* s_i
                         sw, bias, M, N, K, y, yt, nullptr, workspace, workspace_bytes, stream);
   return sq_gemm_fp8(static_cast<const uint8_t*>(xq_buf), sx_buf, static_cast<const uint8_t*>(wq),
                      sw, bias, M, N, K, y, yt, workspace, workspace_bytes, stream);
+}
+
+sq_status sq_gemm_w8a8_noalloc(const int8_t* xq, const float* sx, const int8_t* wq,
+                               const float* sw, const uint16_t* bias, int64_t M, int64_t N,
+                               int64_t K, void* y, sq_dtype yt, void* stream) {
+  sq_status c = check_gemm(xq, sx, wq, sw, bias, M, N, K, y, yt, nullptr);
+  if (c != SQ_OK) return c;
+  if (M == 0) return SQ_OK;
+  // the split-tile scratch this device needs must fit the fixed array
+  if (sqh::gemm_workspace_bytes() > kNoAllocScratchBytes) return SQ_ERR_SCRATCH_TOO_SMALL;
+  void* scratch = noalloc_scratch_ptr();
+  if (!scratch) return SQ_ERR_CUDA;
+  // the array keeps the previous call's contents: the counters the split
+  // tiles synchronize on must start at zero
+  if (cudaMemsetAsync(scratch, 0, sqh::gemm_workspace_counter_bytes(), S(stream)) != cudaSuccess)
+    return SQ_ERR_CUDA;
+  return from_cuda(sqh::launch_gemm(false, reinterpret_cast<const uint8_t*>(xq), sx,
+                                    reinterpret_cast<const uint8_t*>(wq), sw, bias, M, N, K, y,
+                                    yt == SQ_BF16 ? sqh::OutKind::BF16 : sqh::OutKind::F32, nullptr,
+                                    scratch, kNoAllocScratchBytes, S(stream)));
 }
 
 sq_status sq_selftest_fast_division(int64_t* mismatches, void* stream) {

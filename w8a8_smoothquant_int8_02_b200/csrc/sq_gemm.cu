@@ -797,6 +797,8 @@ static bool forced_tile(TileCfg* out) {
   return false;
 }
 
+size_t gemm_workspace_counter_bytes() { return ws_slot_offset(0); }
+
 size_t gemm_workspace_bytes() {
   // the largest need of any tile shape: one 128 x 256 binary32 slot per SM
   return ws_slot_offset(0) + size_t(device_sms()) * 128 * 256 * 4;

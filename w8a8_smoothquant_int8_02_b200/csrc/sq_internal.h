@@ -33,6 +33,7 @@ cudaError_t launch_gemm(bool e4m3, const uint8_t* xq, const float* sx, const uin
                         void* y, OutKind yk, int32_t* acc, void* ws, size_t ws_bytes,
                         cudaStream_t st);
 size_t gemm_workspace_bytes();
+size_t gemm_workspace_counter_bytes();
 
 
 }  // namespace sqh

@@ -18,7 +18,8 @@ import torch
 
 from . import build as _build
 
-SQ_OK, SQ_ERR_INVALID_ARG, SQ_ERR_MISALIGNED, SQ_ERR_UNSUPPORTED, SQ_ERR_CUDA, SQ_ERR_TIMEOUT = range(6)
+(SQ_OK, SQ_ERR_INVALID_ARG, SQ_ERR_MISALIGNED, SQ_ERR_UNSUPPORTED, SQ_ERR_CUDA, SQ_ERR_TIMEOUT,
+ SQ_ERR_SCRATCH_TOO_SMALL) = range(7)
 SQ_F32, SQ_BF16, SQ_I8, SQ_E4M3, SQ_I32 = range(5)
 SQ_AMAX_PER_COLUMN, SQ_AMAX_PER_ROW = 0, 1
 
@@ -26,7 +27,7 @@ EXPORTED = (
     "sq_status_string", "sq_abi_version", "sq_get_device_status", "sq_calibrate_amax",
     "sq_smooth_factors", "sq_quantize_weight", "sq_quantize_act", "sq_gemm_w8a8",
     "sq_gemm_fp8", "sq_linear", "sq_probe_wait_timeout", "sq_selftest_fast_division",
-    "sq_gemm_workspace_bytes",
+    "sq_gemm_workspace_bytes", "sq_gemm_w8a8_noalloc",
 )
 
 _lock = threading.Lock()
@@ -67,6 +68,7 @@ def load(build_if_needed: bool = True) -> ctypes.CDLL:
             lib.sq_gemm_w8a8.argtypes = [P, P, P, P, P, I64, I64, I64, P, I, P, P, SZ, P]
             lib.sq_gemm_fp8.argtypes = [P, P, P, P, P, I64, I64, I64, P, I, P, SZ, P]
             lib.sq_linear.argtypes = [P, I, P, P, P, P, P, I, I64, I64, I64, P, P, P, I, P, SZ, P]
+            lib.sq_gemm_w8a8_noalloc.argtypes = [P, P, P, P, P, I64, I64, I64, P, I, P]
             lib.sq_gemm_workspace_bytes.argtypes = []
             lib.sq_gemm_workspace_bytes.restype = SZ
             lib.sq_probe_wait_timeout.argtypes = [I64, P]
@@ -221,6 +223,20 @@ def gemm_w8a8(xq, sx, wq, sw, bias=None, out_dtype=torch.bfloat16, out=None, acc
     _check(load().sq_gemm_w8a8(_p(xq), _p(sx), _p(wq), _p(sw), _p(bias), M, N, K, _p(out),
                                _fdtype(out), _p(acc), wsp, wsn, _stream(xq.device)),
            "sq_gemm_w8a8")
+    return out
+
+
+def gemm_w8a8_noalloc(xq, sx, wq, sw, bias=None, out_dtype=torch.bfloat16, out=None):
+    """sq_gemm_w8a8_noalloc: the INT8 GEMM with the library's fixed scratch array
+    instead of a caller workspace (allocates nothing itself; `out` may be given)."""
+    _cuda(xq, sx, wq, sw, bias, out)
+    M, K = xq.shape
+    N = wq.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=xq.device)
+    _check(load().sq_gemm_w8a8_noalloc(_p(xq), _p(sx), _p(wq), _p(sw), _p(bias), M, N, K,
+                                       _p(out), _fdtype(out), _stream(xq.device)),
+           "sq_gemm_w8a8_noalloc")
     return out
 
 
