@@ -252,13 +252,17 @@ sq_status sq_gemm_w8a8_noalloc(const int8_t* xq, const float* sx,
                                int64_t K, void* y, sq_dtype yt, void* stream);
 
 /*
- * Self-test of the division shortcut used by sq_quantize_act for bf16 input
- * (an IEEE division x / s_k computed as a reciprocal product corrected with
- * one fused multiply-add residual, after Markstein): runs every bf16
- * significand of x against every binary32 significand of s (2^30 pairs, both
- * signs) and counts results that differ from the IEEE division. Synchronous
- * (waits for `stream`). *mismatches receives the count; 0 means the shortcut
- * is exact wherever sq_quantize_act uses it.
+ * Self-test of the division shortcuts used by sq_quantize_act for bf16 input
+ * (an IEEE division computed as a reciprocal product corrected with one
+ * fused multiply-add residual, after Markstein): runs every bf16 significand
+ * of x against every binary32 significand of s_k (2^30 pairs, both signs),
+ * every binary32 significand of a row maximum divided by 127 and by 448 with
+ * their constant reciprocals, and checks that the refined approximate
+ * reciprocal of every binary32 significand is within one unit in the last
+ * place of the IEEE reciprocal. Synchronous (waits for `stream`).
+ * *mismatches receives the number of failures; 0 means the shortcuts are
+ * exact (or, for the reciprocal, within its bound) wherever sq_quantize_act
+ * uses them.
  */
 sq_status sq_selftest_fast_division(int64_t* mismatches, void* stream);
 

@@ -351,6 +351,46 @@ def test_quantize_act_fast_path_edge_values(qtype):
         np.testing.assert_array_equal(host(xq).view(np.uint8), xq_ref.view(np.uint8))
 
 
+@pytest.mark.parametrize("qtype", ["i8", "e4m3"])
+@pytest.mark.parametrize("K", [64, 208, 4096, 4112, 14336, 16384])
+def test_quantize_act_streaming_rows_edge_values(qtype, K):
+    """Many bf16 rows (the persistent streaming kernel): ordinary rows mixed
+    with rows that leave its fast window (all zeros, all -0, tiny, huge,
+    subnormal) and rows whose elements are zeros of both signs, tiny values
+    or exact ties after smoothing; once with every smoothing factor inside
+    the fast-division window, once with some outside it, once unsmoothed."""
+    M = 700
+    g = np.random.default_rng(K)
+    x = (g.standard_normal((M, K)) * 3).astype(np.float32)
+    x[5] = 0.0
+    x[6] = -0.0
+    x[7] *= 1e-25                      # amax below the fast window
+    x[8] *= 1e28                       # amax above it; no quotient overflows,
+    x[8, 20] = 3e31                    # inputs must keep every x/s finite
+    x[8, 40] = 1e28
+    x[9] = 1e-40                       # subnormal bf16 everywhere
+    x[10, :8] = [0.0, -0.0, 1e-30, -1e-30, 1e-40, -1e-40, 2.0 ** -100, -(2.0 ** -90)]
+    x[11, ::3] = -0.0
+    x[12, :6] = [127.0, 63.5, -0.5, 1.5, 2.5, -126.5]   # ties when s_k = 1
+    x[13:20] = np.round(x[13:20] * 2) / 2                # many half-integers
+    x[20, -1] = 300.0                                    # amax in the last chunk
+    s_in = synth.random_floats(K, seed=K + 3, lo=0.05, hi=20.0)
+    s_in[:6] = 1.0
+    s_in[6:14] = 2.0 ** g.integers(-3, 4, 8).astype(np.float32)
+    # row 12: |x/s| <= ~50 beyond its first six elements, so its amax is 127
+    x[12, 6:] = np.clip(x[12, 6:], -1, 1) * s_in[6:] * 50
+    s_out = s_in.copy()
+    s_out[min(K - 1, 40)] = 2.0 ** -30                   # outside [2^-20, 2^20]
+    xb = synth.to_bf16_bits(x)
+    qt = oracle.E4M3 if qtype == "e4m3" else oracle.INT8
+    for smooth in (s_in, s_out, None):
+        xq_ref, sx_ref = oracle.quantize_act(xb, smooth, qt)
+        xq, sx = ops.quantize_act(dev(xb), None if smooth is None else dev(smooth), qtype)
+        assert ops.device_status() == ops.SQ_OK
+        np.testing.assert_array_equal(host(sx), sx_ref)
+        np.testing.assert_array_equal(host(xq).view(np.uint8), xq_ref.view(np.uint8))
+
+
 # ---------------------------------------------------------- failure path --
 
 def test_bounded_wait_reports_timeout_and_context_survives():
