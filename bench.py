@@ -57,6 +57,45 @@ def rotate_count(case):
     return max(2, -(-int(1.5 * L2_BYTES) // per_set))
 
 
+# DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from
+# one ncu --set full capture of bench.py's own command per workload (the
+# summaries under profiles/), keyed by the sha256 prefix of the kernel's
+# sources at capture time: a kernel changed since reports null.
+PROFILED_TRAFFIC = {
+    ("gemm", "mlp_up_4096x4096x14336"): (75.747328e6 + 82.522624e6, "0d5df644efe1da65"),
+    ("gemm", "fp8_down_4096x14336x4096"): (277.747200e6 + 26.476800e6, "0d5df644efe1da65"),
+    ("quant", "mlp_up_4096x4096x14336"): (33.638144e6 + 0.004608e6, "853c5e0f3819537d"),
+    ("quant", "fp8_down_4096x14336x4096"): (117.617664e6 + 30.590720e6, "853c5e0f3819537d"),
+}
+KERNEL_SOURCES = {"gemm": ("sq_gemm.cu", "sq_common.cuh"), "quant": ("sq_quant.cu", "sq_common.cuh")}
+
+
+def profiled_traffic(kind, workload):
+    """Bytes per launch from the capture, or None if there is none for this
+    workload or the kernel's sources changed since (or a tile is forced)."""
+    import hashlib
+    entry = PROFILED_TRAFFIC.get((kind, workload))
+    if entry is None or (kind == "gemm" and os.environ.get("SQ_GEMM_TILE")):
+        return None
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES[kind]:
+        with open(os.path.join(ROOT, "w8a8_smoothquant_int8_02_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return entry[0] if h.hexdigest()[:16] == entry[1] else None
+
+
+def quant_kernel_name(case):
+    """The activation kernel sq_quantize_act launches for this workload: for
+    bf16 input the persistent streaming form when there are many rows, one
+    CTA per row otherwise; the generic kernel for fp32 input."""
+    sms = 148
+    if case.x_dtype != "bf16" or case.K // 8 > 256 * 8:
+        return "quant_act_kernel"
+    if case.K // 8 <= 2048 and case.M >= 2 * sms:
+        return "quant_act_stream_kernel"
+    return "quant_act_fast_kernel"
+
+
 def _peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -349,10 +388,12 @@ def run_ours(args):
                          "frac_of_sustained": gemm_tops / int8_peak_sus,
                          "ops_note": "INT8 multiply-add counted as 2 ops; peak = 2 x measured "
                                      "bf16 dense (burst)",
-                         "traffic": None, "ms_per_launch": t_gemm},
-            "roofline_quant": {"bound": "hbm", "kernel": "quant_act_kernel",
+                         "traffic": profiled_traffic("gemm", case.name),
+                         "ms_per_launch": t_gemm},
+            "roofline_quant": {"bound": "hbm", "kernel": quant_kernel_name(case),
                                "achieved": q_bytes / (t_quant * 1e-3) / 1e9, "peak": pk["hbm"],
                                "unit": "GB/s", "frac": q_bytes / (t_quant * 1e-3) / 1e9 / pk["hbm"],
+                               "traffic": profiled_traffic("quant", case.name),
                                "ms_per_launch": t_quant},
             "gpu_launches": 2 * K_steps,  # quant_act_stream_kernel + gemm_w8a8_kernel per step
             "clocks": clocks,
