@@ -23,6 +23,11 @@
  *    synchronously on the host and launch nothing when they fail; a failed
  *    launch returns SQ_ERR_CUDA. A device-side wait that gives up (see
  *    sq_get_device_status) is reported through the device status word.
+ *    The many-row activation kernel and the GEMMs are launched with
+ *    programmatic dependent launch: each may be scheduled while the kernel
+ *    before it in the stream finishes, and waits for that kernel to
+ *    complete before touching global memory, so stream order is kept
+ *    (set the environment variable SQ_PDL=0 to launch them plainly).
  *  - K must be a positive multiple of 16 (16-byte rows of 8-bit data for the
  *    tensor-memory-accelerator copies); N a positive multiple of 8 (16-byte
  *    rows of bf16 output). M may be any value >= 0; M == 0 is a no-op that
@@ -33,8 +38,9 @@
  *    reproducible bit for bit against a plain CPU implementation (see
  *    each function for the exact operation order).
  *  - The library allocates no device memory of its own except a 4-byte
- *    device status word and the 8-byte counter of sq_selftest_fast_division.
- *    Scratch memory for the GEMMs is passed in by the caller (see
+ *    device status word, the 8-byte counter of sq_selftest_fast_division and
+ *    the fixed scratch array of sq_gemm_w8a8_noalloc (module data). Scratch
+ *    memory for the other GEMM calls is passed in by the caller (see
  *    sq_gemm_workspace_bytes).
  */
 #ifndef SQ_H

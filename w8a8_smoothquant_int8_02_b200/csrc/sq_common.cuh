@@ -79,6 +79,20 @@ __device__ __forceinline__ float max3_nan(float a, float b, float c) {
   return r;
 }
 
+// ------------------------------------------- programmatic dependent launch --
+// A kernel launched with the programmatic-stream-serialization attribute may
+// start while the kernel before it in the stream is still running (once every
+// CTA of that kernel has called pdl_launch_dependents, or exited). It must
+// call pdl_wait -- which returns when the earlier kernel has completed and its
+// memory is visible -- before it reads or writes any global memory that kernel
+// may touch; work before the wait (barrier set-up, tensor-memory allocation)
+// overlaps the earlier kernel's tail.
+
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ----------------------------------------------------------- shared mem --
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

@@ -217,6 +217,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   if constexpr (CG == 2) cluster_sync_all(); else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // the next kernel waits for this grid to complete before touching memory;
+  // everything above overlapped the previous kernel's tail, everything below
+  // reads its results
+  pdl_launch_dependents();
+  pdl_wait();
 
   const int num_mt = (M + C::kTileM - 1) / C::kTileM;
   const int num_nt = (N + BN - 1) / BN;
@@ -711,19 +716,28 @@ static cudaError_t run_gemm(const void* xq, const void* wq, const float* sx, con
     sk_tiles = 0;
   }
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attrs[1];
+  cudaLaunchAttribute attrs[2];
   cfg.gridDim = dim3(unsigned(units * CG));
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = C::kDynamic;
   cfg.stream = st;
+  unsigned na = 0;
   if (CG == 2) {
-    attrs[0].id = cudaLaunchAttributeClusterDimension;
-    attrs[0].val.clusterDim.x = 2;
-    attrs[0].val.clusterDim.y = 1;
-    attrs[0].val.clusterDim.z = 1;
-    cfg.attrs = attrs;
-    cfg.numAttrs = 1;
+    attrs[na].id = cudaLaunchAttributeClusterDimension;
+    attrs[na].val.clusterDim.x = 2;
+    attrs[na].val.clusterDim.y = 1;
+    attrs[na].val.clusterDim.z = 1;
+    ++na;
   }
+  if (pdl_enabled()) {
+    // may start while the kernel before it (normally the activation
+    // quantization) finishes; the kernel waits before touching memory
+    attrs[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attrs[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  cfg.attrs = attrs;
+  cfg.numAttrs = na;
   int* status = status_ptr();
   return cudaLaunchKernelEx(&cfg, kern, ta, tb, ty, sx, sw, bias, acc, M, N, K, dp_rounds,
                             sk_tiles, static_cast<uint8_t*>(ws), status);

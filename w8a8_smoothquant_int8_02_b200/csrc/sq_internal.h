@@ -35,5 +35,27 @@ cudaError_t launch_gemm(bool e4m3, const uint8_t* xq, const float* sx, const uin
 size_t gemm_workspace_bytes();
 size_t gemm_workspace_counter_bytes();
 
+// Programmatic dependent launch of the streaming kernels (on unless the
+// environment sets SQ_PDL=0): such a launch may start while the previous
+// kernel in the stream finishes; the kernels wait (griddepcontrol.wait)
+// before touching global memory.
+bool pdl_enabled();
+
+template <typename... Params, typename... Args>
+cudaError_t launch_pdl(void (*kern)(Params...), unsigned grid, int threads, size_t smem,
+                       cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(unsigned(threads), 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 
 }  // namespace sqh
