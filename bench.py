@@ -62,10 +62,10 @@ def rotate_count(case):
 # summaries under profiles/), keyed by the sha256 prefix of the kernel's
 # sources at capture time: a kernel changed since reports null.
 PROFILED_TRAFFIC = {
-    ("gemm", "mlp_up_4096x4096x14336"): (75.747328e6 + 82.522624e6, "0d5df644efe1da65"),
-    ("gemm", "fp8_down_4096x14336x4096"): (277.747200e6 + 26.476800e6, "0d5df644efe1da65"),
-    ("quant", "mlp_up_4096x4096x14336"): (33.638144e6 + 0.004608e6, "853c5e0f3819537d"),
-    ("quant", "fp8_down_4096x14336x4096"): (117.617664e6 + 30.590720e6, "853c5e0f3819537d"),
+    ("gemm", "mlp_up_4096x4096x14336"): (75.928576e6 + 82.759680e6, "0d224357d8151d98"),
+    ("gemm", "fp8_down_4096x14336x4096"): (273.935360e6 + 28.075776e6, "0d224357d8151d98"),
+    ("quant", "mlp_up_4096x4096x14336"): (33.648128e6 + 0.008704e6, "616d402bb78b8727"),
+    ("quant", "fp8_down_4096x14336x4096"): (117.738240e6 + 29.602048e6, "616d402bb78b8727"),
 }
 KERNEL_SOURCES = {"gemm": ("sq_gemm.cu", "sq_common.cuh"), "quant": ("sq_quant.cu", "sq_common.cuh")}
 
