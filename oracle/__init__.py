@@ -68,6 +68,7 @@ def _load():
             lib.sqo_smooth_weight.argtypes = [P, I, I64, I64, P, P]
             lib.sqo_quantize_weight.argtypes = [P, I, I64, I64, P, I, P, P]
             lib.sqo_quantize_act.argtypes = [P, I, I64, I64, P, I, P, P]
+            lib.sqo_quantize_act_tensor.argtypes = [P, I, I64, I64, P, I, P, P, P, P]
             lib.sqo_gemm_i8.argtypes = [P, P, I64, I64, I64, P]
             lib.sqo_gemm_e4m3.argtypes = [P, P, I64, I64, I64, P]
             lib.sqo_dequant.argtypes = [ctypes.c_float, ctypes.c_float,
@@ -201,6 +202,23 @@ def quantize_act(x: np.ndarray, s, qtype: int = INT8):
     _load().sqo_quantize_act(_ptr(x), _dtype_code(x), M, K, _ptr(s), qtype,
                              _ptr(xq), _ptr(sx))
     return xq, sx
+
+
+def quantize_act_tensor(x: np.ndarray, s, qtype: int = INT8, scale=None):
+    """Per-tensor scaling: one scale for the whole (smoothed) tensor, the
+    online max|x/s|/Q when `scale` is None, else the given (delayed) scale.
+    Returns (xq [M,K] codes, scale used as float32, amax = max|x/s|)."""
+    x = np.ascontiguousarray(x)
+    M, K = x.shape
+    s = None if s is None else _c(s, np.float32)
+    sc = None if scale is None else np.array([scale], np.float32)
+    xq = np.empty((M, K), np.uint8 if qtype == E4M3 else np.int8)
+    sx = np.empty(max(M, 1), np.float32)
+    amax = np.zeros(1, np.float32)
+    _load().sqo_quantize_act_tensor(_ptr(x), _dtype_code(x), M, K, _ptr(s), qtype, _ptr(sc),
+                                    _ptr(xq), _ptr(sx), _ptr(amax))
+    used = np.float32(scale) if scale is not None else (sx[0] if M else np.float32(0))
+    return xq, np.float32(used), np.float32(amax[0])
 
 
 def gemm_i8(xq, wq) -> np.ndarray:

@@ -285,6 +285,41 @@ void sqo_quantize_act(const void* x, int dtype, int64_t M, int64_t K,
 /* ------------------------------------------------------------------------ */
 
 /* |acc| <= K * 127 * 127, which stays below 2^31 for K < 133144. */
+/* Per-tensor scaling of the (smoothed) activations, [WAQ] §4: one scale for
+ * the whole tensor, q = cast(x/s / scale). Online: scale = max|x/s| / Q over
+ * the tensor. Delayed: the given scale (the previous step's max / Q); values
+ * beyond it saturate (INT8 clamps to +-127, E4M3 to +-448). A zero scale
+ * gives all-zero codes, as for a zero row in per-token scaling. */
+void sqo_quantize_act_tensor(const void* x, int dtype, int64_t M, int64_t K,
+                             const float* s, int qtype, const float* scale_in,
+                             void* xq, float* sx, float* amax_out) {
+    const float qmax = (qtype == 1) ? 448.0f : 127.0f;
+    float amax = 0.0f;
+    for (int64_t i = 0; i < M * K; ++i) {
+        float v = load_elem(x, dtype, i);
+        float xs = s ? smooth_x(v, s[i % K]) : v;
+        float a = fabsf(xs);
+        if (a > amax) amax = a;
+    }
+    *amax_out = amax;
+    const float scale = scale_in ? *scale_in : amax / qmax;
+    #pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m) {
+        sx[m] = scale;
+        for (int64_t k = 0; k < K; ++k) {
+            float v = load_elem(x, dtype, m * K + k);
+            float xs = s ? smooth_x(v, s[k]) : v;
+            if (qtype == 1) {
+                ((uint8_t*)xq)[m * K + k] =
+                    (scale == 0.0f) ? 0 : sqo_e4m3_encode_rn_sat(xs / scale);
+            } else {
+                ((int8_t*)xq)[m * K + k] =
+                    (scale == 0.0f) ? 0 : quant_i8(xs, scale);
+            }
+        }
+    }
+}
+
 void sqo_gemm_i8(const int8_t* xq, const int8_t* wq, int64_t M, int64_t N,
                  int64_t K, int32_t* acc) {
     #pragma omp parallel for schedule(static)

@@ -64,6 +64,16 @@ void sqo_quantize_weight(const void* w, int dtype, int64_t K, int64_t N,
 void sqo_quantize_act(const void* x, int dtype, int64_t M, int64_t K,
                       const float* s, int qtype, void* xq, float* sx);
 
+/* Per-tensor activation scaling ([WAQ] §4 "Per-Tensor Scaling for FP8" and
+ * "FP8 vs INT8 SmoothQuant": per-tensor scaling online, or delayed scaling
+ * from the previous step's max). x: [M,K] (dtype), s: [K] or NULL.
+ * scale_in: the scale to use (delayed scaling), or NULL for the online scale
+ * max|x/s| / Q of this tensor. xq: [M,K] codes; sx: [M] each set to the scale
+ * used; *amax_out: max|x/s| over the whole tensor (the next step's max). */
+void sqo_quantize_act_tensor(const void* x, int dtype, int64_t M, int64_t K,
+                             const float* s, int qtype, const float* scale_in,
+                             void* xq, float* sx, float* amax_out);
+
 /* a6 INT8 x INT8 -> int32 accumulators, acc[m][n] = sum_k xq[m][k]*wq[n][k]. */
 void sqo_gemm_i8(const int8_t* xq, const int8_t* wq, int64_t M, int64_t N,
                  int64_t K, int32_t* acc);

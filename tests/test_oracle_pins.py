@@ -441,3 +441,77 @@ def test_smoothing_reduces_quantization_error_on_outlier_data():
     e_smooth, e_plain = err(s), err(None)
     assert e_smooth < 0.5 * e_plain, (e_smooth, e_plain)
     assert e_smooth < 0.05
+
+
+# ---------------------------------------------------------------------------
+# §4 per-tensor scaling (online, and delayed from the previous step's max).
+# ---------------------------------------------------------------------------
+
+def test_per_tensor_example_spans_tokens():
+    """The §2 row split into two tokens: one per-tensor scale (80/127) for
+    both, so 75 maps to 119 as on the page, where a per-token scale for the
+    second token (75/127) would give it the full 127."""
+    fx = _fixture("per_tensor_scale.txt")
+    row = np.array(fx["row"], np.float32)
+    x = row.reshape(2, 4)
+    xq, scale, amax = oracle.quantize_act_tensor(x, None, oracle.INT8)
+    assert abs(float(scale) - float(fx["scale_approx"][0])) <= \
+        float(fx["scale_rel_tol"][0]) * float(fx["scale_approx"][0])
+    assert amax == np.float32(80.0)
+    np.testing.assert_array_equal(xq.reshape(-1), np.array(fx["codes"], np.int8))
+    per_token, _ = oracle.quantize_act(x, None)
+    assert per_token[1, 1] == 127 and xq[1, 1] == 119
+
+
+@pytest.mark.parametrize("qt", [oracle.INT8, oracle.E4M3])
+def test_per_tensor_one_token_is_per_token(qt):
+    """With a single token the tensor is the row: online per-tensor scaling
+    must equal the (separately pinned) per-token quantization."""
+    g = np.random.default_rng(5)
+    x = (g.standard_normal((1, 96)) * 4).astype(np.float32)
+    s = synth.random_floats(96, seed=6, lo=0.1, hi=10.0)
+    xq_t, scale, amax = oracle.quantize_act_tensor(x, s, qt)
+    xq_r, sx = oracle.quantize_act(x, s, qt)
+    np.testing.assert_array_equal(xq_t, xq_r)
+    assert scale == sx[0]
+    assert amax == np.abs((x / s).astype(np.float32)).max()
+
+
+@pytest.mark.parametrize("qt", [oracle.INT8, oracle.E4M3])
+def test_per_tensor_brute_force(qt):
+    """Element by element in numpy binary32: codes of x/s/scale under the
+    given (delayed) scale, saturating, and the tensor's max |x/s|."""
+    g = np.random.default_rng(7)
+    x = (g.standard_normal((5, 24)) * 3).astype(np.float32)
+    x[2, 3] = 40.0                                     # beyond the delayed scale
+    x[4, 0] = -40.0
+    s = synth.random_floats(24, seed=8, lo=0.5, hi=2.0)
+    s[3] = 1.0
+    s[0] = 1.0
+    scale = np.float32(0.05)                           # Q * scale = 6.35 (INT8), 22.4 (E4M3)
+    xq, used, amax = oracle.quantize_act_tensor(x, s, qt, scale=scale)
+    assert used == scale
+    xs = (x / s).astype(np.float32)
+    assert amax == np.abs(xs).max()
+    for (m, k), v in np.ndenumerate(xs):
+        q = np.float32(v / scale)
+        if qt == oracle.INT8:
+            want = np.int8(min(max(np.rint(q), -127), 127))
+            assert xq[m, k] == want, (m, k)
+        else:
+            assert xq[m, k] == oracle.e4m3_encode(q), (m, k)
+    if qt == oracle.INT8:
+        assert xq[2, 3] == 127 and xq[4, 0] == -127
+    else:
+        assert xq[2, 3] == 0x7E and xq[4, 0] == 0xFE   # +-448: satfinite
+
+
+def test_per_tensor_delayed_with_own_max_is_online_and_zero_scale():
+    g = np.random.default_rng(9)
+    x = (g.standard_normal((6, 32)) * 2).astype(np.float32)
+    xq_o, scale_o, amax = oracle.quantize_act_tensor(x, None, oracle.E4M3)
+    assert scale_o == np.float32(amax / np.float32(448.0))
+    xq_d, _, _ = oracle.quantize_act_tensor(x, None, oracle.E4M3, scale=scale_o)
+    np.testing.assert_array_equal(xq_o, xq_d)
+    xq_z, _, amax_z = oracle.quantize_act_tensor(x, None, oracle.INT8, scale=np.float32(0.0))
+    assert not xq_z.any() and amax_z == amax
