@@ -43,6 +43,9 @@ L2_BYTES = 126 * 2 ** 20
 def metric_for(case):
     if case.name.startswith("mlp_up"):
         return METRIC
+    if case.act_scaling == "tensor":
+        return (f"W8A8 per-tensor FP8 quant+GEMM TOPS and % of FP8 TC peak at "
+                f"M{case.M} K{case.K} N{case.N}")
     kind = "FP8" if case.qtype == "e4m3" else "INT8"
     return (f"W8A8 smooth+quant+GEMM TOPS and % of {kind} TC peak at "
             f"M{case.M} K{case.K} N{case.N}")
@@ -89,6 +92,8 @@ def quant_kernel_name(case):
     bf16 input the persistent streaming form when there are many rows, one
     CTA per row otherwise; the generic kernel for fp32 input."""
     sms = 148
+    if case.act_scaling == "tensor":
+        return "quant_act_tensor_kernel"
     if case.x_dtype != "bf16" or case.K // 8 > 256 * 8:
         return "quant_act_kernel"
     if case.K // 8 <= 2048 and case.M >= 2 * sms:
@@ -207,24 +212,51 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def _oracle_prep(case, d):
+    """The oracle's offline preparation for a workload: (s or None, wq, sw,
+    per-tensor scale or None)."""
+    import oracle
+    qt = oracle.E4M3 if case.qtype == "e4m3" else oracle.INT8
+    s = None
+    if case.smooth:
+        s = oracle.smooth_factors(oracle.amax(d["x_cal"], True), oracle.amax(d["w"], False),
+                                  case.alpha)
+    wq, sw = oracle.quantize_weight(d["w"], s, qt)
+    scale = None
+    if case.act_scaling == "tensor":
+        _, scale, _ = oracle.quantize_act_tensor(d["x_cal"], s, qt)
+    return s, wq, sw, scale
+
+
+def _oracle_runtime(case, xs, s, wq, sw, bias, scale):
+    """The oracle's runtime path on token rows xs: activation quantization,
+    8-bit GEMM, epilogue."""
+    import oracle
+    qt = oracle.E4M3 if case.qtype == "e4m3" else oracle.INT8
+    if scale is None:
+        return oracle.linear(xs, s, wq, sw, bias, qt)
+    xq, sc, _ = oracle.quantize_act_tensor(xs, s, qt, scale=scale)
+    acc = oracle.gemm_e4m3(xq, wq) if qt == oracle.E4M3 else oracle.gemm_i8(xq, wq)
+    sx = np.full(xs.shape[0], sc, np.float32)
+    return oracle.epilogue(acc, sx, sw, bias)
+
+
 def cpu_baseline(case, d, budget_s: float):
     """Oracle throughput on a bounded sample of the workload (rank 0, N=1 only).
     The oracle prepares its own weights (untimed), then runs the runtime path
     (activation quant + 8-bit GEMM + epilogue) on as many token rows as fit
     in about `budget_s` seconds."""
     import oracle
-    qt = oracle.E4M3 if case.qtype == "e4m3" else oracle.INT8
-    s = oracle.smooth_factors(oracle.amax(d["x_cal"], True), oracle.amax(d["w"], False), case.alpha)
-    wq, sw = oracle.quantize_weight(d["w"], s, qt)
+    s, wq, sw, scale = _oracle_prep(case, d)
     rows = 2
     xs = np.ascontiguousarray(d["x"][:rows])
     t0 = time.perf_counter()
-    oracle.linear(xs, s, wq, sw, d["bias"], qt)
+    _oracle_runtime(case, xs, s, wq, sw, d["bias"], scale)
     dt = time.perf_counter() - t0
     rows2 = int(max(2, min(case.M, rows * budget_s / max(dt, 1e-3))))
     xs = np.ascontiguousarray(d["x"][:rows2])
     t0 = time.perf_counter()
-    oracle.linear(xs, s, wq, sw, d["bias"], qt)
+    _oracle_runtime(case, xs, s, wq, sw, d["bias"], scale)
     dt = time.perf_counter() - t0
     return {"value": 2.0 * rows2 * case.N * case.K / dt / 1e12, "unit": UNIT,
             "cores": oracle.num_threads(), "kind": "oracle",
@@ -262,8 +294,18 @@ def run_ours(args):
 
     # ---- offline preparation (untimed) ----
     w = to_dev(d["w"])
-    p = ops.prepare(w, to_dev(d["x_cal"]), alpha=case.alpha, qtype=qt)
-    s, s_inv, wq0, sw = p["s"], p["s_inv"], p["wq"], p["sw"]
+    if case.smooth:
+        p = ops.prepare(w, to_dev(d["x_cal"]), alpha=case.alpha, qtype=qt)
+        s, s_inv, wq0, sw = p["s"], p["s_inv"], p["wq"], p["sw"]
+    else:
+        s = s_inv = None
+        wq0, sw = ops.quantize_weight(w, None, qt)
+    tensor = case.act_scaling == "tensor"
+    # per-tensor (delayed) scaling: step i reads the max written by step i-1;
+    # the first step's comes from the calibration tokens
+    amax_b = torch.zeros(2, dtype=torch.float32, device=dev)
+    if tensor:
+        ops.quantize_act_tensor(to_dev(d["x_cal"]), s, qt, amax_out=amax_b[0:1], s_inv=s_inv)
     bias = to_dev(d["bias"]) if d["bias"] is not None else None
     gemm = ops.gemm_w8a8 if qt == "i8" else ops.gemm_fp8
     del w
@@ -277,10 +319,17 @@ def run_ours(args):
     y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream()
 
-    def step(i):
+    def quantize(i):
         r = i % ROTATE
-        ops.quantize_act(xs[r], s, qt, xq=xq, sx=sx, s_inv=s_inv)
-        gemm(xq, sx, wqs[r], sw, bias, out=y)
+        if tensor:
+            ops.quantize_act_tensor(xs[r], s, qt, amax_prev=amax_b[i % 2:i % 2 + 1], xq=xq, sx=sx,
+                                    amax_out=amax_b[(i + 1) % 2:(i + 1) % 2 + 1], s_inv=s_inv)
+        else:
+            ops.quantize_act(xs[r], s, qt, xq=xq, sx=sx, s_inv=s_inv)
+
+    def step(i):
+        quantize(i)
+        gemm(xq, sx, wqs[i % ROTATE], sw, bias, out=y)
 
     for i in range(max(3, args.warmup)):
         step(i)
@@ -296,7 +345,7 @@ def run_ours(args):
     for i in range(A_steps):
         r = i % ROTATE
         ev[i][0].record(stream)
-        ops.quantize_act(xs[r], s, qt, xq=xq, sx=sx, s_inv=s_inv)
+        quantize(i)
         ev[i][1].record(stream)
         gemm(xq, sx, wqs[r], sw, bias, out=y)
         ev[i][2].record(stream)
@@ -342,7 +391,12 @@ def run_ours(args):
 
         def e2e_step():
             x_dev.copy_(x_host, non_blocking=True)
-            ops.linear(x_dev, s, wq0, sw, bias, qt, out=y, xq_buf=xq, sx_buf=sx, s_inv=s_inv)
+            if tensor:
+                ops.quantize_act_tensor(x_dev, s, qt, amax_prev=amax_b[0:1], xq=xq, sx=sx,
+                                        amax_out=amax_b[1:2], s_inv=s_inv)
+                gemm(xq, sx, wq0, sw, bias, out=y)
+            else:
+                ops.linear(x_dev, s, wq0, sw, bias, qt, out=y, xq_buf=xq, sx_buf=sx, s_inv=s_inv)
             y_host.copy_(y, non_blocking=True)
 
         for _ in range(3):
@@ -372,7 +426,8 @@ def run_ours(args):
         int8_peak_sus = 2.0 * pk["bf16_sus"]
         gemm_tops = case.ops / (t_gemm * 1e-3) / 1e12
         value = ws * case.ops * K_steps / (elapsed_ms * 1e-3) / 1e12
-        q_bytes = M * K * 2 + M * K + M * 4 + K * 4   # read X (bf16) + s, write Xq + sx
+        # read X (bf16) + s, write Xq + sx (per-tensor: + the scale, + the max)
+        q_bytes = M * K * 2 + M * K + M * 4 + (K * 4 if case.smooth else 0)
         g_bytes = M * K + N * K + M * N * 2 + 4 * (M + N) + (2 * N if bias is not None else 0)
         line = {
             "metric": metric_for(case), "value": value, "unit": UNIT, "n_gpus": ws,
@@ -381,7 +436,9 @@ def run_ours(args):
             "dtype": "i8" if qt == "i8" else "e4m3",
             "data": "synthetic (seeded N(0,1) activations with 1% outlier channels x U(20,100), "
                     "N(0,0.02) weights)",
-            "config": {"workload": case.name, "M": M, "K": K, "N": N, "alpha": case.alpha,
+            "config": {"workload": case.name, "M": M, "K": K, "N": N,
+                       "alpha": case.alpha if case.smooth else None,
+                       "act_scaling": ("per-tensor, delayed" if tensor else "per-token"),
                        "bias": bias is not None, "out": "bf16",
                        "l2": (f"{ROTATE} rotating input sets (X + Wq, "
                               f"{ROTATE * (M * K * 2 + N * K) / 2 ** 20:.0f} MiB) > 126 MiB L2"),

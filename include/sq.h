@@ -53,7 +53,7 @@
 extern "C" {
 #endif
 
-#define SQ_ABI_VERSION 3
+#define SQ_ABI_VERSION 4
 
 typedef enum {
     SQ_OK = 0,
@@ -167,6 +167,32 @@ sq_status sq_quantize_weight(const void* w, sq_dtype wt, int64_t K, int64_t N,
 sq_status sq_quantize_act(const void* x, sq_dtype xt, int64_t M, int64_t K,
                           const float* s, const float* s_inv, sq_dtype qt,
                           void* xq, float* sx, void* stream);
+
+/*
+ * Activation smoothing + PER-TENSOR quantization: one scale for the whole
+ * smoothed tensor instead of one per token. Source: "Weight-Activation
+ * Quantization" (infra.bea.ai) §4 "Per-Tensor Scaling for FP8" (q =
+ * cast_fp8(x/s), s = max|x|/448) and its comparison table (per-tensor scaling
+ * online; "delayed scaling uses previous step's max"). The pages have no API
+ * for it; this entry point is this library's.
+ *   x, xt, M, K, s, s_inv, qt, xq : as sq_quantize_act.
+ *   amax_prev : device float[1] holding the previous step's max|x/s|
+ *               (delayed scaling, one pass over x), or NULL for the online
+ *               scale of this tensor (two passes: its max, then the codes).
+ *               The scale is RN(amax / Q), Q = 127 (INT8) or 448 (E4M3).
+ *   sx        : [M], every entry receives the scale used, so the GEMMs take
+ *               it as they take per-token scales.
+ *   amax_out  : device float[1], required, 4-byte aligned, not aliasing
+ *               amax_prev: receives max|x/s| of this tensor (NaN ignored) --
+ *               the next step's amax_prev. M == 0 sets it to 0.
+ * Codes: INT8 clamp(rne(xs / scale), -127, 127), E4M3 round-to-nearest-even
+ * saturating to +-448 (values beyond a delayed scale saturate); a zero scale
+ * gives all-zero codes. Bit-exact against the IEEE definitions.
+ */
+sq_status sq_quantize_act_tensor(const void* x, sq_dtype xt, int64_t M, int64_t K,
+                                 const float* s, const float* s_inv, sq_dtype qt,
+                                 const float* amax_prev, void* xq, float* sx,
+                                 float* amax_out, void* stream);
 
 /*
  * Size in bytes of the GEMM workspace for the current device (its SM count

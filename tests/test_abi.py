@@ -53,7 +53,7 @@ def test_exported_symbols_are_visible_to_the_dynamic_linker():
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.sq_abi_version() == 3
+    assert lib.sq_abi_version() == 4
     for st in range(7):
         assert ops.status_string(st).startswith("SQ_")
     assert "TIMEOUT" in ops.status_string(ops.SQ_ERR_TIMEOUT)
@@ -86,6 +86,31 @@ def test_quantize_act_validation(lib):
     assert call(s=A + 4) == ops.SQ_ERR_MISALIGNED
     assert call(s_inv=A + 4) == ops.SQ_ERR_MISALIGNED
     assert call(M=0) == ops.SQ_OK                      # empty input: no-op
+
+
+def test_quantize_act_tensor_validation(lib):
+    f = lib.sq_quantize_act_tensor
+    ok = dict(x=A, xt=ops.SQ_BF16, M=4, K=64, s=A, qt=ops.SQ_E4M3, prev=A + 64, xq=A, sx=A,
+              out=A + 128)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return f(c(a["x"]), a["xt"], a["M"], a["K"], c(a["s"]), c(a.get("s_inv")), a["qt"],
+                 c(a["prev"]), c(a["xq"]), c(a["sx"]), c(a["out"]), None)
+
+    assert call(out=NUL) == ops.SQ_ERR_INVALID_ARG     # the tensor max is required
+    assert call(out=A + 64) == ops.SQ_ERR_INVALID_ARG  # aliases amax_prev
+    assert call(x=NUL) == ops.SQ_ERR_INVALID_ARG
+    assert call(xq=NUL) == ops.SQ_ERR_INVALID_ARG
+    assert call(sx=NUL) == ops.SQ_ERR_INVALID_ARG
+    assert call(K=24) == ops.SQ_ERR_INVALID_ARG
+    assert call(M=-1) == ops.SQ_ERR_INVALID_ARG
+    assert call(xt=ops.SQ_E4M3) == ops.SQ_ERR_INVALID_ARG
+    assert call(qt=ops.SQ_F32) == ops.SQ_ERR_INVALID_ARG
+    assert call(out=A + 130) == ops.SQ_ERR_MISALIGNED
+    assert call(prev=A + 66) == ops.SQ_ERR_MISALIGNED
+    assert call(x=MIS) == ops.SQ_ERR_MISALIGNED
+    assert call(s=A + 4) == ops.SQ_ERR_MISALIGNED
 
 
 def test_gemm_validation(lib):

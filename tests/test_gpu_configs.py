@@ -1,4 +1,4 @@
-"""The five workloads at full size, in the launch configuration bench.py
+"""The workloads at full size, in the launch configuration bench.py
 times (tile shape chosen by problem size), against the CPU oracle.
 
 Per workload: calibration amaxes bit-exact, smoothing factors within 2 ulp,
@@ -34,24 +34,41 @@ def test_workload_end_to_end(name):
     M, K, N = case.M, case.K, case.N
 
     # ---- offline preparation ----
-    ax = oracle.amax(x_cal, True)
-    aw = oracle.amax(w, False)
-    s = oracle.smooth_factors(ax, aw, case.alpha)
     w_d = dev(w)
-    p = ops.prepare(w_d, dev(x_cal), alpha=case.alpha, qtype=case.qtype)
-    np.testing.assert_array_equal(host(p["amax_x"]), ax)
-    np.testing.assert_array_equal(host(p["amax_w"]), aw)
-    assert ulp_distance(host(p["s"]), s).max() <= 2
+    s = None
+    if case.smooth:
+        ax = oracle.amax(x_cal, True)
+        aw = oracle.amax(w, False)
+        s = oracle.smooth_factors(ax, aw, case.alpha)
+        p = ops.prepare(w_d, dev(x_cal), alpha=case.alpha, qtype=case.qtype)
+        np.testing.assert_array_equal(host(p["amax_x"]), ax)
+        np.testing.assert_array_equal(host(p["amax_w"]), aw)
+        assert ulp_distance(host(p["s"]), s).max() <= 2
+    s_d = None if s is None else dev(s)
+    s_inv_d = None if s is None else dev(_reciprocals(s))
 
     wq_ref, sw_ref = oracle.quantize_weight(w, s, qt)
-    wq_d, sw_d = ops.quantize_weight(w_d, dev(s), case.qtype)
+    wq_d, sw_d = ops.quantize_weight(w_d, s_d, case.qtype)
     del w_d
     np.testing.assert_array_equal(host(sw_d), sw_ref)
     np.testing.assert_array_equal(host(wq_d).view(np.uint8), wq_ref.view(np.uint8))
 
-    # ---- runtime: activation smoothing + per-token quantization ----
-    xq_ref, sx_ref = oracle.quantize_act(x, s, qt)
-    xq_d, sx_d = ops.quantize_act(dev(x), dev(s), case.qtype, s_inv=dev(_reciprocals(s)))
+    if case.act_scaling == "tensor":
+        # ---- runtime: per-tensor delayed scaling, the first step's max from
+        # the calibration tokens (online), then one delayed step ----
+        _, _, amax_cal = oracle.quantize_act_tensor(x_cal, s, qt)
+        _, _, amax_cal_d = ops.quantize_act_tensor(dev(x_cal), s_d, case.qtype, s_inv=s_inv_d)
+        assert host(amax_cal_d)[0] == amax_cal
+        scale = np.float32(amax_cal) / np.float32(448.0 if qt == oracle.E4M3 else 127.0)
+        xq_ref, used, amax_x = oracle.quantize_act_tensor(x, s, qt, scale=scale)
+        sx_ref = np.full(M, used, np.float32)
+        xq_d, sx_d, amax_d = ops.quantize_act_tensor(dev(x), s_d, case.qtype, amax_prev=amax_cal_d,
+                                                     s_inv=s_inv_d)
+        assert host(amax_d)[0] == amax_x
+    else:
+        # ---- runtime: activation smoothing + per-token quantization ----
+        xq_ref, sx_ref = oracle.quantize_act(x, s, qt)
+        xq_d, sx_d = ops.quantize_act(dev(x), s_d, case.qtype, s_inv=s_inv_d)
     np.testing.assert_array_equal(host(sx_d), sx_ref)
     np.testing.assert_array_equal(host(xq_d).view(np.uint8), xq_ref.view(np.uint8))
 
@@ -79,8 +96,10 @@ def test_workload_end_to_end(name):
         assert e.max() <= 1e-3, e.max()
         np.testing.assert_array_equal(yb_got, oracle.f32_to_bf16(yf_got))
 
-    # ---- the fused forward through one C call (same operands) ----
-    y2 = ops.linear(dev(x), dev(s), ops_w, dev(sw_ref), bias_d, case.qtype,
-                    out_dtype=torch.float32, s_inv=dev(_reciprocals(s)))
+    # ---- the fused forward through one C call (same operands; per-token) ----
+    if case.act_scaling == "tensor":
+        return
+    y2 = ops.linear(dev(x), s_d, ops_w, dev(sw_ref), bias_d, case.qtype,
+                    out_dtype=torch.float32, s_inv=s_inv_d)
     assert ops.device_status() == ops.SQ_OK
     np.testing.assert_array_equal(host(y2)[rows, cols], yf_got)

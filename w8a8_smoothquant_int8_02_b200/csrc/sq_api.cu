@@ -175,6 +175,28 @@ sq_status sq_quantize_act(const void* x, sq_dtype xt, int64_t M, int64_t K, cons
                                             S(stream)));
 }
 
+sq_status sq_quantize_act_tensor(const void* x, sq_dtype xt, int64_t M, int64_t K,
+                                 const float* s, const float* s_inv, sq_dtype qt,
+                                 const float* amax_prev, void* xq, float* sx, float* amax_out,
+                                 void* stream) {
+  if (xt != SQ_F32 && xt != SQ_BF16) return SQ_ERR_INVALID_ARG;
+  if (qt != SQ_I8 && qt != SQ_E4M3) return SQ_ERR_INVALID_ARG;
+  if (M < 0 || K <= 0 || K % 16 != 0 || K > 65536 || M > INT32_MAX) return SQ_ERR_INVALID_ARG;
+  if (!amax_out || amax_out == amax_prev) return SQ_ERR_INVALID_ARG;
+  if (!al(amax_out, 4) || (amax_prev && !al(amax_prev, 4))) return SQ_ERR_MISALIGNED;
+  if (M == 0) {  // empty batch: the tensor max is 0
+    return from_cuda(cudaMemsetAsync(amax_out, 0, sizeof(float), S(stream)));
+  }
+  if (!x || !xq || !sx) return SQ_ERR_INVALID_ARG;
+  if (!al(x, 16) || !al(xq, 16) || !al(sx, 4)) return SQ_ERR_MISALIGNED;
+  if (s && !al(s, 16)) return SQ_ERR_MISALIGNED;
+  if (s_inv && !al(s_inv, 16)) return SQ_ERR_MISALIGNED;
+  return from_cuda(sqh::launch_quantize_act_tensor(x, xt == SQ_BF16, M, K, s, s ? s_inv : nullptr,
+                                                   qt == SQ_E4M3, amax_prev,
+                                                   static_cast<uint8_t*>(xq), sx, amax_out,
+                                                   S(stream)));
+}
+
 size_t sq_gemm_workspace_bytes(void) { return sqh::gemm_workspace_bytes(); }
 
 sq_status sq_gemm_w8a8(const int8_t* xq, const float* sx, const int8_t* wq, const float* sw,

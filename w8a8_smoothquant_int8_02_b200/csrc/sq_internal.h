@@ -25,6 +25,10 @@ cudaError_t launch_quantize_weight(const void* w, bool bf16, int64_t K, int64_t 
 cudaError_t launch_quantize_act(const void* x, bool bf16, int64_t M, int64_t K, const float* s,
                                 const float* s_inv, bool e4m3, uint8_t* xq, float* sx,
                                 cudaStream_t st);
+cudaError_t launch_quantize_act_tensor(const void* x, bool bf16, int64_t M, int64_t K,
+                                       const float* s, const float* s_inv, bool e4m3,
+                                       const float* amax_prev, uint8_t* xq, float* sx,
+                                       float* amax_out, cudaStream_t st);
 cudaError_t launch_selftest_fast_division(unsigned long long* mismatches, cudaStream_t st);
 // a6 / a7
 enum class OutKind { BF16, F32 };

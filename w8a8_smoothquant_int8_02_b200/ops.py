@@ -27,7 +27,7 @@ EXPORTED = (
     "sq_status_string", "sq_abi_version", "sq_get_device_status", "sq_calibrate_amax",
     "sq_smooth_factors", "sq_quantize_weight", "sq_quantize_act", "sq_gemm_w8a8",
     "sq_gemm_fp8", "sq_linear", "sq_probe_wait_timeout", "sq_selftest_fast_division",
-    "sq_gemm_workspace_bytes", "sq_gemm_w8a8_noalloc",
+    "sq_gemm_workspace_bytes", "sq_gemm_w8a8_noalloc", "sq_quantize_act_tensor",
 )
 
 _lock = threading.Lock()
@@ -180,6 +180,29 @@ def quantize_act(x: torch.Tensor, s: torch.Tensor | None, qtype: str = "i8", xq=
     _check(load().sq_quantize_act(_p(x), _fdtype(x), M, K, _p(s), _p(s_inv), qt, _p(xq), _p(sx),
                                   _stream(x.device)), "sq_quantize_act")
     return xq, sx
+
+
+def quantize_act_tensor(x: torch.Tensor, s: torch.Tensor | None, qtype: str = "e4m3",
+                        amax_prev: torch.Tensor | None = None, xq=None, sx=None, amax_out=None,
+                        s_inv: torch.Tensor | None = None):
+    """Smoothing + per-tensor quantization: one scale for the whole tensor,
+    RN(amax_prev / Q) (delayed scaling from the previous step's max) or, with
+    amax_prev None, this tensor's own max / Q (online). Returns (xq [M,K],
+    sx [M] = the scale in every entry, amax_out [1] = this tensor's
+    max|x/s|, the next step's amax_prev)."""
+    _cuda(x, s, xq, sx, s_inv, amax_prev, amax_out)
+    M, K = x.shape
+    qt = _qtype(qtype)
+    if xq is None:
+        xq = torch.empty((M, K), dtype=torch.int8 if qt == SQ_I8 else torch.uint8, device=x.device)
+    if sx is None:
+        sx = torch.empty(M, dtype=torch.float32, device=x.device)
+    if amax_out is None:
+        amax_out = torch.empty(1, dtype=torch.float32, device=x.device)
+    _check(load().sq_quantize_act_tensor(_p(x), _fdtype(x), M, K, _p(s), _p(s_inv), qt,
+                                         _p(amax_prev), _p(xq), _p(sx), _p(amax_out),
+                                         _stream(x.device)), "sq_quantize_act_tensor")
+    return xq, sx, amax_out
 
 
 _workspaces: dict = {}

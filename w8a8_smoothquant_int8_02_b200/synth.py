@@ -49,6 +49,8 @@ class LinearCase:
     outlier_factor: float = 0.0   # fixed factor for an explicit list
     bias_std: float = 0.0         # 0 => no bias
     cal_tokens: int = 512         # 0 => calibrate on X itself
+    act_scaling: str = "token"    # "token" (per-token) or "tensor" (per-tensor, delayed)
+    smooth: bool = True           # False => no smoothing factors (plain FP8 / INT8)
     seed: int = 0
     note: str = field(default="")
 

@@ -1,4 +1,5 @@
-"""The five SmoothQuant linear-layer workloads this library is measured on.
+"""The SmoothQuant linear-layer workloads this library is measured on (five
+per-token SmoothQuant cases and one per-tensor FP8 case).
 
 Shapes follow transformer linear layers: Y[M,N] = X[M,K] W[K,N], M tokens,
 K input channels, N output channels.  Prefill / MLP shapes are compute-bound
@@ -45,4 +46,12 @@ DECODE = LinearCase(
     note="X bf16 [16,8192], 1% outlier channels x U(20,100); W bf16 "
          "[8192,28672] N(0,0.02) quantized offline; HBM-bound")
 
-ALL = {c.name: c for c in (TINY, PREFILL, MLP_UP, FP8_DOWN, DECODE)}
+FP8_TENSOR = LinearCase(
+    name="fp8_tensor_4096x4096x14336", M=4096, K=4096, N=14336, x_dtype="bf16",
+    alpha=0.5, qtype="e4m3", w_std=0.02, outlier_frac=0.01, outlier_lo=20.0,
+    outlier_hi=100.0, bias_std=0.01, cal_tokens=512, act_scaling="tensor", smooth=False,
+    note="the MLP-up shape in native FP8: no smoothing, one E4M3 scale for the whole "
+         "activation tensor from the previous step's max (delayed scaling; the first "
+         "step's from the 512 calibration tokens), per-output-channel E4M3 weights")
+
+ALL = {c.name: c for c in (TINY, PREFILL, MLP_UP, FP8_DOWN, DECODE, FP8_TENSOR)}
