@@ -511,10 +511,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; j < 32; ++j) __stcg(dst + j * 128, int32_t(r[j]));
       };
 
+      // a warp whose 32 rows all lie beyond M (the last M-tile of a small
+      // batch) has nothing to store, publish or add: it only keeps the
+      // barrier and counter protocol below
+      const bool slab_live = box_row < M;
       // this warp's chunks are half, half+WPQ, half+2*WPQ, ...; two loads in
       // flight at a time
 #pragma unroll 1
-      for (int c = half; c < NCH && !give_up; c += 2 * WPQ) {
+      for (int c = half; slab_live && c < NCH && !give_up; c += 2 * WPQ) {
         uint32_t r0[32], r1[32];
         const bool two = c + WPQ < NCH;  // warp-uniform
         tmem_ld32(t_addr + uint32_t(c * 32), r0);
