@@ -107,3 +107,34 @@ def test_empty_batch_sets_the_max_to_zero():
     assert xq.shape == (0, 64) and sx.shape == (0,)
     assert host(amax)[0] == 0.0
     assert ops.device_status() == ops.SQ_OK
+
+
+def test_module_delayed_scaling_over_calls():
+    """SmoothQuantLinear(act_scaling='tensor', smooth=False): the first call
+    scales by the calibration max, each later call by the previous call's
+    max; outputs against the oracle (exact E4M3 sums, normalized error)."""
+    from w8a8_smoothquant_int8_02_b200.ops import SmoothQuantLinear
+    from _gpu_util import fp8_normalized_error
+    K, N = 512, 384
+    g = np.random.default_rng(41)
+    w = (g.standard_normal((K, N)) * 0.02).astype(np.float32)
+    x_cal = _x((64, K), seed=42, dtype="bf16")
+    batches = [_x((96, K), seed=43 + i, dtype="bf16") for i in range(3)]
+    layer = SmoothQuantLinear(dev(synth.to_bf16_bits(w)), dev(x_cal), qtype="e4m3",
+                              act_scaling="tensor", smooth=False)
+    wb = synth.to_bf16_bits(w)
+    wq_ref, sw_ref = oracle.quantize_weight(wb, None, oracle.E4M3)
+    _, _, prev = oracle.quantize_act_tensor(x_cal, None, oracle.E4M3)
+    for xb in batches:
+        assert host(layer.last_amax)[0] == prev
+        y = layer(dev(xb), out_dtype=torch.float32)
+        scale = np.float32(prev) / np.float32(448.0)
+        xq_ref, used, prev = oracle.quantize_act_tensor(xb, None, oracle.E4M3, scale=scale)
+        rows, cols = np.divmod(np.arange(96 * N, dtype=np.int64), N)
+        sx_ref = np.full(96, used, np.float32)
+        _, yf_ref, _ = oracle.linear_at(xq_ref, sx_ref, wq_ref, sw_ref, None, rows, cols,
+                                        oracle.E4M3)
+        got = host(y)[rows, cols]
+        e = fp8_normalized_error(got, yf_ref, xq_ref, wq_ref, sx_ref, sw_ref, None, rows, cols)
+        assert e.max() <= 1e-3, e.max()
+    assert ops.device_status() == ops.SQ_OK

@@ -365,16 +365,47 @@ def prepare(w: torch.Tensor, x_cal: torch.Tensor, alpha: float = 0.5, qtype: str
 
 
 class SmoothQuantLinear:
-    """A prepared SmoothQuant W8A8 linear layer: y = x @ W (+ bias)."""
+    """A prepared W8A8 linear layer: y = x @ W (+ bias).
+
+    act_scaling "token" (default): SmoothQuant, per-token activation scales.
+    act_scaling "tensor": one scale for the whole activation tensor, taken
+    from the previous call's max (delayed scaling; the first call's from the
+    calibration tokens); smooth=False skips the smoothing factors (native
+    FP8 without SmoothQuant)."""
 
     def __init__(self, w: torch.Tensor, x_cal: torch.Tensor, alpha: float = 0.5,
-                 qtype: str = "i8", bias: torch.Tensor | None = None):
-        p = prepare(w, x_cal, alpha, qtype)
-        self.s, self.s_inv, self.wq, self.sw = p["s"], p["s_inv"], p["wq"], p["sw"]
+                 qtype: str = "i8", bias: torch.Tensor | None = None,
+                 act_scaling: str = "token", smooth: bool = True):
+        if act_scaling not in ("token", "tensor"):
+            raise ValueError("act_scaling must be 'token' or 'tensor'")
+        if smooth:
+            p = prepare(w, x_cal, alpha, qtype)
+            self.s, self.s_inv, self.wq, self.sw = p["s"], p["s_inv"], p["wq"], p["sw"]
+        else:
+            self.s = self.s_inv = None
+            self.wq, self.sw = quantize_weight(w, None, qtype)
         self.qtype = qtype
         self.bias = bias
+        self.act_scaling = act_scaling
         self.in_features, self.out_features = w.shape
+        if act_scaling == "tensor":
+            # two floats: the max the next call scales by, and the one it writes
+            self._amax = torch.zeros(2, dtype=torch.float32, device=w.device)
+            self._cur = 0
+            quantize_act_tensor(x_cal, self.s, qtype, amax_out=self._amax[0:1], s_inv=self.s_inv)
+
+    @property
+    def last_amax(self) -> torch.Tensor:
+        """The activation max the next call will scale by (tensor scaling)."""
+        return self._amax[self._cur:self._cur + 1]
 
     def __call__(self, x: torch.Tensor, out_dtype=torch.bfloat16) -> torch.Tensor:
-        return linear(x, self.s, self.wq, self.sw, self.bias, self.qtype, out_dtype,
-                      s_inv=self.s_inv)
+        if self.act_scaling == "token":
+            return linear(x, self.s, self.wq, self.sw, self.bias, self.qtype, out_dtype,
+                          s_inv=self.s_inv)
+        c = self._cur
+        xq, sx, _ = quantize_act_tensor(x, self.s, self.qtype, amax_prev=self._amax[c:c + 1],
+                                        amax_out=self._amax[1 - c:2 - c], s_inv=self.s_inv)
+        self._cur = 1 - c
+        g = gemm_w8a8 if self.qtype == "i8" else gemm_fp8
+        return g(xq, sx, self.wq, self.sw, self.bias, out_dtype=out_dtype)
