@@ -1,0 +1,83 @@
+"""Host-side logic of bench.py (no GPU): the L2-defeating rotation, the
+metric names, which activation kernel each workload launches, the
+source-hash guard on profiled DRAM traffic, and the reference arm's
+arithmetic on a tiny case."""
+import importlib.util
+import os
+import shutil
+import sys
+
+import pytest
+
+from w8a8_smoothquant_int8_02_b200 import workloads
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def bench():
+    spec = importlib.util.spec_from_file_location("bench_under_test", os.path.join(ROOT, "bench.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+@pytest.mark.parametrize("name", list(workloads.ALL))
+def test_rotation_exceeds_l2(bench, name):
+    case = workloads.ALL[name]
+    per_set = case.M * case.K * 2 + case.N * case.K
+    r = bench.rotate_count(case)
+    assert r >= 1
+    assert r * per_set >= 1.5 * bench.L2_BYTES or per_set >= 1.5 * bench.L2_BYTES
+
+
+def test_metric_names(bench):
+    assert bench.metric_for(workloads.MLP_UP) == bench.METRIC
+    assert "FP8" in bench.metric_for(workloads.FP8_DOWN)
+    assert "per-tensor" in bench.metric_for(workloads.FP8_TENSOR)
+    assert "M512 K4096 N4096" in bench.metric_for(workloads.PREFILL)
+
+
+def test_activation_kernel_per_workload(bench):
+    assert bench.quant_kernel_name(workloads.TINY) == "quant_act_kernel"              # fp32 input
+    assert bench.quant_kernel_name(workloads.MLP_UP) == "quant_act_stream_kernel"
+    assert bench.quant_kernel_name(workloads.FP8_DOWN) == "quant_act_stream_kernel"
+    assert bench.quant_kernel_name(workloads.DECODE) == "quant_act_fast_kernel"      # 16 rows
+    assert bench.quant_kernel_name(workloads.FP8_TENSOR) == "quant_act_tensor_kernel"
+
+
+def test_profiled_traffic_is_guarded_by_the_kernel_source(bench, tmp_path, monkeypatch):
+    """Traffic is reported only for a workload that was captured and only
+    while the kernel's sources hash as they did at capture time."""
+    assert bench.profiled_traffic("gemm", "decode_16x8192x28672") is None
+    # a copy of the tree whose GEMM source differs by one byte reports null
+    fake = tmp_path / "root"
+    csrc = fake / "w8a8_smoothquant_int8_02_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    for f in ("sq_gemm.cu", "sq_common.cuh", "sq_quant.cu"):
+        shutil.copy(os.path.join(ROOT, "w8a8_smoothquant_int8_02_b200", "csrc", f), csrc / f)
+    monkeypatch.setattr(bench, "ROOT", str(fake))
+    key = ("gemm", "mlp_up_4096x4096x14336")
+    if key in bench.PROFILED_TRAFFIC:
+        expected = bench.profiled_traffic(*key)
+        with open(csrc / "sq_gemm.cu", "a") as f:
+            f.write("\n")
+        assert bench.profiled_traffic(*key) is None
+        assert expected is None or expected > 0
+
+
+def test_reference_arm_cpu_baseline_on_tiny(bench):
+    """The oracle leg runs on a tiny case and reports a positive rate with
+    its sample described."""
+    from w8a8_smoothquant_int8_02_b200 import synth
+    case = workloads.TINY
+    d = synth.generate(case)
+    out = bench.cpu_baseline(case, d, budget_s=0.05)
+    assert out["kind"] == "oracle" and out["value"] > 0 and out["cores"] >= 1
+    assert "token rows" in out["sample"]
+    tensor = workloads.FP8_TENSOR
+    small = synth.LinearCase(**{**tensor.__dict__, "M": 8, "K": 64, "N": 32, "cal_tokens": 16,
+                                "name": "fp8_tensor_small"})
+    d2 = synth.generate(small)
+    out2 = bench.cpu_baseline(small, d2, budget_s=0.05)
+    assert out2["value"] > 0
