@@ -65,10 +65,12 @@ def rotate_count(case):
 # summaries under profiles/), keyed by the sha256 prefix of the kernel's
 # sources at capture time: a kernel changed since reports null.
 PROFILED_TRAFFIC = {
-    ("gemm", "mlp_up_4096x4096x14336"): (75.928576e6 + 82.759680e6, "0d224357d8151d98"),
-    ("gemm", "fp8_down_4096x14336x4096"): (273.935360e6 + 28.075776e6, "0d224357d8151d98"),
-    ("quant", "mlp_up_4096x4096x14336"): (33.648128e6 + 0.008704e6, "616d402bb78b8727"),
-    ("quant", "fp8_down_4096x14336x4096"): (117.738240e6 + 29.602048e6, "616d402bb78b8727"),
+    ("gemm", "mlp_up_4096x4096x14336"): (76.000256e6 + 82.700032e6, "88dbd4d7d330f6de"),
+    ("gemm", "fp8_down_4096x14336x4096"): (267.428864e6 + 26.647040e6, "88dbd4d7d330f6de"),
+    ("gemm", "fp8_tensor_4096x4096x14336"): (75.807744e6 + 85.412864e6, "88dbd4d7d330f6de"),
+    ("quant", "mlp_up_4096x4096x14336"): (33.647872e6 + 0.007168e6, "11715b8dda2dbca9"),
+    ("quant", "fp8_down_4096x14336x4096"): (117.737216e6 + 32.378368e6, "11715b8dda2dbca9"),
+    ("quant", "fp8_tensor_4096x4096x14336"): (33.578240e6 + 0.001024e6, "11715b8dda2dbca9"),
 }
 KERNEL_SOURCES = {"gemm": ("sq_gemm.cu", "sq_common.cuh"), "quant": ("sq_quant.cu", "sq_common.cuh")}
 
