@@ -51,7 +51,10 @@ def test_distributed_calibration_equals_whole_corpus():
     import oracle
     from w8a8_smoothquant_int8_02_b200 import synth, workloads
     world_size = 2
-    manager = mp.Manager()
+    # the result store runs in a spawned process too: this test process may
+    # already have threads (OpenMP in the oracle, torch), and fork would copy
+    # them half-way
+    manager = mp.get_context("spawn").Manager()
     results = manager.dict()
     port = _free_port()
     mp.spawn(_worker, args=(world_size, port, results), nprocs=world_size, join=True)
