@@ -509,7 +509,7 @@ def main():
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--workload", default="mlp_up_4096x4096x14336",
                     help="one of the five workloads (default: the MLP up-projection)")
-    ap.add_argument("--tile", default=None, help="force a GEMM tile shape (c1n128, c1n256, "
+    ap.add_argument("--tile", default=None, help="force a GEMM tile shape (c1n128, c1n224, c1n256, "
                     "c2n224, c2n256); default: chosen by problem size")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -771,18 +771,21 @@ static cudaError_t dispatch_epilogue(const void* xq, const void* wq, const float
 
 // Tile shapes compiled in. Each entry: CTAs per tile (1 or 2), N per tile,
 // pipeline depth.
-enum class TileCfg { C1_N128, C1_N256, C2_N224, C2_N256 };
+enum class TileCfg { C1_N128, C1_N224, C1_N256, C2_N224, C2_N256 };
 
 static TileCfg choose_tile(int64_t M, int64_t N, bool can_split) {
   // Estimated time ~ (number of rounds of tiles over the SMs) x (work per
   // tile) / (relative MAC throughput of the tile shape, measured on B200 at
   // 4096 x 4096 x 14336: 256x256 pairs 1.0, 256x224 pairs 0.89, 128x256
-  // single CTAs 0.90, 128x128 single CTAs 0.62).
+  // single CTAs 0.90, 128x224 single CTAs 0.85, 128x128 single CTAs 0.62).
+  // For a single M-tile (decode) the work per tile is its Wq panel, so the
+  // same estimate favours the tile width that spreads N over the most SMs.
   const int sms = device_sms();
   struct Cand { TileCfg c; int cg, bm, bn; double eff; };
   const Cand cands[] = {{TileCfg::C2_N256, 2, 256, 256, 1.0},
                         {TileCfg::C2_N224, 2, 256, 224, 0.89},
                         {TileCfg::C1_N256, 1, 128, 256, 0.90},
+                        {TileCfg::C1_N224, 1, 128, 224, 0.85},
                         {TileCfg::C1_N128, 1, 128, 128, 0.62}};
   double best = 1e30;
   TileCfg pick = TileCfg::C1_N128;
@@ -802,13 +805,14 @@ static TileCfg choose_tile(int64_t M, int64_t N, bool can_split) {
   return pick;
 }
 
-// SQ_GEMM_TILE = c1n128 | c1n256 | c2n224 | c2n256 forces one tile shape
+// SQ_GEMM_TILE = c1n128 | c1n224 | c1n256 | c2n224 | c2n256 forces one tile shape
 // (used to test every shape and to compare them); unset or anything else
 // selects by problem size.
 static bool forced_tile(TileCfg* out) {
   const char* e = getenv("SQ_GEMM_TILE");
   if (!e) return false;
   if (!strcmp(e, "c1n128")) { *out = TileCfg::C1_N128; return true; }
+  if (!strcmp(e, "c1n224")) { *out = TileCfg::C1_N224; return true; }
   if (!strcmp(e, "c1n256")) { *out = TileCfg::C1_N256; return true; }
   if (!strcmp(e, "c2n224")) { *out = TileCfg::C2_N224; return true; }
   if (!strcmp(e, "c2n256")) { *out = TileCfg::C2_N256; return true; }
@@ -836,6 +840,7 @@ cudaError_t launch_gemm(bool e4m3, const uint8_t* xq, const float* sx, const uin
     case TileCfg::C2_N256: SQ_CASE(2, 256, 6);
     case TileCfg::C2_N224: SQ_CASE(2, 224, 7);
     case TileCfg::C1_N256: SQ_CASE(1, 256, 4);
+    case TileCfg::C1_N224: SQ_CASE(1, 224, 5);
     default: SQ_CASE(1, 128, 6);
   }
 #undef SQ_CASE

@@ -326,7 +326,7 @@ def probe_wait_timeout(timeout_ns: int, device=None):
 
 
 # GEMM tile shapes compiled into libsq.so (CTAs per tile x N per tile).
-GEMM_TILES = ("c1n128", "c1n256", "c2n224", "c2n256")
+GEMM_TILES = ("c1n128", "c1n224", "c1n256", "c2n224", "c2n256")
 
 
 class gemm_tile:
