@@ -65,12 +65,12 @@ def rotate_count(case):
 # summaries under profiles/), keyed by the sha256 prefix of the kernel's
 # sources at capture time: a kernel changed since reports null.
 PROFILED_TRAFFIC = {
-    ("gemm", "mlp_up_4096x4096x14336"): (76.000256e6 + 82.700032e6, "88dbd4d7d330f6de"),
-    ("gemm", "fp8_down_4096x14336x4096"): (267.428864e6 + 26.647040e6, "88dbd4d7d330f6de"),
-    ("gemm", "fp8_tensor_4096x4096x14336"): (75.807744e6 + 85.412864e6, "88dbd4d7d330f6de"),
-    ("quant", "mlp_up_4096x4096x14336"): (33.647872e6 + 0.007168e6, "11715b8dda2dbca9"),
-    ("quant", "fp8_down_4096x14336x4096"): (117.737216e6 + 32.378368e6, "11715b8dda2dbca9"),
-    ("quant", "fp8_tensor_4096x4096x14336"): (33.578240e6 + 0.001024e6, "11715b8dda2dbca9"),
+    ("gemm", "mlp_up_4096x4096x14336"): (75.886592e6 + 83.189248e6, "38e67a6ddb8053cd"),
+    ("gemm", "fp8_down_4096x14336x4096"): (277.412096e6 + 26.567424e6, "38e67a6ddb8053cd"),
+    ("gemm", "fp8_tensor_4096x4096x14336"): (75.913984e6 + 84.172288e6, "38e67a6ddb8053cd"),
+    ("quant", "mlp_up_4096x4096x14336"): (33.647616e6 + 0.003072e6, "11715b8dda2dbca9"),
+    ("quant", "fp8_down_4096x14336x4096"): (117.746432e6 + 29.849344e6, "11715b8dda2dbca9"),
+    ("quant", "fp8_tensor_4096x4096x14336"): (33.578496e6 + 0.003840e6, "11715b8dda2dbca9"),
 }
 KERNEL_SOURCES = {"gemm": ("sq_gemm.cu", "sq_common.cuh"), "quant": ("sq_quant.cu", "sq_common.cuh")}
 
