@@ -66,6 +66,7 @@ def _load():
             lib.sqo_smooth_factors.argtypes = [P, P, I64, ctypes.c_double, P]
             lib.sqo_smooth_act.argtypes = [P, I, I64, I64, P, P]
             lib.sqo_smooth_weight.argtypes = [P, I, I64, I64, P, P]
+            lib.sqo_fold_smoothing.argtypes = [P, I, I64, I64, P, I, P]
             lib.sqo_quantize_weight.argtypes = [P, I, I64, I64, P, I, P, P]
             lib.sqo_quantize_act.argtypes = [P, I, I64, I64, P, I, P, P]
             lib.sqo_quantize_act_tensor.argtypes = [P, I, I64, I64, P, I, P, P, P, P]
@@ -169,6 +170,22 @@ def smooth_weight(w: np.ndarray, s) -> np.ndarray:
     s = _c(s, np.float32)
     out = np.empty((K, N), np.float32)
     _load().sqo_smooth_weight(_ptr(w), _dtype_code(w), K, N, _ptr(s), _ptr(out))
+    return out
+
+
+def fold_smoothing(p: np.ndarray, s, per_column: bool = True) -> np.ndarray:
+    """The producer's per-channel parameters divided by s (float32): channel =
+    column (per_column) or row; the producer then emits X~ = X diag(s)^-1."""
+    p = np.ascontiguousarray(p)
+    if p.ndim == 1:
+        p = p.reshape(1, -1) if per_column else p.reshape(-1, 1)
+    rows, cols = p.shape
+    s = _c(s, np.float32)
+    if s.size != (cols if per_column else rows):
+        raise ValueError("s must have one entry per channel")
+    out = np.empty((rows, cols), np.float32)
+    _load().sqo_fold_smoothing(_ptr(p), _dtype_code(p), rows, cols, _ptr(s), int(per_column),
+                               _ptr(out))
     return out
 
 

@@ -146,6 +146,20 @@ void sqo_smooth_weight(const void* w, int dtype, int64_t K, int64_t N,
             out[k * N + n] = smooth_w(load_elem(w, dtype, k * N + n), s[k]);
 }
 
+/* The smoothing is offline ([LES] §2: the transform happens during model
+ * preparation, with no runtime overhead; [WAQ] §3 Step 1 lists X~ = X
+ * diag(1/s) under offline preparation). Reading taken: the op that produces
+ * X carries one parameter, or one row / column of a weight, per channel k of
+ * X, and dividing those by s_k -- the same binary32 division smooth_x applies
+ * to x -- makes it emit X~. */
+void sqo_fold_smoothing(const void* p, int dtype, int64_t rows, int64_t cols,
+                        const float* s, int per_column, float* out) {
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < cols; ++c)
+            out[r * cols + c] = smooth_x(load_elem(p, dtype, r * cols + c),
+                                         per_column ? s[c] : s[r]);
+}
+
 int sqo_num_threads(void) {
 #ifdef _OPENMP
     return omp_get_max_threads();

@@ -53,6 +53,14 @@ void sqo_smooth_act(const void* x, int dtype, int64_t M, int64_t K,
 void sqo_smooth_weight(const void* w, int dtype, int64_t K, int64_t N,
                        const float* s, float* out);
 
+/* Offline fold of the activation division into the layer that produces X:
+ * its parameters for channel k of X are divided by s[k] once, so it emits
+ * X~ itself and the runtime quantization runs without s.
+ * p: [rows, cols] (dtype); per_column != 0: channel = column,
+ * out[r][c] = p[r][c] / s[c]; else channel = row, out[r][c] = p[r][c] / s[r]. */
+void sqo_fold_smoothing(const void* p, int dtype, int64_t rows, int64_t cols,
+                        const float* s, int per_column, float* out);
+
 /* a4 offline weight smoothing + per-output-channel quantization.
  * w: [K,N] (dtype), s: [K] or NULL (no smoothing).
  * wq: [N,K] int8 or E4M3 codes, sw: [N] binary32 scales. */

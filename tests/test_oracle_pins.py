@@ -515,3 +515,87 @@ def test_per_tensor_delayed_with_own_max_is_online_and_zero_scale():
     np.testing.assert_array_equal(xq_o, xq_d)
     xq_z, _, amax_z = oracle.quantize_act_tensor(x, None, oracle.INT8, scale=np.float32(0.0))
     assert not xq_z.any() and amax_z == amax
+
+
+# ---------------------------------------------------------------------------
+# The smoothing is offline: 1/s folded once into the layer that produces X.
+# ---------------------------------------------------------------------------
+
+def test_fold_worked_example_gain_emits_the_smoothed_values():
+    """A producer with unit gain on the worked example's channel, folded with
+    s = 8, has gain 1/8 and emits the smoothed values printed in §3."""
+    fx = _fixture("worked_example.txt")
+    x = np.array(fx["x"], np.float32)
+    s = np.array(fx["s"], np.float32)
+    g = oracle.fold_smoothing(np.ones(3, np.float32), s)[0]
+    np.testing.assert_array_equal(g, np.full(3, 0.125, np.float32))
+    np.testing.assert_array_equal((x * g).astype(np.float32),
+                                  np.array(fx["x_smoothed"], np.float32))
+
+
+def test_fold_power_of_two_is_an_exact_scaling():
+    """Division by 2^e is the exact scaling by 2^-e, along either axis."""
+    rng = np.random.default_rng(61)
+    p = rng.standard_normal((5, 40)).astype(np.float32)
+    ec = rng.integers(-12, 13, size=40)
+    er = rng.integers(-12, 13, size=5)
+    sc = np.ldexp(np.ones(40), ec).astype(np.float32)
+    sr = np.ldexp(np.ones(5), er).astype(np.float32)
+    np.testing.assert_array_equal(oracle.fold_smoothing(p, sc, per_column=True),
+                                  np.ldexp(p.astype(np.float64), -ec[None, :]).astype(np.float32))
+    np.testing.assert_array_equal(oracle.fold_smoothing(p, sr, per_column=False),
+                                  np.ldexp(p.astype(np.float64), -er[:, None]).astype(np.float32))
+
+
+@pytest.mark.parametrize("bf16", [False, True])
+def test_fold_general_s_is_the_correctly_rounded_quotient(bf16):
+    """A binary64 quotient of two binary32 values rounded once to binary32 is
+    their correctly rounded binary32 quotient (53 >= 2*24 + 2 significant
+    bits, so the double rounding is harmless): an independent route to the
+    fold's result. bf16 parameters widen exactly first."""
+    rng = np.random.default_rng(62)
+    p = (rng.standard_normal((7, 33)) * np.exp(rng.uniform(-20, 20, (7, 33)))).astype(np.float32)
+    s = np.exp(rng.uniform(np.log(1e-3), np.log(1e3), 33)).astype(np.float32)
+    if bf16:
+        pin = synth.to_bf16_bits(p)
+        pw = oracle.bf16_to_f32(pin)
+    else:
+        pin = pw = p
+    want = (pw.astype(np.float64) / s.astype(np.float64)[None, :]).astype(np.float32)
+    np.testing.assert_array_equal(oracle.fold_smoothing(pin, s, per_column=True), want)
+
+
+def test_fold_axes_are_transposes_of_each_other():
+    """Channel = column of p [R,K] and channel = row of p^T [K,R] give
+    transposed results (a swapped index would fail on this non-square p)."""
+    rng = np.random.default_rng(63)
+    p = rng.standard_normal((6, 11)).astype(np.float32)
+    s = rng.uniform(0.05, 20.0, 11).astype(np.float32)
+    a = oracle.fold_smoothing(p, s, per_column=True)
+    b = oracle.fold_smoothing(np.ascontiguousarray(p.T), s, per_column=False)
+    np.testing.assert_array_equal(a, b.T)
+    assert not np.array_equal(a, p / s[0])
+
+
+@pytest.mark.parametrize("qt", [oracle.INT8, oracle.E4M3])
+def test_folded_producer_feeds_the_same_codes(qt):
+    """A gain producer x * g: folded (gain g/s, then quantization without s)
+    and unfolded (gain g, then x/s inside the quantization) give the same
+    codes and scales when s is a power of two, and X~ within two roundings
+    on each side otherwise."""
+    rng = np.random.default_rng(64)
+    M, K = 9, 64
+    x = (rng.standard_normal((M, K)) * 3).astype(np.float32)
+    x[:, [5, 40]] *= 50
+    g = rng.uniform(0.5, 2.0, K).astype(np.float32)
+    s = np.ldexp(np.ones(K), rng.integers(-4, 8, K)).astype(np.float32)
+    folded = (x * oracle.fold_smoothing(g, s)[0]).astype(np.float32)
+    unfolded = (x * g).astype(np.float32)
+    q1, sx1 = oracle.quantize_act(folded, None, qt)
+    q2, sx2 = oracle.quantize_act(unfolded, s, qt)
+    np.testing.assert_array_equal(q1, q2)
+    np.testing.assert_array_equal(sx1, sx2)
+    s = rng.uniform(0.05, 20.0, K).astype(np.float32)
+    folded = (x * oracle.fold_smoothing(g, s)[0]).astype(np.float64)
+    exact = x.astype(np.float64) * g.astype(np.float64) / s.astype(np.float64)
+    assert np.all(np.abs(folded - exact) <= 2.0 ** -22 * np.abs(exact))
