@@ -53,7 +53,7 @@
 extern "C" {
 #endif
 
-#define SQ_ABI_VERSION 4
+#define SQ_ABI_VERSION 5
 
 typedef enum {
     SQ_OK = 0,
@@ -193,6 +193,32 @@ sq_status sq_quantize_act_tensor(const void* x, sq_dtype xt, int64_t M, int64_t 
                                  const float* s, const float* s_inv, sq_dtype qt,
                                  const float* amax_prev, void* xq, float* sx,
                                  float* amax_out, void* stream);
+
+/*
+ * Offline fold of the activation smoothing into the layer that produces X.
+ * Source: "Weight-Activation Quantization" (infra.bea.ai) §3, the two-step
+ * pipeline (X_tilde = X diag(1/s) is part of offline model preparation), and
+ * the grasp.study lesson on W8A16 vs W8A8, §2 (the transform happens offline,
+ * with no runtime overhead). The pages name no producer; this library takes
+ * it to carry one parameter, or one row or column of a weight, per channel k
+ * of X (a normalization's gain, a preceding linear layer's weight and bias).
+ * Dividing those by s_k once makes the producer emit X_tilde, and this
+ * layer's activations are then quantized with s = NULL.
+ *   p    : [rows, cols] row-major, SQ_F32 or SQ_BF16, aligned to its element
+ *   s    : the smoothing factors (sq_smooth_factors), one per channel
+ *   axis : SQ_AMAX_PER_COLUMN -> channel = column: out[r,c] = p[r,c] / s[c]
+ *          (s has `cols` entries; a gain vector as [1,K], or a producer
+ *          weight [R,K] in this library's [in,out] layout);
+ *          SQ_AMAX_PER_ROW    -> channel = row: out[r,c] = p[r,c] / s[r]
+ *          (s has `rows` entries; a producer weight stored [K,R]).
+ *   out  : [rows, cols] binary32, not aliasing p (SQ_ERR_INVALID_ARG if
+ *          out == p).
+ * Each element is one IEEE binary32 division, the operation the runtime
+ * kernels apply to x, so the result is bit-exact against it. rows or cols
+ * == 0 is a no-op.
+ */
+sq_status sq_fold_smoothing(const void* p, sq_dtype pt, int64_t rows, int64_t cols,
+                            const float* s, sq_axis axis, float* out, void* stream);
 
 /*
  * Size in bytes of the GEMM workspace for the current device (its SM count

@@ -53,7 +53,7 @@ def test_exported_symbols_are_visible_to_the_dynamic_linker():
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.sq_abi_version() == 4
+    assert lib.sq_abi_version() == 5
     for st in range(7):
         assert ops.status_string(st).startswith("SQ_")
     assert "TIMEOUT" in ops.status_string(ops.SQ_ERR_TIMEOUT)
@@ -111,6 +111,32 @@ def test_quantize_act_tensor_validation(lib):
     assert call(prev=A + 66) == ops.SQ_ERR_MISALIGNED
     assert call(x=MIS) == ops.SQ_ERR_MISALIGNED
     assert call(s=A + 4) == ops.SQ_ERR_MISALIGNED
+
+
+def test_fold_smoothing_validation(lib):
+    f = lib.sq_fold_smoothing
+    ok = dict(p=A, pt=ops.SQ_BF16, rows=3, cols=40, s=A + 4096, axis=ops.SQ_AMAX_PER_COLUMN,
+              out=A + 8192)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return f(c(a["p"]), a["pt"], a["rows"], a["cols"], c(a["s"]), a["axis"], c(a["out"]), None)
+
+    assert call(p=NUL) == ops.SQ_ERR_INVALID_ARG
+    assert call(s=NUL) == ops.SQ_ERR_INVALID_ARG
+    assert call(out=NUL) == ops.SQ_ERR_INVALID_ARG
+    assert call(out=A) == ops.SQ_ERR_INVALID_ARG          # in place is aliasing
+    assert call(pt=ops.SQ_I8) == ops.SQ_ERR_INVALID_ARG
+    assert call(axis=2) == ops.SQ_ERR_INVALID_ARG
+    assert call(rows=-1) == ops.SQ_ERR_INVALID_ARG
+    assert call(rows=2 ** 40, cols=2 ** 40) == ops.SQ_ERR_INVALID_ARG   # rows*cols overflows
+    assert call(p=A + 1) == ops.SQ_ERR_MISALIGNED          # bf16 wants 2-byte alignment
+    assert call(p=A + 2, pt=ops.SQ_F32) == ops.SQ_ERR_MISALIGNED
+    assert call(s=A + 2) == ops.SQ_ERR_MISALIGNED
+    assert call(out=A + 8194) == ops.SQ_ERR_MISALIGNED
+    # empty: a no-op that accepts NULL pointers
+    assert call(rows=0, p=NUL, s=NUL, out=NUL) == ops.SQ_OK
+    assert call(cols=0, p=NUL, s=NUL, out=NUL) == ops.SQ_OK
 
 
 def test_gemm_validation(lib):

@@ -42,6 +42,7 @@ def _host(shape, dtype):
     lambda: ops.quantize_act_tensor(_host((4, 64), torch.bfloat16), None, "e4m3"),
     lambda: ops.quantize_weight(_host((64, 32), torch.bfloat16), None, "i8"),
     lambda: ops.calibrate_amax(_host((4, 64), torch.bfloat16), "column"),
+    lambda: ops.fold_smoothing(_host(64, torch.float32), _host(64, torch.float32)),
     lambda: ops.gemm_w8a8(_host((4, 64), torch.int8), _host(4, torch.float32),
                           _host((32, 64), torch.int8), _host(32, torch.float32)),
     lambda: ops.gemm_fp8(_host((4, 64), torch.uint8), _host(4, torch.float32),

@@ -197,6 +197,19 @@ sq_status sq_quantize_act_tensor(const void* x, sq_dtype xt, int64_t M, int64_t 
                                                    S(stream)));
 }
 
+sq_status sq_fold_smoothing(const void* p, sq_dtype pt, int64_t rows, int64_t cols,
+                            const float* s, sq_axis axis, float* out, void* stream) {
+  if (pt != SQ_F32 && pt != SQ_BF16) return SQ_ERR_INVALID_ARG;
+  if (axis != SQ_AMAX_PER_COLUMN && axis != SQ_AMAX_PER_ROW) return SQ_ERR_INVALID_ARG;
+  if (rows < 0 || cols < 0) return SQ_ERR_INVALID_ARG;
+  if (rows == 0 || cols == 0) return SQ_OK;  // nothing to fold: pointers may be NULL
+  if (rows > INT64_MAX / cols) return SQ_ERR_INVALID_ARG;
+  if (!p || !s || !out || static_cast<const void*>(out) == p) return SQ_ERR_INVALID_ARG;
+  if (!al(p, pt == SQ_BF16 ? 2 : 4) || !al(s, 4) || !al(out, 4)) return SQ_ERR_MISALIGNED;
+  return from_cuda(sqh::launch_fold_smoothing(p, pt == SQ_BF16, rows, cols, s,
+                                              axis == SQ_AMAX_PER_COLUMN, out, S(stream)));
+}
+
 size_t sq_gemm_workspace_bytes(void) { return sqh::gemm_workspace_bytes(); }
 
 sq_status sq_gemm_w8a8(const int8_t* xq, const float* sx, const int8_t* wq, const float* sw,

@@ -29,6 +29,9 @@ cudaError_t launch_quantize_act_tensor(const void* x, bool bf16, int64_t M, int6
                                        const float* s, const float* s_inv, bool e4m3,
                                        const float* amax_prev, uint8_t* xq, float* sx,
                                        float* amax_out, cudaStream_t st);
+// offline fold of 1/s into the producer of X
+cudaError_t launch_fold_smoothing(const void* p, bool bf16, int64_t rows, int64_t cols,
+                                  const float* s, bool per_column, float* out, cudaStream_t st);
 cudaError_t launch_selftest_fast_division(unsigned long long* mismatches, cudaStream_t st);
 // a6 / a7
 enum class OutKind { BF16, F32 };

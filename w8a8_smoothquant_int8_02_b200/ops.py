@@ -28,6 +28,7 @@ EXPORTED = (
     "sq_smooth_factors", "sq_quantize_weight", "sq_quantize_act", "sq_gemm_w8a8",
     "sq_gemm_fp8", "sq_linear", "sq_probe_wait_timeout", "sq_selftest_fast_division",
     "sq_gemm_workspace_bytes", "sq_gemm_w8a8_noalloc", "sq_quantize_act_tensor",
+    "sq_fold_smoothing",
 )
 
 _lock = threading.Lock()
@@ -64,6 +65,7 @@ def load(build_if_needed: bool = True) -> ctypes.CDLL:
             lib.sq_smooth_factors.argtypes = [P, P, I64, D, P, P, P]
             lib.sq_quantize_weight.argtypes = [P, I, I64, I64, P, I, P, P, P]
             lib.sq_quantize_act.argtypes = [P, I, I64, I64, P, P, I, P, P, P]
+            lib.sq_fold_smoothing.argtypes = [P, I, I64, I64, P, I, P, P]
             SZ = ctypes.c_size_t
             lib.sq_gemm_w8a8.argtypes = [P, P, P, P, P, I64, I64, I64, P, I, P, P, SZ, P]
             lib.sq_gemm_fp8.argtypes = [P, P, P, P, P, I64, I64, I64, P, I, P, SZ, P]
@@ -139,6 +141,34 @@ def calibrate_amax(x: torch.Tensor, axis: str = "column", out: torch.Tensor | No
         out = torch.empty(n, dtype=torch.float32, device=x.device)
     _check(load().sq_calibrate_amax(_p(x), _fdtype(x), rows, cols, ax, _p(out), int(accumulate),
                                     _stream(x.device)), "sq_calibrate_amax")
+    return out
+
+
+def fold_smoothing(p: torch.Tensor, s: torch.Tensor, axis: str = "column",
+                   out: torch.Tensor | None = None) -> torch.Tensor:
+    """Offline: the producer's per-channel parameters divided by s (float32),
+    so that it emits X~ = X diag(s)^-1 and the quantization runs without s.
+    axis "column": channel = column of p (a gain vector, or a producer weight
+    [R,K] in the [in,out] layout); "row": channel = row (a weight stored
+    [K,R]). A 1-D p holds one value per channel."""
+    _cuda(p, s, out)
+    if axis not in ("column", "row"):
+        raise ValueError("axis must be 'column' or 'row'")
+    if p.dim() == 1:
+        rows, cols = (1, p.numel()) if axis == "column" else (p.numel(), 1)
+    elif p.dim() == 2:
+        rows, cols = p.shape
+    else:
+        raise ValueError("p must be 1-D or 2-D")
+    if s.dtype != torch.float32 or s.numel() != (cols if axis == "column" else rows):
+        raise ValueError("s must be float32 with one entry per channel")
+    if out is None:
+        out = torch.empty(p.shape, dtype=torch.float32, device=p.device)
+    elif out.shape != p.shape or out.dtype != torch.float32:
+        raise ValueError("out must be float32 with p's shape")
+    ax = SQ_AMAX_PER_COLUMN if axis == "column" else SQ_AMAX_PER_ROW
+    _check(load().sq_fold_smoothing(_p(p), _fdtype(p), rows, cols, _p(s), ax, _p(out),
+                                    _stream(p.device)), "sq_fold_smoothing")
     return out
 
 
@@ -384,6 +414,7 @@ class SmoothQuantLinear:
         else:
             self.s = self.s_inv = None
             self.wq, self.sw = quantize_weight(w, None, qtype)
+        self.folded_s = None
         self.qtype = qtype
         self.bias = bias
         self.act_scaling = act_scaling
@@ -393,6 +424,20 @@ class SmoothQuantLinear:
             self._amax = torch.zeros(2, dtype=torch.float32, device=w.device)
             self._cur = 0
             quantize_act_tensor(x_cal, self.s, qtype, amax_out=self._amax[0:1], s_inv=self.s_inv)
+
+    def fold_smoothing_into(self, p: torch.Tensor, axis: str = "column") -> torch.Tensor:
+        """Offline: fold this layer's 1/s into the parameters p of the layer
+        that produces its input (see fold_smoothing for the axes) and take the
+        producer's output as already smoothed from then on, so the runtime
+        quantization runs without the division. Returns the folded float32
+        parameters for the producer. A layer folds once; any other
+        parameter of the producer on the same channels (its bias, say) takes
+        fold_smoothing(bias, layer.folded_s)."""
+        if self.s is None:
+            raise RuntimeError("no smoothing factors to fold (smooth=False, or already folded)")
+        out = fold_smoothing(p, self.s, axis)
+        self.folded_s, self.s, self.s_inv = self.s, None, None
+        return out
 
     @property
     def last_amax(self) -> torch.Tensor:
