@@ -494,8 +494,7 @@ def run_ours(args):
             "steps": K_steps, "warmup": args.warmup, "ms_per_step": elapsed_ms / K_steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "i8" if qt == "i8" else "e4m3",
-            "data": "synthetic (seeded N(0,1) activations with 1% outlier channels x U(20,100), "
-                    "N(0,0.02) weights)",
+            "data": f"synthetic, seeded: {case.note}",
             "config": {"workload": case.name, "M": M, "K": K, "N": N,
                        "alpha": case.alpha if case.smooth else None,
                        "act_scaling": ("per-tensor, delayed" if tensor else "per-token"),
@@ -522,7 +521,7 @@ def run_ours(args):
                                "unit": "GB/s", "frac": q_bytes / (t_quant * 1e-3) / 1e9 / pk["hbm"],
                                "traffic": profiled_traffic("quant", case.name),
                                "ms_per_launch": t_quant},
-            "gpu_launches": 2 * K_steps,  # quant_act_stream_kernel + gemm_w8a8_kernel per step
+            "gpu_launches": 2 * K_steps,  # the activation kernel + gemm_w8a8_kernel per step
             "clocks": clocks,
             "e2e": e2e,
             "cpu_baseline": cpu,
