@@ -176,39 +176,51 @@ def _dist():
     return ws, rank, local
 
 
+REF_BUDGET_S = 120.0
+
+
 def run_reference(args):
-    """The reference arm: the CPU oracle, on a bounded sample per step."""
+    """The reference arm: the CPU oracle on the same workload as our arm, a
+    bounded sample of its token rows per step (full K and N)."""
     import oracle
     from w8a8_smoothquant_int8_02_b200 import synth, workloads
 
     ws, rank, _ = _dist()
     if rank != 0:
         return
-    case = workloads.MLP_UP
+    case = workloads.ALL[args.workload]
     d = synth.generate(case)
-    s = oracle.smooth_factors(oracle.amax(d["x_cal"], True), oracle.amax(d["w"], False), case.alpha)
-    wq, sw = oracle.quantize_weight(d["w"], s)
-    rows = max(1, args.ref_rows)
+    s, wq, sw, scale = _oracle_prep(case, d)
+    bias = d["bias"]
+    # one untimed row sizes the per-step sample so that the K steps take
+    # about REF_BUDGET_S seconds at most (at least one row per step)
+    t0 = time.perf_counter()
+    _oracle_runtime(case, np.ascontiguousarray(d["x"][:1]), s, wq, sw, bias, scale)
+    t_row = max(time.perf_counter() - t0, 1e-6)
+    rows = max(1, min(args.ref_rows, case.M, int(REF_BUDGET_S / (args.steps * t_row))))
     xs = np.ascontiguousarray(d["x"][:rows])
-    for _ in range(args.warmup if args.warmup < 1 else 1):
-        oracle.linear(xs, s, wq, sw, d["bias"])
+    _oracle_runtime(case, xs, s, wq, sw, bias, scale)   # warm-up at the sample size
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle.linear(xs, s, wq, sw, d["bias"])
+        _oracle_runtime(case, xs, s, wq, sw, bias, scale)
     dt = time.perf_counter() - t0
     ops = 2.0 * rows * case.N * case.K * args.steps
     val = ops / dt / 1e12
     line = {
-        "impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": ws,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "i8",
-        "data": "synthetic",
+        "impl": "reference", "metric": metric_for(case), "value": val, "unit": UNIT,
+        "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "i8" if case.qtype == "i8" else "e4m3",
+        "data": f"synthetic, seeded: {case.note}",
         "config": {"workload": case.name, "M": case.M, "K": case.K, "N": case.N,
-                   "alpha": case.alpha, "bias": True},
+                   "alpha": case.alpha if case.smooth else None,
+                   "act_scaling": ("per-tensor, delayed" if case.act_scaling == "tensor"
+                                   else "per-token"),
+                   "bias": bias is not None, "out": "bf16"},
         "cpu_baseline": {"value": val, "unit": UNIT, "cores": oracle.num_threads(),
                          "kind": "oracle",
-                         "sample": f"{rows} of {case.M} token rows per step through the whole "
-                                   f"layer (act quant + INT8 GEMM + epilogue), full K and N"},
+                         "sample": f"{rows} of {case.M} token rows per step through the runtime "
+                                   f"path (act quant + 8-bit GEMM + epilogue), full K and N"},
         "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
