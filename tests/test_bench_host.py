@@ -81,3 +81,22 @@ def test_reference_arm_cpu_baseline_on_tiny(bench):
     d2 = synth.generate(small)
     out2 = bench.cpu_baseline(small, d2, budget_s=0.05)
     assert out2["value"] > 0
+
+
+def test_reference_arm_line(bench, capsys, monkeypatch):
+    """--impl reference prints one JSON line for the selected workload with
+    the base contract's keys; ranks other than 0 print nothing."""
+    import argparse
+    import json
+    args = argparse.Namespace(workload="tiny_16x64x64", steps=3, warmup=3, ref_rows=8)
+    bench.run_reference(args)
+    line = json.loads(capsys.readouterr().out.strip())
+    assert line["impl"] == "reference" and line["value"] > 0
+    assert line["metric"] == bench.metric_for(workloads.TINY)
+    assert line["config"]["workload"] == "tiny_16x64x64"
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    bench.run_reference(args)
+    assert capsys.readouterr().out == ""
