@@ -104,6 +104,7 @@ def test_quantize_act_tensor_validation(lib):
     assert call(xq=NUL) == ops.SQ_ERR_INVALID_ARG
     assert call(sx=NUL) == ops.SQ_ERR_INVALID_ARG
     assert call(K=24) == ops.SQ_ERR_INVALID_ARG
+    assert call(K=65536 + 16) == ops.SQ_ERR_INVALID_ARG
     assert call(M=-1) == ops.SQ_ERR_INVALID_ARG
     assert call(xt=ops.SQ_E4M3) == ops.SQ_ERR_INVALID_ARG
     assert call(qt=ops.SQ_F32) == ops.SQ_ERR_INVALID_ARG

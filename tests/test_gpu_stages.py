@@ -100,7 +100,7 @@ def test_quantize_weight(qtype, dtype, smooth, K, N):
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("smooth", [True, False])
 @pytest.mark.parametrize("M,K", [(1, 64), (17, 96), (129, 4096), (16, 8192), (3, 14336), (5, 16),
-                                 (2, 20000)])
+                                 (2, 20000), (2, 65536)])
 def test_quantize_act(qtype, dtype, smooth, M, K):
     x = _x((M, K), seed=M * 31 + K, dtype=dtype)
     s = synth.random_floats(K, seed=K + 1, lo=0.05, hi=20.0) if smooth else None
@@ -237,6 +237,31 @@ def test_gemm_w8a8_extreme_accumulators():
     a = host(acc)
     assert a[0, 0] == K * 127 * 127 and a[1, 0] == -K * 127 * 127 and a[1, 5] == K * 127 * 127
     assert a[0, 7] == 127 and a[1, 7] == -127
+    np.testing.assert_array_equal(a, oracle.gemm_i8(xq, wq))
+
+
+def test_gemm_w8a8_maximum_k():
+    """The largest K the int32 accumulator admits (K * 127^2 < 2^31, K a
+    multiple of 16): all-extreme rows reach +-2,147,350,544 exactly, and the
+    K tail (K mod 128 = 16) is summed."""
+    M, N, K = 3, 16, 133136
+    assert K * 127 * 127 < 2 ** 31 <= (K + 16) * 127 * 127
+    xq = np.full((M, K), 127, np.int8)
+    xq[1] = -127
+    xq[2] = synth.random_matrix((1, K), np.int8, seed=91)[0]
+    wq = np.full((N, K), 127, np.int8)
+    wq[3] = -127
+    wq[4] = synth.random_matrix((1, K), np.int8, seed=92)[0]
+    wq[5] = 0
+    wq[5, K - 1] = 7                   # only the last element of the tail
+    sx = np.ones(M, np.float32)
+    sw = np.ones(N, np.float32)
+    acc = torch.empty((M, N), dtype=torch.int32, device="cuda")
+    ops.gemm_w8a8(dev(xq), dev(sx), dev(wq), dev(sw), out_dtype=torch.float32, acc=acc)
+    assert ops.device_status() == ops.SQ_OK
+    a = host(acc)
+    assert a[0, 0] == K * 127 * 127 and a[1, 0] == -K * 127 * 127 and a[0, 3] == -K * 127 * 127
+    assert a[0, 5] == 7 * 127 and a[1, 5] == -7 * 127
     np.testing.assert_array_equal(a, oracle.gemm_i8(xq, wq))
 
 

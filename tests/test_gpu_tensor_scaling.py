@@ -58,7 +58,8 @@ def _reciprocals(s):
 @pytest.mark.parametrize("qtype", ["i8", "e4m3"])
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 @pytest.mark.parametrize("smooth", [True, False])
-@pytest.mark.parametrize("M,K", [(1, 64), (37, 208), (700, 4096), (16, 8192), (300, 14336)])
+@pytest.mark.parametrize("M,K", [(1, 64), (37, 208), (700, 4096), (16, 8192), (300, 14336),
+                                 (3, 65536)])
 def test_online_and_delayed(qtype, dtype, smooth, M, K):
     x = _x((M, K), seed=M + K, dtype=dtype)
     s = synth.random_floats(K, seed=K + 5, lo=0.05, hi=20.0) if smooth else None
