@@ -262,16 +262,17 @@ def cpu_baseline(case, d, budget_s: float):
     in about `budget_s` seconds."""
     import oracle
     s, wq, sw, scale = _oracle_prep(case, d)
-    rows = 2
-    xs = np.ascontiguousarray(d["x"][:rows])
-    t0 = time.perf_counter()
-    _oracle_runtime(case, xs, s, wq, sw, d["bias"], scale)
-    dt = time.perf_counter() - t0
-    rows2 = int(max(2, min(case.M, rows * budget_s / max(dt, 1e-3))))
-    xs = np.ascontiguousarray(d["x"][:rows2])
-    t0 = time.perf_counter()
-    _oracle_runtime(case, xs, s, wq, sw, d["bias"], scale)
-    dt = time.perf_counter() - t0
+    # grow the sample until it takes about budget_s (a small first sample
+    # underestimates the per-row rate: thread start-up, rows < threads)
+    rows2, dt = 2, 0.0
+    for _ in range(4):
+        xs = np.ascontiguousarray(d["x"][:rows2])
+        t0 = time.perf_counter()
+        _oracle_runtime(case, xs, s, wq, sw, d["bias"], scale)
+        dt = time.perf_counter() - t0
+        if dt >= 0.5 * budget_s or rows2 >= case.M:
+            break
+        rows2 = int(max(rows2 + 1, min(case.M, rows2 * budget_s / max(dt, 1e-3))))
     return {"value": 2.0 * rows2 * case.N * case.K / dt / 1e12, "unit": UNIT,
             "cores": oracle.num_threads(), "kind": "oracle",
             "sample": f"{rows2} of {case.M} token rows through the runtime path (act quant + "
