@@ -49,7 +49,7 @@ def test_activation_kernel_per_workload(bench):
 def test_profiled_traffic_is_guarded_by_the_kernel_source(bench, tmp_path, monkeypatch):
     """Traffic is reported only for a workload that was captured and only
     while the kernel's sources hash as they did at capture time."""
-    assert bench.profiled_traffic("gemm", "decode_16x8192x28672") is None
+    assert bench.profiled_traffic("gemm", "prefill_512x4096x4096") is None
     # a copy of the tree whose GEMM source differs by one byte reports null
     fake = tmp_path / "root"
     csrc = fake / "w8a8_smoothquant_int8_02_b200" / "csrc"
@@ -100,3 +100,18 @@ def test_reference_arm_line(bench, capsys, monkeypatch):
     monkeypatch.setenv("WORLD_SIZE", "2")
     bench.run_reference(args)
     assert capsys.readouterr().out == ""
+
+
+def test_gemm_roofline_bound_follows_the_ridge_point(bench):
+    """The decode shape (few tokens, the weight streamed once) is reported
+    against HBM; the MLP-up and prefill shapes against the tensor peak."""
+    def entry(case):
+        M, K, N = case.M, case.K, case.N
+        nbytes = M * K + N * K + M * N * 2 + 4 * (M + N)
+        return bench.gemm_roofline(case.ops, nbytes, 0.1, 3285.6, 2840.0, 6538.0, None)
+    assert entry(workloads.DECODE)["bound"] == "hbm"
+    assert entry(workloads.DECODE)["unit"] == "GB/s"
+    assert entry(workloads.MLP_UP)["bound"] == "tensor"
+    assert entry(workloads.PREFILL)["bound"] == "tensor"
+    e = entry(workloads.MLP_UP)
+    assert abs(e["frac"] - e["achieved"] / 3285.6) < 1e-12
