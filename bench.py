@@ -68,13 +68,14 @@ PROFILED_TRAFFIC = {
     ("gemm", "mlp_up_4096x4096x14336"): (75.886592e6 + 83.189248e6, "38e67a6ddb8053cd"),
     ("gemm", "fp8_down_4096x14336x4096"): (277.412096e6 + 26.567424e6, "38e67a6ddb8053cd"),
     ("gemm", "fp8_tensor_4096x4096x14336"): (75.913984e6 + 84.172288e6, "38e67a6ddb8053cd"),
-    ("gemm", "decode_16x8192x28672"): (235.188480e6 + 3.869440e6, "38e67a6ddb8053cd"),
     ("quant", "mlp_up_4096x4096x14336"): (33.647616e6 + 0.003072e6, "11715b8dda2dbca9"),
     ("quant", "fp8_down_4096x14336x4096"): (117.746432e6 + 29.849344e6, "11715b8dda2dbca9"),
     ("quant", "fp8_tensor_4096x4096x14336"): (33.578496e6 + 0.003840e6, "11715b8dda2dbca9"),
     ("quant", "decode_16x8192x28672"): (0.362240e6 + 0.0, "11715b8dda2dbca9"),
 }
-KERNEL_SOURCES = {"gemm": ("sq_gemm.cu", "sq_common.cuh"), "quant": ("sq_quant.cu", "sq_common.cuh")}
+KERNEL_SOURCES = {"gemm": ("sq_gemm.cu", "sq_common.cuh"),
+                  "gemm_skinny": ("sq_gemm_skinny.cu", "sq_common.cuh"),
+                  "quant": ("sq_quant.cu", "sq_common.cuh")}
 
 
 def profiled_traffic(kind, workload):
@@ -82,7 +83,7 @@ def profiled_traffic(kind, workload):
     workload or the kernel's sources changed since (or a tile is forced)."""
     import hashlib
     entry = PROFILED_TRAFFIC.get((kind, workload))
-    if entry is None or (kind == "gemm" and os.environ.get("SQ_GEMM_TILE")):
+    if entry is None or (kind.startswith("gemm") and os.environ.get("SQ_GEMM_TILE")):
         return None
     h = hashlib.sha256()
     for f in KERNEL_SOURCES[kind]:
@@ -91,24 +92,34 @@ def profiled_traffic(kind, workload):
     return entry[0] if h.hexdigest()[:16] == entry[1] else None
 
 
-def gemm_roofline(ops, nbytes, ms, tops_peak, tops_peak_sus, hbm_gbs, traffic):
+def gemm_roofline(ops, nbytes, ms, tops_peak, tops_peak_sus, hbm_gbs, traffic,
+                  kernel="gemm_w8a8_kernel"):
     """The GEMM's roofline entry: against the 8-bit tensor peak when its
     arithmetic intensity (ops per compulsory byte) is above the ridge point
     of the two measured peaks, else against HBM bandwidth (the few-token
     decode shape, which streams the weight once)."""
     if ops / nbytes >= tops_peak * 1e12 / (hbm_gbs * 1e9):
         tops = ops / (ms * 1e-3) / 1e12
-        return {"bound": "tensor", "kernel": "gemm_w8a8_kernel", "achieved": tops,
+        return {"bound": "tensor", "kernel": kernel, "achieved": tops,
                 "peak": tops_peak, "unit": "TFLOP/s", "frac": tops / tops_peak,
                 "frac_of_sustained": tops / tops_peak_sus,
                 "ops_note": "INT8 multiply-add counted as 2 ops; peak = 2 x measured bf16 dense "
                             "(burst)",
                 "traffic": traffic, "ms_per_launch": ms}
     gbs = nbytes / (ms * 1e-3) / 1e9
-    return {"bound": "hbm", "kernel": "gemm_w8a8_kernel", "achieved": gbs, "peak": hbm_gbs,
+    return {"bound": "hbm", "kernel": kernel, "achieved": gbs, "peak": hbm_gbs,
             "unit": "GB/s", "frac": gbs / hbm_gbs,
             "bytes_note": "compulsory bytes: Xq + Wq read once, Y written, scales and bias",
             "traffic": traffic, "ms_per_launch": ms}
+
+
+def gemm_kind(case, forced_tile=None):
+    """Which GEMM kernel the library runs for this workload: the
+    weight-streaming form for at most 16 tokens (unless a tile shape is
+    forced), else the tiled kernel. Returns (traffic key, kernel name)."""
+    if case.M <= 16 and not forced_tile:
+        return "gemm_skinny", "gemm_skinny_kernel"
+    return "gemm", "gemm_w8a8_kernel"
 
 
 def quant_kernel_name(case):
@@ -517,6 +528,7 @@ def run_ours(args):
 
     if rank == 0:
         pk = _peaks()
+        g_kind, g_name = gemm_kind(case, os.environ.get("SQ_GEMM_TILE"))
         int8_peak = 2.0 * pk["bf16"]        # dense INT8 / FP8 = 2x dense bf16 (4.5 vs 2.25 P)
         int8_peak_sus = 2.0 * pk["bf16_sus"]
         gemm_tops = case.ops / (t_gemm * 1e-3) / 1e12
@@ -545,13 +557,13 @@ def run_ours(args):
             "int8_peak_source": f"2 x {pk['src']} bf16 dense ({pk['bf16']} TFLOP/s burst)",
             "gemm_hbm_gbs": g_bytes / (t_gemm * 1e-3) / 1e9,
             "roofline": gemm_roofline(case.ops, g_bytes, t_gemm, int8_peak, int8_peak_sus,
-                                      pk["hbm"], profiled_traffic("gemm", case.name)),
+                                      pk["hbm"], profiled_traffic(g_kind, case.name), g_name),
             "roofline_quant": {"bound": "hbm", "kernel": quant_kernel_name(case),
                                "achieved": q_bytes / (t_quant * 1e-3) / 1e9, "peak": pk["hbm"],
                                "unit": "GB/s", "frac": q_bytes / (t_quant * 1e-3) / 1e9 / pk["hbm"],
                                "traffic": profiled_traffic("quant", case.name),
                                "ms_per_launch": t_quant},
-            "gpu_launches": 2 * K_steps,  # the activation kernel + gemm_w8a8_kernel per step
+            "gpu_launches": 2 * K_steps,  # the activation kernel + the GEMM per step
             "clocks": clocks,
             "e2e": e2e,
             "cpu_baseline": cpu,

@@ -115,3 +115,13 @@ def test_gemm_roofline_bound_follows_the_ridge_point(bench):
     assert entry(workloads.PREFILL)["bound"] == "tensor"
     e = entry(workloads.MLP_UP)
     assert abs(e["frac"] - e["achieved"] / 3285.6) < 1e-12
+
+
+def test_gemm_kernel_per_workload(bench):
+    """At most 16 tokens run the weight-streaming kernel unless a tile shape
+    is forced; every other workload the tiled kernel."""
+    assert bench.gemm_kind(workloads.DECODE) == ("gemm_skinny", "gemm_skinny_kernel")
+    assert bench.gemm_kind(workloads.TINY) == ("gemm_skinny", "gemm_skinny_kernel")
+    assert bench.gemm_kind(workloads.DECODE, "c1n224") == ("gemm", "gemm_w8a8_kernel")
+    assert bench.gemm_kind(workloads.MLP_UP) == ("gemm", "gemm_w8a8_kernel")
+    assert bench.gemm_kind(workloads.PREFILL) == ("gemm", "gemm_w8a8_kernel")

@@ -13,7 +13,7 @@ import torch
 import oracle
 from w8a8_smoothquant_int8_02_b200 import ops, synth
 
-from _gpu_util import dev, fp8_normalized_error, host, ulp_distance
+from _gpu_util import dev, fp8_normalized_error, host, sample_points, ulp_distance
 
 pytestmark = pytest.mark.gpu
 
@@ -306,6 +306,81 @@ def test_gemm_fp8(M, N, K, with_bias):
     # the bf16 output is the nearest-even rounding of the same binary32 values
     # (the tensor-core summation order is fixed for a given launch shape)
     np.testing.assert_array_equal(host(yb), oracle.f32_to_bf16(host(yf)))
+
+
+# ------------------------------------------- few tokens: weight streaming --
+
+SKINNY_SHAPES = [(1, 8, 16), (5, 136, 1040), (16, 1000, 208), (16, 4096, 8192), (3, 28672, 256)]
+
+
+@pytest.mark.parametrize("M,N,K", SKINNY_SHAPES)
+@pytest.mark.parametrize("with_bias", [False, True])
+def test_gemm_few_tokens_int8(M, N, K, with_bias, monkeypatch):
+    """M <= 16 runs the weight-streaming kernel (operand roles swapped): int32
+    accumulators, binary32 and bf16 outputs bit for bit against the oracle
+    and against the tiled kernel forced on the same inputs."""
+    xq = synth.random_matrix((M, K), np.int8, seed=M + 3 * K)
+    wq = synth.random_matrix((N, K), np.int8, seed=N + 5 * K)
+    xq[0, :8] = 127
+    wq[:, :8] = -127
+    sx = synth.random_floats(M, seed=31, lo=1e-3, hi=0.5)
+    sw = synth.random_floats(N, seed=32, lo=1e-4, hi=1e-2)
+    bias = synth.to_bf16_bits(synth.random_floats(N, seed=33, std=0.1)) if with_bias else None
+    acc_ref = oracle.gemm_i8(xq, wq)
+    yf_ref, yb_ref = oracle.epilogue(acc_ref, sx, sw, bias)
+    d = [dev(a) for a in (xq, sx, wq, sw)]
+    b = None if bias is None else dev(bias)
+    acc = torch.empty((M, N), dtype=torch.int32, device="cuda")
+    yf = ops.gemm_w8a8(*d, bias=b, out_dtype=torch.float32, acc=acc)
+    yb = ops.gemm_w8a8(*d, bias=b, out_dtype=torch.bfloat16)
+    yn = ops.gemm_w8a8_noalloc(*d, bias=b)
+    assert ops.device_status() == ops.SQ_OK
+    np.testing.assert_array_equal(host(acc), acc_ref)
+    np.testing.assert_array_equal(host(yf), yf_ref)
+    np.testing.assert_array_equal(host(yb), yb_ref)
+    np.testing.assert_array_equal(host(yn), yb_ref)
+    monkeypatch.setenv("SQ_GEMM_TILE", "c1n128")
+    yt = ops.gemm_w8a8(*d, bias=b, out_dtype=torch.bfloat16)
+    assert torch.equal(yt.view(torch.int16), yb.view(torch.int16))
+
+
+@pytest.mark.parametrize("M,N,K", SKINNY_SHAPES)
+def test_gemm_few_tokens_fp8(M, N, K):
+    g = np.random.default_rng(M * 7 + N + K)
+    mag = np.abs(oracle.e4m3_decode(E4M3_FINITE))
+    codes = E4M3_FINITE[(mag <= 64.0)]
+    xq = g.choice(codes, size=(M, K)).astype(np.uint8)
+    wq = g.choice(codes, size=(N, K)).astype(np.uint8)
+    sx = synth.random_floats(M, seed=34, lo=1e-3, hi=0.5)
+    sw = synth.random_floats(N, seed=35, lo=1e-4, hi=1e-2)
+    bias = synth.to_bf16_bits(synth.random_floats(N, seed=36, std=0.1))
+    yf_ref, _ = oracle.epilogue(oracle.gemm_e4m3(xq, wq), sx, sw, bias)
+    yf = ops.gemm_fp8(dev(xq), dev(sx), dev(wq), dev(sw), bias=dev(bias), out_dtype=torch.float32)
+    yb = ops.gemm_fp8(dev(xq), dev(sx), dev(wq), dev(sw), bias=dev(bias))
+    assert ops.device_status() == ops.SQ_OK
+    if M * N <= 50000:
+        rows, cols = np.divmod(np.arange(M * N, dtype=np.int64), N)
+    else:
+        rows, cols = sample_points(M, N, seed=37)
+    yfh = host(yf)
+    e = fp8_normalized_error(yfh[rows, cols], yf_ref[rows, cols], xq, wq, sx, sw, bias, rows, cols)
+    assert e.max() <= 1e-3, e.max()
+    np.testing.assert_array_equal(host(yb), oracle.f32_to_bf16(yfh))
+
+
+def test_gemm_few_tokens_does_not_write_outside_output():
+    M, N, K = 7, 200, 96
+    xq = synth.random_matrix((M, K), np.int8, seed=41)
+    wq = synth.random_matrix((N, K), np.int8, seed=42)
+    sx = synth.random_floats(M, seed=43, lo=0.01, hi=0.1)
+    sw = synth.random_floats(N, seed=44, lo=0.01, hi=0.1)
+    guard = 4096
+    buf = torch.full((M * N + 2 * guard,), -7777.0, dtype=torch.float32, device="cuda")
+    out = buf[guard:guard + M * N].view(M, N)
+    ops.gemm_w8a8(dev(xq), dev(sx), dev(wq), dev(sw), out=out)
+    h = host(buf)
+    assert (h[:guard] == -7777.0).all() and (h[guard + M * N:] == -7777.0).all()
+    np.testing.assert_array_equal(host(out), oracle.epilogue(oracle.gemm_i8(xq, wq), sx, sw)[0])
 
 
 # --------------------------------------------------------- the whole layer --

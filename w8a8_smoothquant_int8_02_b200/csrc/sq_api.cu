@@ -65,6 +65,18 @@ sq_status check_gemm(const void* xq, const float* sx, const void* wq, const floa
   return SQ_OK;
 }
 
+// Few tokens (M <= 16) take the weight-streaming form with the operand roles
+// swapped (sq_gemm_skinny.cu, same results, no workspace); SQ_GEMM_TILE or
+// SQ_GEMM_NO_SKINNY in the environment keep the tiled kernel for every M.
+cudaError_t run_gemm_any(bool e4m3, const uint8_t* xq, const float* sx, const uint8_t* wq,
+                         const float* sw, const uint16_t* bias, int64_t M, int64_t N, int64_t K,
+                         void* y, sqh::OutKind yk, int32_t* acc, void* ws, size_t ws_bytes,
+                         cudaStream_t st) {
+  if (sqh::gemm_skinny_applies(M))
+    return sqh::launch_gemm_skinny(e4m3, xq, sx, wq, sw, bias, M, N, K, y, yk, acc, st);
+  return sqh::launch_gemm(e4m3, xq, sx, wq, sw, bias, M, N, K, y, yk, acc, ws, ws_bytes, st);
+}
+
 // ---------------------------------------------------------------------------
 // Scratch of the allocation-free GEMM entry point (sq_gemm_w8a8_noalloc):
 // a fixed array in the library's own device image, so the call allocates
@@ -219,7 +231,7 @@ sq_status sq_gemm_w8a8(const int8_t* xq, const float* sx, const int8_t* wq, cons
   if (c != SQ_OK) return c;
   if (M == 0) return SQ_OK;
   if (workspace && !al(workspace, 256)) return SQ_ERR_MISALIGNED;
-  return from_cuda(sqh::launch_gemm(false, reinterpret_cast<const uint8_t*>(xq), sx,
+  return from_cuda(run_gemm_any(false, reinterpret_cast<const uint8_t*>(xq), sx,
                                     reinterpret_cast<const uint8_t*>(wq), sw, bias, M, N, K, y,
                                     yt == SQ_BF16 ? sqh::OutKind::BF16 : sqh::OutKind::F32, acc,
                                     workspace, workspace_bytes, S(stream)));
@@ -232,7 +244,7 @@ sq_status sq_gemm_fp8(const uint8_t* xq, const float* sx, const uint8_t* wq, con
   if (c != SQ_OK) return c;
   if (M == 0) return SQ_OK;
   if (workspace && !al(workspace, 256)) return SQ_ERR_MISALIGNED;
-  return from_cuda(sqh::launch_gemm(true, xq, sx, wq, sw, bias, M, N, K, y,
+  return from_cuda(run_gemm_any(true, xq, sx, wq, sw, bias, M, N, K, y,
                                     yt == SQ_BF16 ? sqh::OutKind::BF16 : sqh::OutKind::F32, nullptr,
                                     workspace, workspace_bytes, S(stream)));
 }
@@ -260,6 +272,13 @@ sq_status sq_gemm_w8a8_noalloc(const int8_t* xq, const float* sx, const int8_t* 
   sq_status c = check_gemm(xq, sx, wq, sw, bias, M, N, K, y, yt, nullptr);
   if (c != SQ_OK) return c;
   if (M == 0) return SQ_OK;
+  if (sqh::gemm_skinny_applies(M))  // the few-token form uses no scratch
+    return from_cuda(sqh::launch_gemm_skinny(false, reinterpret_cast<const uint8_t*>(xq), sx,
+                                             reinterpret_cast<const uint8_t*>(wq), sw, bias, M,
+                                             N, K, y,
+                                             yt == SQ_BF16 ? sqh::OutKind::BF16
+                                                           : sqh::OutKind::F32,
+                                             nullptr, S(stream)));
   // the split-tile scratch this device needs must fit the fixed array
   if (sqh::gemm_workspace_bytes() > kNoAllocScratchBytes) return SQ_ERR_SCRATCH_TOO_SMALL;
   void* scratch = noalloc_scratch_ptr();
@@ -268,7 +287,7 @@ sq_status sq_gemm_w8a8_noalloc(const int8_t* xq, const float* sx, const int8_t* 
   // tiles synchronize on must start at zero
   if (cudaMemsetAsync(scratch, 0, sqh::gemm_workspace_counter_bytes(), S(stream)) != cudaSuccess)
     return SQ_ERR_CUDA;
-  return from_cuda(sqh::launch_gemm(false, reinterpret_cast<const uint8_t*>(xq), sx,
+  return from_cuda(run_gemm_any(false, reinterpret_cast<const uint8_t*>(xq), sx,
                                     reinterpret_cast<const uint8_t*>(wq), sw, bias, M, N, K, y,
                                     yt == SQ_BF16 ? sqh::OutKind::BF16 : sqh::OutKind::F32, nullptr,
                                     scratch, kNoAllocScratchBytes, S(stream)));

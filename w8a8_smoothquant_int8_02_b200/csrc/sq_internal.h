@@ -39,6 +39,11 @@ cudaError_t launch_gemm(bool e4m3, const uint8_t* xq, const float* sx, const uin
                         const float* sw, const uint16_t* bias, int64_t M, int64_t N, int64_t K,
                         void* y, OutKind yk, int32_t* acc, void* ws, size_t ws_bytes,
                         cudaStream_t st);
+// a6 / a7 for M <= 16: the weight-streaming form (sq_gemm_skinny.cu)
+bool gemm_skinny_applies(int64_t M);
+cudaError_t launch_gemm_skinny(bool e4m3, const uint8_t* xq, const float* sx, const uint8_t* wq,
+                               const float* sw, const uint16_t* bias, int64_t M, int64_t N,
+                               int64_t K, void* y, OutKind yk, int32_t* acc, cudaStream_t st);
 size_t gemm_workspace_bytes();
 size_t gemm_workspace_counter_bytes();
 
