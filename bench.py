@@ -68,6 +68,7 @@ PROFILED_TRAFFIC = {
     ("gemm", "mlp_up_4096x4096x14336"): (75.886592e6 + 83.189248e6, "38e67a6ddb8053cd"),
     ("gemm", "fp8_down_4096x14336x4096"): (277.412096e6 + 26.567424e6, "38e67a6ddb8053cd"),
     ("gemm", "fp8_tensor_4096x4096x14336"): (75.913984e6 + 84.172288e6, "38e67a6ddb8053cd"),
+    ("gemm_skinny", "decode_16x8192x28672"): (235.154432e6 + 4.865280e6, "c40f47cedac0f9ac"),
     ("quant", "mlp_up_4096x4096x14336"): (33.647616e6 + 0.003072e6, "11715b8dda2dbca9"),
     ("quant", "fp8_down_4096x14336x4096"): (117.746432e6 + 29.849344e6, "11715b8dda2dbca9"),
     ("quant", "fp8_tensor_4096x4096x14336"): (33.578496e6 + 0.003840e6, "11715b8dda2dbca9"),
