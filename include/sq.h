@@ -246,6 +246,11 @@ size_t sq_gemm_workspace_bytes(void);
  * acc[m,n] = sum_k xq[m,k]*wq[n,k] (exact in int32 for K < 133144);
  * t = float(acc) (nearest-even); t = t*sx[m]; t = t*sw[n]; t = t + bias[n];
  * y = t (SQ_F32) or bf16(t) rounded to nearest-even (SQ_BF16).
+ * Kernels: M <= 16 runs a weight-streaming kernel (the weight rows are the
+ * 128-row tensor-core operand, the tokens a 16-column one; no workspace),
+ * every other M the tiled kernel. Results are the same either way. Setting
+ * SQ_GEMM_NO_SKINNY or SQ_GEMM_TILE in the environment keeps the tiled
+ * kernel for every M.
  */
 sq_status sq_gemm_w8a8(const int8_t* xq, const float* sx, const int8_t* wq,
                        const float* sw, const uint16_t* bias, int64_t M,
