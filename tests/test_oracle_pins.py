@@ -321,6 +321,39 @@ def test_act_quant_zero_row_and_no_smoothing():
     np.testing.assert_array_equal(sx, sx1)
 
 
+def test_scale_that_underflows_to_zero_gives_zero_codes():
+    """A row / column whose amax / Q underflows to a zero scale (amax a few
+    subnormal steps) is stored with scale 0 and all codes 0, although its
+    elements are not zero; dividing by that zero scale would give +-inf and
+    saturated codes instead."""
+    tiny = np.float32(2.0 ** -147)          # amax / 127 rounds to 0 in binary32
+    assert np.float32(tiny / np.float32(127.0)) == 0 and tiny > 0
+    x = np.zeros((2, 16), np.float32)
+    x[0, 3], x[0, 9] = tiny, -tiny
+    x[1] = 1.0
+    for qt in (oracle.INT8, oracle.E4M3):
+        xq, sx = oracle.quantize_act(x, None, qt)
+        assert sx[0] == 0 and not xq[0].view(np.uint8).any(), qt
+        assert sx[1] > 0
+        wq, sw = oracle.quantize_weight(np.ascontiguousarray(x.T), None, qt)
+        assert sw[0] == 0 and not wq[0].view(np.uint8).any(), qt
+
+
+def test_quantize_weight_e4m3_scale_and_extreme():
+    """E4M3 weights: sw[n] = amax_n / 448 and the largest element of each
+    output channel is stored as +-448 (code 0x7E / 0xFE)."""
+    K, N = 32, 24
+    rng = np.random.default_rng(14)
+    w = (rng.standard_normal((K, N)) * 0.02).astype(np.float32)
+    w[5, 7] = -0.5
+    wq, sw = oracle.quantize_weight(w, None, oracle.E4M3)
+    amax = np.abs(w).max(axis=0)
+    np.testing.assert_array_equal(sw, (amax / np.float32(448.0)).astype(np.float32))
+    assert wq[7, 5] == 0xFE
+    top = np.abs(w).argmax(axis=0)
+    assert np.all((wq[np.arange(N), top] & 0x7F) == 0x7E)
+
+
 def test_act_quant_e4m3_bound():
     rng = np.random.default_rng(13)
     x = (rng.standard_normal((8, 64)) * 5).astype(np.float32)
