@@ -81,6 +81,11 @@ MUTANTS = [
     ("e4m3_gemm_uses_x_twice",
      "a += table[xq[m * K + k]] * table[wq[n * K + k]];",
      "a += table[xq[m * K + k]] * table[xq[m * K + k]];"),
+    ("sampled_int8_output_wrong_sign",
+     "d += (int32_t)xr[k] * (int32_t)wr[k];", "d -= (int32_t)xr[k] * (int32_t)wr[k];"),
+    ("sampled_e4m3_output_uses_w_twice",
+     "for (int64_t k = 0; k < K; ++k) d += table[xr[k]] * table[wr[k]];",
+     "for (int64_t k = 0; k < K; ++k) d += table[wr[k]] * table[wr[k]];"),
     ("epilogue_drops_the_bias",
      "if (has_bias) t = t + sqo_bf16_to_f32(bias_bf16);", "if (has_bias) t = t + 0.0f;"),
     ("epilogue_skips_the_channel_scale", "    t = t * sw_n;\n", "\n"),

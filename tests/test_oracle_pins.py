@@ -436,18 +436,21 @@ def test_epilogue_relative_error_bound():
     assert np.all(np.abs(yf - exact) <= 3.01 * 2.0 ** -24 * np.abs(exact))
 
 
-def test_linear_at_matches_full_path():
+@pytest.mark.parametrize("qt", [oracle.INT8, oracle.E4M3])
+def test_linear_at_matches_full_path(qt):
+    """The sampled-output function the full-size GPU tests use equals the
+    full product at the sampled points, for both code types."""
     case = workloads.TINY
     d = synth.generate(case)
     ax = oracle.amax(d["x_cal"], True)
     aw = oracle.amax(d["w"], False)
     s = oracle.smooth_factors(ax, aw, case.alpha)
-    wq, sw = oracle.quantize_weight(d["w"], s)
+    wq, sw = oracle.quantize_weight(d["w"], s, qt)
     bias = synth.to_bf16_bits(synth.random_floats(case.N, seed=4, std=0.1))
-    full = oracle.linear(d["x"], s, wq, sw, bias)
-    rows = np.array([0, 3, 15, 8], np.int64)
-    cols = np.array([0, 63, 41, 7], np.int64)
-    acc, yf, yb = oracle.linear_at(full["xq"], full["sx"], wq, sw, bias, rows, cols)
+    full = oracle.linear(d["x"], s, wq, sw, bias, qt)
+    rows = np.array([0, 3, 15, 8, 2, 9], np.int64)
+    cols = np.array([0, 63, 41, 7, 3, 12], np.int64)
+    acc, yf, yb = oracle.linear_at(full["xq"], full["sx"], wq, sw, bias, rows, cols, qt)
     np.testing.assert_array_equal(acc, full["acc"][rows, cols].astype(np.float64))
     np.testing.assert_array_equal(yf, full["y_f32"][rows, cols])
     np.testing.assert_array_equal(yb, full["y_bf16"][rows, cols])
