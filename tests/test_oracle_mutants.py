@@ -103,6 +103,26 @@ MUTANTS = [
      "ldexp((double)m, -9)", "ldexp((double)m, -10)"),
     ("e4m3_exponent_bias_wrong",
      "ldexp((double)(8 + m), e - 10)", "ldexp((double)(8 + m), e - 11)"),
+    ("column_amax_starts_at_one",
+     "for (int64_t c = 0; c < cols; ++c) out[c] = 0.0f;",
+     "for (int64_t c = 0; c < cols; ++c) out[c] = 1.0f;"),
+    ("act_e4m3_codes_multiply_by_the_scale",
+     "float scale = amax / qmax;\n        sx[m] = scale;\n        for (int64_t k = 0; k < K; ++k) {\n            float v = load_elem(x, dtype, m * K + k);\n            float xs = s ? smooth_x(v, s[k]) : v;\n            if (qtype == 1) {\n                ((uint8_t*)xq)[m * K + k] =\n                    (scale == 0.0f) ? 0 : sqo_e4m3_encode_rn_sat(xs / scale);",
+     "float scale = amax / qmax;\n        sx[m] = scale;\n        for (int64_t k = 0; k < K; ++k) {\n            float v = load_elem(x, dtype, m * K + k);\n            float xs = s ? smooth_x(v, s[k]) : v;\n            if (qtype == 1) {\n                ((uint8_t*)xq)[m * K + k] =\n                    (scale == 0.0f) ? 0 : sqo_e4m3_encode_rn_sat(xs * scale);"),
+    ("weight_e4m3_codes_unscaled",
+     "(scale == 0.0f) ? 0 : sqo_e4m3_encode_rn_sat(wt / scale);",
+     "(scale == 0.0f) ? 0 : sqo_e4m3_encode_rn_sat(wt);"),
+    ("e4m3_sign_dropped",
+     "uint8_t sign = signbit(x) ? 0x80 : 0x00;", "uint8_t sign = 0x00;"),
+    ("per_tensor_max_of_unsmoothed_values",
+     "float a = fabsf(xs);\n        if (a > amax) amax = a;\n    }\n    *amax_out = amax;",
+     "float a = fabsf(v);\n        if (a > amax) amax = a;\n    }\n    *amax_out = amax;"),
+    ("per_tensor_reports_the_scale_as_max",
+     "*amax_out = amax;", "*amax_out = amax / qmax;"),
+    ("bf16_widening_shifted_wrong",
+     "return bits_f32((uint32_t)h << 16);", "return bits_f32((uint32_t)h << 15);"),
+    ("fold_reads_the_transpose",
+     "smooth_x(load_elem(p, dtype, r * cols + c),", "smooth_x(load_elem(p, dtype, c * rows + r),"),
     ("fold_multiplies",
      "out[r * cols + c] = smooth_x(load_elem(p, dtype, r * cols + c),",
      "out[r * cols + c] = smooth_w(load_elem(p, dtype, r * cols + c),"),

@@ -269,6 +269,19 @@ def test_amax_axes(dtype):
     np.testing.assert_array_equal(oracle.amax(src, False), np.abs(xf).max(axis=1))
 
 
+def test_amax_of_small_and_zero_channels():
+    """Channels whose values all lie below 1 in magnitude, and all-zero ones,
+    along both axes (a calibration scaled like layer activations after a
+    normalization)."""
+    rng = np.random.default_rng(15)
+    x = (rng.uniform(-1, 1, (9, 24)) * 1e-3).astype(np.float32)
+    x[:, 4] = 0.0
+    x[6] = 0.0
+    np.testing.assert_array_equal(oracle.amax(x, True), np.abs(x).max(axis=0))
+    np.testing.assert_array_equal(oracle.amax(x, False), np.abs(x).max(axis=1))
+    assert oracle.amax(x, True)[4] == 0 and oracle.amax(x, False)[6] == 0
+
+
 def test_quantize_weight_layout_and_scale():
     K, N = 48, 40
     w = np.full((K, N), 0.001, np.float32)
