@@ -114,11 +114,14 @@ def gemm_roofline(ops, nbytes, ms, tops_peak, tops_peak_sus, hbm_gbs, traffic,
             "traffic": traffic, "ms_per_launch": ms}
 
 
+SKINNY_MAX_M = 16  # the library's weight-streaming GEMM takes M <= 16 (sq_gemm_skinny.cu)
+
+
 def gemm_kind(case, forced_tile=None):
     """Which GEMM kernel the library runs for this workload: the
     weight-streaming form for at most 16 tokens (unless a tile shape is
     forced), else the tiled kernel. Returns (traffic key, kernel name)."""
-    if case.M <= 16 and not forced_tile:
+    if case.M <= SKINNY_MAX_M and not forced_tile:
         return "gemm_skinny", "gemm_skinny_kernel"
     return "gemm", "gemm_w8a8_kernel"
 

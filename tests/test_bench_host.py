@@ -125,3 +125,17 @@ def test_gemm_kernel_per_workload(bench):
     assert bench.gemm_kind(workloads.DECODE, "c1n224") == ("gemm", "gemm_w8a8_kernel")
     assert bench.gemm_kind(workloads.MLP_UP) == ("gemm", "gemm_w8a8_kernel")
     assert bench.gemm_kind(workloads.PREFILL) == ("gemm", "gemm_w8a8_kernel")
+
+
+def test_few_token_threshold_matches_the_library(bench):
+    """bench.py names the kernel by the same token threshold the library
+    dispatches on."""
+    import re
+    src = open(os.path.join(ROOT, "w8a8_smoothquant_int8_02_b200", "csrc",
+                            "sq_gemm_skinny.cu")).read()
+    mp = int(re.search(r"constexpr int kSkMP = (\d+);", src).group(1))
+    assert mp == bench.SKINNY_MAX_M
+    from w8a8_smoothquant_int8_02_b200 import synth
+    at = workloads.DECODE.__dict__
+    assert bench.gemm_kind(synth.LinearCase(**{**at, "M": mp}))[0] == "gemm_skinny"
+    assert bench.gemm_kind(synth.LinearCase(**{**at, "M": mp + 1}))[0] == "gemm"
