@@ -60,3 +60,11 @@ def test_non_contiguous_tensors_are_rejected():
     assert not x.is_contiguous()
     with pytest.raises(ValueError):
         ops._cuda(x)
+
+
+def test_missing_library_raises(monkeypatch, tmp_path):
+    """Without libsq.so the binding raises instead of computing anything."""
+    monkeypatch.setattr(ops, "_lib", None)
+    monkeypatch.setattr(ops._build, "LIB", str(tmp_path / "libsq.so"))
+    with pytest.raises(RuntimeError, match="libsq.so not found"):
+        ops.load(build_if_needed=False)
