@@ -139,3 +139,24 @@ def test_few_token_threshold_matches_the_library(bench):
     at = workloads.DECODE.__dict__
     assert bench.gemm_kind(synth.LinearCase(**{**at, "M": mp}))[0] == "gemm_skinny"
     assert bench.gemm_kind(synth.LinearCase(**{**at, "M": mp + 1}))[0] == "gemm"
+
+
+def test_bench_line_carries_every_contract_key():
+    """The JSON line bench.py prints (the dict literal in run_ours and the
+    one in run_reference) names every key of the measurement contract."""
+    import ast
+    tree = ast.parse(open(os.path.join(ROOT, "bench.py")).read())
+    required = {"metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "cpu_baseline", "e2e"}
+    found = {}
+    for fn in (n for n in tree.body if isinstance(n, ast.FunctionDef)
+               and n.name in ("run_ours", "run_reference")):
+        for node in ast.walk(fn):
+            if isinstance(node, ast.Assign) and any(getattr(t, "id", None) == "line"
+                                                    for t in node.targets):
+                assert isinstance(node.value, ast.Dict)
+                found[fn.name] = {k.value for k in node.value.keys
+                                  if isinstance(k, ast.Constant)}
+    assert required | {"roofline", "clocks", "gpu_launches"} <= found["run_ours"]
+    assert required | {"impl"} <= found["run_reference"]
