@@ -43,6 +43,10 @@ MUTANTS = [
     ("epsilon_clamp_dropped",
      "double ax = (double)amax_x[k] > eps ? (double)amax_x[k] : eps;",
      "double ax = (double)amax_x[k];"),
+    ("epsilon_too_small", "const double eps = 1e-5;", "const double eps = 1e-6;"),
+    ("weight_epsilon_clamp_dropped",
+     "double aw = (double)amax_w[k] > eps ? (double)amax_w[k] : eps;",
+     "double aw = (double)amax_w[k];"),
     ("column_amax_without_abs",
      "float a = fabsf(load_elem(x, dtype, r * cols + c));\n                if (a > out[c])",
      "float a = load_elem(x, dtype, r * cols + c);\n                if (a > out[c])"),
