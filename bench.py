@@ -323,6 +323,10 @@ def run_ours(args):
     from w8a8_smoothquant_int8_02_b200 import dist as sqdist, ops, synth, workloads
 
     ws, rank, local = _dist()
+    if args.gpus != ws:
+        raise SystemExit(f"--gpus {args.gpus} but {ws} process(es): launch N > 1 GPUs with "
+                         f"python -m torch.distributed.run --nproc-per-node {args.gpus} bench.py "
+                         f"--gpus {args.gpus}")
     if args.tile:
         os.environ["SQ_GEMM_TILE"] = args.tile
     torch.cuda.set_device(local)
@@ -593,7 +597,7 @@ def main():
     ap.add_argument("--no-graph", action="store_true",
                     help="launch the timed steps one by one instead of replaying a CUDA graph")
     ap.add_argument("--workload", default="mlp_up_4096x4096x14336",
-                    help="one of the five workloads (default: the MLP up-projection)")
+                    help="one of the six workloads in workloads.py (default: the MLP up-projection)")
     ap.add_argument("--tile", default=None, help="force a GEMM tile shape (c1n128, c1n224, c1n256, "
                     "c2n224, c2n256); default: chosen by problem size")
     args = ap.parse_args()

@@ -160,3 +160,12 @@ def test_bench_line_carries_every_contract_key():
                                   if isinstance(k, ast.Constant)}
     assert required | {"roofline", "clocks", "gpu_launches"} <= found["run_ours"]
     assert required | {"impl"} <= found["run_reference"]
+
+
+def test_gpu_count_must_match_the_process_count(bench, monkeypatch):
+    """--gpus N without N processes stops before touching a GPU."""
+    import argparse
+    monkeypatch.delenv("WORLD_SIZE", raising=False)
+    args = argparse.Namespace(gpus=2, tile=None, workload="tiny_16x64x64")
+    with pytest.raises(SystemExit, match="torch.distributed.run"):
+        bench.run_ours(args)
