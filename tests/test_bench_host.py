@@ -169,3 +169,11 @@ def test_gpu_count_must_match_the_process_count(bench, monkeypatch):
     args = argparse.Namespace(gpus=2, tile=None, workload="tiny_16x64x64")
     with pytest.raises(SystemExit, match="torch.distributed.run"):
         bench.run_ours(args)
+    # one GPU, one process: the check passes (and, without a GPU here, the
+    # first CUDA call is what stops it)
+    import torch
+    if not torch.cuda.is_available():
+        args.gpus = 1
+        with pytest.raises(Exception) as exc:
+            bench.run_ours(args)
+        assert not isinstance(exc.value, SystemExit)
