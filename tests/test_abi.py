@@ -195,3 +195,20 @@ def test_smooth_factor_and_calibration_validation(lib):
     assert lin(c(A), ops.SQ_BF16, None, None, c(A), c(A), None, ops.SQ_I8, 0, 64, 64, c(A), c(A),
                c(A), ops.SQ_BF16, None, 0, None) == ops.SQ_OK
     assert lib.sq_probe_wait_timeout(10, None) == ops.SQ_ERR_INVALID_ARG
+
+
+def test_abi_from_plain_c(tmp_path):
+    """include/sq.h compiles as C11 and libsq.so links and answers from a C
+    program (tests/c/abi_from_c.c): validation failures, empty no-ops and
+    the version, no GPU touched."""
+    import subprocess
+    lib = ops.library_path()
+    exe = tmp_path / "abi_from_c"
+    src = os.path.join(ROOT, "tests", "c", "abi_from_c.c")
+    subprocess.run(["gcc", "-std=c11", "-Wall", "-Wextra", "-Werror", "-I",
+                    os.path.join(ROOT, "include"), src, "-o", str(exe),
+                    "-L", os.path.dirname(lib), "-l:" + os.path.basename(lib),
+                    "-Wl,-rpath," + os.path.dirname(lib)], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert out.returncode == 0, out.stderr
+    assert out.stdout.strip() == "ok"
