@@ -202,6 +202,7 @@ def test_abi_from_plain_c(tmp_path):
     program (tests/c/abi_from_c.c): validation failures, empty no-ops and
     the version, no GPU touched."""
     import subprocess
+    ops.load()  # builds libsq.so first if it is missing or stale
     lib = ops.library_path()
     exe = tmp_path / "abi_from_c"
     src = os.path.join(ROOT, "tests", "c", "abi_from_c.c")
