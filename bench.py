@@ -38,6 +38,9 @@ sys.path.insert(0, ROOT)
 METRIC = "W8A8 smooth+quant+GEMM TOPS and % of INT8 TC peak at M4096 K4096 N14336"
 UNIT = "TOPS"
 L2_BYTES = 126 * 2 ** 20
+# B200 dense INT8 / FP8 tensor-core rate from NVIDIA's datasheet (9 POPS is
+# with 2:4 sparsity); reported beside the measured-peak fraction
+DATASHEET_8BIT_TOPS = 4500.0
 
 
 def metric_for(case):
@@ -138,6 +141,12 @@ def quant_kernel_name(case):
     if case.K // 8 <= 2048 and case.M >= 2 * sms:
         return "quant_act_stream_kernel"
     return "quant_act_fast_kernel"
+
+
+def launches_per_step(case):
+    """Kernels of this library launched per step: the activation kernel and
+    the GEMM."""
+    return 2
 
 
 def _peaks():
@@ -383,9 +392,11 @@ def run_ours(args):
         else:
             ops.quantize_act(xs[r], s, qt, xq=xq, sx=sx, s_inv=s_inv)
 
+    split = bool(args.split)
+
     def step(i):
         quantize(i)
-        gemm(xq, sx, wqs[i % ROTATE], sw, bias, out=y)
+        gemm(xq, sx, wqs[i % ROTATE], sw, bias, out=y, split=split)
 
     for i in range(max(3, args.warmup)):
         step(i)
@@ -403,7 +414,7 @@ def run_ours(args):
         ev[i][0].record(stream)
         quantize(i)
         ev[i][1].record(stream)
-        gemm(xq, sx, wqs[r], sw, bias, out=y)
+        gemm(xq, sx, wqs[r], sw, bias, out=y, split=split)
         ev[i][2].record(stream)
     torch.cuda.synchronize()
     t_quant = float(np.mean([e[0].elapsed_time(e[1]) for e in ev]))
@@ -415,9 +426,20 @@ def run_ours(args):
     # region; the kernels and their programmatic dependencies are the same.
     # Falls back to launching the steps one by one if capture fails. ----
     graph = None
+    tail = None
+    K_steps = args.steps
+    g_steps = ROTATE * max(1, 6 // ROTATE)
+    tail_steps = K_steps % g_steps
+
+    def capture(n_steps, first):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=side):
+            for i in range(first, first + n_steps):
+                step(i)
+        return g
+
     if not args.no_graph:
         try:
-            g_steps = ROTATE * max(1, 6 // ROTATE)
             side = torch.cuda.Stream(device=dev)
             side.wait_stream(stream)
             with torch.cuda.stream(side):
@@ -425,24 +447,32 @@ def run_ours(args):
                     step(i)
             stream.wait_stream(side)
             torch.cuda.synchronize()
-            graph = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(graph, stream=side):
-                for i in range(g_steps):
-                    step(i)
+            graph = capture(g_steps, 0)
+            # the last K mod g steps, so that exactly K steps are timed
+            tail = capture(tail_steps, 0) if tail_steps else None
             torch.cuda.synchronize()
             graph.replay()
+            if tail is not None:
+                tail.replay()
             torch.cuda.synchronize()
             if ops.device_status() != ops.SQ_OK:
                 raise RuntimeError("device status after a graph replay")
         except Exception as exc:  # noqa: BLE001 - report and run without the graph
             print(f"graph capture unavailable ({exc}); launching steps one by one",
                   file=sys.stderr)
-            graph = None
+            graph = tail = None
 
-    # ---- timed region: K steps back to back, events only at both ends ----
-    K_steps = args.steps
-    if graph is not None:
-        K_steps = max(g_steps, (args.steps + g_steps - 1) // g_steps * g_steps)
+    def run_steps(n):
+        if graph is not None:
+            for _ in range(n // g_steps):
+                graph.replay()
+            if n % g_steps:
+                tail.replay()
+        else:
+            for i in range(n):
+                step(i)
+
+    # ---- timed region: exactly K steps back to back, events only at both ends ----
     sampler = ClockSampler(local) if not args.no_clocks else None
     if sampler:
         sampler.start()
@@ -454,12 +484,7 @@ def run_ours(args):
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     start.record(stream)
-    if graph is not None:
-        for _ in range(K_steps // g_steps):
-            graph.replay()
-    else:
-        for i in range(K_steps):
-            step(i)
+    run_steps(K_steps)
     end.record(stream)
     torch.cuda.synchronize()
     t_wall1 = time.time()
@@ -471,6 +496,37 @@ def run_ours(args):
         raise RuntimeError(f"device status after timed region: {ops.status_string(st)}")
     elapsed_ms = start.elapsed_time(end)
     elapsed_ms = sqdist.max_over_ranks(elapsed_ms, device=dev)
+
+    # ---- sustained: the same steps repeated for about args.sustained_s
+    # seconds (clocks settle under the power cap), timed the same way ----
+    sustained = None
+    if args.sustained_s > 0:
+        n_sus = max(g_steps, int(args.sustained_s * 1e3 / max(elapsed_ms / K_steps, 1e-3)))
+        n_sus = (n_sus + g_steps - 1) // g_steps * g_steps
+        sampler2 = ClockSampler(local) if not args.no_clocks else None
+        if sampler2:
+            sampler2.start()
+            time.sleep(0.3)
+        if ws > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        t_s0 = time.time()
+        a_ev = torch.cuda.Event(enable_timing=True)
+        b_ev = torch.cuda.Event(enable_timing=True)
+        a_ev.record(stream)
+        run_steps(n_sus)
+        b_ev.record(stream)
+        torch.cuda.synchronize()
+        t_s1 = time.time()
+        if ws > 1:
+            dist.barrier()
+        clocks2 = sampler2.stop(t_s0, t_s1) if sampler2 else None
+        sus_ms = sqdist.max_over_ranks(a_ev.elapsed_time(b_ev), device=dev)
+        if ops.device_status() != ops.SQ_OK:
+            raise RuntimeError("device status after the sustained run")
+        sustained = {"value": ws * case.ops * n_sus / (sus_ms * 1e-3) / 1e12, "unit": UNIT,
+                     "steps": n_sus, "seconds": sus_ms * 1e-3, "ms_per_step": sus_ms / n_sus,
+                     "clocks": clocks2}
 
     # ---- end to end through the public API with host buffers: every step
     # copies its input X from pinned host memory and its output Y back, in a
@@ -526,9 +582,14 @@ def run_ours(args):
         b.record(s_d2h)
         torch.cuda.synchronize()
         e_ms = sqdist.max_over_ranks(a.elapsed_time(b), device=dev)
+        step_s = e_ms * 1e-3 / e_steps
         e2e = {"value": ws * case.ops * e_steps / (e_ms * 1e-3) / 1e12, "unit": UNIT,
                "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2,
-               "steps": e_steps, "pipeline": "H2D / kernels / D2H on three streams"}
+               "steps": e_steps, "pipeline": "H2D / kernels / D2H on three streams",
+               # the copies' achieved rates over the step (each direction has
+               # its own PCIe link budget): the larger one bounds the step
+               "h2d_gbs": M * K * 2 / step_s / 1e9, "d2h_gbs": M * N * 2 / step_s / 1e9,
+               "bound": ("D2H copy of Y" if M * N >= M * K else "H2D copy of X")}
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
@@ -557,11 +618,15 @@ def run_ours(args):
                        "l2": (f"{ROTATE} rotating input sets (X + Wq, "
                               f"{ROTATE * (M * K * 2 + N * K) / 2 ** 20:.0f} MiB) > 126 MiB L2"),
                        "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU",
-                       "launch": (f"CUDA graph of {g_steps} steps, replayed" if graph is not None
-                                  else "one launch per kernel"),
+                       "launch": ((f"CUDA graph of {g_steps} steps, replayed"
+                                   + (f", then one of {tail_steps}" if tail_steps else ""))
+                                  if graph is not None else "one launch per kernel"),
+                       "split_last_wave": split,
                        "gemm_tile": os.environ.get("SQ_GEMM_TILE", "auto")},
             "frac_of_int8_peak": value / ws / int8_peak,
+            "frac_of_datasheet": value / ws / DATASHEET_8BIT_TOPS,
             "int8_peak_tops": int8_peak,
+            "datasheet_8bit_tops": DATASHEET_8BIT_TOPS,
             "int8_peak_source": f"2 x {pk['src']} bf16 dense ({pk['bf16']} TFLOP/s burst)",
             "gemm_hbm_gbs": g_bytes / (t_gemm * 1e-3) / 1e9,
             "roofline": gemm_roofline(case.ops, g_bytes, t_gemm, int8_peak, int8_peak_sus,
@@ -571,8 +636,9 @@ def run_ours(args):
                                "unit": "GB/s", "frac": q_bytes / (t_quant * 1e-3) / 1e9 / pk["hbm"],
                                "traffic": profiled_traffic("quant", case.name),
                                "ms_per_launch": t_quant},
-            "gpu_launches": 2 * K_steps,  # the activation kernel + the GEMM per step
+            "gpu_launches": launches_per_step(case) * K_steps,
             "clocks": clocks,
+            "sustained": sustained,
             "e2e": e2e,
             "cpu_baseline": cpu,
         }
@@ -580,6 +646,61 @@ def run_ours(args):
     if ws > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def measure_peaks(args):
+    """Black-box 8-bit tensor-core rates of cuBLAS on this GPU (no code of this
+    repository on the path): torch._int_mm (INT8 x INT8 -> int32) and
+    torch._scaled_mm (E4M3 x E4M3 -> bf16, per-tensor scales), each at
+    8192^3 and at every workload shape with at least 17 tokens. One JSON line
+    per (kind, shape): mean CUDA-event time of `steps` launches after
+    `warmup`, TOPS, and the SM clocks sampled meanwhile."""
+    import torch
+    from w8a8_smoothquant_int8_02_b200 import workloads
+
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    shapes = [("cube_8192", 8192, 8192, 8192)]
+    shapes += [(c.name, c.M, c.K, c.N) for c in workloads.ALL.values() if c.M > 16]
+    g = torch.Generator(device=dev)
+    g.manual_seed(0)
+    for name, M, K, N in shapes:
+        for kind in ("int8", "e4m3"):
+            a8 = torch.randint(-127, 128, (M, K), dtype=torch.int8, device=dev, generator=g)
+            b8 = torch.randint(-127, 128, (N, K), dtype=torch.int8, device=dev, generator=g)
+            if kind == "int8":
+                fn = lambda: torch._int_mm(a8, b8.t())  # noqa: E731
+            else:
+                af = (a8.float() / 32).to(torch.float8_e4m3fn)
+                bf = (b8.float() / 32).to(torch.float8_e4m3fn)
+                one = torch.ones((), dtype=torch.float32, device=dev)
+                fn = lambda: torch._scaled_mm(af, bf.t(), scale_a=one, scale_b=one,  # noqa: E731
+                                              out_dtype=torch.bfloat16)
+            for _ in range(max(3, args.warmup)):
+                fn()
+            torch.cuda.synchronize()
+            n = max(20, args.steps)
+            sampler = ClockSampler(0) if not args.no_clocks else None
+            if sampler:
+                sampler.start()
+                time.sleep(0.3)
+            t0 = time.time()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(n):
+                fn()
+            e1.record()
+            torch.cuda.synchronize()
+            t1 = time.time()
+            clocks = sampler.stop(t0, t1) if sampler else None
+            ms = e0.elapsed_time(e1) / n
+            print(json.dumps({"peak_probe": f"cublas_{kind}", "shape": name, "M": M, "K": K,
+                              "N": N, "us_per_launch": ms * 1e3,
+                              "tops": 2.0 * M * N * K / (ms * 1e-3) / 1e12, "launches": n,
+                              "clocks": clocks}), flush=True)
+            del a8, b8
+            torch.cuda.empty_cache()
 
 
 def main():
@@ -598,6 +719,14 @@ def main():
                     help="launch the timed steps one by one instead of replaying a CUDA graph")
     ap.add_argument("--workload", default="mlp_up_4096x4096x14336",
                     help="one of the six workloads in workloads.py (default: the MLP up-projection)")
+    ap.add_argument("--split", action="store_true",
+                    help="pass the GEMM workspace so the last partial wave of tiles is split "
+                         "along K over all SMs (stream-K)")
+    ap.add_argument("--sustained-s", type=float, default=1.5,
+                    help="seconds of extra replays for the sustained figure (0: skip)")
+    ap.add_argument("--measure-peaks", action="store_true",
+                    help="time the library-free 8-bit peaks instead: cuBLAS INT8 (torch._int_mm) "
+                         "and FP8 (torch._scaled_mm) as black boxes at 8192^3 and each workload")
     ap.add_argument("--tile", default=None, help="force a GEMM tile shape (c1n128, c1n224, c1n256, "
                     "c2n224, c2n256); default: chosen by problem size")
     args = ap.parse_args()
@@ -605,6 +734,8 @@ def main():
         args.warmup = 3
     if args.impl == "reference":
         run_reference(args)
+    elif args.measure_peaks:
+        measure_peaks(args)
     else:
         run_ours(args)
 

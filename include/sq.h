@@ -292,16 +292,20 @@ sq_status sq_linear(const void* x, sq_dtype xt, const float* s,
  * afford the device-wide synchronization cudaMalloc / cudaFree may imply --
  * and so cannot provide the workspace the split-tile GEMM needs. This entry
  * point takes the same inputs and outputs as sq_gemm_w8a8 (without acc and
- * without a workspace) and uses a fixed 20 MiB array inside the library's
- * device image as its scratch instead. It calls no cudaMalloc / cudaFree or
- * other allocating routine.
+ * without a workspace) and uses a fixed array inside the library's device
+ * image as its scratch instead: 20 MiB + 4 KiB, the split-tile workspace of
+ * a GPU with up to 160 SMs. It calls no cudaMalloc / cudaFree or other
+ * allocating routine.
  *  - Limit: the scratch this call needs (see sq_gemm_workspace_bytes; it
- *    depends on the GPU's SM count, not on M, N, K) must fit 20 MiB,
- *    otherwise SQ_ERR_SCRATCH_TOO_SMALL and nothing is launched. Every GPU
- *    that loads the library holds the 20 MiB array until the process exits.
+ *    depends on the GPU's SM count, not on M, N, K) must fit the array, so
+ *    GPUs with more than 160 SMs get SQ_ERR_SCRATCH_TOO_SMALL and nothing is
+ *    launched. Every GPU that loads the library holds the array until the
+ *    process exits.
  *  - Set-up: the first call on each device looks up the array's device
- *    address (cudaGetSymbolAddress) with that device current; make that first
- *    call before any stream capture.
+ *    address (cudaGetSymbolAddress) with that device current and caches it;
+ *    make that first call before any stream capture. The cached address is
+ *    not valid after cudaDeviceReset: do not call this entry point on a
+ *    device after resetting it.
  *  - Every call shares the one array, which keeps the last call's contents;
  *    each call first clears the part that must start at zero (an async
  *    memset on `stream`). Calls that overlap on the GPU (different streams,

@@ -58,6 +58,7 @@ def _load():
             lib.sqo_bf16_to_f32.restype = ctypes.c_float
             lib.sqo_f32_to_bf16_rne.argtypes = [ctypes.c_float]
             lib.sqo_f32_to_bf16_rne.restype = ctypes.c_uint16
+            lib.sqo_f32_to_bf16_rne_n.argtypes = [P, P, I64]
             lib.sqo_e4m3_decode.argtypes = [ctypes.c_uint8]
             lib.sqo_e4m3_decode.restype = ctypes.c_double
             lib.sqo_e4m3_encode_rn_sat.argtypes = [ctypes.c_float]
@@ -114,15 +115,18 @@ def bf16_to_f32(h) -> np.ndarray:
     return out.reshape(h.shape)
 
 
+def bf16_to_f32_array(h) -> np.ndarray:
+    """bf16_to_f32 for whole arrays: the bits move up 16 (exact)."""
+    h = _c(h, np.uint16)
+    return (h.astype(np.uint32) << 16).view(np.float32)
+
+
 def f32_to_bf16(x) -> np.ndarray:
-    lib = _load()
+    """Round float32 to bf16 (nearest-even), returned as raw uint16 bits."""
     x = _c(x, np.float32)
-    flat = x.reshape(-1)
-    out = np.empty(flat.shape, np.uint16)
-    f = lib.sqo_f32_to_bf16_rne
-    for i in range(flat.size):
-        out[i] = f(float(flat[i]))
-    return out.reshape(x.shape)
+    out = np.empty(x.shape, np.uint16)
+    _load().sqo_f32_to_bf16_rne_n(_ptr(x), _ptr(out), x.size)
+    return out
 
 
 def e4m3_decode(codes) -> np.ndarray:

@@ -73,6 +73,11 @@ uint16_t sqo_f32_to_bf16_rne(float f) {
     return (uint16_t)kept;
 }
 
+/* The same rounding over an array (a loop over sqo_f32_to_bf16_rne). */
+void sqo_f32_to_bf16_rne_n(const float* x, uint16_t* out, int64_t n) {
+    for (int64_t i = 0; i < n; ++i) out[i] = sqo_f32_to_bf16_rne(x[i]);
+}
+
 /* E4M3: 1 sign bit, 4 exponent bits (bias 7), 3 mantissa bits, no infinity,
  * S.1111.111 is NaN, largest finite value 1.75 * 2^8 = 448 ([WAQ] §4 gives
  * the range [-448, 448]). Normal: (1 + m/8) 2^(e-7) = (8+m) 2^(e-10).

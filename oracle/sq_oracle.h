@@ -31,6 +31,7 @@ extern "C" {
 /* bfloat16 <-> binary32 (definition of the format; widening is exact). */
 float    sqo_bf16_to_f32(uint16_t h);
 uint16_t sqo_f32_to_bf16_rne(float f);
+void     sqo_f32_to_bf16_rne_n(const float* x, uint16_t* out, int64_t n);
 
 /* FP8 E4M3: value of a code, and round-to-nearest-even saturating encode. */
 double   sqo_e4m3_decode(uint8_t code);

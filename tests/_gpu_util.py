@@ -54,3 +54,28 @@ def sample_points(M, N, seed, n_random=4096, full_rows=4, full_cols=4):
     rows = [np.repeat(rsel, N), np.tile(np.arange(M), csel.size), g.integers(0, M, n_random)]
     cols = [np.tile(np.arange(N), rsel.size), np.repeat(csel, M), g.integers(0, N, n_random)]
     return np.concatenate(rows).astype(np.int64), np.concatenate(cols).astype(np.int64)
+
+
+def fp8_error_denominator(xq, wq, sx, sw, bias, rows_per_chunk=1024):
+    """sx[m]*sw[n]*sum_k |a_mk b_nk| + |bias[n]| for every output element: the
+    magnitude sums as one binary64 matrix product per row block."""
+    table = np.abs(oracle.e4m3_decode(np.arange(256, dtype=np.uint8)))
+    b_mag = table[np.ascontiguousarray(wq)].T.copy()                 # [K,N]
+    sw64 = np.asarray(sw, np.float64)
+    bias_abs = 0.0 if bias is None else np.abs(oracle.bf16_to_f32_array(bias).astype(np.float64))
+    M = xq.shape[0]
+    den = np.empty((M, b_mag.shape[1]), np.float64)
+    for r0 in range(0, M, rows_per_chunk):
+        r1 = min(M, r0 + rows_per_chunk)
+        mag = table[np.ascontiguousarray(xq[r0:r1])] @ b_mag
+        den[r0:r1] = np.asarray(sx[r0:r1], np.float64)[:, None] * sw64[None, :] * mag + bias_abs
+    return den
+
+
+def fp8_normalized_error_full(y, y_ref, xq=None, wq=None, sx=None, sw=None, bias=None, den=None):
+    """The same metric as fp8_normalized_error on whole [M,N] outputs (pass
+    `den` from fp8_error_denominator to reuse it across outputs)."""
+    if den is None:
+        den = fp8_error_denominator(xq, wq, sx, sw, bias)
+    num = np.abs(np.asarray(y, np.float64) - np.asarray(y_ref, np.float64))
+    return np.where(den > 0, num / np.where(den > 0, den, 1.0), num)

@@ -170,6 +170,45 @@ def test_gemm_validation(lib):
     assert g(c(A), c(A), c(A), c(A), None, 0, 64, 64, c(A), ops.SQ_BF16, None, 0, None) == ops.SQ_OK
 
 
+def test_gemm_noalloc_validation(lib):
+    """The allocation-free GEMM rejects bad arguments on the host exactly as
+    sq_gemm_w8a8 does (same checks, no launch), and M == 0 is a no-op."""
+    f = lib.sq_gemm_w8a8_noalloc
+    ok = dict(xq=A, sx=A, wq=A, sw=A, bias=None, M=16, N=64, K=64, y=A, yt=ops.SQ_BF16)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return f(c(a["xq"]), c(a["sx"]), c(a["wq"]), c(a["sw"]), c(a["bias"]), a["M"], a["N"],
+                 a["K"], c(a["y"]), a["yt"], None)
+
+    assert call(xq=NUL) == ops.SQ_ERR_INVALID_ARG
+    assert call(sx=NUL) == ops.SQ_ERR_INVALID_ARG
+    assert call(wq=NUL) == ops.SQ_ERR_INVALID_ARG
+    assert call(sw=NUL) == ops.SQ_ERR_INVALID_ARG
+    assert call(y=NUL) == ops.SQ_ERR_INVALID_ARG
+    assert call(M=-1) == ops.SQ_ERR_INVALID_ARG
+    assert call(N=0) == ops.SQ_ERR_INVALID_ARG
+    assert call(N=12) == ops.SQ_ERR_INVALID_ARG        # not a multiple of 8
+    assert call(K=0) == ops.SQ_ERR_INVALID_ARG
+    assert call(K=40) == ops.SQ_ERR_INVALID_ARG        # not a multiple of 16
+    assert call(K=133152) == ops.SQ_ERR_UNSUPPORTED    # int32 accumulator could overflow
+    assert call(yt=ops.SQ_I8) == ops.SQ_ERR_INVALID_ARG
+    assert call(yt=ops.SQ_E4M3) == ops.SQ_ERR_INVALID_ARG
+    assert call(xq=A + 8) == ops.SQ_ERR_MISALIGNED
+    assert call(wq=A + 2) == ops.SQ_ERR_MISALIGNED
+    assert call(y=A + 8) == ops.SQ_ERR_MISALIGNED
+    assert call(sx=A + 2) == ops.SQ_ERR_MISALIGNED
+    assert call(sw=A + 4) == ops.SQ_ERR_MISALIGNED
+    assert call(bias=A + 2) == ops.SQ_ERR_MISALIGNED
+    assert call(M=0) == ops.SQ_OK
+    assert call(M=0, xq=NUL, sx=NUL, y=NUL) == ops.SQ_OK
+
+
+def test_scratch_too_small_has_its_own_message(lib):
+    msg = ops.status_string(ops.SQ_ERR_SCRATCH_TOO_SMALL)
+    assert msg.startswith("SQ_ERR_SCRATCH_TOO_SMALL") and "160 SMs" in msg
+
+
 def test_smooth_factor_and_calibration_validation(lib):
     sf = lib.sq_smooth_factors
     assert sf(c(A), c(A), 64, 1.5, c(A), None, None) == ops.SQ_ERR_INVALID_ARG

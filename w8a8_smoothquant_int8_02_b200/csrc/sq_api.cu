@@ -2,6 +2,7 @@
 //
 // Argument validation happens here, synchronously, before anything is
 // launched; the launchers in sq_quant.cu / sq_gemm.cu assume valid input.
+#include <atomic>
 #include <cstdint>
 #include <cuda_runtime.h>
 
@@ -80,27 +81,35 @@ cudaError_t run_gemm_any(bool e4m3, const uint8_t* xq, const float* sx, const ui
 // ---------------------------------------------------------------------------
 // Scratch of the allocation-free GEMM entry point (sq_gemm_w8a8_noalloc):
 // a fixed array in the library's own device image, so the call allocates
-// nothing. 20 MiB holds the split-tile workspace of every tile shape on a GPU
-// with up to 160 SMs (4 KiB of counters + one 128 x 256 x 4-byte slot per SM).
-// Every GPU that loads the library keeps this array until the process exits.
+// nothing. Its size is the split-tile workspace of a GPU with kNoAllocMaxSms
+// SMs: the counter block plus one 128 x 256 x 4-byte partial-sum slot per SM
+// (sq_gemm_workspace_bytes on such a GPU). Every GPU that loads the library
+// keeps this array until the process exits.
 // ---------------------------------------------------------------------------
-constexpr size_t kNoAllocScratchBytes = size_t(20) << 20;
-static __device__ __align__(256) unsigned char g_sq_noalloc_scratch[kNoAllocScratchBytes];
+constexpr size_t kNoAllocMaxSms = 160;
+constexpr size_t kNoAllocSlotBytes = size_t(128) * 256 * 4;
+static __device__ __align__(256) unsigned char
+    g_sq_noalloc_scratch[size_t(4096) + kNoAllocMaxSms * kNoAllocSlotBytes];
+constexpr size_t kNoAllocScratchBytes = sizeof(g_sq_noalloc_scratch);
 
 // Device address of the array for the current device. Host code must not use
 // the array's name as a pointer (it is a host-side stand-in); the runtime
-// gives the device address, looked up once per device and cached.
+// gives the device address. It is looked up once per device with that device
+// current and cached; concurrent first calls may both look it up and store
+// the same value (atomic stores). After cudaDeviceReset the module is loaded
+// again and the cached address is stale, so a process that resets a device
+// must not call the entry point on it afterwards.
 void* noalloc_scratch_ptr() {
-  static void* ptrs[64] = {nullptr};
+  static std::atomic<void*> ptrs[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  if (!ptrs[dev]) {
-    void* p = nullptr;
+  void* p = ptrs[dev].load(std::memory_order_acquire);
+  if (!p) {
     if (cudaGetSymbolAddress(&p, g_sq_noalloc_scratch) != cudaSuccess || p == nullptr)
       return nullptr;
-    ptrs[dev] = p;
+    ptrs[dev].store(p, std::memory_order_release);
   }
-  return ptrs[dev];
+  return p;
 }
 
 }  // namespace
@@ -116,8 +125,8 @@ const char* sq_status_string(sq_status st) {
     case SQ_ERR_CUDA: return "SQ_ERR_CUDA: CUDA runtime error";
     case SQ_ERR_TIMEOUT: return "SQ_ERR_TIMEOUT: a bounded device wait gave up";
     case SQ_ERR_SCRATCH_TOO_SMALL:
-      return "SQ_ERR_SCRATCH_TOO_SMALL: this call needs more scratch than the fixed 20 MiB array "
-             "of the allocation-free entry point";
+      return "SQ_ERR_SCRATCH_TOO_SMALL: this call needs more scratch than the fixed array of "
+             "the allocation-free entry point (sized for GPUs with up to 160 SMs)";
   }
   return "SQ_ERR_UNKNOWN";
 }
