@@ -80,6 +80,9 @@ def _load():
             lib.sqo_linear_at.argtypes = [P, P, P, P, P, I, I64, P, P, I64,
                                           P, P, P]
             lib.sqo_num_threads.restype = I
+            lib.sqo_quantize_weight_i4.argtypes = [P, I, I64, I64, P, P]
+            lib.sqo_unpack_i4.argtypes = [P, I64, I64, P]
+            lib.sqo_gemm_weight_only.argtypes = [P, P, I, P, P, I64, I64, I64, P]
             _lib = lib
     return _lib
 
@@ -313,3 +316,47 @@ def linear(x, s, wq, sw, bias=None, qtype: int = INT8):
     acc = gemm_e4m3(xq, wq) if qtype == E4M3 else gemm_i8(xq, wq)
     yf, yb = epilogue(acc, sx, sw, bias)
     return dict(xq=xq, sx=sx, acc=acc, y_f32=yf, y_bf16=yb)
+
+
+# ---- weight-only quantization (W8A16 / W4A16) -------------------------------
+
+def quantize_weight_i4(w: np.ndarray):
+    """Per-output-channel symmetric INT4 weights: (wq4 [N, K/2] uint8, two codes
+    per byte, low nibble = even k; sw [N] float32 = amax / 7)."""
+    w = np.ascontiguousarray(w)
+    K, N = w.shape
+    if K % 2:
+        raise ValueError("K must be even for packed INT4 weights")
+    wq4 = np.empty((N, K // 2), np.uint8)
+    sw = np.empty(N, np.float32)
+    _load().sqo_quantize_weight_i4(_ptr(w), _dtype_code(w), K, N, _ptr(wq4), _ptr(sw))
+    return wq4, sw
+
+
+def unpack_i4(wq4: np.ndarray) -> np.ndarray:
+    """Codes (int8 [N, K]) of packed INT4 weights [N, K/2]."""
+    wq4 = _c(wq4, np.uint8)
+    N, half = wq4.shape
+    codes = np.empty((N, 2 * half), np.int8)
+    _load().sqo_unpack_i4(_ptr(wq4), N, 2 * half, _ptr(codes))
+    return codes
+
+
+def gemm_weight_only(x, wq, sw, bias=None, bits: int = 8) -> np.ndarray:
+    """y = x @ (codes * sw).T + bias in binary64 (x: bf16 bits [M,K]; wq: int8
+    [N,K] for bits 8, packed uint8 [N,K/2] for bits 4)."""
+    x = _c(x, np.uint16)
+    M, K = x.shape
+    wq = np.ascontiguousarray(wq)
+    N = wq.shape[0]
+    if bits == 8:
+        assert wq.dtype == np.int8 and wq.shape[1] == K
+    elif bits == 4:
+        assert wq.dtype == np.uint8 and 2 * wq.shape[1] == K
+    else:
+        raise ValueError("bits must be 8 or 4")
+    sw = _c(sw, np.float32)
+    bias = None if bias is None else _c(bias, np.uint16)
+    y = np.empty((M, N), np.float64)
+    _load().sqo_gemm_weight_only(_ptr(x), _ptr(wq), bits, _ptr(sw), _ptr(bias), M, N, K, _ptr(y))
+    return y

@@ -422,3 +422,88 @@ void sqo_linear_at(const void* xq, const float* sx, const void* wq,
         if (y_bf16) y_bf16[i] = sqo_f32_to_bf16_rne(t);
     }
 }
+
+/* ------------------------------------------------------------------------ */
+/* Weight-only quantization, the comparison the pages draw for decode       */
+/* ([WAQ] §1 table, W4A16 row: "INT4 -> dequant to FP16, then FP16 x FP16";  */
+/* [ACT]: the runtime dequantizes the weights on the fly to multiply them    */
+/* against the BF16 activations; [LES] §1 and §3: W8A16, 8-bit weights       */
+/* de-quantized back to 16-bit and multiplied with 16-bit activations; the   */
+/* zenaique page "W8A8 vs W4A16": W4A16 reads 4x fewer weight bytes, which   */
+/* is what bandwidth-bound decode needs).                                   */
+/*                                                                          */
+/* Readings: the weights are quantized per output channel, symmetric, with  */
+/* the same rule as the W8A8 weights (the pages' per-channel scaling), for  */
+/* INT4 with Q = 7 (codes -7..7; group-wise scales belong to the AWQ / GPTQ  */
+/* methods, which are not built). The dequantized weight is the real value  */
+/* q[n][k] * sw[n]; the activations are bf16, used as they are (no          */
+/* smoothing: no activation is quantized). The product is taken in binary64: */
+/* y[m][n] = sum_k x[m][k] * (q[n][k] * sw[n]) + bias[n]. Every product is   */
+/* exact in binary64 (8 x 8 x 24 significant bits); only the sum rounds, so  */
+/* the result is within a few binary64 ulps of the real value.              */
+/* ------------------------------------------------------------------------ */
+
+/* INT4 code of v at scale `scale` (scale > 0): round-half-even of the binary32
+ * quotient, clamped to +-7. */
+static int8_t quant_i4(float v, float scale) {
+    float c = nearbyintf(v / scale);
+    if (c > 7.0f) c = 7.0f;
+    if (c < -7.0f) c = -7.0f;
+    return (int8_t)c;
+}
+
+/* The two's-complement nibble of a code in -8..7, and back. */
+static uint8_t nibble_of(int8_t q) { return (uint8_t)q & 0x0Fu; }
+static int8_t code_of_nibble(uint8_t nb) { return (int8_t)((nb & 0x08u) ? (int)nb - 16 : (int)nb); }
+
+void sqo_quantize_weight_i4(const void* w, int dtype, int64_t K, int64_t N,
+                            uint8_t* wq4, float* sw) {
+    #pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n) {
+        float amax = 0.0f;
+        for (int64_t k = 0; k < K; ++k) {
+            float a = fabsf(load_elem(w, dtype, k * N + n));
+            if (a > amax) amax = a;
+        }
+        float scale = amax / 7.0f;
+        sw[n] = scale;
+        /* byte k/2 of row n: code of even k in the low nibble, odd k in the high */
+        for (int64_t k = 0; k < K; k += 2) {
+            int8_t q0 = (scale == 0.0f) ? 0 : quant_i4(load_elem(w, dtype, k * N + n), scale);
+            int8_t q1 = (scale == 0.0f) ? 0
+                                        : quant_i4(load_elem(w, dtype, (k + 1) * N + n), scale);
+            wq4[n * (K / 2) + k / 2] = (uint8_t)(nibble_of(q0) | (nibble_of(q1) << 4));
+        }
+    }
+}
+
+void sqo_unpack_i4(const uint8_t* wq4, int64_t N, int64_t K, int8_t* codes) {
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k) {
+            uint8_t b = wq4[n * (K / 2) + k / 2];
+            codes[n * K + k] = code_of_nibble((k & 1) ? (uint8_t)(b >> 4) : (uint8_t)(b & 0x0Fu));
+        }
+}
+
+void sqo_gemm_weight_only(const uint16_t* x, const void* wq, int bits, const float* sw,
+                          const uint16_t* bias, int64_t M, int64_t N, int64_t K,
+                          double* y) {
+    #pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; ++k) {
+                int8_t q;
+                if (bits == 4) {
+                    uint8_t b = ((const uint8_t*)wq)[n * (K / 2) + k / 2];
+                    q = code_of_nibble((k & 1) ? (uint8_t)(b >> 4) : (uint8_t)(b & 0x0Fu));
+                } else {
+                    q = ((const int8_t*)wq)[n * K + k];
+                }
+                double w_deq = (double)q * (double)sw[n];
+                acc += (double)sqo_bf16_to_f32(x[m * K + k]) * w_deq;
+            }
+            if (bias) acc += (double)sqo_bf16_to_f32(bias[n]);
+            y[m * N + n] = acc;
+        }
+}

@@ -112,6 +112,22 @@ void sqo_linear_at(const void* xq, const float* sx, const void* wq,
                    int64_t count, double* acc_out, float* y_f32,
                    uint16_t* y_bf16);
 
+/* Weight-only quantization (W8A16 / W4A16). INT4 weights: per output channel
+ * sw[n] = max_k |w[k][n]| / 7, codes clamp(round-half-even(w / sw), -7, 7)
+ * (0 where sw is 0), packed two per byte into wq4 [N, K/2]: byte k/2 of row n
+ * holds the code of even k in its low nibble and of odd k in its high nibble
+ * (two's complement). K must be even. */
+void sqo_quantize_weight_i4(const void* w, int dtype, int64_t K, int64_t N,
+                            uint8_t* wq4, float* sw);
+/* The codes of a packed INT4 matrix, one int8 per element: codes [N,K]. */
+void sqo_unpack_i4(const uint8_t* wq4, int64_t N, int64_t K, int8_t* codes);
+/* y[m][n] = sum_k x[m][k] * (q[n][k] * sw[n]) + bias[n] in binary64, with x
+ * [M,K] bf16 bits, q the codes of wq (bits 8: int8 [N,K]; bits 4: packed
+ * [N,K/2]), sw [N] and bias [N] bf16 or NULL. */
+void sqo_gemm_weight_only(const uint16_t* x, const void* wq, int bits, const float* sw,
+                          const uint16_t* bias, int64_t M, int64_t N, int64_t K,
+                          double* y);
+
 /* Threads OpenMP will use (1 when built without OpenMP). */
 int sqo_num_threads(void);
 

@@ -648,3 +648,97 @@ def test_folded_producer_feeds_the_same_codes(qt):
     folded = (x * oracle.fold_smoothing(g, s)[0]).astype(np.float64)
     exact = x.astype(np.float64) * g.astype(np.float64) / s.astype(np.float64)
     assert np.all(np.abs(folded - exact) <= 2.0 ** -22 * np.abs(exact))
+
+
+# ---------------------------------------------------------------------------
+# Weight-only quantization (W8A16 / W4A16): infra.bea.ai §1 table (W4A16 row,
+# weights dequantized, then a 16-bit multiply), the zenaique flashcard (the
+# runtime dequantizes weights on the fly against BF16 activations), the
+# grasp.study lesson §1 / §3 (W8A16).
+# ---------------------------------------------------------------------------
+
+def test_int4_weight_codes_and_packing_by_hand():
+    """A column with amax 7 has scale 1: codes are the half-even roundings
+    clamped to +-7, and each byte holds an even-k code (low nibble) and the
+    following odd-k code (high nibble), two's complement."""
+    w = np.zeros((6, 3), np.float32)
+    w[:, 0] = [7.0, -3.5, 2.5, 0.5, -6.49, 1.0]   # ties go to even: -3.5 -> -4, 2.5 -> 2, 0.5 -> 0
+    w[:, 1] = [0.0, 0.0, 0.0, 0.0, 0.0, -14.0]    # amax 14 -> scale 2; -14 / 2 = -7
+    wq4, sw = oracle.quantize_weight_i4(w)
+    assert sw.tolist() == [1.0, 2.0, 0.0]
+    assert wq4[0].tolist() == [0xC7, 0x02, 0x1A]  # (7, -4), (2, 0), (-6, 1)
+    assert wq4[1].tolist() == [0x00, 0x00, 0x90]  # (0, 0), (0, 0), (0, -7)
+    assert not wq4[2].any()                       # an all-zero channel
+    np.testing.assert_array_equal(oracle.unpack_i4(wq4)[0], [7, -4, 2, 0, -6, 1])
+
+
+@pytest.mark.parametrize("bf16", [False, True])
+def test_int4_weight_quant_brute_force(bf16):
+    w = synth.random_floats((64, 40), seed=41, std=0.02)
+    w[:, 3] = 0.0
+    w[5, 7] = 0.5                                  # one dominant weight per channel
+    if bf16:
+        w = synth.to_bf16_bits(w)
+    wf = oracle.bf16_to_f32_array(w) if bf16 else w
+    amax = np.abs(wf).max(axis=0)
+    scale = (amax / np.float32(7.0)).astype(np.float32)
+    safe = np.where(scale > 0, scale, np.float32(1.0))
+    codes = np.clip(np.rint(wf / safe[None, :]), -7, 7).astype(np.int8).T
+    codes[scale == 0] = 0
+    wq4, sw = oracle.quantize_weight_i4(w)
+    np.testing.assert_array_equal(sw, scale)
+    np.testing.assert_array_equal(oracle.unpack_i4(wq4), codes)
+    lo = (codes[:, 0::2].astype(np.int16) & 0xF)
+    hi = (codes[:, 1::2].astype(np.int16) & 0xF)
+    np.testing.assert_array_equal(wq4, (lo | (hi << 4)).astype(np.uint8))
+    # the largest weight of a channel maps to +-7 and the error is half a step
+    assert (np.abs(oracle.unpack_i4(wq4)[7]).max() == 7)
+    err = np.abs(wf.T - codes * sw[:, None])
+    assert (err <= sw[:, None] / 2 * (1 + 2 ** -20)).all()
+
+
+@pytest.mark.parametrize("bits", [8, 4])
+def test_weight_only_gemm_brute_force(bits):
+    M, K, N = 5, 96, 24
+    x = synth.to_bf16_bits(synth.random_floats((M, K), seed=42, std=1.0) *
+                           np.float32(3.0))
+    w = synth.random_floats((K, N), seed=43, std=0.02)
+    bias = synth.to_bf16_bits(synth.random_floats(N, seed=44, std=0.05))
+    if bits == 8:
+        wq, sw = oracle.quantize_weight(w, None)
+        codes = wq
+    else:
+        wq, sw = oracle.quantize_weight_i4(w)
+        codes = oracle.unpack_i4(wq)
+    xf = oracle.bf16_to_f32_array(x).astype(np.float64)
+    ref = xf @ (codes.astype(np.float64) * sw.astype(np.float64)[:, None]).T
+    ref += oracle.bf16_to_f32_array(bias).astype(np.float64)[None, :]
+    y = oracle.gemm_weight_only(x, wq, sw, bias, bits)
+    np.testing.assert_allclose(y, ref, rtol=1e-13, atol=1e-13)
+    y0 = oracle.gemm_weight_only(x, wq, sw, None, bits)
+    np.testing.assert_allclose(y - y0, np.broadcast_to(
+        oracle.bf16_to_f32_array(bias).astype(np.float64), y.shape), rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("bits", [8, 4])
+def test_weight_only_one_hot_row_reads_one_dequantized_weight(bits):
+    K, N = 32, 16
+    w = synth.random_floats((K, N), seed=45, std=0.02)
+    wq, sw = oracle.quantize_weight(w, None) if bits == 8 else oracle.quantize_weight_i4(w)
+    codes = wq if bits == 8 else oracle.unpack_i4(wq)
+    x = np.zeros((K, K), np.float32)
+    x[np.arange(K), np.arange(K)] = 1.0            # row j is e_j
+    y = oracle.gemm_weight_only(synth.to_bf16_bits(x), wq, sw, None, bits)
+    np.testing.assert_array_equal(y, (codes.astype(np.float64) * sw.astype(np.float64)[:, None]).T)
+
+
+def test_weight_only_on_integer_activations_is_the_int8_gemm_scaled():
+    """With integer activations (|x| <= 127, exact in bf16) the weight-only
+    product equals the INT8 GEMM of the same codes times the channel scale."""
+    M, K, N = 7, 160, 40
+    xi = synth.random_matrix((M, K), np.int8, seed=46)
+    w = synth.random_floats((K, N), seed=47, std=0.02)
+    wq, sw = oracle.quantize_weight(w, None)
+    y = oracle.gemm_weight_only(synth.to_bf16_bits(xi.astype(np.float32)), wq, sw, None, 8)
+    acc = oracle.gemm_i8(xi, wq).astype(np.float64)
+    np.testing.assert_array_equal(y, acc * sw.astype(np.float64)[None, :])
