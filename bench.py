@@ -43,9 +43,17 @@ L2_BYTES = 126 * 2 ** 20
 DATASHEET_8BIT_TOPS = 4500.0
 
 
+def weight_bits(case):
+    """Weight bits of a weight-only workload (W8A16 / W4A16), else None."""
+    return {"w8": 8, "w4": 4}.get(case.qtype)
+
+
 def metric_for(case):
     if case.name.startswith("mlp_up"):
         return METRIC
+    if weight_bits(case):
+        return (f"W{weight_bits(case)}A16 weight-only GEMM TOPS and % of HBM roofline at "
+                f"M{case.M} K{case.K} N{case.N}")
     if case.act_scaling == "tensor":
         return (f"W8A8 per-tensor FP8 quant+GEMM TOPS and % of FP8 TC peak at "
                 f"M{case.M} K{case.K} N{case.N}")
@@ -57,7 +65,7 @@ def metric_for(case):
 def rotate_count(case):
     """Input sets to rotate through so that the inputs of one step are not
     left in L2 by the previous steps (X and Wq of all sets > 1.5 x L2)."""
-    per_set = case.M * case.K * 2 + case.N * case.K
+    per_set = case.M * case.K * 2 + case.N * case.K * (weight_bits(case) or 8) // 8
     if per_set >= 1.5 * L2_BYTES:
         return 1
     return max(2, -(-int(1.5 * L2_BYTES) // per_set))
@@ -78,6 +86,7 @@ PROFILED_TRAFFIC = {
     ("quant", "decode_16x8192x28672"): (0.362240e6 + 0.0, "11715b8dda2dbca9"),
 }
 KERNEL_SOURCES = {"gemm": ("sq_gemm.cu", "sq_common.cuh"),
+                  "gemm_wonly": ("sq_gemm_wonly.cu", "sq_common.cuh"),
                   "gemm_skinny": ("sq_gemm_skinny.cu", "sq_common.cuh"),
                   "quant": ("sq_quant.cu", "sq_common.cuh")}
 
@@ -121,9 +130,12 @@ SKINNY_MAX_M = 16  # the library's weight-streaming GEMM takes M <= 16 (sq_gemm_
 
 
 def gemm_kind(case, forced_tile=None):
-    """Which GEMM kernel the library runs for this workload: the
-    weight-streaming form for at most 16 tokens (unless a tile shape is
-    forced), else the tiled kernel. Returns (traffic key, kernel name)."""
+    """Which GEMM kernel the library runs for this workload: the weight-only
+    kernel for W8A16 / W4A16, the weight-streaming form for at most 16 tokens
+    (unless a tile shape is forced), else the tiled kernel. Returns (traffic
+    key, kernel name)."""
+    if weight_bits(case):
+        return "gemm_wonly", "gemm_wonly_kernel"
     if case.M <= SKINNY_MAX_M and not forced_tile:
         return "gemm_skinny", "gemm_skinny_kernel"
     return "gemm", "gemm_w8a8_kernel"
@@ -134,6 +146,8 @@ def quant_kernel_name(case):
     bf16 input the persistent streaming form when there are many rows, one
     CTA per row otherwise; the generic kernel for fp32 input."""
     sms = 148
+    if weight_bits(case):
+        return None
     if case.act_scaling == "tensor":
         return "quant_act_tensor_kernel"
     if case.x_dtype != "bf16" or case.K // 8 > 256 * 8:
@@ -143,10 +157,15 @@ def quant_kernel_name(case):
     return "quant_act_fast_kernel"
 
 
+def path_desc(case):
+    return ("weight-only GEMM on bf16 activations + epilogue" if weight_bits(case)
+            else "act quant + 8-bit GEMM + epilogue")
+
+
 def launches_per_step(case):
     """Kernels of this library launched per step: the activation kernel and
-    the GEMM."""
-    return 2
+    the GEMM (the weight-only GEMM alone for W8A16 / W4A16)."""
+    return 1 if weight_bits(case) else 2
 
 
 def _peaks():
@@ -256,7 +275,8 @@ def run_reference(args):
         "impl": "reference", "metric": metric_for(case), "value": val, "unit": UNIT,
         "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "i8" if case.qtype == "i8" else "e4m3",
+        "vs_baseline": None,
+        "dtype": "bf16" if weight_bits(case) else ("i8" if case.qtype == "i8" else "e4m3"),
         "data": f"synthetic, seeded: {case.note}",
         "config": {"workload": case.name, "M": case.M, "K": case.K, "N": case.N,
                    "alpha": case.alpha if case.smooth else None,
@@ -266,7 +286,7 @@ def run_reference(args):
         "cpu_baseline": {"value": val, "unit": UNIT, "cores": oracle.num_threads(),
                          "kind": "oracle",
                          "sample": f"{rows} of {case.M} token rows per step through the runtime "
-                                   f"path (act quant + 8-bit GEMM + epilogue), full K and N"},
+                                   f"path ({path_desc(case)}), full K and N"},
         "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -276,6 +296,12 @@ def _oracle_prep(case, d):
     """The oracle's offline preparation for a workload: (s or None, wq, sw,
     per-tensor scale or None)."""
     import oracle
+    if weight_bits(case) == 8:
+        wq, sw = oracle.quantize_weight(d["w"], None)
+        return None, wq, sw, None
+    if weight_bits(case) == 4:
+        wq, sw = oracle.quantize_weight_i4(d["w"])
+        return None, wq, sw, None
     qt = oracle.E4M3 if case.qtype == "e4m3" else oracle.INT8
     s = None
     if case.smooth:
@@ -290,8 +316,10 @@ def _oracle_prep(case, d):
 
 def _oracle_runtime(case, xs, s, wq, sw, bias, scale):
     """The oracle's runtime path on token rows xs: activation quantization,
-    8-bit GEMM, epilogue."""
+    8-bit GEMM, epilogue (the weight-only product for W8A16 / W4A16)."""
     import oracle
+    if weight_bits(case):
+        return oracle.gemm_weight_only(xs, wq, sw, bias, weight_bits(case))
     qt = oracle.E4M3 if case.qtype == "e4m3" else oracle.INT8
     if scale is None:
         return oracle.linear(xs, s, wq, sw, bias, qt)
@@ -321,8 +349,8 @@ def cpu_baseline(case, d, budget_s: float):
         rows2 = int(max(rows2 + 1, min(case.M, rows2 * budget_s / max(dt, 1e-3))))
     return {"value": 2.0 * rows2 * case.N * case.K / dt / 1e12, "unit": UNIT,
             "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": f"{rows2} of {case.M} token rows through the runtime path (act quant + "
-                      f"8-bit GEMM + epilogue), full K={case.K} and N={case.N}; {dt:.1f} s"}
+            "sample": f"{rows2} of {case.M} token rows through the runtime path "
+                      f"({path_desc(case)}), full K={case.K} and N={case.N}; {dt:.1f} s"}
 
 
 def run_ours(args):
@@ -359,7 +387,11 @@ def run_ours(args):
 
     # ---- offline preparation (untimed) ----
     w = to_dev(d["w"])
-    if case.smooth:
+    wbits = weight_bits(case)
+    if wbits:
+        s = s_inv = None
+        wq0, sw = ops.quantize_weight(w, None, "i8" if wbits == 8 else "i4")
+    elif case.smooth:
         p = ops.prepare(w, to_dev(d["x_cal"]), alpha=case.alpha, qtype=qt)
         s, s_inv, wq0, sw = p["s"], p["s_inv"], p["wq"], p["sw"]
     else:
@@ -373,6 +405,9 @@ def run_ours(args):
         ops.quantize_act_tensor(to_dev(d["x_cal"]), s, qt, amax_out=amax_b[0:1], s_inv=s_inv)
     bias = to_dev(d["bias"]) if d["bias"] is not None else None
     gemm = ops.gemm_w8a8 if qt == "i8" else ops.gemm_fp8
+    if wbits:
+        def gemm(xin, sx_, wq_, sw_, bias_, out, split=False):  # noqa: E306
+            return ops.gemm_weight_only(xin, wq_, sw_, bias_, wbits, out=out)
     del w
     xs = [to_dev(d["x"])] + [None] * (ROTATE - 1)
     wqs = [wq0] + [None] * (ROTATE - 1)
@@ -395,6 +430,9 @@ def run_ours(args):
     split = bool(args.split)
 
     def step(i):
+        if wbits:
+            gemm(xs[i % ROTATE], None, wqs[i % ROTATE], sw, bias, out=y)
+            return
         quantize(i)
         gemm(xq, sx, wqs[i % ROTATE], sw, bias, out=y, split=split)
 
@@ -412,9 +450,10 @@ def run_ours(args):
     for i in range(A_steps):
         r = i % ROTATE
         ev[i][0].record(stream)
-        quantize(i)
+        if not wbits:
+            quantize(i)
         ev[i][1].record(stream)
-        gemm(xq, sx, wqs[r], sw, bias, out=y, split=split)
+        gemm(xs[r] if wbits else xq, sx, wqs[r], sw, bias, out=y, split=split)
         ev[i][2].record(stream)
     torch.cuda.synchronize()
     t_quant = float(np.mean([e[0].elapsed_time(e[1]) for e in ev]))
@@ -544,7 +583,9 @@ def run_ours(args):
         s_h2d, s_comp, s_d2h = (torch.cuda.Stream(device=dev) for _ in range(3))
 
         def compute(xd, yd):
-            if tensor:
+            if wbits:
+                gemm(xd, None, wq0, sw, bias, out=yd)
+            elif tensor:
                 ops.quantize_act_tensor(xd, s, qt, amax_prev=amax_b[0:1], xq=xq, sx=sx,
                                         amax_out=amax_b[1:2], s_inv=s_inv)
                 gemm(xq, sx, wq0, sw, bias, out=yd)
@@ -605,37 +646,43 @@ def run_ours(args):
         # read X (bf16) + s, write Xq + sx (per-tensor: + the scale, + the max)
         q_bytes = M * K * 2 + M * K + M * 4 + (K * 4 if case.smooth else 0)
         g_bytes = M * K + N * K + M * N * 2 + 4 * (M + N) + (2 * N if bias is not None else 0)
+        if wbits:
+            # bf16 X, the packed weight codes once, Y bf16, scales and bias
+            g_bytes = (M * K * 2 + N * K * wbits // 8 + M * N * 2 + 4 * N
+                       + (2 * N if bias is not None else 0))
+        w_set = N * K * (wbits or 8) // 8
         line = {
             "metric": metric_for(case), "value": value, "unit": UNIT, "n_gpus": ws,
             "steps": K_steps, "warmup": args.warmup, "ms_per_step": elapsed_ms / K_steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "i8" if qt == "i8" else "e4m3",
+            "dtype": "bf16" if wbits else ("i8" if qt == "i8" else "e4m3"),
             "data": f"synthetic, seeded: {case.note}",
             "config": {"workload": case.name, "M": M, "K": K, "N": N,
                        "alpha": case.alpha if case.smooth else None,
-                       "act_scaling": ("per-tensor, delayed" if tensor else "per-token"),
+                       "act_scaling": ("none (weight-only)" if wbits else
+                                       "per-tensor, delayed" if tensor else "per-token"),
                        "bias": bias is not None, "out": "bf16",
                        "l2": (f"{ROTATE} rotating input sets (X + Wq, "
-                              f"{ROTATE * (M * K * 2 + N * K) / 2 ** 20:.0f} MiB) > 126 MiB L2"),
+                              f"{ROTATE * (M * K * 2 + w_set) / 2 ** 20:.0f} MiB) > 126 MiB L2"),
                        "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU",
                        "launch": ((f"CUDA graph of {g_steps} steps, replayed"
                                    + (f", then one of {tail_steps}" if tail_steps else ""))
                                   if graph is not None else "one launch per kernel"),
                        "split_last_wave": split,
                        "gemm_tile": os.environ.get("SQ_GEMM_TILE", "auto")},
-            "frac_of_int8_peak": value / ws / int8_peak,
-            "frac_of_datasheet": value / ws / DATASHEET_8BIT_TOPS,
+            "frac_of_int8_peak": None if wbits else value / ws / int8_peak,
+            "frac_of_datasheet": None if wbits else value / ws / DATASHEET_8BIT_TOPS,
             "int8_peak_tops": int8_peak,
             "datasheet_8bit_tops": DATASHEET_8BIT_TOPS,
             "int8_peak_source": f"2 x {pk['src']} bf16 dense ({pk['bf16']} TFLOP/s burst)",
             "gemm_hbm_gbs": g_bytes / (t_gemm * 1e-3) / 1e9,
             "roofline": gemm_roofline(case.ops, g_bytes, t_gemm, int8_peak, int8_peak_sus,
                                       pk["hbm"], profiled_traffic(g_kind, case.name), g_name),
-            "roofline_quant": {"bound": "hbm", "kernel": quant_kernel_name(case),
-                               "achieved": q_bytes / (t_quant * 1e-3) / 1e9, "peak": pk["hbm"],
-                               "unit": "GB/s", "frac": q_bytes / (t_quant * 1e-3) / 1e9 / pk["hbm"],
-                               "traffic": profiled_traffic("quant", case.name),
-                               "ms_per_launch": t_quant},
+            "roofline_quant": None if wbits else {
+                "bound": "hbm", "kernel": quant_kernel_name(case),
+                "achieved": q_bytes / (t_quant * 1e-3) / 1e9, "peak": pk["hbm"],
+                "unit": "GB/s", "frac": q_bytes / (t_quant * 1e-3) / 1e9 / pk["hbm"],
+                "traffic": profiled_traffic("quant", case.name), "ms_per_launch": t_quant},
             "gpu_launches": launches_per_step(case) * K_steps,
             "clocks": clocks,
             "sustained": sustained,

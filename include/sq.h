@@ -53,7 +53,7 @@
 extern "C" {
 #endif
 
-#define SQ_ABI_VERSION 5
+#define SQ_ABI_VERSION 6
 
 typedef enum {
     SQ_OK = 0,
@@ -70,7 +70,8 @@ typedef enum {
     SQ_BF16 = 1,  /* bfloat16 (raw 16-bit patterns)                          */
     SQ_I8 = 2,    /* signed 8-bit integer code                               */
     SQ_E4M3 = 3,  /* FP8 E4M3 code: bias 7, no infinity, max finite 448      */
-    SQ_I32 = 4    /* signed 32-bit integer                                   */
+    SQ_I32 = 4,   /* signed 32-bit integer                                   */
+    SQ_I4 = 5     /* signed 4-bit code (-7..7), two per byte, low nibble first */
 } sq_dtype;
 
 typedef enum {
@@ -133,13 +134,18 @@ sq_status sq_smooth_factors(const float* amax_x, const float* amax_w,
  * quantize(W_tilde)); §4 "Per-Tensor Scaling for FP8" for qt = SQ_E4M3.
  *   w  : [K,N] row-major, dtype wt (SQ_F32 or SQ_BF16)
  *   s  : [K] smoothing factors, or NULL for no smoothing
- *   qt : SQ_I8 or SQ_E4M3
+ *   qt : SQ_I8, SQ_E4M3 or SQ_I4 (below)
  *   wq : [N,K] output codes (transposed, K contiguous)
  *   sw : [N] output scales
  * For each n: wt[k] = s[k]*w[k,n]; sw[n] = max_k|wt[k]| / Q (Q = 127 for
  * INT8, 448 for E4M3); wq[n,k] = clamp(rne(wt[k]/sw[n]), -127, 127) for INT8,
  * or the E4M3 code of wt[k]/sw[n] (nearest-even, saturating to +-448). A
  * column with sw[n] == 0 gets all-zero codes.
+ * qt = SQ_I4 (weight-only W4A16, see sq_gemm_weight_only): s must be NULL
+ * (SQ_ERR_UNSUPPORTED otherwise) and K a multiple of 32; sw[n] = max_k|w[k,n]|
+ * / 7, codes clamp(rne(w[k,n]/sw[n]), -7, 7), stored packed as wq [N, K/2]
+ * bytes: byte k/2 of row n holds the code of even k in its low nibble and of
+ * odd k in its high nibble (two's complement).
  */
 sq_status sq_quantize_weight(const void* w, sq_dtype wt, int64_t K, int64_t N,
                              const float* s, sq_dtype qt, void* wq, float* sw,
@@ -269,6 +275,33 @@ sq_status sq_gemm_fp8(const uint8_t* xq, const float* sx, const uint8_t* wq,
                       const float* sw, const uint16_t* bias, int64_t M,
                       int64_t N, int64_t K, void* y, sq_dtype yt,
                       void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Weight-only quantized linear layer for few tokens (decode): W8A16 and
+ * W4A16, the schemes the pages set against W8A8. Source: "Weight-Activation
+ * Quantization" (infra.bea.ai) §1 table (W4A16: INT4 weights dequantized,
+ * then a 16-bit multiply); the zenaique flashcard on activation quantization
+ * (the weights are dequantized on the fly to multiply the BF16
+ * activations); the grasp.study lesson on W8A16 vs W8A8, §1 and §3; the
+ * zenaique page "W8A8 vs W4A16" (decode is bound by the weight read; 4-bit
+ * weights halve it again).
+ *   x   : [M,K] bf16 activations (not quantized, not smoothed)
+ *   wq  : per-output-channel weight codes from sq_quantize_weight with s =
+ *         NULL: wqt = SQ_I8 -> int8 [N,K]; wqt = SQ_I4 -> packed [N,K/2]
+ *   sw  : [N] channel scales (4-byte aligned); bias : [N] bf16 or NULL
+ *   y   : [M,N], yt = SQ_BF16 or SQ_F32
+ * y[m,n] = bf16( RN(sum_k x[m,k] * q[n,k]) * sw[n] + bias[n] ): the codes are
+ * widened exactly to bf16 and multiplied by x on the tensor cores with
+ * binary32 accumulation (order unspecified); the channel scale multiplies
+ * the sum, then the bias is added, each step rounded in binary32. The result
+ * differs from the exact sum_k x * (q * sw) only by that accumulation.
+ * K must be a multiple of 16 (SQ_I8) or 32 (SQ_I4); N a multiple of 8. Built
+ * for M <= 16 (one pass over the weights); larger M runs one pass per 16
+ * tokens.
+ */
+sq_status sq_gemm_weight_only(const void* x, const void* wq, sq_dtype wqt, const float* sw,
+                              const uint16_t* bias, int64_t M, int64_t N, int64_t K, void* y,
+                              sq_dtype yt, void* stream);
 
 /*
  * Runtime forward of one SmoothQuant linear layer: sq_quantize_act followed

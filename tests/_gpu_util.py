@@ -79,3 +79,14 @@ def fp8_normalized_error_full(y, y_ref, xq=None, wq=None, sx=None, sw=None, bias
         den = fp8_error_denominator(xq, wq, sx, sw, bias)
     num = np.abs(np.asarray(y, np.float64) - np.asarray(y_ref, np.float64))
     return np.where(den > 0, num / np.where(den > 0, den, 1.0), num)
+
+
+def weight_only_error_denominator(x_bf16, codes, sw, bias):
+    """sw[n] * sum_k |x[m,k] q[n,k]| + |bias[n]| for the weight-only GEMM: the
+    magnitude its binary32 accumulation error is measured against."""
+    xa = np.abs(oracle.bf16_to_f32_array(x_bf16).astype(np.float64))
+    mag = xa @ np.abs(codes.astype(np.float64)).T
+    den = mag * np.asarray(sw, np.float64)[None, :]
+    if bias is not None:
+        den = den + np.abs(oracle.bf16_to_f32_array(bias).astype(np.float64))[None, :]
+    return np.where(den > 0, den, 1.0)

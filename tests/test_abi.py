@@ -53,7 +53,7 @@ def test_exported_symbols_are_visible_to_the_dynamic_linker():
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.sq_abi_version() == 5
+    assert lib.sq_abi_version() == 6
     for st in range(7):
         assert ops.status_string(st).startswith("SQ_")
     assert "TIMEOUT" in ops.status_string(ops.SQ_ERR_TIMEOUT)

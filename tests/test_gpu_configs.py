@@ -14,7 +14,8 @@ import torch
 import oracle
 from w8a8_smoothquant_int8_02_b200 import ops, synth, workloads
 
-from _gpu_util import dev, fp8_normalized_error_full, host, ulp_distance
+from _gpu_util import (dev, fp8_normalized_error_full, host, ulp_distance,
+                       weight_only_error_denominator)
 
 pytestmark = pytest.mark.gpu
 
@@ -25,9 +26,40 @@ def _reciprocals(s):
     return np.where(inside, np.float32(1.0) / np.where(inside, s, 1), np.float32(np.nan)).astype(np.float32)
 
 
+def _weight_only_end_to_end(case):
+    """Weight-only workloads: per-channel weight codes and scales bit-exact,
+    then every output element of the GEMM within 1e-3 of the binary64 product
+    (normalized by sw * sum_k |x q| + |bias|), bf16 the rounding of binary32."""
+    bits = workloads.WEIGHT_ONLY_BITS[case.qtype]
+    d = synth.generate(case)
+    x, w, bias = d["x"], d["w"], d["bias"]
+    if bits == 8:
+        wq_ref, sw_ref = oracle.quantize_weight(w, None)
+    else:
+        wq_ref, sw_ref = oracle.quantize_weight_i4(w)
+    wq_d, sw_d = ops.quantize_weight(dev(w), None, "i8" if bits == 8 else "i4")
+    np.testing.assert_array_equal(host(sw_d), sw_ref)
+    np.testing.assert_array_equal(host(wq_d).view(np.uint8), wq_ref.view(np.uint8))
+    bias_d = None if bias is None else dev(bias)
+    xd = dev(x)
+    yf = ops.gemm_weight_only(xd, wq_d, sw_d, bias_d, bits, out_dtype=torch.float32)
+    yb = ops.gemm_weight_only(xd, wq_d, sw_d, bias_d, bits)
+    assert ops.device_status() == ops.SQ_OK
+    y_ref = oracle.gemm_weight_only(x, wq_ref, sw_ref, bias, bits)
+    codes = wq_ref if bits == 8 else oracle.unpack_i4(wq_ref)
+    den = weight_only_error_denominator(x, codes, sw_ref, bias)
+    got = host(yf)
+    e = np.abs(got.astype(np.float64) - y_ref) / den
+    assert e.max() <= 1e-3, e.max()
+    np.testing.assert_array_equal(host(yb), oracle.f32_to_bf16(got))
+
+
 @pytest.mark.parametrize("name", list(workloads.ALL))
 def test_workload_end_to_end(name):
     case = workloads.ALL[name]
+    if case.qtype in workloads.WEIGHT_ONLY_BITS:
+        _weight_only_end_to_end(case)
+        return
     qt = oracle.E4M3 if case.qtype == "e4m3" else oracle.INT8
     d = synth.generate(case)
     x, x_cal, w, bias = d["x"], d["x_cal"], d["w"], d["bias"]

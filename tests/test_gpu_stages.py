@@ -491,6 +491,42 @@ def test_quantize_act_streaming_rows_edge_values(qtype, K):
         np.testing.assert_array_equal(host(xq).view(np.uint8), xq_ref.view(np.uint8))
 
 
+@pytest.mark.parametrize("qtype", ["i8", "e4m3"])
+@pytest.mark.parametrize("M,K", [(40000, 1024), (12000, 4096), (9000, 4112), (5000, 8192),
+                                 (2000, 14336)])
+def test_quantize_act_many_rows_per_cta(qtype, M, K):
+    """Enough rows that every persistent CTA of the many-row kernel handles
+    many of them (its ring slots are refilled and its per-row buffers reused
+    several times), with the edge rows of the test above repeated every 500
+    rows; with and without the caller's reciprocals."""
+    g = np.random.default_rng(M + K)
+    x = (g.standard_normal((M, K)) * 3).astype(np.float32)
+    ch = g.choice(K, size=K // 100, replace=False)
+    x[:, ch] *= g.uniform(20, 100, ch.size).astype(np.float32)
+    for r0 in range(0, M - 16, 500):
+        x[r0 + 0] = 0.0
+        x[r0 + 1] = -0.0
+        x[r0 + 2] *= 1e-25
+        x[r0 + 3] *= 1e28
+        x[r0 + 4] = 1e-40
+        x[r0 + 5, :8] = [0.0, -0.0, 1e-30, -1e-30, 1e-40, -1e-40, 2.0 ** -100, -(2.0 ** -90)]
+        x[r0 + 6, :6] = [127.0, 63.5, -0.5, 1.5, 2.5, -126.5]
+        x[r0 + 7:r0 + 12] = np.round(x[r0 + 7:r0 + 12] * 2) / 2
+        x[r0 + 12, -1] = 3000.0
+    s = synth.random_floats(K, seed=K + 5, lo=0.05, hi=20.0)
+    s[:6] = 1.0
+    xb = synth.to_bf16_bits(x)
+    qt = oracle.E4M3 if qtype == "e4m3" else oracle.INT8
+    xd = dev(xb)
+    for smooth, inv in ((s, reciprocals(s)), (s, None), (None, None)):
+        xq_ref, sx_ref = oracle.quantize_act(xb, smooth, qt)
+        xq, sx = ops.quantize_act(xd, None if smooth is None else dev(smooth), qtype,
+                                  s_inv=None if inv is None else dev(inv))
+        assert ops.device_status() == ops.SQ_OK
+        np.testing.assert_array_equal(host(sx), sx_ref)
+        np.testing.assert_array_equal(host(xq).view(np.uint8), xq_ref.view(np.uint8))
+
+
 # ---------------------------------------------------------- failure path --
 
 def test_bounded_wait_reports_timeout_and_context_survives():

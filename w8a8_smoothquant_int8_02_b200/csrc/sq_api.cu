@@ -172,11 +172,16 @@ sq_status sq_quantize_weight(const void* w, sq_dtype wt, int64_t K, int64_t N, c
                              sq_dtype qt, void* wq, float* sw, void* stream) {
   if (!w || !wq || !sw) return SQ_ERR_INVALID_ARG;
   if (wt != SQ_F32 && wt != SQ_BF16) return SQ_ERR_INVALID_ARG;
-  if (qt != SQ_I8 && qt != SQ_E4M3) return SQ_ERR_INVALID_ARG;
+  if (qt != SQ_I8 && qt != SQ_E4M3 && qt != SQ_I4) return SQ_ERR_INVALID_ARG;
   if (K <= 0 || N <= 0 || K % 16 != 0 || N % 8 != 0 || K > INT32_MAX || N > INT32_MAX)
     return SQ_ERR_INVALID_ARG;
+  if (qt == SQ_I4 && K % 32 != 0) return SQ_ERR_INVALID_ARG;
+  if (qt == SQ_I4 && s) return SQ_ERR_UNSUPPORTED;  // weight-only: no smoothing
   if (!al(w, 16) || !al(wq, 16) || !al(sw, 16)) return SQ_ERR_MISALIGNED;
   if (s && !al(s, 4)) return SQ_ERR_MISALIGNED;
+  if (qt == SQ_I4)
+    return from_cuda(sqh::launch_quantize_weight_i4(w, wt == SQ_BF16, K, N,
+                                                    static_cast<uint8_t*>(wq), sw, S(stream)));
   return from_cuda(sqh::launch_quantize_weight(w, wt == SQ_BF16, K, N, s, qt == SQ_E4M3,
                                                static_cast<uint8_t*>(wq), sw, S(stream)));
 }
@@ -300,6 +305,23 @@ sq_status sq_gemm_w8a8_noalloc(const int8_t* xq, const float* sx, const int8_t* 
                                     reinterpret_cast<const uint8_t*>(wq), sw, bias, M, N, K, y,
                                     yt == SQ_BF16 ? sqh::OutKind::BF16 : sqh::OutKind::F32, nullptr,
                                     scratch, kNoAllocScratchBytes, S(stream)));
+}
+
+sq_status sq_gemm_weight_only(const void* x, const void* wq, sq_dtype wqt, const float* sw,
+                              const uint16_t* bias, int64_t M, int64_t N, int64_t K, void* y,
+                              sq_dtype yt, void* stream) {
+  if (wqt != SQ_I8 && wqt != SQ_I4) return SQ_ERR_INVALID_ARG;
+  if (M < 0 || N <= 0 || K <= 0 || N % 8 != 0) return SQ_ERR_INVALID_ARG;
+  if (K % (wqt == SQ_I4 ? 32 : 16) != 0) return SQ_ERR_INVALID_ARG;
+  if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return SQ_ERR_INVALID_ARG;
+  if (yt != SQ_BF16 && yt != SQ_F32) return SQ_ERR_INVALID_ARG;
+  if (M == 0) return SQ_OK;  // empty batch: pointers may be NULL
+  if (!x || !wq || !sw || !y) return SQ_ERR_INVALID_ARG;
+  if (!al(x, 16) || !al(wq, 16) || !al(y, 16) || !al(sw, 4)) return SQ_ERR_MISALIGNED;
+  if (bias && !al(bias, 2)) return SQ_ERR_MISALIGNED;
+  return from_cuda(sqh::launch_gemm_weight_only(
+      wqt == SQ_I4 ? 4 : 8, static_cast<const uint16_t*>(x), wq, sw, bias, M, N, K, y,
+      yt == SQ_BF16 ? sqh::OutKind::BF16 : sqh::OutKind::F32, S(stream)));
 }
 
 sq_status sq_selftest_fast_division(int64_t* mismatches, void* stream) {

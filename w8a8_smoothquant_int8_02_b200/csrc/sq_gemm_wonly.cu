@@ -1,0 +1,465 @@
+// sq_gemm_wonly.cu -- weight-only quantized GEMM for few tokens (decode),
+// sm_100a (tcgen05 + TMA + tensor memory): W8A16 and W4A16.
+//
+//   y[m,n] = bf16( float( sum_k x[m,k] * q[n,k] ) * sw[n] + bias[n] )
+//
+// x is bf16 [M,K]; q are the per-output-channel weight codes (INT8 [N,K], or
+// INT4 packed two per byte [N,K/2], low nibble = even k) with scales sw [N].
+// Source: the pages' weight-only schemes -- "Weight-Activation
+// Quantization" (infra.bea.ai) §1 table (W4A16: INT4 weights dequantized to
+// 16 bits, then a 16-bit multiply), the zenaique flashcard on activation
+// quantization (the runtime dequantizes the weights on the fly against BF16
+// activations), the grasp.study lesson on W8A16 vs W8A8 §1 and §3, and the
+// zenaique "W8A8 vs W4A16" page (decode is bound by the weight read; 4-bit
+// weights read half the bytes of 8-bit ones).
+//
+// Dequantization: every INT8 / INT4 code is exactly representable in bf16,
+// so the weights are widened to bf16 codes in shared memory and multiplied by
+// the bf16 activations on the tensor cores (kind::f16, binary32 accumulators
+// in tensor memory); the channel scale sw[n] is constant along k, so it is
+// applied once to the sum in the epilogue: sum_k x * (q * sw) = sw * sum_k x*q.
+//
+// Roles are swapped as in the few-token W8A8 kernel: 128 weight rows are the
+// M = 128 operand, the (up to) 16 token rows the N = 16 operand, D[n][m] in
+// 128 lanes x 16 columns of tensor memory. One CTA per 128 output channels
+// and 16 tokens (grid.y walks token tiles of larger batches).
+//   warp 0      : TMA producer -- per stage one 128-byte-wide K slice of the
+//                 packed weights [128 rows x 128 B] (128 k for INT8, 256 for
+//                 INT4) and the matching bf16 token slices [16 rows x 64 k]
+//   warp 1      : tensor memory (32 columns); one thread issues the MMAs
+//                 (K = 16 per instruction) and frees buffers by tcgen05.commit
+//   warps 2..9  : widen the weight codes of each stage into bf16 sub-tiles
+//                 [128 rows x 64 k] (128-byte swizzle, the layout the MMA
+//                 reads); warps 2..5 then run the epilogue
+// Every barrier wait is bounded: a wait that gives up records
+// SQ_ERR_TIMEOUT, the CTA skips its remaining work, waits (bounded) for its
+// copies and MMAs in flight and still frees tensor memory.
+#include <cstdint>
+#include <cstdlib>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "sq_common.cuh"
+#include "sq_internal.h"
+
+namespace sqk {
+
+constexpr int kWoTokens = 16;                 // token columns (N of the instruction)
+constexpr int kWoConvWarps = 8;               // warps widening the weight codes
+constexpr int kWoThreads = 64 + 32 * kWoConvWarps;
+constexpr uint32_t kWoWBytes = 128 * 128;     // packed weight slice of one stage
+constexpr uint32_t kWoSubBytes = 128 * 128;   // bf16 weight sub-tile [128 x 64 k]
+constexpr uint32_t kWoXSub = kWoTokens * 128; // bf16 token sub-tile [16 x 64 k]
+
+template <int BITS>
+struct WoCfg {
+  static constexpr int KS = BITS == 8 ? 128 : 256;   // k per stage
+  static constexpr int SUBS = KS / 64;               // bf16 sub-tiles per stage
+  static constexpr int STAGES = 3;                   // packed-weight ring
+  static constexpr int NA = BITS == 8 ? 3 : 2;       // bf16 weight ring
+  static constexpr uint32_t kXBytes = SUBS * kWoXSub;
+  static constexpr uint32_t kStageBytes = kWoWBytes + kXBytes;
+  static constexpr uint32_t kRingA = STAGES * kStageBytes;          // 1024-aligned
+  static constexpr uint32_t kBarOff = kRingA + NA * kWoSubBytes;
+  // barriers: full[S], empty[S], afull[NA], aempty[NA], tfull, drain
+  static constexpr uint32_t kMiscOff = kBarOff + (2 * STAGES + 2 * NA + 2) * 8;
+  static constexpr uint32_t kDynamic = kMiscOff + 16 + 1024;  // slack for 1024-B alignment
+  static_assert(kStageBytes % 1024 == 0, "stages must keep 1024-byte alignment");
+  static_assert(2 * (kDynamic + 1024) <= 233472, "two CTAs per SM must fit");
+};
+
+// Instruction descriptor of tcgen05.mma kind::f16 with bf16 A and B (both
+// K-major) and binary32 accumulators: bits 4-5 D format, 7-9 / 10-12 A / B
+// formats, 17-22 N/8, 24-28 M/16.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int m, int n) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(n >> 3) << 17) | (uint32_t(m >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                         uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  return __byte_perm(a, b, sel);
+}
+
+// Four offset-binary bytes u (= code + OFF) of `u4` -> two words of two bf16
+// codes each (elements in byte order). 0x4B0000uu is the binary32 2^23 + u,
+// so subtracting 2^23 + OFF leaves the code exactly, and a code of at most 8
+// significant bits is its own bf16 (the upper half of its binary32 word).
+template <int OFF>
+__device__ __forceinline__ void widen4(uint32_t u4, uint32_t& w01, uint32_t& w23) {
+  constexpr uint32_t kExp = 0x4B000000u;
+  constexpr float kBias = 8388608.0f + float(OFF);
+  const uint64_t bias2 = f2_make(kBias, kBias);
+  float a, b, c, d;
+  f2_split(f2_sub(f2_make(__uint_as_float(prmt(u4, kExp, 0x7440)),
+                          __uint_as_float(prmt(u4, kExp, 0x7441))), bias2), a, b);
+  f2_split(f2_sub(f2_make(__uint_as_float(prmt(u4, kExp, 0x7442)),
+                          __uint_as_float(prmt(u4, kExp, 0x7443))), bias2), c, d);
+  w01 = prmt(__float_as_uint(a), __float_as_uint(b), 0x7632);
+  w23 = prmt(__float_as_uint(c), __float_as_uint(d), 0x7632);
+}
+
+// Two offset-binary nibble bytes (even elements in `lo`, odd in `hi`, byte i
+// of each holding elements 2i and 2i + 1) -> four words of bf16 pairs in
+// element order.
+__device__ __forceinline__ void widen8_nibbles(uint32_t lo, uint32_t hi, uint32_t (&w)[4]) {
+  constexpr uint32_t kExp = 0x4B000000u;
+  constexpr float kBias = 8388608.0f + 8.0f;
+  const uint64_t bias2 = f2_make(kBias, kBias);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float a, b;
+    f2_split(f2_sub(f2_make(__uint_as_float(prmt(lo, kExp, 0x7440 + i)),
+                            __uint_as_float(prmt(hi, kExp, 0x7440 + i))), bias2), a, b);
+    w[i] = prmt(__float_as_uint(a), __float_as_uint(b), 0x7632);
+  }
+}
+
+__device__ __forceinline__ uint32_t sw128_off(uint32_t row, uint32_t chunk) {
+  return row * 128u + ((chunk ^ (row & 7u)) << 4);
+}
+
+__device__ __forceinline__ void tmem_ld16_wait_wo(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32"
+      " {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+
+template <int BITS, bool OUT_BF16, bool HAS_BIAS>
+__global__ void __launch_bounds__(kWoThreads, 2)
+    gemm_wonly_kernel(const __grid_constant__ CUtensorMap tm_w,
+                      const __grid_constant__ CUtensorMap tm_x, const float* __restrict__ sw,
+                      const uint16_t* __restrict__ bias, void* __restrict__ y, int M, int N,
+                      int K, int* status) {
+  using C = WoCfg<BITS>;
+  constexpr int S = C::STAGES, NA = C::NA, SUBS = C::SUBS;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t s_base = smem_u32(smem);
+  const uint32_t s_a = s_base + C::kRingA;
+  const uint32_t bar_full = s_base + C::kBarOff;
+  const uint32_t bar_empty = bar_full + S * 8;
+  const uint32_t bar_afull = bar_empty + S * 8;
+  const uint32_t bar_aempty = bar_afull + NA * 8;
+  const uint32_t bar_tfull = bar_aempty + NA * 8;
+  const uint32_t bar_drain = bar_tfull + 8;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < S; ++i) {
+      mbar_init(bar_full + 8 * i, 1);
+      mbar_init(bar_empty + 8 * i, kWoConvWarps + 1);  // every widening warp + the MMAs
+    }
+    for (int i = 0; i < NA; ++i) {
+      mbar_init(bar_afull + 8 * i, kWoConvWarps);
+      mbar_init(bar_aempty + 8 * i, 1);
+    }
+    mbar_init(bar_tfull, 1);
+    mbar_init(bar_drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    tma_prefetch_map(&tm_w);
+    tma_prefetch_map(&tm_x);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 32);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  // set-up above overlaps the previous kernel; its results are read below
+  pdl_launch_dependents();
+  pdl_wait();
+
+  const int n0 = int(blockIdx.x) * 128;
+  const int m0 = int(blockIdx.y) * kWoTokens;
+  const int nk = (K + C::KS - 1) / C::KS;
+  auto give_up = [&]() {
+    record_status(status, kStatusTimeout);
+    *abort_flag = 1;
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer --
+    if (lane == 0) {
+      int issued = 0;
+#pragma unroll 1
+      for (int kb = 0; kb < nk; ++kb) {
+        const uint32_t st = uint32_t(kb % S), ph = uint32_t(kb / S) & 1u;
+        if (*abort_flag || !mbar_wait(bar_empty + 8 * st, ph ^ 1u)) {
+          give_up();
+          break;
+        }
+        const uint32_t dst = s_base + st * C::kStageBytes;
+        mbar_arrive_expect_tx(bar_full + 8 * st, C::kStageBytes);
+        tma_load_2d(dst, &tm_w, bar_full + 8 * st, kb * 128, n0);
+#pragma unroll
+        for (int t = 0; t < SUBS; ++t)
+          tma_load_2d(dst + kWoWBytes + t * kWoXSub, &tm_x, bar_full + 8 * st,
+                      kb * C::KS + t * 64, m0);
+        ++issued;
+      }
+      // no copy may still be writing shared memory when the CTA exits
+      const int first = issued > S ? issued - S : 0;
+#pragma unroll 1
+      for (int j = first; j < issued; ++j)
+        (void)mbar_wait(bar_full + 8 * uint32_t(j % S), uint32_t(j / S) & 1u);
+    }
+  } else if (warp == 1) {
+    // ----------------------------------------------------------------- MMA --
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(128, kWoTokens);
+      bool ok = true;
+      uint32_t ia = 0;
+#pragma unroll 1
+      for (int kb = 0; kb < nk && ok; ++kb) {
+        const uint32_t st = uint32_t(kb % S), ph = uint32_t(kb / S) & 1u;
+        if (*abort_flag || !mbar_wait(bar_full + 8 * st, ph)) {
+          give_up();
+          ok = false;
+          break;
+        }
+        const uint32_t x_addr = s_base + st * C::kStageBytes + kWoWBytes;
+#pragma unroll 1
+        for (int t = 0; t < SUBS; ++t, ++ia) {
+          const uint32_t slot = ia % NA;
+          if (*abort_flag || !mbar_wait(bar_afull + 8 * slot, (ia / NA) & 1u)) {
+            give_up();
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = s_a + slot * kWoSubBytes;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t ad = sw128_desc(a_addr + kk * 32);
+            const uint64_t bd = sw128_desc(x_addr + t * kWoXSub + kk * 32);
+            mma_bf16(tmem_base, ad, bd, idesc, (kb > 0 || t > 0 || kk > 0) ? 1u : 0u);
+          }
+          tc_commit(bar_aempty + 8 * slot);
+        }
+        if (!ok) break;
+        tc_commit(bar_empty + 8 * st);  // the token slices of this stage are read
+      }
+      if (ok) tc_commit(bar_tfull);
+      // every MMA issued has finished before tensor memory can be freed
+      tc_commit(bar_drain);
+      (void)mbar_wait(bar_drain, 0);
+    }
+  } else {
+    // ------------------------------------------- widening, then epilogue --
+    const int cw = warp - 2;                   // 0 .. kWoConvWarps - 1
+    const uint32_t row = uint32_t(cw & 3) * 32u + uint32_t(lane);   // weight row of the tile
+    const int part = cw >> 2;                  // which half of the row's source chunks
+    uint32_t ia = 0;
+    bool ok = true;
+#pragma unroll 1
+    for (int kb = 0; kb < nk && ok; ++kb) {
+      const uint32_t st = uint32_t(kb % S), ph = uint32_t(kb / S) & 1u;
+      if (*abort_flag || !mbar_wait(bar_full + 8 * st, ph)) {
+        give_up();
+        ok = false;
+        break;
+      }
+      const uint8_t* wsrc = smem + st * C::kStageBytes;
+#pragma unroll 1
+      for (int t = 0; t < SUBS; ++t, ++ia) {
+        const uint32_t slot = ia % NA;
+        if (*abort_flag || !mbar_wait(bar_aempty + 8 * slot, ((ia / NA) & 1u) ^ 1u)) {
+          give_up();
+          ok = false;
+          break;
+        }
+        uint8_t* adst = smem + C::kRingA + slot * kWoSubBytes;
+        if constexpr (BITS == 8) {
+          // sub-tile t holds source chunks 4t .. 4t+3 (16 codes each); this
+          // warp widens two of them per row: 4 bf16 chunks of 8 codes
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const uint32_t j = uint32_t(4 * t + 2 * part + h);
+            const uint4 q = *reinterpret_cast<const uint4*>(wsrc + sw128_off(row, j));
+            uint4 o0, o1;
+            widen4<128>(q.x ^ 0x80808080u, o0.x, o0.y);
+            widen4<128>(q.y ^ 0x80808080u, o0.z, o0.w);
+            widen4<128>(q.z ^ 0x80808080u, o1.x, o1.y);
+            widen4<128>(q.w ^ 0x80808080u, o1.z, o1.w);
+            const uint32_t c0 = 2u * (j - 4u * uint32_t(t));
+            *reinterpret_cast<uint4*>(adst + sw128_off(row, c0)) = o0;
+            *reinterpret_cast<uint4*>(adst + sw128_off(row, c0 + 1)) = o1;
+          }
+        } else {
+          // sub-tile t holds source chunks 2t, 2t+1 (32 codes each); this
+          // warp widens one of them per row: 4 bf16 chunks of 8 codes
+          const uint32_t j = uint32_t(2 * t + part);
+          const uint4 q = *reinterpret_cast<const uint4*>(wsrc + sw128_off(row, j));
+          const uint32_t qw[4] = {q.x, q.y, q.z, q.w};
+          const uint32_t c0 = 4u * uint32_t(part);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            // nibble ^ 8 is the offset-binary code + 8
+            const uint32_t lo = (qw[i] & 0x0F0F0F0Fu) ^ 0x08080808u;
+            const uint32_t hi = ((qw[i] >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;
+            uint32_t w[4];
+            widen8_nibbles(lo, hi, w);
+            *reinterpret_cast<uint4*>(adst + sw128_off(row, c0 + uint32_t(i))) =
+                make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        }
+        // the tensor cores read the sub-tile through the async proxy
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_afull + 8 * slot);
+      }
+      if (!ok) break;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_empty + 8 * st);  // this warp is done with the stage
+    }
+    if (cw < 4) {
+      // epilogue: warp w reads TMEM lanes 32*(w%4) .. +31 = output channels
+      const int sub = warp & 3;
+      const int n = n0 + sub * 32 + lane;
+      if (!ok || *abort_flag || !mbar_wait(bar_tfull, 0)) {
+        give_up();
+      } else {
+        tc_fence_after();
+        uint32_t r[16];
+        tmem_ld16_wait_wo(tmem_base + (uint32_t(sub * 32) << 16), r);
+        if (n < N) {
+          const float swn = __ldg(sw + n);
+          float bn = 0.0f;
+          if constexpr (HAS_BIAS) bn = __uint_as_float(uint32_t(__ldg(bias + n)) << 16);
+#pragma unroll
+          for (int j = 0; j < kWoTokens; ++j) {
+            const int m = m0 + j;
+            if (m < M) {
+              float a = __fmul_rn(__uint_as_float(r[j]), swn);
+              if constexpr (HAS_BIAS) a = __fadd_rn(a, bn);
+              const int64_t off = int64_t(m) * N + n;
+              if constexpr (OUT_BF16)
+                static_cast<uint16_t*>(y)[off] = uint16_t(pack_bf16x2(a, 0.0f) & 0xFFFFu);
+              else
+                static_cast<float*>(y)[off] = a;
+            }
+          }
+        }
+      }
+    }
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 32);
+  }
+}
+
+}  // namespace sqk
+
+namespace sqh {
+
+using namespace sqk;
+
+typedef CUresult (*WoEncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                    const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static WoEncodeTiledFn wo_encoder() {
+  static WoEncodeTiledFn enc = nullptr;
+  if (!enc) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      enc = reinterpret_cast<WoEncodeTiledFn>(p);
+  }
+  return enc;
+}
+
+// Row-major [rows, cols] matrix of `elem` bytes per element: box = box_cols x
+// box_rows (box_cols * elem = 128 bytes), 128-byte swizzle, zero fill.
+static bool wo_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int elem,
+                   int64_t rows, int64_t cols, int box_cols, int box_rows) {
+  WoEncodeTiledFn enc = wo_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {cuuint64_t(cols), cuuint64_t(rows)};
+  cuuint64_t strides[1] = {cuuint64_t(cols) * cuuint64_t(elem)};
+  cuuint32_t box[2] = {cuuint32_t(box_cols), cuuint32_t(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int BITS, bool OUT_BF16, bool HAS_BIAS>
+static cudaError_t run_wonly(const void* x, const void* wq, const float* sw, const uint16_t* bias,
+                             void* y, int M, int N, int K, cudaStream_t st) {
+  using C = WoCfg<BITS>;
+  auto kern = gemm_wonly_kernel<BITS, OUT_BF16, HAS_BIAS>;
+  CUtensorMap tw, tx;
+  const int64_t wcols = BITS == 8 ? K : K / 2;  // bytes per weight row
+  if (!wo_map(&tw, wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, wcols, 128, 128) ||
+      !wo_map(&tx, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, K, 64, kWoTokens))
+    return cudaErrorInvalidValue;
+  static uint64_t attr_set = 0;  // one bit per device ordinal
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 64 || !((attr_set >> dev) & 1u)) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         int(C::kDynamic));
+    if (e != cudaSuccess) return e;
+    if (dev < 64) attr_set |= uint64_t(1) << dev;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(unsigned((N + 127) / 128), unsigned((M + kWoTokens - 1) / kWoTokens), 1);
+  cfg.blockDim = dim3(kWoThreads, 1, 1);
+  cfg.dynamicSmemBytes = C::kDynamic;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, tw, tx, sw, bias, y, M, N, K, status_ptr());
+}
+
+cudaError_t launch_gemm_weight_only(int bits, const uint16_t* x, const void* wq, const float* sw,
+                                    const uint16_t* bias, int64_t M, int64_t N, int64_t K,
+                                    void* y, OutKind yk, cudaStream_t st) {
+  const int m = int(M), n = int(N), k = int(K);
+  const int key = (bits == 4 ? 4 : 0) | (yk == OutKind::BF16 ? 2 : 0) | (bias ? 1 : 0);
+#define SQ_WO(B, O, H) return run_wonly<B, O, H>(x, wq, sw, bias, y, m, n, k, st)
+  switch (key) {
+    case 0: SQ_WO(8, false, false);
+    case 1: SQ_WO(8, false, true);
+    case 2: SQ_WO(8, true, false);
+    case 3: SQ_WO(8, true, true);
+    case 4: SQ_WO(4, false, false);
+    case 5: SQ_WO(4, false, true);
+    case 6: SQ_WO(4, true, false);
+    default: SQ_WO(4, true, true);
+  }
+#undef SQ_WO
+}
+
+}  // namespace sqh

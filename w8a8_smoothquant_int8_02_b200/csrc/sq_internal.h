@@ -44,6 +44,12 @@ bool gemm_skinny_applies(int64_t M);
 cudaError_t launch_gemm_skinny(bool e4m3, const uint8_t* xq, const float* sx, const uint8_t* wq,
                                const float* sw, const uint16_t* bias, int64_t M, int64_t N,
                                int64_t K, void* y, OutKind yk, int32_t* acc, cudaStream_t st);
+// weight-only W8A16 / W4A16 GEMM for few tokens (sq_gemm_wonly.cu)
+cudaError_t launch_gemm_weight_only(int bits, const uint16_t* x, const void* wq, const float* sw,
+                                    const uint16_t* bias, int64_t M, int64_t N, int64_t K,
+                                    void* y, OutKind yk, cudaStream_t st);
+cudaError_t launch_quantize_weight_i4(const void* w, bool bf16, int64_t K, int64_t N,
+                                      uint8_t* wq4, float* sw, cudaStream_t st);
 size_t gemm_workspace_bytes();
 size_t gemm_workspace_counter_bytes();
 

@@ -20,7 +20,7 @@ from . import build as _build
 
 (SQ_OK, SQ_ERR_INVALID_ARG, SQ_ERR_MISALIGNED, SQ_ERR_UNSUPPORTED, SQ_ERR_CUDA, SQ_ERR_TIMEOUT,
  SQ_ERR_SCRATCH_TOO_SMALL) = range(7)
-SQ_F32, SQ_BF16, SQ_I8, SQ_E4M3, SQ_I32 = range(5)
+SQ_F32, SQ_BF16, SQ_I8, SQ_E4M3, SQ_I32, SQ_I4 = range(6)
 SQ_AMAX_PER_COLUMN, SQ_AMAX_PER_ROW = 0, 1
 
 EXPORTED = (
@@ -28,7 +28,7 @@ EXPORTED = (
     "sq_smooth_factors", "sq_quantize_weight", "sq_quantize_act", "sq_gemm_w8a8",
     "sq_gemm_fp8", "sq_linear", "sq_probe_wait_timeout", "sq_selftest_fast_division",
     "sq_gemm_workspace_bytes", "sq_gemm_w8a8_noalloc", "sq_quantize_act_tensor",
-    "sq_fold_smoothing",
+    "sq_fold_smoothing", "sq_gemm_weight_only",
 )
 
 _lock = threading.Lock()
@@ -71,6 +71,7 @@ def load(build_if_needed: bool = True) -> ctypes.CDLL:
             lib.sq_gemm_fp8.argtypes = [P, P, P, P, P, I64, I64, I64, P, I, P, SZ, P]
             lib.sq_linear.argtypes = [P, I, P, P, P, P, P, I, I64, I64, I64, P, P, P, I, P, SZ, P]
             lib.sq_gemm_w8a8_noalloc.argtypes = [P, P, P, P, P, I64, I64, I64, P, I, P]
+            lib.sq_gemm_weight_only.argtypes = [P, P, I, P, P, I64, I64, I64, P, I, P]
             lib.sq_gemm_workspace_bytes.argtypes = []
             lib.sq_gemm_workspace_bytes.restype = SZ
             lib.sq_probe_wait_timeout.argtypes = [I64, P]
@@ -112,7 +113,9 @@ def _qtype(q: str) -> int:
         return SQ_I8
     if q in ("e4m3", "fp8"):
         return SQ_E4M3
-    raise ValueError(f"qtype must be 'i8' or 'e4m3', got {q!r}")
+    if q in ("i4", "int4"):
+        return SQ_I4
+    raise ValueError(f"qtype must be 'i8', 'e4m3' or 'i4', got {q!r}")
 
 
 def _cuda(*ts):
@@ -185,11 +188,16 @@ def smooth_factors(amax_x: torch.Tensor, amax_w: torch.Tensor, alpha: float,
 
 
 def quantize_weight(w: torch.Tensor, s: torch.Tensor | None, qtype: str = "i8"):
-    """a4: returns (wq [N,K] int8 / uint8-E4M3, sw [N] float32)."""
+    """a4: returns (wq [N,K] int8 / uint8-E4M3, sw [N] float32); qtype "i4"
+    (weight-only, s None): wq [N,K/2] uint8, two codes per byte."""
     _cuda(w, s)
     K, N = w.shape
     qt = _qtype(qtype)
-    wq = torch.empty((N, K), dtype=torch.int8 if qt == SQ_I8 else torch.uint8, device=w.device)
+    if qt == SQ_I4:
+        wq = torch.empty((N, K // 2), dtype=torch.uint8, device=w.device)
+    else:
+        wq = torch.empty((N, K), dtype=torch.int8 if qt == SQ_I8 else torch.uint8,
+                         device=w.device)
     sw = torch.empty(N, dtype=torch.float32, device=w.device)
     _check(load().sq_quantize_weight(_p(w), _fdtype(w), K, N, _p(s), qt, _p(wq), _p(sw),
                                      _stream(w.device)), "sq_quantize_weight")
@@ -304,6 +312,24 @@ def gemm_fp8(xq, sx, wq, sw, bias=None, out_dtype=torch.bfloat16, out=None, spli
     wsp, wsn = _ws_args(split, xq.device)
     _check(load().sq_gemm_fp8(_p(xq), _p(sx), _p(wq), _p(sw), _p(bias), M, N, K, _p(out),
                               _fdtype(out), wsp, wsn, _stream(xq.device)), "sq_gemm_fp8")
+    return out
+
+
+def gemm_weight_only(x, wq, sw, bias=None, bits=8, out_dtype=torch.bfloat16, out=None):
+    """Weight-only W8A16 (bits 8: wq int8 [N,K]) or W4A16 (bits 4: wq packed
+    uint8 [N,K/2]) linear layer on bf16 activations x [M,K]."""
+    _cuda(x, wq, sw, bias, out)
+    if x.dtype != torch.bfloat16:
+        raise TypeError("x must be bfloat16")
+    M, K = x.shape
+    N = wq.shape[0]
+    if bits not in (8, 4):
+        raise ValueError("bits must be 8 or 4")
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=x.device)
+    _check(load().sq_gemm_weight_only(_p(x), _p(wq), SQ_I8 if bits == 8 else SQ_I4, _p(sw),
+                                      _p(bias), M, N, K, _p(out), _fdtype(out),
+                                      _stream(x.device)), "sq_gemm_weight_only")
     return out
 
 

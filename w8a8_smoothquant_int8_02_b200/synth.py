@@ -40,7 +40,7 @@ class LinearCase:
     N: int
     x_dtype: str                 # "f32" or "bf16"
     alpha: float
-    qtype: str                   # "i8" or "e4m3"
+    qtype: str                   # "i8" or "e4m3"; weight-only: "w8" / "w4"
     w_std: float
     outlier_frac: float = 0.01
     outlier_lo: float = 20.0
@@ -49,7 +49,7 @@ class LinearCase:
     outlier_factor: float = 0.0   # fixed factor for an explicit list
     bias_std: float = 0.0         # 0 => no bias
     cal_tokens: int = 512         # 0 => calibrate on X itself
-    act_scaling: str = "token"    # "token" (per-token) or "tensor" (per-tensor, delayed)
+    act_scaling: str = "token"    # "token" (per-token), "tensor" (per-tensor, delayed), "none"
     smooth: bool = True           # False => no smoothing factors (plain FP8 / INT8)
     seed: int = 0
     note: str = field(default="")

@@ -1,5 +1,6 @@
-"""The SmoothQuant linear-layer workloads this library is measured on (five
-per-token SmoothQuant cases and one per-tensor FP8 case).
+"""The linear-layer workloads this library is measured on: five per-token
+SmoothQuant cases, one per-tensor FP8 case, and the two weight-only schemes
+(W8A16, W4A16) at the decode shape.
 
 Shapes follow transformer linear layers: Y[M,N] = X[M,K] W[K,N], M tokens,
 K input channels, N output channels.  Prefill / MLP shapes are compute-bound
@@ -54,4 +55,24 @@ FP8_TENSOR = LinearCase(
          "activation tensor from the previous step's max (delayed scaling; the first "
          "step's from the 512 calibration tokens), per-output-channel E4M3 weights")
 
-ALL = {c.name: c for c in (TINY, PREFILL, MLP_UP, FP8_DOWN, DECODE, FP8_TENSOR)}
+# The weight-only schemes the pages set against W8A8 at decode (W8A16, W4A16):
+# bf16 activations as they are, per-output-channel INT8 / INT4 weights, the
+# decode shape above. Bound by the weight read from HBM.
+DECODE_W8A16 = LinearCase(
+    name="decode_w8a16_16x8192x28672", M=16, K=8192, N=28672, x_dtype="bf16",
+    alpha=0.5, qtype="w8", w_std=0.02, outlier_frac=0.01, outlier_lo=20.0,
+    outlier_hi=100.0, cal_tokens=0, act_scaling="none", smooth=False,
+    note="weight-only W8A16: X bf16 [16,8192], 1% outlier channels x U(20,100), not "
+         "quantized; W bf16 [8192,28672] N(0,0.02) as per-channel INT8 codes; HBM-bound")
+
+DECODE_W4A16 = LinearCase(
+    name="decode_w4a16_16x8192x28672", M=16, K=8192, N=28672, x_dtype="bf16",
+    alpha=0.5, qtype="w4", w_std=0.02, outlier_frac=0.01, outlier_lo=20.0,
+    outlier_hi=100.0, cal_tokens=0, act_scaling="none", smooth=False,
+    note="weight-only W4A16: X bf16 [16,8192], 1% outlier channels x U(20,100), not "
+         "quantized; W bf16 [8192,28672] N(0,0.02) as per-channel INT4 codes packed two per "
+         "byte; HBM-bound")
+
+ALL = {c.name: c for c in (TINY, PREFILL, MLP_UP, FP8_DOWN, DECODE, FP8_TENSOR, DECODE_W8A16,
+                           DECODE_W4A16)}
+WEIGHT_ONLY_BITS = {"w8": 8, "w4": 4}   # qtype of a weight-only workload -> weight bits
