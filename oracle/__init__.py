@@ -321,12 +321,13 @@ def linear(x, s, wq, sw, bias=None, qtype: int = INT8):
 # ---- weight-only quantization (W8A16 / W4A16) -------------------------------
 
 def quantize_weight_i4(w: np.ndarray):
-    """Per-output-channel symmetric INT4 weights: (wq4 [N, K/2] uint8, two codes
-    per byte, low nibble = even k; sw [N] float32 = amax / 7)."""
+    """Per-output-channel symmetric INT4 weights: (wq4 [N, K/2] uint8, sw [N]
+    float32 = amax / 7). Each 32-bit little-endian word packs the codes of 8
+    consecutive k: the even ones in bits 0,4,8,12, the odd ones in 16,20,24,28."""
     w = np.ascontiguousarray(w)
     K, N = w.shape
-    if K % 2:
-        raise ValueError("K must be even for packed INT4 weights")
+    if K % 8:
+        raise ValueError("K must be a multiple of 8 for packed INT4 weights")
     wq4 = np.empty((N, K // 2), np.uint8)
     sw = np.empty(N, np.float32)
     _load().sqo_quantize_weight_i4(_ptr(w), _dtype_code(w), K, N, _ptr(wq4), _ptr(sw))
@@ -344,7 +345,7 @@ def unpack_i4(wq4: np.ndarray) -> np.ndarray:
 
 def gemm_weight_only(x, wq, sw, bias=None, bits: int = 8) -> np.ndarray:
     """y = x @ (codes * sw).T + bias in binary64 (x: bf16 bits [M,K]; wq: int8
-    [N,K] for bits 8, packed uint8 [N,K/2] for bits 4)."""
+    [N,K] for bits 8, packed uint8 [N,K/2] for bits 4, see quantize_weight_i4)."""
     x = _c(x, np.uint16)
     M, K = x.shape
     wq = np.ascontiguousarray(wq)

@@ -456,6 +456,20 @@ static int8_t quant_i4(float v, float scale) {
 static uint8_t nibble_of(int8_t q) { return (uint8_t)q & 0x0Fu; }
 static int8_t code_of_nibble(uint8_t nb) { return (int8_t)((nb & 0x08u) ? (int)nb - 16 : (int)nb); }
 
+/* Packed INT4 layout (the pages fix none; this is the library's format): the
+ * codes of k = 8g .. 8g+7 form the little-endian 32-bit word at byte 4g of
+ * the row, code(8g + 2j) in bits 4j..4j+3 and code(8g + 2j + 1) in bits
+ * 16+4j..16+4j+3, j = 0..3 (the even codes in the low half-word, the odd ones
+ * in the high half-word). */
+static int nibble_shift(int64_t k) { return (int)((k & 1) ? 16 + 4 * ((k & 7) >> 1) : 4 * ((k & 7) >> 1)); }
+
+static int8_t unpack_code(const uint8_t* row, int64_t k) {
+    const uint8_t* wb = row + 4 * (k / 8);
+    uint32_t word = (uint32_t)wb[0] | ((uint32_t)wb[1] << 8) | ((uint32_t)wb[2] << 16) |
+                    ((uint32_t)wb[3] << 24);
+    return code_of_nibble((uint8_t)((word >> nibble_shift(k)) & 0x0Fu));
+}
+
 void sqo_quantize_weight_i4(const void* w, int dtype, int64_t K, int64_t N,
                             uint8_t* wq4, float* sw) {
     #pragma omp parallel for schedule(static)
@@ -467,22 +481,21 @@ void sqo_quantize_weight_i4(const void* w, int dtype, int64_t K, int64_t N,
         }
         float scale = amax / 7.0f;
         sw[n] = scale;
-        /* byte k/2 of row n: code of even k in the low nibble, odd k in the high */
-        for (int64_t k = 0; k < K; k += 2) {
-            int8_t q0 = (scale == 0.0f) ? 0 : quant_i4(load_elem(w, dtype, k * N + n), scale);
-            int8_t q1 = (scale == 0.0f) ? 0
-                                        : quant_i4(load_elem(w, dtype, (k + 1) * N + n), scale);
-            wq4[n * (K / 2) + k / 2] = (uint8_t)(nibble_of(q0) | (nibble_of(q1) << 4));
+        uint8_t* row = wq4 + n * (K / 2);
+        for (int64_t g = 0; g < K / 8; ++g) {
+            uint32_t word = 0;
+            for (int64_t k = 8 * g; k < 8 * g + 8; ++k) {
+                int8_t q = (scale == 0.0f) ? 0 : quant_i4(load_elem(w, dtype, k * N + n), scale);
+                word |= (uint32_t)nibble_of(q) << nibble_shift(k);
+            }
+            for (int b = 0; b < 4; ++b) row[4 * g + b] = (uint8_t)(word >> (8 * b));
         }
     }
 }
 
 void sqo_unpack_i4(const uint8_t* wq4, int64_t N, int64_t K, int8_t* codes) {
     for (int64_t n = 0; n < N; ++n)
-        for (int64_t k = 0; k < K; ++k) {
-            uint8_t b = wq4[n * (K / 2) + k / 2];
-            codes[n * K + k] = code_of_nibble((k & 1) ? (uint8_t)(b >> 4) : (uint8_t)(b & 0x0Fu));
-        }
+        for (int64_t k = 0; k < K; ++k) codes[n * K + k] = unpack_code(wq4 + n * (K / 2), k);
 }
 
 void sqo_gemm_weight_only(const uint16_t* x, const void* wq, int bits, const float* sw,
@@ -495,8 +508,7 @@ void sqo_gemm_weight_only(const uint16_t* x, const void* wq, int bits, const flo
             for (int64_t k = 0; k < K; ++k) {
                 int8_t q;
                 if (bits == 4) {
-                    uint8_t b = ((const uint8_t*)wq)[n * (K / 2) + k / 2];
-                    q = code_of_nibble((k & 1) ? (uint8_t)(b >> 4) : (uint8_t)(b & 0x0Fu));
+                    q = unpack_code((const uint8_t*)wq + n * (K / 2), k);
                 } else {
                     q = ((const int8_t*)wq)[n * K + k];
                 }

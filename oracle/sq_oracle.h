@@ -114,9 +114,10 @@ void sqo_linear_at(const void* xq, const float* sx, const void* wq,
 
 /* Weight-only quantization (W8A16 / W4A16). INT4 weights: per output channel
  * sw[n] = max_k |w[k][n]| / 7, codes clamp(round-half-even(w / sw), -7, 7)
- * (0 where sw is 0), packed two per byte into wq4 [N, K/2]: byte k/2 of row n
- * holds the code of even k in its low nibble and of odd k in its high nibble
- * (two's complement). K must be even. */
+ * (0 where sw is 0), packed into wq4 [N, K/2] bytes: the codes of k = 8g ..
+ * 8g+7 form the little-endian 32-bit word at byte 4g of the row, code(8g+2j)
+ * in bits 4j..4j+3 and code(8g+2j+1) in bits 16+4j..16+4j+3 (two's
+ * complement nibbles). K must be a multiple of 8. */
 void sqo_quantize_weight_i4(const void* w, int dtype, int64_t K, int64_t N,
                             uint8_t* wq4, float* sw);
 /* The codes of a packed INT4 matrix, one int8 per element: codes [N,K]. */

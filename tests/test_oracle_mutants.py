@@ -135,18 +135,21 @@ MUTANTS = [
     ("int4_scale_divides_by_8", "float scale = amax / 7.0f;", "float scale = amax / 8.0f;"),
     ("int4_truncates",
      "float c = nearbyintf(v / scale);", "float c = truncf(v / scale);"),
-    ("int4_nibbles_swapped",
-     "(uint8_t)(nibble_of(q0) | (nibble_of(q1) << 4))",
-     "(uint8_t)(nibble_of(q1) | (nibble_of(q0) << 4))"),
+    ("int4_even_and_odd_halves_swapped",
+     "static int nibble_shift(int64_t k) { return (int)((k & 1) ? 16 + 4 * ((k & 7) >> 1) : 4 * ((k & 7) >> 1)); }",
+     "static int nibble_shift(int64_t k) { return (int)((k & 1) ? 4 * ((k & 7) >> 1) : 16 + 4 * ((k & 7) >> 1)); }"),
+    ("int4_word_bytes_big_endian",
+     "for (int b = 0; b < 4; ++b) row[4 * g + b] = (uint8_t)(word >> (8 * b));",
+     "for (int b = 0; b < 4; ++b) row[4 * g + b] = (uint8_t)(word >> (24 - 8 * b));"),
     ("int4_nibble_not_sign_extended",
      "return (int8_t)((nb & 0x08u) ? (int)nb - 16 : (int)nb);", "return (int8_t)nb;"),
     ("weight_only_drops_the_scale",
      "double w_deq = (double)q * (double)sw[n];", "double w_deq = (double)q;"),
     ("weight_only_drops_the_bias",
      "if (bias) acc += (double)sqo_bf16_to_f32(bias[n]);", "(void)bias;"),
-    ("weight_only_reads_the_wrong_nibble",
-     "q = code_of_nibble((k & 1) ? (uint8_t)(b >> 4) : (uint8_t)(b & 0x0Fu));",
-     "q = code_of_nibble((k & 1) ? (uint8_t)(b & 0x0Fu) : (uint8_t)(b >> 4));"),
+    ("weight_only_reads_the_wrong_code",
+     "q = unpack_code((const uint8_t*)wq + n * (K / 2), k);",
+     "q = unpack_code((const uint8_t*)wq + n * (K / 2), k ^ 1);"),
     ("weight_only_wrong_channel_scale",
      "double w_deq = (double)q * (double)sw[n];", "double w_deq = (double)q * (double)sw[m % N];"),
 ]

@@ -659,17 +659,18 @@ def test_folded_producer_feeds_the_same_codes(qt):
 
 def test_int4_weight_codes_and_packing_by_hand():
     """A column with amax 7 has scale 1: codes are the half-even roundings
-    clamped to +-7, and each byte holds an even-k code (low nibble) and the
-    following odd-k code (high nibble), two's complement."""
-    w = np.zeros((6, 3), np.float32)
-    w[:, 0] = [7.0, -3.5, 2.5, 0.5, -6.49, 1.0]   # ties go to even: -3.5 -> -4, 2.5 -> 2, 0.5 -> 0
-    w[:, 1] = [0.0, 0.0, 0.0, 0.0, 0.0, -14.0]    # amax 14 -> scale 2; -14 / 2 = -7
+    clamped to +-7. The 8 codes of one k-group form one little-endian word,
+    even k in bits 0,4,8,12 and odd k in bits 16,20,24,28 (two's complement)."""
+    w = np.zeros((8, 3), np.float32)
+    w[:, 0] = [7.0, -3.5, 2.5, 0.5, -6.49, 1.0, 3.0, -6.6]  # ties to even: -3.5 -> -4, 2.5 -> 2
+    w[7, 1] = -14.0                                           # amax 14 -> scale 2; -14 / 2 = -7
     wq4, sw = oracle.quantize_weight_i4(w)
     assert sw.tolist() == [1.0, 2.0, 0.0]
-    assert wq4[0].tolist() == [0xC7, 0x02, 0x1A]  # (7, -4), (2, 0), (-6, 1)
-    assert wq4[1].tolist() == [0x00, 0x00, 0x90]  # (0, 0), (0, 0), (0, -7)
-    assert not wq4[2].any()                       # an all-zero channel
-    np.testing.assert_array_equal(oracle.unpack_i4(wq4)[0], [7, -4, 2, 0, -6, 1])
+    # codes (7, -4, 2, 0, -6, 1, 3, -7): even k 7, 2, -6, 3 -> 0x3A27; odd k -4, 0, 1, -7 -> 0x910C
+    assert wq4[0].tolist() == [0x27, 0x3A, 0x0C, 0x91]
+    assert wq4[1].tolist() == [0x00, 0x00, 0x00, 0x90]      # code -7 at k = 7 (bits 28..31)
+    assert not wq4[2].any()                                   # an all-zero channel
+    np.testing.assert_array_equal(oracle.unpack_i4(wq4)[0], [7, -4, 2, 0, -6, 1, 3, -7])
 
 
 @pytest.mark.parametrize("bf16", [False, True])
@@ -688,9 +689,12 @@ def test_int4_weight_quant_brute_force(bf16):
     wq4, sw = oracle.quantize_weight_i4(w)
     np.testing.assert_array_equal(sw, scale)
     np.testing.assert_array_equal(oracle.unpack_i4(wq4), codes)
-    lo = (codes[:, 0::2].astype(np.int16) & 0xF)
-    hi = (codes[:, 1::2].astype(np.int16) & 0xF)
-    np.testing.assert_array_equal(wq4, (lo | (hi << 4)).astype(np.uint8))
+    nib = codes.astype(np.int64).reshape(codes.shape[0], -1, 8) & 0xF   # [N, K/8, 8]
+    words = np.zeros(nib.shape[:2], np.int64)
+    for j in range(4):
+        words |= nib[:, :, 2 * j] << (4 * j)
+        words |= nib[:, :, 2 * j + 1] << (16 + 4 * j)
+    np.testing.assert_array_equal(wq4, words.astype("<u4").view(np.uint8).reshape(wq4.shape))
     # the largest weight of a channel maps to +-7 and the error is half a step
     assert (np.abs(oracle.unpack_i4(wq4)[7]).max() == 7)
     err = np.abs(wf.T - codes * sw[:, None])
