@@ -71,7 +71,7 @@ typedef enum {
     SQ_I8 = 2,    /* signed 8-bit integer code                               */
     SQ_E4M3 = 3,  /* FP8 E4M3 code: bias 7, no infinity, max finite 448      */
     SQ_I32 = 4,   /* signed 32-bit integer                                   */
-    SQ_I4 = 5     /* signed 4-bit code (-7..7), two per byte, low nibble first */
+    SQ_I4 = 5     /* signed 4-bit code (-7..7), packed 8 per 32-bit word       */
 } sq_dtype;
 
 typedef enum {
@@ -144,8 +144,10 @@ sq_status sq_smooth_factors(const float* amax_x, const float* amax_w,
  * qt = SQ_I4 (weight-only W4A16, see sq_gemm_weight_only): s must be NULL
  * (SQ_ERR_UNSUPPORTED otherwise) and K a multiple of 32; sw[n] = max_k|w[k,n]|
  * / 7, codes clamp(rne(w[k,n]/sw[n]), -7, 7), stored packed as wq [N, K/2]
- * bytes: byte k/2 of row n holds the code of even k in its low nibble and of
- * odd k in its high nibble (two's complement).
+ * bytes: the codes of k = 8g .. 8g+7 form the little-endian 32-bit word at
+ * byte 4g of row n, code(8g+2j) in bits 4j..4j+3 and code(8g+2j+1) in bits
+ * 16+4j..16+4j+3 (two's-complement nibbles; the pages fix no packing, and
+ * this one lets the GEMM widen two codes with two masks and one subtraction).
  */
 sq_status sq_quantize_weight(const void* w, sq_dtype wt, int64_t K, int64_t N,
                              const float* s, sq_dtype qt, void* wq, float* sw,
@@ -287,7 +289,8 @@ sq_status sq_gemm_fp8(const uint8_t* xq, const float* sx, const uint8_t* wq,
  * weights halve it again).
  *   x   : [M,K] bf16 activations (not quantized, not smoothed)
  *   wq  : per-output-channel weight codes from sq_quantize_weight with s =
- *         NULL: wqt = SQ_I8 -> int8 [N,K]; wqt = SQ_I4 -> packed [N,K/2]
+ *         NULL: wqt = SQ_I8 -> int8 [N,K]; wqt = SQ_I4 -> packed [N,K/2] (the
+ *         layout sq_quantize_weight documents)
  *   sw  : [N] channel scales (4-byte aligned); bias : [N] bf16 or NULL
  *   y   : [M,N], yt = SQ_BF16 or SQ_F32
  * y[m,n] = bf16( RN(sum_k x[m,k] * q[n,k]) * sw[n] + bias[n] ): the codes are

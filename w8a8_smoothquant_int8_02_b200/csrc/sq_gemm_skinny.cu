@@ -22,11 +22,18 @@
 //   warp 0    : TMA producer (Wq slice [128 rows x 128 B] + Xq slice
 //               [16 rows x 128 B], 128-byte swizzle; token rows beyond M read
 //               as zero)
-//   warp 1    : allocates 32 tensor-memory columns; one thread issues the
-//               MMAs (K = 32 per instruction) and frees ring slots with
-//               tcgen05.commit
+//   warp 1    : allocates 128 tensor-memory columns (eight accumulators of
+//               16 columns); one thread issues the MMAs (K = 32 per
+//               instruction) into the eight accumulators in turn -- an MMA of
+//               128 x 16 x 32 is far shorter than the latency of the
+//               accumulator it would otherwise wait for -- and frees ring
+//               slots with tcgen05.commit
 //   warps 2-5 : epilogue -- warp w reads lanes 32*(w%4)..+31 (its output
-//               channels) x 16 columns (the tokens), dequantizes and stores.
+//               channels) x 16 columns (the tokens) of each accumulator, adds
+//               them (int32, exact; E4M3 binary32 in a fixed order),
+//               dequantizes and stores.
+// Each CTA starts its k loop at a different k-block: all CTAs read the same
+// token slices, which would otherwise be requested by every CTA at once.
 // Every barrier wait is bounded: a wait that gives up records SQ_ERR_TIMEOUT,
 // the CTA skips its remaining work, waits (bounded) for its copies and MMAs
 // in flight and still frees tensor memory.
@@ -51,7 +58,8 @@ constexpr uint32_t kSkBarOff = kSkStages * kSkStageBytes;
 // barriers: full[S], empty[S], tfull, drain; then the TMEM slot and abort flag
 constexpr uint32_t kSkMiscOff = kSkBarOff + (2 * kSkStages + 2) * 8;
 constexpr uint32_t kSkDynamic = kSkMiscOff + 16 + 1024;  // slack for 1024-B alignment
-constexpr uint32_t kSkTmemCols = 32;                     // smallest allocation
+constexpr int kSkNAcc = 8;                               // independent accumulators
+constexpr uint32_t kSkTmemCols = kSkNAcc * 16;          // 16 columns each
 static_assert(kSkStageBytes % 1024 == 0, "stages must keep 1024-byte alignment");
 static_assert(kSkDynamic * 2 + 2048 <= 233472, "two CTAs per SM must fit");
 
@@ -114,6 +122,10 @@ __global__ void __launch_bounds__(kSkThreads, 2)
 
   const int n0 = int(blockIdx.x) * 128;
   const int nk = (K + kSkBK - 1) / kSkBK;
+  // every CTA reads the same token slices; starting each CTA at a different
+  // k-block spreads those reads over the L2 instead of all CTAs asking for
+  // the same lines at once (integer sums do not depend on the order)
+  const int kb_rot = int(blockIdx.x) % nk;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer --
@@ -128,9 +140,10 @@ __global__ void __launch_bounds__(kSkThreads, 2)
           break;
         }
         const uint32_t dst = s_base + st * kSkStageBytes;
+        const int kbe = kb + kb_rot < nk ? kb + kb_rot : kb + kb_rot - nk;
         mbar_arrive_expect_tx(bar_full + 8 * st, kSkStageBytes);
-        tma_load_2d(dst, &tm_w, bar_full + 8 * st, kb * kSkBK, n0);
-        tma_load_2d(dst + kSkABytes, &tm_x, bar_full + 8 * st, kb * kSkBK, 0);
+        tma_load_2d(dst, &tm_w, bar_full + 8 * st, kbe * kSkBK, n0);
+        tma_load_2d(dst + kSkABytes, &tm_x, bar_full + 8 * st, kbe * kSkBK, 0);
         ++issued;
       }
       // no copy may still be writing shared memory when the CTA exits: wait
@@ -158,13 +171,17 @@ __global__ void __launch_bounds__(kSkThreads, 2)
         tc_fence_after();
         const uint32_t a_addr = s_base + st * kSkStageBytes;
         const uint32_t b_addr = a_addr + kSkABytes;
+        // MMA j accumulates into accumulator j % kSkNAcc: consecutive MMAs
+        // do not wait for one another's result
 #pragma unroll
         for (int kk = 0; kk < kSkBK / 32; ++kk) {
+          const uint32_t j = uint32_t(kb) * uint32_t(kSkBK / 32) + uint32_t(kk);
           const uint64_t ad = sw128_desc(a_addr + kk * 32);
           const uint64_t bd = sw128_desc(b_addr + kk * 32);
-          const uint32_t accum = (kb > 0 || kk > 0) ? 1u : 0u;
-          if constexpr (E4M3) mma_f8(tmem_base, ad, bd, idesc, accum);
-          else mma_i8(tmem_base, ad, bd, idesc, accum);
+          const uint32_t d = tmem_base + (j % kSkNAcc) * 16u;
+          const uint32_t accum = j >= uint32_t(kSkNAcc) ? 1u : 0u;
+          if constexpr (E4M3) mma_f8(d, ad, bd, idesc, accum);
+          else mma_i8(d, ad, bd, idesc, accum);
         }
         tc_commit(bar_empty + 8 * st);
       }
@@ -182,8 +199,23 @@ __global__ void __launch_bounds__(kSkThreads, 2)
       *abort_flag = 1;
     } else {
       tc_fence_after();
+      // the sum of the accumulators (exact for INT8; in a fixed order for E4M3)
       uint32_t r[16];
       tmem_ld16_wait(tmem_base + (uint32_t(sub * 32) << 16), r);
+      // accumulators that received an MMA (all of them unless K is tiny)
+      const int n_acc = nk * (kSkBK / 32) < kSkNAcc ? nk * (kSkBK / 32) : kSkNAcc;
+#pragma unroll 1
+      for (int c = 1; c < n_acc; ++c) {
+        uint32_t r2[16];
+        tmem_ld16_wait(tmem_base + (uint32_t(sub * 32) << 16) + uint32_t(c * 16), r2);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          if constexpr (E4M3)
+            r[j] = __float_as_uint(__fadd_rn(__uint_as_float(r[j]), __uint_as_float(r2[j])));
+          else
+            r[j] = uint32_t(int32_t(r[j]) + int32_t(r2[j]));
+        }
+      }
       if (n < N) {
         const float swn = __ldg(sw + n);
         float bn = 0.0f;

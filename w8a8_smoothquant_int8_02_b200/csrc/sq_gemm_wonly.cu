@@ -4,8 +4,8 @@
 //   y[m,n] = bf16( float( sum_k x[m,k] * q[n,k] ) * sw[n] + bias[n] )
 //
 // x is bf16 [M,K]; q are the per-output-channel weight codes (INT8 [N,K], or
-// INT4 packed two per byte [N,K/2], low nibble = even k) with scales sw [N].
-// Source: the pages' weight-only schemes -- "Weight-Activation
+// INT4 [N,K/2] packed eight per 32-bit word, see sq_quantize_weight) with
+// scales sw [N]. Source: the pages' weight-only schemes -- "Weight-Activation
 // Quantization" (infra.bea.ai) §1 table (W4A16: INT4 weights dequantized to
 // 16 bits, then a 16-bit multiply), the zenaique flashcard on activation
 // quantization (the runtime dequantizes the weights on the fly against BF16
@@ -14,23 +14,34 @@
 // weights read half the bytes of 8-bit ones).
 //
 // Dequantization: every INT8 / INT4 code is exactly representable in bf16,
-// so the weights are widened to bf16 codes in shared memory and multiplied by
-// the bf16 activations on the tensor cores (kind::f16, binary32 accumulators
-// in tensor memory); the channel scale sw[n] is constant along k, so it is
-// applied once to the sum in the epilogue: sum_k x * (q * sw) = sw * sum_k x*q.
+// so the codes are widened to bf16 and multiplied by the bf16 activations on
+// the tensor cores (kind::f16, binary32 accumulators in tensor memory); the
+// channel scale sw[n] is constant along k, so it is applied once to the sum
+// in the epilogue: sum_k x * (q * sw) = sw * sum_k x * q.
 //
 // Roles are swapped as in the few-token W8A8 kernel: 128 weight rows are the
 // M = 128 operand, the (up to) 16 token rows the N = 16 operand, D[n][m] in
 // 128 lanes x 16 columns of tensor memory. One CTA per 128 output channels
-// and 16 tokens (grid.y walks token tiles of larger batches).
+// and 16 tokens (grid.y walks token tiles of larger batches); two CTAs per SM.
 //   warp 0      : TMA producer -- per stage one 128-byte-wide K slice of the
 //                 packed weights [128 rows x 128 B] (128 k for INT8, 256 for
 //                 INT4) and the matching bf16 token slices [16 rows x 64 k]
-//   warp 1      : tensor memory (32 columns); one thread issues the MMAs
-//                 (K = 16 per instruction) and frees buffers by tcgen05.commit
-//   warps 2..9  : widen the weight codes of each stage into bf16 sub-tiles
-//                 [128 rows x 64 k] (128-byte swizzle, the layout the MMA
-//                 reads); warps 2..5 then run the epilogue
+//                 into a 5- (INT8) or 4-stage (INT4) shared-memory ring
+//   warp 1      : tensor memory (256 columns: eight accumulators and a
+//                 4-deep ring of bf16 weight sub-tiles); one thread issues
+//                 the MMAs (A from tensor memory, B = the token slice from
+//                 shared memory, K = 16 per instruction), rotating over the
+//                 eight accumulators so that consecutive MMAs are independent
+//                 (one MMA of 128 x 16 x 16 is far shorter than the latency
+//                 of the accumulator it would otherwise wait for), and frees
+//                 buffers by tcgen05.commit
+//   warps 2..9  : two groups of four (one warp per lane quarter) taking
+//                 alternate 64-k sub-tiles: each thread widens its weight
+//                 row's 64 codes to 32 bf16 pairs and stores them to tensor
+//                 memory (tcgen05.st); warps 2..5 then run the epilogue,
+//                 which adds the eight accumulators in a fixed order
+// Each CTA starts its k loop at a different k-block: all CTAs read the same
+// token slices, which would otherwise be requested by every CTA at once.
 // Every barrier wait is bounded: a wait that gives up records
 // SQ_ERR_TIMEOUT, the CTA skips its remaining work, waits (bounded) for its
 // copies and MMAs in flight and still frees tensor memory.
@@ -45,82 +56,85 @@
 namespace sqk {
 
 constexpr int kWoTokens = 16;                 // token columns (N of the instruction)
-constexpr int kWoConvWarps = 8;               // warps widening the weight codes
+constexpr int kWoConvWarps = 8;               // two groups of four, alternating sub-tiles
 constexpr int kWoThreads = 64 + 32 * kWoConvWarps;
 constexpr uint32_t kWoWBytes = 128 * 128;     // packed weight slice of one stage
-constexpr uint32_t kWoSubBytes = 128 * 128;   // bf16 weight sub-tile [128 x 64 k]
 constexpr uint32_t kWoXSub = kWoTokens * 128; // bf16 token sub-tile [16 x 64 k]
+constexpr uint32_t kWoTmemCols = 256;         // per CTA: accumulators + A ring
+constexpr int kWoNAcc = 8;                    // independent accumulators (16 columns each)
+constexpr uint32_t kWoAColBase = kWoNAcc * 16;  // first A column
+constexpr int kWoNA = 4;                      // A sub-tiles in tensor memory (32 columns each)
 
 template <int BITS>
 struct WoCfg {
   static constexpr int KS = BITS == 8 ? 128 : 256;   // k per stage
-  static constexpr int SUBS = KS / 64;               // bf16 sub-tiles per stage
-  static constexpr int STAGES = 3;                   // packed-weight ring
-  static constexpr int NA = BITS == 8 ? 3 : 2;       // bf16 weight ring
+  static constexpr int SUBS = KS / 64;               // 64-k sub-tiles per stage
+  static constexpr int STAGES = BITS == 8 ? 5 : 4;   // packed-weight ring
   static constexpr uint32_t kXBytes = SUBS * kWoXSub;
   static constexpr uint32_t kStageBytes = kWoWBytes + kXBytes;
-  static constexpr uint32_t kRingA = STAGES * kStageBytes;          // 1024-aligned
-  static constexpr uint32_t kBarOff = kRingA + NA * kWoSubBytes;
+  static constexpr uint32_t kBarOff = STAGES * kStageBytes;
   // barriers: full[S], empty[S], afull[NA], aempty[NA], tfull, drain
-  static constexpr uint32_t kMiscOff = kBarOff + (2 * STAGES + 2 * NA + 2) * 8;
+  static constexpr uint32_t kMiscOff = kBarOff + (2 * STAGES + 2 * kWoNA + 2) * 8;
   static constexpr uint32_t kDynamic = kMiscOff + 16 + 1024;  // slack for 1024-B alignment
   static_assert(kStageBytes % 1024 == 0, "stages must keep 1024-byte alignment");
   static_assert(2 * (kDynamic + 1024) <= 233472, "two CTAs per SM must fit");
 };
+static_assert(kWoAColBase + kWoNA * 32 <= kWoTmemCols, "A ring must fit the allocation");
 
-// Instruction descriptor of tcgen05.mma kind::f16 with bf16 A and B (both
-// K-major) and binary32 accumulators: bits 4-5 D format, 7-9 / 10-12 A / B
-// formats, 17-22 N/8, 24-28 M/16.
+// Instruction descriptor of tcgen05.mma kind::f16 with bf16 A and B and
+// binary32 accumulators: bits 4-5 D format, 7-9 / 10-12 A / B formats,
+// 17-22 N/8, 24-28 M/16 (A and B not transposed).
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int m, int n) {
   return (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(n >> 3) << 17) | (uint32_t(m >> 4) << 24);
 }
 
-__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                         uint32_t idesc, uint32_t accumulate) {
+// D[tmem] (+)= A[tmem] * B[smem]^T, bf16 operands, binary32 accumulators: A
+// is read from tensor memory (row m in lane m, two k per 32-bit column).
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 
-__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
-  return __byte_perm(a, b, sel);
+// registers -> 32 lanes x 32 consecutive 32-bit columns of tensor memory
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0],"
+      " {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16,"
+      " %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};"
+      ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
+        "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]),
+        "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]),
+        "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]),
+        "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
-// Four offset-binary bytes u (= code + OFF) of `u4` -> two words of two bf16
-// codes each (elements in byte order). 0x4B0000uu is the binary32 2^23 + u,
-// so subtracting 2^23 + OFF leaves the code exactly, and a code of at most 8
-// significant bits is its own bf16 (the upper half of its binary32 word).
-template <int OFF>
-__device__ __forceinline__ void widen4(uint32_t u4, uint32_t& w01, uint32_t& w23) {
-  constexpr uint32_t kExp = 0x4B000000u;
-  constexpr float kBias = 8388608.0f + float(OFF);
-  const uint64_t bias2 = f2_make(kBias, kBias);
-  float a, b, c, d;
-  f2_split(f2_sub(f2_make(__uint_as_float(prmt(u4, kExp, 0x7440)),
-                          __uint_as_float(prmt(u4, kExp, 0x7441))), bias2), a, b);
-  f2_split(f2_sub(f2_make(__uint_as_float(prmt(u4, kExp, 0x7442)),
-                          __uint_as_float(prmt(u4, kExp, 0x7443))), bias2), c, d);
-  w01 = prmt(__float_as_uint(a), __float_as_uint(b), 0x7632);
-  w23 = prmt(__float_as_uint(c), __float_as_uint(d), 0x7632);
+// bf16x2 a - b, rounded to nearest (exact here: every result is a small integer)
+__device__ __forceinline__ uint32_t bf16x2_sub(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
 }
 
-// Two offset-binary nibble bytes (even elements in `lo`, odd in `hi`, byte i
-// of each holding elements 2i and 2i + 1) -> four words of bf16 pairs in
-// element order.
-__device__ __forceinline__ void widen8_nibbles(uint32_t lo, uint32_t hi, uint32_t (&w)[4]) {
-  constexpr uint32_t kExp = 0x4B000000u;
-  constexpr float kBias = 8388608.0f + 8.0f;
-  const uint64_t bias2 = f2_make(kBias, kBias);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    float a, b;
-    f2_split(f2_sub(f2_make(__uint_as_float(prmt(lo, kExp, 0x7440 + i)),
-                            __uint_as_float(prmt(hi, kExp, 0x7440 + i))), bias2), a, b);
-    w[i] = prmt(__float_as_uint(a), __float_as_uint(b), 0x7632);
-  }
+// Widening of codes to bf16 without a conversion instruction. A code c with
+// |c| < 2^(B-1) is split into its low bits v and its sign bit s (two's
+// complement: c = v - s * 2^(B-1)). The bf16 with bits 0x4300 | v is 128 + v
+// (exponent 2^7, one unit per mantissa step) and 0x4300 | (sign bit in place)
+// is 128 + s * 2^(B-1); their bf16 difference is c exactly. Two codes at bit
+// 0 and bit 16 of a word give two bf16 at once (the low half is the first).
+template <int B>
+__device__ __forceinline__ uint32_t codes_to_bf16x2(uint32_t w) {
+  constexpr uint32_t kLow = B == 8 ? 0x007F007Fu : 0x00070007u;
+  constexpr uint32_t kSign = B == 8 ? 0x00800080u : 0x00080008u;
+  return bf16x2_sub((w & kLow) | 0x43004300u, (w & kSign) | 0x43004300u);
 }
 
 __device__ __forceinline__ uint32_t sw128_off(uint32_t row, uint32_t chunk) {
@@ -146,12 +160,11 @@ __global__ void __launch_bounds__(kWoThreads, 2)
                       const uint16_t* __restrict__ bias, void* __restrict__ y, int M, int N,
                       int K, int* status) {
   using C = WoCfg<BITS>;
-  constexpr int S = C::STAGES, NA = C::NA, SUBS = C::SUBS;
+  constexpr int S = C::STAGES, NA = kWoNA, SUBS = C::SUBS;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const uint32_t s_base = smem_u32(smem);
-  const uint32_t s_a = s_base + C::kRingA;
   const uint32_t bar_full = s_base + C::kBarOff;
   const uint32_t bar_empty = bar_full + S * 8;
   const uint32_t bar_afull = bar_empty + S * 8;
@@ -168,7 +181,7 @@ __global__ void __launch_bounds__(kWoThreads, 2)
       mbar_init(bar_empty + 8 * i, kWoConvWarps + 1);  // every widening warp + the MMAs
     }
     for (int i = 0; i < NA; ++i) {
-      mbar_init(bar_afull + 8 * i, kWoConvWarps);
+      mbar_init(bar_afull + 8 * i, 4);                 // the four warps of one group
       mbar_init(bar_aempty + 8 * i, 1);
     }
     mbar_init(bar_tfull, 1);
@@ -179,7 +192,7 @@ __global__ void __launch_bounds__(kWoThreads, 2)
     tma_prefetch_map(&tm_x);
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), 32);
+    tmem_alloc(smem_u32(tmem_slot), kWoTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -193,6 +206,10 @@ __global__ void __launch_bounds__(kWoThreads, 2)
   const int n0 = int(blockIdx.x) * 128;
   const int m0 = int(blockIdx.y) * kWoTokens;
   const int nk = (K + C::KS - 1) / C::KS;
+  // every CTA reads the same token slices; starting each CTA at a different
+  // k-block spreads those reads over the L2 instead of all CTAs asking for
+  // the same lines at once (the sum is the same up to binary32 rounding)
+  const int kb_rot = int(blockIdx.x) % nk;
   auto give_up = [&]() {
     record_status(status, kStatusTimeout);
     *abort_flag = 1;
@@ -210,12 +227,13 @@ __global__ void __launch_bounds__(kWoThreads, 2)
           break;
         }
         const uint32_t dst = s_base + st * C::kStageBytes;
+        const int kbe = kb + kb_rot < nk ? kb + kb_rot : kb + kb_rot - nk;
         mbar_arrive_expect_tx(bar_full + 8 * st, C::kStageBytes);
-        tma_load_2d(dst, &tm_w, bar_full + 8 * st, kb * 128, n0);
+        tma_load_2d(dst, &tm_w, bar_full + 8 * st, kbe * 128, n0);
 #pragma unroll
         for (int t = 0; t < SUBS; ++t)
           tma_load_2d(dst + kWoWBytes + t * kWoXSub, &tm_x, bar_full + 8 * st,
-                      kb * C::KS + t * 64, m0);
+                      kbe * C::KS + t * 64, m0);
         ++issued;
       }
       // no copy may still be writing shared memory when the CTA exits
@@ -248,12 +266,15 @@ __global__ void __launch_bounds__(kWoThreads, 2)
             break;
           }
           tc_fence_after();
-          const uint32_t a_addr = s_a + slot * kWoSubBytes;
+          const uint32_t a_tmem = tmem_base + kWoAColBase + slot * 32u;
+          // MMA j accumulates into accumulator j % kWoNAcc: consecutive MMAs
+          // do not wait for one another's result
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t ad = sw128_desc(a_addr + kk * 32);
+            const uint32_t j = ia * 4u + uint32_t(kk);
             const uint64_t bd = sw128_desc(x_addr + t * kWoXSub + kk * 32);
-            mma_bf16(tmem_base, ad, bd, idesc, (kb > 0 || t > 0 || kk > 0) ? 1u : 0u);
+            mma_bf16_ts(tmem_base + (j % kWoNAcc) * 16u, a_tmem + uint32_t(kk * 8), bd, idesc,
+                        j >= uint32_t(kWoNAcc) ? 1u : 0u);
           }
           tc_commit(bar_aempty + 8 * slot);
         }
@@ -268,8 +289,10 @@ __global__ void __launch_bounds__(kWoThreads, 2)
   } else {
     // ------------------------------------------- widening, then epilogue --
     const int cw = warp - 2;                   // 0 .. kWoConvWarps - 1
-    const uint32_t row = uint32_t(cw & 3) * 32u + uint32_t(lane);   // weight row of the tile
-    const int part = cw >> 2;                  // which half of the row's source chunks
+    const int quarter = warp & 3;              // TMEM lane quarter this warp may access
+    const int group = cw >> 2;                 // sub-tiles ia with ia % 2 == group
+    const uint32_t row = uint32_t(quarter) * 32u + uint32_t(lane);  // weight row of the tile
+    const uint32_t lane_off = uint32_t(quarter * 32) << 16;
     uint32_t ia = 0;
     bool ok = true;
 #pragma unroll 1
@@ -283,49 +306,47 @@ __global__ void __launch_bounds__(kWoThreads, 2)
       const uint8_t* wsrc = smem + st * C::kStageBytes;
 #pragma unroll 1
       for (int t = 0; t < SUBS; ++t, ++ia) {
+        if (int(ia & 1u) != group) continue;
         const uint32_t slot = ia % NA;
         if (*abort_flag || !mbar_wait(bar_aempty + 8 * slot, ((ia / NA) & 1u) ^ 1u)) {
           give_up();
           ok = false;
           break;
         }
-        uint8_t* adst = smem + C::kRingA + slot * kWoSubBytes;
+        tc_fence_after();
+        // this row's 64 codes of sub-tile t -> 32 bf16 pairs (k order)
+        uint32_t a[32];
         if constexpr (BITS == 8) {
-          // sub-tile t holds source chunks 4t .. 4t+3 (16 codes each); this
-          // warp widens two of them per row: 4 bf16 chunks of 8 codes
+          // source chunks 4t .. 4t+3 of the row, 16 codes each
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const uint32_t j = uint32_t(4 * t + 2 * part + h);
-            const uint4 q = *reinterpret_cast<const uint4*>(wsrc + sw128_off(row, j));
-            uint4 o0, o1;
-            widen4<128>(q.x ^ 0x80808080u, o0.x, o0.y);
-            widen4<128>(q.y ^ 0x80808080u, o0.z, o0.w);
-            widen4<128>(q.z ^ 0x80808080u, o1.x, o1.y);
-            widen4<128>(q.w ^ 0x80808080u, o1.z, o1.w);
-            const uint32_t c0 = 2u * (j - 4u * uint32_t(t));
-            *reinterpret_cast<uint4*>(adst + sw128_off(row, c0)) = o0;
-            *reinterpret_cast<uint4*>(adst + sw128_off(row, c0 + 1)) = o1;
+          for (int h = 0; h < 4; ++h) {
+            const uint4 q = *reinterpret_cast<const uint4*>(wsrc + sw128_off(row, uint32_t(4 * t + h)));
+            const uint32_t qw[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              // bytes (c0 c1 c2 c3) -> (c0 c2 c1 c3): c0, c1 at bits 0 / 16
+              const uint32_t p = __byte_perm(qw[i], 0u, 0x3120);
+              a[8 * h + 2 * i] = codes_to_bf16x2<8>(p);
+              a[8 * h + 2 * i + 1] = codes_to_bf16x2<8>(p >> 8);
+            }
           }
         } else {
-          // sub-tile t holds source chunks 2t, 2t+1 (32 codes each); this
-          // warp widens one of them per row: 4 bf16 chunks of 8 codes
-          const uint32_t j = uint32_t(2 * t + part);
-          const uint4 q = *reinterpret_cast<const uint4*>(wsrc + sw128_off(row, j));
-          const uint32_t qw[4] = {q.x, q.y, q.z, q.w};
-          const uint32_t c0 = 4u * uint32_t(part);
+          // source chunks 2t, 2t+1 of the row, 32 codes each; each 32-bit
+          // word holds 8 codes: even k at bits 0,4,8,12, odd k at 16,20,24,28
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            // nibble ^ 8 is the offset-binary code + 8
-            const uint32_t lo = (qw[i] & 0x0F0F0F0Fu) ^ 0x08080808u;
-            const uint32_t hi = ((qw[i] >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;
-            uint32_t w[4];
-            widen8_nibbles(lo, hi, w);
-            *reinterpret_cast<uint4*>(adst + sw128_off(row, c0 + uint32_t(i))) =
-                make_uint4(w[0], w[1], w[2], w[3]);
+          for (int h = 0; h < 2; ++h) {
+            const uint4 q = *reinterpret_cast<const uint4*>(wsrc + sw128_off(row, uint32_t(2 * t + h)));
+            const uint32_t qw[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+#pragma unroll
+              for (int j = 0; j < 4; ++j) a[16 * h + 4 * i + j] = codes_to_bf16x2<4>(qw[i] >> (4 * j));
+            }
           }
         }
-        // the tensor cores read the sub-tile through the async proxy
-        fence_proxy_async_smem();
+        tmem_st32(tmem_base + lane_off + kWoAColBase + slot * 32u, a);
+        tmem_wait_st();
+        tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar_afull + 8 * slot);
       }
@@ -335,14 +356,24 @@ __global__ void __launch_bounds__(kWoThreads, 2)
     }
     if (cw < 4) {
       // epilogue: warp w reads TMEM lanes 32*(w%4) .. +31 = output channels
-      const int sub = warp & 3;
-      const int n = n0 + sub * 32 + lane;
+      const int n = n0 + quarter * 32 + lane;
       if (!ok || *abort_flag || !mbar_wait(bar_tfull, 0)) {
         give_up();
       } else {
         tc_fence_after();
+        // the sum of the accumulators, in a fixed order
         uint32_t r[16];
-        tmem_ld16_wait_wo(tmem_base + (uint32_t(sub * 32) << 16), r);
+        tmem_ld16_wait_wo(tmem_base + lane_off, r);
+        // accumulators that received an MMA (all of them unless K is tiny)
+        const int n_acc = nk * SUBS * 4 < kWoNAcc ? nk * SUBS * 4 : kWoNAcc;
+#pragma unroll 1
+        for (int c = 1; c < n_acc; ++c) {
+          uint32_t r2[16];
+          tmem_ld16_wait_wo(tmem_base + lane_off + uint32_t(c * 16), r2);
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            r[j] = __float_as_uint(__fadd_rn(__uint_as_float(r[j]), __uint_as_float(r2[j])));
+        }
         if (n < N) {
           const float swn = __ldg(sw + n);
           float bn = 0.0f;
@@ -351,13 +382,13 @@ __global__ void __launch_bounds__(kWoThreads, 2)
           for (int j = 0; j < kWoTokens; ++j) {
             const int m = m0 + j;
             if (m < M) {
-              float a = __fmul_rn(__uint_as_float(r[j]), swn);
-              if constexpr (HAS_BIAS) a = __fadd_rn(a, bn);
+              float v = __fmul_rn(__uint_as_float(r[j]), swn);
+              if constexpr (HAS_BIAS) v = __fadd_rn(v, bn);
               const int64_t off = int64_t(m) * N + n;
               if constexpr (OUT_BF16)
-                static_cast<uint16_t*>(y)[off] = uint16_t(pack_bf16x2(a, 0.0f) & 0xFFFFu);
+                static_cast<uint16_t*>(y)[off] = uint16_t(pack_bf16x2(v, 0.0f) & 0xFFFFu);
               else
-                static_cast<float*>(y)[off] = a;
+                static_cast<float*>(y)[off] = v;
             }
           }
         }
@@ -369,7 +400,7 @@ __global__ void __launch_bounds__(kWoThreads, 2)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, 32);
+    tmem_dealloc(tmem_base, kWoTmemCols);
   }
 }
 
