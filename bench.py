@@ -427,7 +427,7 @@ def run_ours(args):
         else:
             ops.quantize_act(xs[r], s, qt, xq=xq, sx=sx, s_inv=s_inv)
 
-    split = bool(args.split)
+    split = not args.no_split
 
     def step(i):
         if wbits:
@@ -588,9 +588,10 @@ def run_ours(args):
             elif tensor:
                 ops.quantize_act_tensor(xd, s, qt, amax_prev=amax_b[0:1], xq=xq, sx=sx,
                                         amax_out=amax_b[1:2], s_inv=s_inv)
-                gemm(xq, sx, wq0, sw, bias, out=yd)
+                gemm(xq, sx, wq0, sw, bias, out=yd, split=split)
             else:
-                ops.linear(xd, s, wq0, sw, bias, qt, out=yd, xq_buf=xq, sx_buf=sx, s_inv=s_inv)
+                ops.linear(xd, s, wq0, sw, bias, qt, out=yd, xq_buf=xq, sx_buf=sx, s_inv=s_inv,
+                           split=split)
 
         def run_pipeline(n):
             ev = [[torch.cuda.Event() for _ in range(3)] for _ in range(n)]
@@ -668,7 +669,7 @@ def run_ours(args):
                        "launch": ((f"CUDA graph of {g_steps} steps, replayed"
                                    + (f", then one of {tail_steps}" if tail_steps else ""))
                                   if graph is not None else "one launch per kernel"),
-                       "split_last_wave": split,
+                       "gemm_workspace": ("passed: the last partial round of tiles is split where that pays" if split else "not passed"),
                        "gemm_tile": os.environ.get("SQ_GEMM_TILE", "auto")},
             "frac_of_int8_peak": None if wbits else value / ws / int8_peak,
             "frac_of_datasheet": None if wbits else value / ws / DATASHEET_8BIT_TOPS,
@@ -766,9 +767,9 @@ def main():
                     help="launch the timed steps one by one instead of replaying a CUDA graph")
     ap.add_argument("--workload", default="mlp_up_4096x4096x14336",
                     help="one of the six workloads in workloads.py (default: the MLP up-projection)")
-    ap.add_argument("--split", action="store_true",
-                    help="pass the GEMM workspace so the last partial wave of tiles is split "
-                         "along K over all SMs (stream-K)")
+    ap.add_argument("--no-split", action="store_true",
+                    help="launch the GEMM without its workspace (by default the library may split "
+                         "the last partial round of tiles along K over all SMs where that pays)")
     ap.add_argument("--sustained-s", type=float, default=1.5,
                     help="seconds of extra replays for the sustained figure (0: skip)")
     ap.add_argument("--measure-peaks", action="store_true",

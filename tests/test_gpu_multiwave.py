@@ -68,9 +68,16 @@ def test_shape_gives_every_tile_shape_several_tiles_per_unit():
         assert tiles / (SMS // cg) >= 3.0, name
 
 
+@pytest.fixture
+def force_split(monkeypatch):
+    """Split the last partial round on every tile shape (the library
+    otherwise splits only where it pays)."""
+    monkeypatch.setenv("SQ_GEMM_FORCE_SPLIT", "1")
+
+
 @pytest.mark.parametrize("split", [False, True])
 @pytest.mark.parametrize("tile", ops.GEMM_TILES)
-def test_int8_multiwave_bit_exact(int8_case, tile, split):
+def test_int8_multiwave_bit_exact(int8_case, tile, split, force_split):
     c = int8_case
     d = [dev(c[k]) for k in ("xq", "sx", "wq", "sw")]
     acc = torch.empty((M, N), dtype=torch.int32, device="cuda")
@@ -85,7 +92,7 @@ def test_int8_multiwave_bit_exact(int8_case, tile, split):
 
 @pytest.mark.parametrize("split", [False, True])
 @pytest.mark.parametrize("tile", ops.GEMM_TILES)
-def test_fp8_multiwave_full_range_codes(fp8_case, tile, split):
+def test_fp8_multiwave_full_range_codes(fp8_case, tile, split, force_split):
     c = fp8_case
     d = [dev(c[k]) for k in ("xq", "sx", "wq", "sw")]
     with ops.gemm_tile(tile):

@@ -164,8 +164,10 @@ def test_gemm_w8a8(M, N, K, with_bias):
 @pytest.mark.parametrize("M,N,K", [(300, 392, 4096), (129, 200, 96), (513, 520, 208),
                                    (1, 16, 32), (256, 448, 1024), (1100, 904, 272)])
 @pytest.mark.parametrize("qtype", ["i8", "e4m3"])
-def test_gemm_every_tile_shape(tile, M, N, K, qtype, split):
-    """Every compiled tile shape (1-CTA and SM-pair) on ragged sizes."""
+def test_gemm_every_tile_shape(tile, M, N, K, qtype, split, monkeypatch):
+    """Every compiled tile shape (1-CTA and SM-pair) on ragged sizes; with
+    split=True the last partial round is always split."""
+    monkeypatch.setenv("SQ_GEMM_FORCE_SPLIT", "1")
     g = np.random.default_rng(M + N + K)
     if qtype == "i8":
         xq = synth.random_matrix((M, K), np.int8, seed=M * 3 + K)
@@ -202,9 +204,10 @@ def test_gemm_every_tile_shape(tile, M, N, K, qtype, split):
         np.testing.assert_array_equal(host(yb), oracle.f32_to_bf16(host(yf)))
 
 
-def test_split_tiles_leave_workspace_clean_and_match_whole_tiles():
+def test_split_tiles_leave_workspace_clean_and_match_whole_tiles(monkeypatch):
     """Stream-K split tiles give the same bits as whole tiles (INT8 partial
     sums are exact) and the workspace counters are zero again afterwards."""
+    monkeypatch.setenv("SQ_GEMM_FORCE_SPLIT", "1")
     M, N, K = 1000, 2056, 2048
     xq = synth.random_matrix((M, K), np.int8, seed=41)
     wq = synth.random_matrix((N, K), np.int8, seed=42)

@@ -647,12 +647,27 @@ static int device_sms() {
   return n[dev];
 }
 
-// Whole-tile rounds first; when the last round would leave units idle, the
-// last one or two rounds' worth of tiles become a stream-K region shared by
-// all units (needs a workspace).
+// Whether splitting the last partial round pays: measured on B200, the split
+// region costs more than it saves unless whole-tile rounds waste at least a
+// tenth of the time (FP8 down 4096 x 14336 x 4096: 256 tiles on 74 SM pairs,
+// 4 rounds for 3.46 rounds of work, 180 -> 170 us; MLP up: 13 rounds for
+// 12.1, 163 -> 164 us; fewer tiles than units, as at 512 tokens: 22 -> 25 us).
+// SQ_GEMM_FORCE_SPLIT=1 in the environment splits every partial round (used
+// by the tests to reach the split path on every tile shape).
+static bool split_pays(int64_t tiles, int64_t units) {
+  const int64_t full = tiles / units, rem = tiles % units;
+  if (rem == 0) return false;
+  const char* force = getenv("SQ_GEMM_FORCE_SPLIT");
+  if (force && force[0] == '1') return true;
+  if (full == 0) return false;
+  return double(tiles) / double(units) <= 0.9 * double(full + 1);
+}
+
+// Whole-tile rounds first; when split_pays, the last one or two rounds' worth
+// of tiles become a stream-K region shared by all units (needs a workspace).
 static void plan_schedule(int num_tiles, int units, bool can_split, int* dp_rounds, int* sk_tiles) {
-  const int full = num_tiles / units, rem = num_tiles % units;
-  const bool split = can_split && rem != 0 && (full == 0 || rem < units * 85 / 100);
+  const int full = num_tiles / units;
+  const bool split = can_split && split_pays(num_tiles, units);
   if (!split) {
     *dp_rounds = (num_tiles + units - 1) / units;
     *sk_tiles = 0;
@@ -712,7 +727,9 @@ static cudaError_t run_gemm(const void* xq, const void* wq, const float* sx, con
   const size_t need = ws_slot_offset(0) + size_t(units_max) * CG * 128 * BN * 4;
   const bool can_split = ws != nullptr && ws_bytes >= need && !getenv("SQ_GEMM_NO_SPLIT");
   int units = tiles < units_max ? tiles : units_max;
-  if (can_split && tiles > 0 && int64_t(tiles) * ((K + kBK - 1) / kBK) >= units_max) units = units_max;
+  if (can_split && tiles > 0 && split_pays(tiles, units_max) &&
+      int64_t(tiles) * ((K + kBK - 1) / kBK) >= units_max)
+    units = units_max;
   int dp_rounds = 0, sk_tiles = 0;
   plan_schedule(tiles, units, can_split, &dp_rounds, &sk_tiles);
   if (sk_tiles > kMaxSkTiles) {
@@ -794,8 +811,9 @@ static TileCfg choose_tile(int64_t M, int64_t N, bool can_split) {
     const int64_t units = sms / c.cg;
     // with split tiles the last wave is shared (fractional rounds, plus a
     // small cost for the partial sums); without, whole rounds
-    const double rounds = can_split ? double(tiles) / double(units) + (tiles % units ? 0.1 : 0.0)
-                                    : double((tiles + units - 1) / units);
+    const double rounds = (can_split && split_pays(tiles, units))
+                              ? double(tiles) / double(units) + 0.1
+                              : double((tiles + units - 1) / units);
     const double t = rounds * double(c.bm) * double(c.bn) / (double(c.cg) * c.eff);
     if (t < best * 0.999) {
       best = t;

@@ -22,12 +22,14 @@
 //   warp 0    : TMA producer (Wq slice [128 rows x 128 B] + Xq slice
 //               [16 rows x 128 B], 128-byte swizzle; token rows beyond M read
 //               as zero)
-//   warp 1    : allocates 128 tensor-memory columns (eight accumulators of
-//               16 columns); one thread issues the MMAs (K = 32 per
-//               instruction) into the eight accumulators in turn -- an MMA of
-//               128 x 16 x 32 is far shorter than the latency of the
-//               accumulator it would otherwise wait for -- and frees ring
-//               slots with tcgen05.commit
+//   warps 1, 6: warp 1 allocates 128 tensor-memory columns (eight
+//               accumulators of 16 columns); one thread of each issues the
+//               MMAs of alternate k-blocks (K = 32 per instruction) into its
+//               own four accumulators in turn, and frees ring slots with
+//               tcgen05.commit. An MMA of 128 x 16 x 32 is short next to the
+//               latency of the accumulator it updates, and every commit
+//               stalls the issuing thread's stream; two issuers and four
+//               accumulators each keep the tensor cores busy.
 //   warps 2-5 : epilogue -- warp w reads lanes 32*(w%4)..+31 (its output
 //               channels) x 16 columns (the tokens) of each accumulator, adds
 //               them (int32, exact; E4M3 binary32 in a fixed order),
@@ -50,7 +52,8 @@ namespace sqk {
 constexpr int kSkBK = 128;       // bytes of K per stage
 constexpr int kSkMP = 16;        // token columns (N of the instruction)
 constexpr int kSkStages = 6;
-constexpr int kSkThreads = 192;  // producer, MMA, four epilogue warps
+constexpr int kSkThreads = 224;  // producer, MMA, four epilogue warps, second MMA warp
+constexpr int kSkMmaWarp1 = 6;   // the second MMA-issuing warp
 constexpr uint32_t kSkABytes = 128 * kSkBK;     // weight slice
 constexpr uint32_t kSkBBytes = kSkMP * kSkBK;   // token slice
 constexpr uint32_t kSkStageBytes = kSkABytes + kSkBBytes;
@@ -101,8 +104,8 @@ __global__ void __launch_bounds__(kSkThreads, 2)
       mbar_init(bar_full + 8 * i, 1);
       mbar_init(bar_empty + 8 * i, 1);
     }
-    mbar_init(bar_tfull, 1);
-    mbar_init(bar_drain, 1);
+    mbar_init(bar_tfull, 2);  // both MMA threads
+    mbar_init(bar_drain, 2);
     *abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_map(&tm_w);
@@ -154,13 +157,15 @@ __global__ void __launch_bounds__(kSkThreads, 2)
       for (int j = first; j < issued; ++j)
         (void)mbar_wait(bar_full + 8 * uint32_t(j % kSkStages), uint32_t(j / kSkStages) & 1u);
     }
-  } else if (warp == 1) {
+  } else if (warp == 1 || warp == kSkMmaWarp1) {
     // ----------------------------------------------------------------- MMA --
     if (lane == 0) {
       constexpr uint32_t idesc = E4M3 ? idesc_e4m3_f32(128, kSkMP) : idesc_s8_s32(128, kSkMP);
+      const int grp = warp == 1 ? 0 : 1;
       bool ok = true;
+      uint32_t j = 0;  // this thread's MMAs
 #pragma unroll 1
-      for (int kb = 0; kb < nk; ++kb) {
+      for (int kb = grp; kb < nk; kb += 2) {
         const uint32_t st = uint32_t(kb % kSkStages), ph = uint32_t(kb / kSkStages) & 1u;
         if (!mbar_wait(bar_full + 8 * st, ph) || *abort_flag) {
           record_status(status, kStatusTimeout);
@@ -171,15 +176,14 @@ __global__ void __launch_bounds__(kSkThreads, 2)
         tc_fence_after();
         const uint32_t a_addr = s_base + st * kSkStageBytes;
         const uint32_t b_addr = a_addr + kSkABytes;
-        // MMA j accumulates into accumulator j % kSkNAcc: consecutive MMAs
-        // do not wait for one another's result
+        // this thread's MMA j accumulates into accumulator 4 * grp + j % 4:
+        // consecutive MMAs do not wait for one another's result
 #pragma unroll
-        for (int kk = 0; kk < kSkBK / 32; ++kk) {
-          const uint32_t j = uint32_t(kb) * uint32_t(kSkBK / 32) + uint32_t(kk);
+        for (int kk = 0; kk < kSkBK / 32; ++kk, ++j) {
           const uint64_t ad = sw128_desc(a_addr + kk * 32);
           const uint64_t bd = sw128_desc(b_addr + kk * 32);
-          const uint32_t d = tmem_base + (j % kSkNAcc) * 16u;
-          const uint32_t accum = j >= uint32_t(kSkNAcc) ? 1u : 0u;
+          const uint32_t d = tmem_base + (4u * uint32_t(grp) + j % 4u) * 16u;
+          const uint32_t accum = j >= 4u ? 1u : 0u;
           if constexpr (E4M3) mma_f8(d, ad, bd, idesc, accum);
           else mma_i8(d, ad, bd, idesc, accum);
         }
@@ -202,8 +206,9 @@ __global__ void __launch_bounds__(kSkThreads, 2)
       // the sum of the accumulators (exact for INT8; in a fixed order for E4M3)
       uint32_t r[16];
       tmem_ld16_wait(tmem_base + (uint32_t(sub * 32) << 16), r);
-      // accumulators that received an MMA (all of them unless K is tiny)
-      const int n_acc = nk * (kSkBK / 32) < kSkNAcc ? nk * (kSkBK / 32) : kSkNAcc;
+      // accumulators that received an MMA: the four of the first MMA thread,
+      // and those of the second when there are at least two k-blocks
+      const int n_acc = nk >= 2 ? kSkNAcc : 4;
 #pragma unroll 1
       for (int c = 1; c < n_acc; ++c) {
         uint32_t r2[16];

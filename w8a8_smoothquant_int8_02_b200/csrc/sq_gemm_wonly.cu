@@ -27,14 +27,16 @@
 //                 packed weights [128 rows x 128 B] (128 k for INT8, 256 for
 //                 INT4) and the matching bf16 token slices [16 rows x 64 k]
 //                 into a 5- (INT8) or 4-stage (INT4) shared-memory ring
-//   warp 1      : tensor memory (256 columns: eight accumulators and a
-//                 4-deep ring of bf16 weight sub-tiles); one thread issues
-//                 the MMAs (A from tensor memory, B = the token slice from
-//                 shared memory, K = 16 per instruction), rotating over the
-//                 eight accumulators so that consecutive MMAs are independent
-//                 (one MMA of 128 x 16 x 16 is far shorter than the latency
-//                 of the accumulator it would otherwise wait for), and frees
-//                 buffers by tcgen05.commit
+//   warps 1, 10 : warp 1 allocates tensor memory (256 columns: eight
+//                 accumulators and a 4-deep ring of bf16 weight sub-tiles);
+//                 one thread of each issues the MMAs of alternate sub-tiles
+//                 (A from tensor memory, B = the token slice from shared
+//                 memory, K = 16 per instruction) into its own four
+//                 accumulators in turn, and frees buffers by tcgen05.commit.
+//                 An MMA of 128 x 16 x 16 is short next to the latency of the
+//                 accumulator it updates, and every commit stalls the
+//                 issuing thread's stream; two issuers and four accumulators
+//                 each keep the tensor cores busy.
 //   warps 2..9  : two groups of four (one warp per lane quarter) taking
 //                 alternate 64-k sub-tiles: each thread widens its weight
 //                 row's 64 codes to 32 bf16 pairs and stores them to tensor
@@ -57,7 +59,8 @@ namespace sqk {
 
 constexpr int kWoTokens = 16;                 // token columns (N of the instruction)
 constexpr int kWoConvWarps = 8;               // two groups of four, alternating sub-tiles
-constexpr int kWoThreads = 64 + 32 * kWoConvWarps;
+constexpr int kWoMmaWarp1 = 2 + kWoConvWarps;  // the second MMA-issuing warp
+constexpr int kWoThreads = 96 + 32 * kWoConvWarps;
 constexpr uint32_t kWoWBytes = 128 * 128;     // packed weight slice of one stage
 constexpr uint32_t kWoXSub = kWoTokens * 128; // bf16 token sub-tile [16 x 64 k]
 constexpr uint32_t kWoTmemCols = 256;         // per CTA: accumulators + A ring
@@ -178,14 +181,14 @@ __global__ void __launch_bounds__(kWoThreads, 2)
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) {
       mbar_init(bar_full + 8 * i, 1);
-      mbar_init(bar_empty + 8 * i, kWoConvWarps + 1);  // every widening warp + the MMAs
+      mbar_init(bar_empty + 8 * i, kWoConvWarps + 2);  // every widening warp + both MMA threads
     }
     for (int i = 0; i < NA; ++i) {
       mbar_init(bar_afull + 8 * i, 4);                 // the four warps of one group
       mbar_init(bar_aempty + 8 * i, 1);
     }
-    mbar_init(bar_tfull, 1);
-    mbar_init(bar_drain, 1);
+    mbar_init(bar_tfull, 2);
+    mbar_init(bar_drain, 2);
     *abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_map(&tm_w);
@@ -242,12 +245,16 @@ __global__ void __launch_bounds__(kWoThreads, 2)
       for (int j = first; j < issued; ++j)
         (void)mbar_wait(bar_full + 8 * uint32_t(j % S), uint32_t(j / S) & 1u);
     }
-  } else if (warp == 1) {
+  } else if (warp == 1 || warp == kWoMmaWarp1) {
     // ----------------------------------------------------------------- MMA --
+    // Two issuing threads, one per group of sub-tiles (ia % 2), each into its
+    // own four accumulators: a tcgen05.commit stalls the stream of the thread
+    // that issues it, so two streams keep the tensor cores busy.
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(128, kWoTokens);
+      const uint32_t grp = warp == 1 ? 0u : 1u;
       bool ok = true;
-      uint32_t ia = 0;
+      uint32_t ia = 0, j = 0;  // sub-tile counter (all groups); this thread's MMAs
 #pragma unroll 1
       for (int kb = 0; kb < nk && ok; ++kb) {
         const uint32_t st = uint32_t(kb % S), ph = uint32_t(kb / S) & 1u;
@@ -259,6 +266,7 @@ __global__ void __launch_bounds__(kWoThreads, 2)
         const uint32_t x_addr = s_base + st * C::kStageBytes + kWoWBytes;
 #pragma unroll 1
         for (int t = 0; t < SUBS; ++t, ++ia) {
+          if ((ia & 1u) != grp) continue;
           const uint32_t slot = ia % NA;
           if (*abort_flag || !mbar_wait(bar_afull + 8 * slot, (ia / NA) & 1u)) {
             give_up();
@@ -267,14 +275,13 @@ __global__ void __launch_bounds__(kWoThreads, 2)
           }
           tc_fence_after();
           const uint32_t a_tmem = tmem_base + kWoAColBase + slot * 32u;
-          // MMA j accumulates into accumulator j % kWoNAcc: consecutive MMAs
-          // do not wait for one another's result
+          // this thread's MMA j accumulates into accumulator 4 * grp + j % 4:
+          // consecutive MMAs do not wait for one another's result
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint32_t j = ia * 4u + uint32_t(kk);
+          for (int kk = 0; kk < 4; ++kk, ++j) {
             const uint64_t bd = sw128_desc(x_addr + t * kWoXSub + kk * 32);
-            mma_bf16_ts(tmem_base + (j % kWoNAcc) * 16u, a_tmem + uint32_t(kk * 8), bd, idesc,
-                        j >= uint32_t(kWoNAcc) ? 1u : 0u);
+            mma_bf16_ts(tmem_base + (4u * grp + j % 4u) * 16u, a_tmem + uint32_t(kk * 8), bd,
+                        idesc, j >= 4u ? 1u : 0u);
           }
           tc_commit(bar_aempty + 8 * slot);
         }
@@ -361,13 +368,12 @@ __global__ void __launch_bounds__(kWoThreads, 2)
         give_up();
       } else {
         tc_fence_after();
-        // the sum of the accumulators, in a fixed order
+        // the sum of the accumulators, in a fixed order (every one received
+        // MMAs: each MMA thread has at least one sub-tile, 4 MMAs each)
         uint32_t r[16];
         tmem_ld16_wait_wo(tmem_base + lane_off, r);
-        // accumulators that received an MMA (all of them unless K is tiny)
-        const int n_acc = nk * SUBS * 4 < kWoNAcc ? nk * SUBS * 4 : kWoNAcc;
 #pragma unroll 1
-        for (int c = 1; c < n_acc; ++c) {
+        for (int c = 1; c < kWoNAcc; ++c) {
           uint32_t r2[16];
           tmem_ld16_wait_wo(tmem_base + lane_off + uint32_t(c * 16), r2);
 #pragma unroll
