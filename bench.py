@@ -87,6 +87,7 @@ PROFILED_TRAFFIC = {
 }
 KERNEL_SOURCES = {"gemm": ("sq_gemm.cu", "sq_common.cuh"),
                   "gemm_wonly": ("sq_gemm_wonly.cu", "sq_common.cuh"),
+                  "gemm_small": ("sq_gemm_small.cu", "sq_common.cuh"),
                   "gemm_skinny": ("sq_gemm_skinny.cu", "sq_common.cuh"),
                   "quant": ("sq_quant.cu", "sq_common.cuh")}
 
@@ -131,13 +132,17 @@ SKINNY_MAX_M = 16  # the library's weight-streaming GEMM takes M <= 16 (sq_gemm_
 
 def gemm_kind(case, forced_tile=None):
     """Which GEMM kernel the library runs for this workload: the weight-only
-    kernel for W8A16 / W4A16, the weight-streaming form for at most 16 tokens
-    (unless a tile shape is forced), else the tiled kernel. Returns (traffic
-    key, kernel name)."""
+    kernel for W8A16 / W4A16, the weight-streaming form for at most 16 tokens,
+    the four-issuer form when the 128 x 128 tiles fit in one wave (unless a
+    tile shape is forced), else the tiled kernel. Returns (traffic key,
+    kernel name)."""
     if weight_bits(case):
         return "gemm_wonly", "gemm_wonly_kernel"
     if case.M <= SKINNY_MAX_M and not forced_tile:
         return "gemm_skinny", "gemm_skinny_kernel"
+    tiles = -(-case.M // 128) * -(-case.N // 128)
+    if tiles <= 148 and case.K >= 1024 and not forced_tile:
+        return "gemm_small", "gemm_small_kernel"
     return "gemm", "gemm_w8a8_kernel"
 
 

@@ -119,12 +119,31 @@ def test_gemm_roofline_bound_follows_the_ridge_point(bench):
 
 def test_gemm_kernel_per_workload(bench):
     """At most 16 tokens run the weight-streaming kernel unless a tile shape
-    is forced; every other workload the tiled kernel."""
+    is forced; single-wave problems (prefill: 4 x 32 tiles of 128 x 128) the
+    four-issuer kernel; weight-only workloads their own kernel; every other
+    workload the tiled kernel."""
     assert bench.gemm_kind(workloads.DECODE) == ("gemm_skinny", "gemm_skinny_kernel")
     assert bench.gemm_kind(workloads.TINY) == ("gemm_skinny", "gemm_skinny_kernel")
     assert bench.gemm_kind(workloads.DECODE, "c1n224") == ("gemm", "gemm_w8a8_kernel")
     assert bench.gemm_kind(workloads.MLP_UP) == ("gemm", "gemm_w8a8_kernel")
-    assert bench.gemm_kind(workloads.PREFILL) == ("gemm", "gemm_w8a8_kernel")
+    assert bench.gemm_kind(workloads.PREFILL) == ("gemm_small", "gemm_small_kernel")
+    assert bench.gemm_kind(workloads.PREFILL, "c2n256") == ("gemm", "gemm_w8a8_kernel")
+    assert bench.gemm_kind(workloads.DECODE_W4A16) == ("gemm_wonly", "gemm_wonly_kernel")
+
+
+def test_single_wave_rule_matches_the_library(bench):
+    """bench.py names the four-issuer kernel by the same tile and K rule the
+    library dispatches on (128 x 128 tiles, at most one per SM, K of at least
+    two 128-byte k-blocks per issuing thread)."""
+    import re
+    src = open(os.path.join(ROOT, "w8a8_smoothquant_int8_02_b200", "csrc",
+                            "sq_gemm_small.cu")).read()
+    assert int(re.search(r"constexpr int kSmTile = (\d+);", src).group(1)) == 128
+    assert int(re.search(r"constexpr int kSmIssuers = (\d+);", src).group(1)) * 2 * 128 == 1024
+    from w8a8_smoothquant_int8_02_b200 import synth
+    at = workloads.PREFILL.__dict__
+    assert bench.gemm_kind(synth.LinearCase(**{**at, "K": 1008}))[0] == "gemm"
+    assert bench.gemm_kind(synth.LinearCase(**{**at, "M": 640}))[0] == "gemm"   # 5 x 32 > 148
 
 
 def test_few_token_threshold_matches_the_library(bench):

@@ -67,14 +67,19 @@ sq_status check_gemm(const void* xq, const float* sx, const void* wq, const floa
 }
 
 // Few tokens (M <= 16) take the weight-streaming form with the operand roles
-// swapped (sq_gemm_skinny.cu, same results, no workspace); SQ_GEMM_TILE or
-// SQ_GEMM_NO_SKINNY in the environment keep the tiled kernel for every M.
+// swapped (sq_gemm_skinny.cu); problems whose 128 x 128 tiles fit in one wave
+// the four-issuer form (sq_gemm_small.cu); everything else the persistent
+// tiled kernel (sq_gemm.cu). Same results (INT8 bit for bit), no workspace
+// for the first two. SQ_GEMM_TILE in the environment keeps the tiled kernel
+// for every shape; SQ_GEMM_NO_SKINNY / SQ_GEMM_NO_SMALL skip one form.
 cudaError_t run_gemm_any(bool e4m3, const uint8_t* xq, const float* sx, const uint8_t* wq,
                          const float* sw, const uint16_t* bias, int64_t M, int64_t N, int64_t K,
                          void* y, sqh::OutKind yk, int32_t* acc, void* ws, size_t ws_bytes,
                          cudaStream_t st) {
   if (sqh::gemm_skinny_applies(M))
     return sqh::launch_gemm_skinny(e4m3, xq, sx, wq, sw, bias, M, N, K, y, yk, acc, st);
+  if (sqh::gemm_small_applies(M, N, K))
+    return sqh::launch_gemm_small(e4m3, xq, sx, wq, sw, bias, M, N, K, y, yk, acc, st);
   return sqh::launch_gemm(e4m3, xq, sx, wq, sw, bias, M, N, K, y, yk, acc, ws, ws_bytes, st);
 }
 

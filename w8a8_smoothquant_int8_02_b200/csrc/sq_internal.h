@@ -44,6 +44,11 @@ bool gemm_skinny_applies(int64_t M);
 cudaError_t launch_gemm_skinny(bool e4m3, const uint8_t* xq, const float* sx, const uint8_t* wq,
                                const float* sw, const uint16_t* bias, int64_t M, int64_t N,
                                int64_t K, void* y, OutKind yk, int32_t* acc, cudaStream_t st);
+// a6 / a7 when the 128 x 128 tiles fit in one wave (sq_gemm_small.cu)
+bool gemm_small_applies(int64_t M, int64_t N, int64_t K);
+cudaError_t launch_gemm_small(bool e4m3, const uint8_t* xq, const float* sx, const uint8_t* wq,
+                              const float* sw, const uint16_t* bias, int64_t M, int64_t N,
+                              int64_t K, void* y, OutKind yk, int32_t* acc, cudaStream_t st);
 // weight-only W8A16 / W4A16 GEMM for few tokens (sq_gemm_wonly.cu)
 cudaError_t launch_gemm_weight_only(int bits, const uint16_t* x, const void* wq, const float* sw,
                                     const uint16_t* bias, int64_t M, int64_t N, int64_t K,
