@@ -22,14 +22,15 @@
 //   warp 0    : TMA producer (Wq slice [128 rows x 128 B] + Xq slice
 //               [16 rows x 128 B], 128-byte swizzle; token rows beyond M read
 //               as zero)
-//   warps 1, 6: warp 1 allocates 128 tensor-memory columns (eight
-//               accumulators of 16 columns); one thread of each issues the
-//               MMAs of alternate k-blocks (K = 32 per instruction) into its
-//               own four accumulators in turn, and frees ring slots with
-//               tcgen05.commit. An MMA of 128 x 16 x 32 is short next to the
-//               latency of the accumulator it updates, and every commit
-//               stalls the issuing thread's stream; two issuers and four
-//               accumulators each keep the tensor cores busy.
+//   warps 1, 6-8: warp 1 allocates 128 tensor-memory columns (eight
+//               accumulators of 16 columns); one thread of each warp issues
+//               the MMAs of every fourth k-block (K = 32 per instruction)
+//               into its own two accumulators in turn, and frees ring slots
+//               with tcgen05.commit. An MMA of 128 x 16 x 32 is short, and a
+//               single thread's stream of them is slow once commits are
+//               interleaved (on the order of a hundred nanoseconds or more
+//               per instruction, measured on B200), while the streams of
+//               different warps overlap: four issuers keep up with HBM.
 //   warps 2-5 : epilogue -- warp w reads lanes 32*(w%4)..+31 (its output
 //               channels) x 16 columns (the tokens) of each accumulator, adds
 //               them (int32, exact; E4M3 binary32 in a fixed order),
@@ -52,8 +53,9 @@ namespace sqk {
 constexpr int kSkBK = 128;       // bytes of K per stage
 constexpr int kSkMP = 16;        // token columns (N of the instruction)
 constexpr int kSkStages = 6;
-constexpr int kSkThreads = 224;  // producer, MMA, four epilogue warps, second MMA warp
-constexpr int kSkMmaWarp1 = 6;   // the second MMA-issuing warp
+constexpr int kSkIssuers = 4;    // MMA-issuing threads: warp 1, then warps 6 ..
+constexpr int kSkMmaWarpB = 6;   // warp of the second issuer
+constexpr int kSkThreads = 32 * (kSkMmaWarpB + kSkIssuers - 1);  // producer, MMA, 4 epilogue, MMA
 constexpr uint32_t kSkABytes = 128 * kSkBK;     // weight slice
 constexpr uint32_t kSkBBytes = kSkMP * kSkBK;   // token slice
 constexpr uint32_t kSkStageBytes = kSkABytes + kSkBBytes;
@@ -61,7 +63,7 @@ constexpr uint32_t kSkBarOff = kSkStages * kSkStageBytes;
 // barriers: full[S], empty[S], tfull, drain; then the TMEM slot and abort flag
 constexpr uint32_t kSkMiscOff = kSkBarOff + (2 * kSkStages + 2) * 8;
 constexpr uint32_t kSkDynamic = kSkMiscOff + 16 + 1024;  // slack for 1024-B alignment
-constexpr int kSkNAcc = 8;                               // independent accumulators
+constexpr int kSkNAcc = 2 * kSkIssuers;                  // two accumulators per issuer
 constexpr uint32_t kSkTmemCols = kSkNAcc * 16;          // 16 columns each
 static_assert(kSkStageBytes % 1024 == 0, "stages must keep 1024-byte alignment");
 static_assert(kSkDynamic * 2 + 2048 <= 233472, "two CTAs per SM must fit");
@@ -98,14 +100,16 @@ __global__ void __launch_bounds__(kSkThreads, 2)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kSkMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kSkMiscOff + 4);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nk = (K + kSkBK - 1) / kSkBK;
+  const int n_active = nk < kSkIssuers ? nk : kSkIssuers;  // issuers with k-blocks
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kSkStages; ++i) {
       mbar_init(bar_full + 8 * i, 1);
       mbar_init(bar_empty + 8 * i, 1);
     }
-    mbar_init(bar_tfull, 2);  // both MMA threads
-    mbar_init(bar_drain, 2);
+    mbar_init(bar_tfull, uint32_t(n_active));  // the MMA threads with k-blocks
+    mbar_init(bar_drain, kSkIssuers);
     *abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_map(&tm_w);
@@ -124,7 +128,6 @@ __global__ void __launch_bounds__(kSkThreads, 2)
   pdl_wait();
 
   const int n0 = int(blockIdx.x) * 128;
-  const int nk = (K + kSkBK - 1) / kSkBK;
   // every CTA reads the same token slices; starting each CTA at a different
   // k-block spreads those reads over the L2 instead of all CTAs asking for
   // the same lines at once (integer sums do not depend on the order)
@@ -157,16 +160,27 @@ __global__ void __launch_bounds__(kSkThreads, 2)
       for (int j = first; j < issued; ++j)
         (void)mbar_wait(bar_full + 8 * uint32_t(j % kSkStages), uint32_t(j / kSkStages) & 1u);
     }
-  } else if (warp == 1 || warp == kSkMmaWarp1) {
+  } else if (warp == 1 || warp >= kSkMmaWarpB) {
     // ----------------------------------------------------------------- MMA --
     if (lane == 0) {
       constexpr uint32_t idesc = E4M3 ? idesc_e4m3_f32(128, kSkMP) : idesc_s8_s32(128, kSkMP);
-      const int grp = warp == 1 ? 0 : 1;
+      const int q = warp == 1 ? 0 : warp - kSkMmaWarpB + 1;
       bool ok = true;
       uint32_t j = 0;  // this thread's MMAs
 #pragma unroll 1
-      for (int kb = grp; kb < nk; kb += 2) {
+      for (int kb = q; kb < nk; kb += kSkIssuers) {
         const uint32_t st = uint32_t(kb % kSkStages), ph = uint32_t(kb / kSkStages) & 1u;
+        // The uses of a ring slot pass from issuer to issuer (six stages,
+        // four issuers), so the previous use of this one may be another
+        // thread's: wait for its commit (the phase the producer waits for
+        // before refilling) first. Then the full barrier cannot be two phases
+        // behind this wait, where its parity would match a completed phase.
+        if (kb >= kSkStages && (!mbar_wait(bar_empty + 8 * st, ph ^ 1u) || *abort_flag)) {
+          record_status(status, kStatusTimeout);
+          *abort_flag = 1;
+          ok = false;
+          break;
+        }
         if (!mbar_wait(bar_full + 8 * st, ph) || *abort_flag) {
           record_status(status, kStatusTimeout);
           *abort_flag = 1;
@@ -176,20 +190,19 @@ __global__ void __launch_bounds__(kSkThreads, 2)
         tc_fence_after();
         const uint32_t a_addr = s_base + st * kSkStageBytes;
         const uint32_t b_addr = a_addr + kSkABytes;
-        // this thread's MMA j accumulates into accumulator 4 * grp + j % 4:
-        // consecutive MMAs do not wait for one another's result
+        // this thread's MMA j accumulates into accumulator 2 * q + j % 2
 #pragma unroll
         for (int kk = 0; kk < kSkBK / 32; ++kk, ++j) {
           const uint64_t ad = sw128_desc(a_addr + kk * 32);
           const uint64_t bd = sw128_desc(b_addr + kk * 32);
-          const uint32_t d = tmem_base + (4u * uint32_t(grp) + j % 4u) * 16u;
-          const uint32_t accum = j >= 4u ? 1u : 0u;
+          const uint32_t d = tmem_base + (2u * uint32_t(q) + j % 2u) * 16u;
+          const uint32_t accum = j >= 2u ? 1u : 0u;
           if constexpr (E4M3) mma_f8(d, ad, bd, idesc, accum);
           else mma_i8(d, ad, bd, idesc, accum);
         }
         tc_commit(bar_empty + 8 * st);
       }
-      if (ok) tc_commit(bar_tfull);
+      if (ok && q < n_active) tc_commit(bar_tfull);  // the issuers with k-blocks
       // every MMA issued has finished before tensor memory can be freed
       tc_commit(bar_drain);
       (void)mbar_wait(bar_drain, 0);
@@ -206,9 +219,9 @@ __global__ void __launch_bounds__(kSkThreads, 2)
       // the sum of the accumulators (exact for INT8; in a fixed order for E4M3)
       uint32_t r[16];
       tmem_ld16_wait(tmem_base + (uint32_t(sub * 32) << 16), r);
-      // accumulators that received an MMA: the four of the first MMA thread,
-      // and those of the second when there are at least two k-blocks
-      const int n_acc = nk >= 2 ? kSkNAcc : 4;
+      // accumulators that received an MMA: both of every issuer with a
+      // k-block (each k-block is four MMAs)
+      const int n_acc = 2 * n_active;
 #pragma unroll 1
       for (int c = 1; c < n_acc; ++c) {
         uint32_t r2[16];

@@ -142,6 +142,16 @@ __global__ void __launch_bounds__(kSmThreads, 1)
 #pragma unroll 1
       for (int kb = q; kb < nk; kb += kSmIssuers) {
         const uint32_t st = uint32_t(kb % kSmStages), ph = uint32_t(kb / kSmStages) & 1u;
+        // The uses of a ring slot pass from issuer to issuer (six stages,
+        // four issuers), so the previous use of this one may be another
+        // thread's: wait for its commit (the phase the producer waits for
+        // before refilling) first. Then the full barrier cannot be two phases
+        // behind this wait, where its parity would match a completed phase.
+        if (kb >= kSmStages && (*abort_flag || !mbar_wait(bar_empty + 8 * st, ph ^ 1u))) {
+          give_up();
+          ok = false;
+          break;
+        }
         if (*abort_flag || !mbar_wait(bar_full + 8 * st, ph)) {
           give_up();
           ok = false;

@@ -59,14 +59,15 @@ namespace sqk {
 
 constexpr int kWoTokens = 16;                 // token columns (N of the instruction)
 constexpr int kWoConvWarps = 8;               // two groups of four, alternating sub-tiles
-constexpr int kWoMmaWarp1 = 2 + kWoConvWarps;  // the second MMA-issuing warp
-constexpr int kWoThreads = 96 + 32 * kWoConvWarps;
+constexpr int kWoIssuers = 4;                 // MMA-issuing threads, one accumulator each
+constexpr int kWoMmaWarpB = 2 + kWoConvWarps;  // warps of issuers 1.. (issuer 0 is warp 1)
+constexpr int kWoThreads = 32 * (2 + kWoConvWarps + kWoIssuers - 1);
 constexpr uint32_t kWoWBytes = 128 * 128;     // packed weight slice of one stage
 constexpr uint32_t kWoXSub = kWoTokens * 128; // bf16 token sub-tile [16 x 64 k]
 constexpr uint32_t kWoTmemCols = 256;         // per CTA: accumulators + A ring
-constexpr int kWoNAcc = 8;                    // independent accumulators (16 columns each)
+constexpr int kWoNAcc = kWoIssuers;           // accumulators (16 columns each)
 constexpr uint32_t kWoAColBase = kWoNAcc * 16;  // first A column
-constexpr int kWoNA = 4;                      // A sub-tiles in tensor memory (32 columns each)
+constexpr int kWoNA = 6;                      // A sub-tiles in tensor memory (32 columns each)
 
 template <int BITS>
 struct WoCfg {
@@ -83,6 +84,7 @@ struct WoCfg {
   static_assert(2 * (kDynamic + 1024) <= 233472, "two CTAs per SM must fit");
 };
 static_assert(kWoAColBase + kWoNA * 32 <= kWoTmemCols, "A ring must fit the allocation");
+static_assert(kWoNA >= kWoIssuers, "every issuer needs an A slot of its own in flight");
 
 // Instruction descriptor of tcgen05.mma kind::f16 with bf16 A and B and
 // binary32 accumulators: bits 4-5 D format, 7-9 / 10-12 A / B formats,
@@ -177,18 +179,27 @@ __global__ void __launch_bounds__(kWoThreads, 2)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nk = (K + C::KS - 1) / C::KS;
+  // issuer q takes the sub-tiles ia with ia % kWoIssuers == q: a stage holds
+  // SUBS consecutive sub-tiles, so SUBS issuers (at most all) use each one
+  constexpr int kStageIssuers = SUBS < kWoIssuers ? SUBS : kWoIssuers;
+  static_assert(kWoIssuers % SUBS == 0 || SUBS % kWoIssuers == 0,
+                "the issuers of a stage must be SUBS distinct threads");
+  const int n_sub = nk * SUBS;
+  const int n_active = n_sub < kWoIssuers ? n_sub : kWoIssuers;  // issuers with sub-tiles
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) {
       mbar_init(bar_full + 8 * i, 1);
-      mbar_init(bar_empty + 8 * i, kWoConvWarps + 2);  // every widening warp + both MMA threads
+      // every widening warp + the issuers with a sub-tile in the stage
+      mbar_init(bar_empty + 8 * i, kWoConvWarps + kStageIssuers);
     }
     for (int i = 0; i < NA; ++i) {
       mbar_init(bar_afull + 8 * i, 4);                 // the four warps of one group
       mbar_init(bar_aempty + 8 * i, 1);
     }
-    mbar_init(bar_tfull, 2);
-    mbar_init(bar_drain, 2);
+    mbar_init(bar_tfull, uint32_t(n_active));
+    mbar_init(bar_drain, kWoIssuers);
     *abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_map(&tm_w);
@@ -208,7 +219,6 @@ __global__ void __launch_bounds__(kWoThreads, 2)
 
   const int n0 = int(blockIdx.x) * 128;
   const int m0 = int(blockIdx.y) * kWoTokens;
-  const int nk = (K + C::KS - 1) / C::KS;
   // every CTA reads the same token slices; starting each CTA at a different
   // k-block spreads those reads over the L2 instead of all CTAs asking for
   // the same lines at once (the sum is the same up to binary32 rounding)
@@ -245,19 +255,35 @@ __global__ void __launch_bounds__(kWoThreads, 2)
       for (int j = first; j < issued; ++j)
         (void)mbar_wait(bar_full + 8 * uint32_t(j % S), uint32_t(j / S) & 1u);
     }
-  } else if (warp == 1 || warp == kWoMmaWarp1) {
+  } else if (warp == 1 || warp >= kWoMmaWarpB) {
     // ----------------------------------------------------------------- MMA --
-    // Two issuing threads, one per group of sub-tiles (ia % 2), each into its
-    // own four accumulators: a tcgen05.commit stalls the stream of the thread
-    // that issues it, so two streams keep the tensor cores busy.
+    // Four issuing threads, issuer q taking the sub-tiles ia = q (mod 4),
+    // each into its own accumulator: a single thread's tcgen05.mma stream is
+    // slow for these short instructions once commits are interleaved, while
+    // the streams of different warps overlap.
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(128, kWoTokens);
-      const uint32_t grp = warp == 1 ? 0u : 1u;
+      const uint32_t q = warp == 1 ? 0u : uint32_t(warp - kWoMmaWarpB + 1);
+      const uint32_t d = tmem_base + q * 16u;
       bool ok = true;
-      uint32_t ia = 0, j = 0;  // sub-tile counter (all groups); this thread's MMAs
+      uint32_t j = 0;  // this thread's MMAs so far
 #pragma unroll 1
       for (int kb = 0; kb < nk && ok; ++kb) {
+        // sub-tiles SUBS*kb .. SUBS*kb + SUBS-1: is one of them this thread's?
+        const uint32_t ia0 = uint32_t(kb) * SUBS;
+        const uint32_t t0 = (q + kWoIssuers - ia0 % kWoIssuers) % kWoIssuers;
+        if (t0 >= uint32_t(SUBS)) continue;
         const uint32_t st = uint32_t(kb % S), ph = uint32_t(kb / S) & 1u;
+        // The issuers of a stage change from one use of it to the next, so
+        // the previous use may be other threads': wait for its release (the
+        // phase the producer waits for before refilling) first. Then the
+        // full barrier cannot be two phases behind this wait, where its
+        // parity would match a completed phase.
+        if (kb >= S && (*abort_flag || !mbar_wait(bar_empty + 8 * st, ph ^ 1u))) {
+          give_up();
+          ok = false;
+          break;
+        }
         if (*abort_flag || !mbar_wait(bar_full + 8 * st, ph)) {
           give_up();
           ok = false;
@@ -265,9 +291,17 @@ __global__ void __launch_bounds__(kWoThreads, 2)
         }
         const uint32_t x_addr = s_base + st * C::kStageBytes + kWoWBytes;
 #pragma unroll 1
-        for (int t = 0; t < SUBS; ++t, ++ia) {
-          if ((ia & 1u) != grp) continue;
+        for (uint32_t t = t0; t < uint32_t(SUBS); t += kWoIssuers) {
+          const uint32_t ia = ia0 + t;
           const uint32_t slot = ia % NA;
+          // the same for the A slots: the previous use of this slot may
+          // have been another issuer's
+          if (ia >= uint32_t(NA) &&
+              (*abort_flag || !mbar_wait(bar_aempty + 8 * slot, ((ia / NA) & 1u) ^ 1u))) {
+            give_up();
+            ok = false;
+            break;
+          }
           if (*abort_flag || !mbar_wait(bar_afull + 8 * slot, (ia / NA) & 1u)) {
             give_up();
             ok = false;
@@ -275,20 +309,17 @@ __global__ void __launch_bounds__(kWoThreads, 2)
           }
           tc_fence_after();
           const uint32_t a_tmem = tmem_base + kWoAColBase + slot * 32u;
-          // this thread's MMA j accumulates into accumulator 4 * grp + j % 4:
-          // consecutive MMAs do not wait for one another's result
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk, ++j) {
             const uint64_t bd = sw128_desc(x_addr + t * kWoXSub + kk * 32);
-            mma_bf16_ts(tmem_base + (4u * grp + j % 4u) * 16u, a_tmem + uint32_t(kk * 8), bd,
-                        idesc, j >= 4u ? 1u : 0u);
+            mma_bf16_ts(d, a_tmem + uint32_t(kk * 8), bd, idesc, j > 0u ? 1u : 0u);
           }
           tc_commit(bar_aempty + 8 * slot);
         }
         if (!ok) break;
-        tc_commit(bar_empty + 8 * st);  // the token slices of this stage are read
+        tc_commit(bar_empty + 8 * st);  // this thread is done with the stage's token slices
       }
-      if (ok) tc_commit(bar_tfull);
+      if (ok && q < uint32_t(n_active)) tc_commit(bar_tfull);
       // every MMA issued has finished before tensor memory can be freed
       tc_commit(bar_drain);
       (void)mbar_wait(bar_drain, 0);
@@ -368,12 +399,12 @@ __global__ void __launch_bounds__(kWoThreads, 2)
         give_up();
       } else {
         tc_fence_after();
-        // the sum of the accumulators, in a fixed order (every one received
-        // MMAs: each MMA thread has at least one sub-tile, 4 MMAs each)
+        // the sum of the accumulators of the issuers that had sub-tiles, in
+        // a fixed order
         uint32_t r[16];
         tmem_ld16_wait_wo(tmem_base + lane_off, r);
 #pragma unroll 1
-        for (int c = 1; c < kWoNAcc; ++c) {
+        for (int c = 1; c < n_active; ++c) {
           uint32_t r2[16];
           tmem_ld16_wait_wo(tmem_base + lane_off + uint32_t(c * 16), r2);
 #pragma unroll
