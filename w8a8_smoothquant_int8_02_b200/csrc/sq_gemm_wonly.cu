@@ -23,25 +23,28 @@
 // M = 128 operand, the (up to) 16 token rows the N = 16 operand, D[n][m] in
 // 128 lanes x 16 columns of tensor memory. One CTA per 128 output channels
 // and 16 tokens (grid.y walks token tiles of larger batches); two CTAs per SM.
-//   warp 0      : TMA producer -- per stage one 128-byte-wide K slice of the
-//                 packed weights [128 rows x 128 B] (128 k for INT8, 256 for
-//                 INT4) and the matching bf16 token slices [16 rows x 64 k]
-//                 into a 5- (INT8) or 4-stage (INT4) shared-memory ring
-//   warps 1, 10 : warp 1 allocates tensor memory (256 columns: eight
-//                 accumulators and a 4-deep ring of bf16 weight sub-tiles);
-//                 one thread of each issues the MMAs of alternate sub-tiles
-//                 (A from tensor memory, B = the token slice from shared
-//                 memory, K = 16 per instruction) into its own four
-//                 accumulators in turn, and frees buffers by tcgen05.commit.
-//                 An MMA of 128 x 16 x 16 is short next to the latency of the
-//                 accumulator it updates, and every commit stalls the
-//                 issuing thread's stream; two issuers and four accumulators
-//                 each keep the tensor cores busy.
+//   warp 0      : weight producer -- per stage one 128-byte-wide K slice of
+//                 the packed weights [128 rows x 128 B] (128 k for INT8, 256
+//                 for INT4) into a 5-stage ring (128-byte swizzle)
+//   warp 10     : token producer -- the matching bf16 token slices [16 rows
+//                 x 64 k] into a ring of their own
 //   warps 2..9  : two groups of four (one warp per lane quarter) taking
-//                 alternate 64-k sub-tiles: each thread widens its weight
-//                 row's 64 codes to 32 bf16 pairs and stores them to tensor
-//                 memory (tcgen05.st); warps 2..5 then run the epilogue,
-//                 which adds the eight accumulators in a fixed order
+//                 alternate 64-k sub-tiles of each stage: each thread loads
+//                 its weight row's codes of the stage into registers and
+//                 releases the weight slot at once (the weight stream never
+//                 waits for the tensor cores), then widens the codes to bf16
+//                 pairs and stores them to tensor memory (tcgen05.st), a
+//                 6-deep ring of A sub-tiles; warps 2..5 then run the
+//                 epilogue, which adds the accumulators in a fixed order
+//   warps 1, 11..13: warp 1 allocates tensor memory (256 columns: four
+//                 accumulators and the A ring); one thread of each warp
+//                 issues the MMAs of every fourth sub-tile (A from tensor
+//                 memory, B = the token slice from shared memory, K = 16 per
+//                 instruction) into its own accumulator, and frees A slots
+//                 and token slots by tcgen05.commit. A single thread's stream
+//                 of these short instructions is slow once commits are
+//                 interleaved (about 200 ns per instruction, measured on
+//                 B200); the streams of different warps overlap.
 // Each CTA starts its k loop at a different k-block: all CTAs read the same
 // token slices, which would otherwise be requested by every CTA at once.
 // Every barrier wait is bounded: a wait that gives up records
@@ -60,8 +63,9 @@ namespace sqk {
 constexpr int kWoTokens = 16;                 // token columns (N of the instruction)
 constexpr int kWoConvWarps = 8;               // two groups of four, alternating sub-tiles
 constexpr int kWoIssuers = 4;                 // MMA-issuing threads, one accumulator each
-constexpr int kWoMmaWarpB = 2 + kWoConvWarps;  // warps of issuers 1.. (issuer 0 is warp 1)
-constexpr int kWoThreads = 32 * (2 + kWoConvWarps + kWoIssuers - 1);
+constexpr int kWoXWarp = 2 + kWoConvWarps;     // the token-slice producer
+constexpr int kWoMmaWarpB = kWoXWarp + 1;      // warps of issuers 1.. (issuer 0 is warp 1)
+constexpr int kWoThreads = 32 * (kWoMmaWarpB + kWoIssuers - 1);
 constexpr uint32_t kWoWBytes = 128 * 128;     // packed weight slice of one stage
 constexpr uint32_t kWoXSub = kWoTokens * 128; // bf16 token sub-tile [16 x 64 k]
 constexpr uint32_t kWoTmemCols = 256;         // per CTA: accumulators + A ring
@@ -69,19 +73,28 @@ constexpr int kWoNAcc = kWoIssuers;           // accumulators (16 columns each)
 constexpr uint32_t kWoAColBase = kWoNAcc * 16;  // first A column
 constexpr int kWoNA = 6;                      // A sub-tiles in tensor memory (32 columns each)
 
+// Two rings: packed weight slices (released by the widening warps as soon as
+// they hold their codes in registers) and the matching token slices (released
+// by the MMAs that read them), so the weight stream does not wait for the
+// tensor cores.
 template <int BITS>
 struct WoCfg {
-  static constexpr int KS = BITS == 8 ? 128 : 256;   // k per stage
+  static constexpr int KS = BITS == 8 ? 128 : 256;   // k per weight stage (128 B per row)
   static constexpr int SUBS = KS / 64;               // 64-k sub-tiles per stage
-  static constexpr int STAGES = BITS == 8 ? 5 : 4;   // packed-weight ring
+  static constexpr int SW = 5;                       // weight ring
+  static constexpr int SX = BITS == 8 ? 7 : 3;       // token ring
   static constexpr uint32_t kXBytes = SUBS * kWoXSub;
-  static constexpr uint32_t kStageBytes = kWoWBytes + kXBytes;
-  static constexpr uint32_t kBarOff = STAGES * kStageBytes;
-  // barriers: full[S], empty[S], afull[NA], aempty[NA], tfull, drain
-  static constexpr uint32_t kMiscOff = kBarOff + (2 * STAGES + 2 * kWoNA + 2) * 8;
+  static constexpr uint32_t kXOff = SW * kWoWBytes;
+  static constexpr uint32_t kBarOff = kXOff + SX * kXBytes;
+  // barriers: wfull[SW], wempty[SW], xfull[SX], xempty[SX], afull[NA],
+  // aempty[NA], tfull, drain; then the TMEM slot and the abort flag
+  static constexpr uint32_t kMiscOff = kBarOff + (2 * SW + 2 * SX + 2 * kWoNA + 2) * 8;
   static constexpr uint32_t kDynamic = kMiscOff + 16 + 1024;  // slack for 1024-B alignment
-  static_assert(kStageBytes % 1024 == 0, "stages must keep 1024-byte alignment");
+  static_assert(kWoWBytes % 1024 == 0 && kXBytes % 1024 == 0,
+                "ring slots must keep 1024-byte alignment");
   static_assert(2 * (kDynamic + 1024) <= 233472, "two CTAs per SM must fit");
+  static_assert(SUBS % 2 == 0 && kWoNA % 2 == 0,
+                "each A slot must be filled by one widening group only");
 };
 static_assert(kWoAColBase + kWoNA * 32 <= kWoTmemCols, "A ring must fit the allocation");
 static_assert(kWoNA >= kWoIssuers, "every issuer needs an A slot of its own in flight");
@@ -129,17 +142,22 @@ __device__ __forceinline__ uint32_t bf16x2_sub(uint32_t a, uint32_t b) {
   return r;
 }
 
-// Widening of codes to bf16 without a conversion instruction. A code c with
-// |c| < 2^(B-1) is split into its low bits v and its sign bit s (two's
-// complement: c = v - s * 2^(B-1)). The bf16 with bits 0x4300 | v is 128 + v
-// (exponent 2^7, one unit per mantissa step) and 0x4300 | (sign bit in place)
-// is 128 + s * 2^(B-1); their bf16 difference is c exactly. Two codes at bit
+// Widening of 8-bit codes to bf16 without a conversion instruction. A code c
+// is split into its low seven bits v and its sign bit s (two's complement:
+// c = v - 128 s). The bf16 with bits 0x4300 | v is 128 + v (exponent 2^7,
+// one unit per mantissa step) and 0x4300 | (sign bit in place) is
+// 128 + 128 s; their bf16 difference is c exactly. Two codes at bit
 // 0 and bit 16 of a word give two bf16 at once (the low half is the first).
-template <int B>
 __device__ __forceinline__ uint32_t codes_to_bf16x2(uint32_t w) {
-  constexpr uint32_t kLow = B == 8 ? 0x007F007Fu : 0x00070007u;
-  constexpr uint32_t kSign = B == 8 ? 0x00800080u : 0x00080008u;
-  return bf16x2_sub((w & kLow) | 0x43004300u, (w & kSign) | 0x43004300u);
+  return bf16x2_sub((w & 0x007F007Fu) | 0x43004300u, (w & 0x00800080u) | 0x43004300u);
+}
+
+// The same for 4-bit codes in one logic operation: a code c in [-8, 7] is
+// the nibble n = c mod 16, and n ^ 8 = c + 8. (w & 0x000F000F) ^ 0x43084308
+// keeps bits 0-2 of each nibble, inverts bit 3 and sets the bits of 0x4300,
+// giving the bf16 128 + (c + 8); subtracting 136 leaves c exactly.
+__device__ __forceinline__ uint32_t nibbles_to_bf16x2(uint32_t w) {
+  return bf16x2_sub((w & 0x000F000Fu) ^ 0x43084308u, 0x43084308u);
 }
 
 __device__ __forceinline__ uint32_t sw128_off(uint32_t row, uint32_t chunk) {
@@ -165,14 +183,16 @@ __global__ void __launch_bounds__(kWoThreads, 2)
                       const uint16_t* __restrict__ bias, void* __restrict__ y, int M, int N,
                       int K, int* status) {
   using C = WoCfg<BITS>;
-  constexpr int S = C::STAGES, NA = kWoNA, SUBS = C::SUBS;
+  constexpr int SW = C::SW, SX = C::SX, NA = kWoNA, SUBS = C::SUBS;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const uint32_t s_base = smem_u32(smem);
-  const uint32_t bar_full = s_base + C::kBarOff;
-  const uint32_t bar_empty = bar_full + S * 8;
-  const uint32_t bar_afull = bar_empty + S * 8;
+  const uint32_t bar_wfull = s_base + C::kBarOff;
+  const uint32_t bar_wempty = bar_wfull + SW * 8;
+  const uint32_t bar_xfull = bar_wempty + SW * 8;
+  const uint32_t bar_xempty = bar_xfull + SX * 8;
+  const uint32_t bar_afull = bar_xempty + SX * 8;
   const uint32_t bar_aempty = bar_afull + NA * 8;
   const uint32_t bar_tfull = bar_aempty + NA * 8;
   const uint32_t bar_drain = bar_tfull + 8;
@@ -189,10 +209,13 @@ __global__ void __launch_bounds__(kWoThreads, 2)
   const int n_active = n_sub < kWoIssuers ? n_sub : kWoIssuers;  // issuers with sub-tiles
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < S; ++i) {
-      mbar_init(bar_full + 8 * i, 1);
-      // every widening warp + the issuers with a sub-tile in the stage
-      mbar_init(bar_empty + 8 * i, kWoConvWarps + kStageIssuers);
+    for (int i = 0; i < SW; ++i) {
+      mbar_init(bar_wfull + 8 * i, 1);
+      mbar_init(bar_wempty + 8 * i, kWoConvWarps);    // every widening warp
+    }
+    for (int i = 0; i < SX; ++i) {
+      mbar_init(bar_xfull + 8 * i, 1);
+      mbar_init(bar_xempty + 8 * i, kStageIssuers);   // the issuers with a sub-tile in it
     }
     for (int i = 0; i < NA; ++i) {
       mbar_init(bar_afull + 8 * i, 4);                 // the four warps of one group
@@ -228,38 +251,47 @@ __global__ void __launch_bounds__(kWoThreads, 2)
     *abort_flag = 1;
   };
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer --
+  if (warp == 0 || warp == kWoXWarp) {
+    // ----------------------------------------------------------- producers --
+    // warp 0 streams the packed weights, the token-slice warp the matching
+    // bf16 token slices; each is the only writer of its ring
     if (lane == 0) {
+      const bool is_w = warp == 0;
+      const int ns = is_w ? SW : SX;
+      const uint32_t full = is_w ? bar_wfull : bar_xfull;
+      const uint32_t empty = is_w ? bar_wempty : bar_xempty;
       int issued = 0;
 #pragma unroll 1
       for (int kb = 0; kb < nk; ++kb) {
-        const uint32_t st = uint32_t(kb % S), ph = uint32_t(kb / S) & 1u;
-        if (*abort_flag || !mbar_wait(bar_empty + 8 * st, ph ^ 1u)) {
+        const uint32_t st = uint32_t(kb % ns), ph = uint32_t(kb / ns) & 1u;
+        if (*abort_flag || !mbar_wait(empty + 8 * st, ph ^ 1u)) {
           give_up();
           break;
         }
-        const uint32_t dst = s_base + st * C::kStageBytes;
         const int kbe = kb + kb_rot < nk ? kb + kb_rot : kb + kb_rot - nk;
-        mbar_arrive_expect_tx(bar_full + 8 * st, C::kStageBytes);
-        tma_load_2d(dst, &tm_w, bar_full + 8 * st, kbe * 128, n0);
+        if (is_w) {
+          mbar_arrive_expect_tx(full + 8 * st, kWoWBytes);
+          tma_load_2d(s_base + st * kWoWBytes, &tm_w, full + 8 * st, kbe * 128, n0);
+        } else {
+          const uint32_t dst = s_base + C::kXOff + st * C::kXBytes;
+          mbar_arrive_expect_tx(full + 8 * st, C::kXBytes);
 #pragma unroll
-        for (int t = 0; t < SUBS; ++t)
-          tma_load_2d(dst + kWoWBytes + t * kWoXSub, &tm_x, bar_full + 8 * st,
-                      kbe * C::KS + t * 64, m0);
+          for (int t = 0; t < SUBS; ++t)
+            tma_load_2d(dst + t * kWoXSub, &tm_x, full + 8 * st, kbe * C::KS + t * 64, m0);
+        }
         ++issued;
       }
       // no copy may still be writing shared memory when the CTA exits
-      const int first = issued > S ? issued - S : 0;
+      const int first = issued > ns ? issued - ns : 0;
 #pragma unroll 1
       for (int j = first; j < issued; ++j)
-        (void)mbar_wait(bar_full + 8 * uint32_t(j % S), uint32_t(j / S) & 1u);
+        (void)mbar_wait(full + 8 * uint32_t(j % ns), uint32_t(j / ns) & 1u);
     }
   } else if (warp == 1 || warp >= kWoMmaWarpB) {
     // ----------------------------------------------------------------- MMA --
     // Four issuing threads, issuer q taking the sub-tiles ia = q (mod 4),
-    // each into its own accumulator: a single thread's tcgen05.mma stream is
-    // slow for these short instructions once commits are interleaved, while
+    // each into its own accumulator: a single thread's stream of these short
+    // tcgen05.mma instructions is slow once commits are interleaved, while
     // the streams of different warps overlap.
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(128, kWoTokens);
@@ -273,23 +305,23 @@ __global__ void __launch_bounds__(kWoThreads, 2)
         const uint32_t ia0 = uint32_t(kb) * SUBS;
         const uint32_t t0 = (q + kWoIssuers - ia0 % kWoIssuers) % kWoIssuers;
         if (t0 >= uint32_t(SUBS)) continue;
-        const uint32_t st = uint32_t(kb % S), ph = uint32_t(kb / S) & 1u;
-        // The issuers of a stage change from one use of it to the next, so
-        // the previous use may be other threads': wait for its release (the
-        // phase the producer waits for before refilling) first. Then the
-        // full barrier cannot be two phases behind this wait, where its
+        const uint32_t xs = uint32_t(kb % SX), ph = uint32_t(kb / SX) & 1u;
+        // The issuers of a token slot change from one use of it to the next,
+        // so the previous use may be other threads': wait for its release
+        // (the phase the producer waits for before refilling) first. Then
+        // the full barrier cannot be two phases behind this wait, where its
         // parity would match a completed phase.
-        if (kb >= S && (*abort_flag || !mbar_wait(bar_empty + 8 * st, ph ^ 1u))) {
+        if (kb >= SX && (*abort_flag || !mbar_wait(bar_xempty + 8 * xs, ph ^ 1u))) {
           give_up();
           ok = false;
           break;
         }
-        if (*abort_flag || !mbar_wait(bar_full + 8 * st, ph)) {
+        if (*abort_flag || !mbar_wait(bar_xfull + 8 * xs, ph)) {
           give_up();
           ok = false;
           break;
         }
-        const uint32_t x_addr = s_base + st * C::kStageBytes + kWoWBytes;
+        const uint32_t x_addr = s_base + C::kXOff + xs * C::kXBytes;
 #pragma unroll 1
         for (uint32_t t = t0; t < uint32_t(SUBS); t += kWoIssuers) {
           const uint32_t ia = ia0 + t;
@@ -317,7 +349,7 @@ __global__ void __launch_bounds__(kWoThreads, 2)
           tc_commit(bar_aempty + 8 * slot);
         }
         if (!ok) break;
-        tc_commit(bar_empty + 8 * st);  // this thread is done with the stage's token slices
+        tc_commit(bar_xempty + 8 * xs);  // this thread is done with the slot's token slices
       }
       if (ok && q < uint32_t(n_active)) tc_commit(bar_tfull);
       // every MMA issued has finished before tensor memory can be freed
@@ -328,57 +360,69 @@ __global__ void __launch_bounds__(kWoThreads, 2)
     // ------------------------------------------- widening, then epilogue --
     const int cw = warp - 2;                   // 0 .. kWoConvWarps - 1
     const int quarter = warp & 3;              // TMEM lane quarter this warp may access
-    const int group = cw >> 2;                 // sub-tiles ia with ia % 2 == group
+    const int group = cw >> 2;                 // sub-tiles t of a stage with t % 2 == group
     const uint32_t row = uint32_t(quarter) * 32u + uint32_t(lane);  // weight row of the tile
     const uint32_t lane_off = uint32_t(quarter * 32) << 16;
-    uint32_t ia = 0;
+    constexpr int kChunks = BITS == 8 ? 4 : 2;  // 16-byte chunks of a row per sub-tile
+    constexpr int kMySubs = SUBS / 2;           // this group's sub-tiles per stage
     bool ok = true;
 #pragma unroll 1
     for (int kb = 0; kb < nk && ok; ++kb) {
-      const uint32_t st = uint32_t(kb % S), ph = uint32_t(kb / S) & 1u;
-      if (*abort_flag || !mbar_wait(bar_full + 8 * st, ph)) {
+      const uint32_t st = uint32_t(kb % SW), ph = uint32_t(kb / SW) & 1u;
+      if (*abort_flag || !mbar_wait(bar_wfull + 8 * st, ph)) {
         give_up();
         ok = false;
         break;
       }
-      const uint8_t* wsrc = smem + st * C::kStageBytes;
-#pragma unroll 1
-      for (int t = 0; t < SUBS; ++t, ++ia) {
-        if (int(ia & 1u) != group) continue;
-        const uint32_t slot = ia % NA;
+      // this thread's codes of the stage into registers, then the weight
+      // slot is released: the producer refills it while the codes are widened
+      uint4 raw[kMySubs * kChunks];
+      const uint8_t* wsrc = smem + st * kWoWBytes;
+#pragma unroll
+      for (int u = 0; u < kMySubs; ++u)
+#pragma unroll
+        for (int h = 0; h < kChunks; ++h)
+          raw[u * kChunks + h] = *reinterpret_cast<const uint4*>(
+              wsrc + sw128_off(row, uint32_t(kChunks * (2 * u + group) + h)));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_wempty + 8 * st);
+#pragma unroll
+      for (int u = 0; u < kMySubs; ++u) {
+        const uint32_t ia = uint32_t(kb) * SUBS + uint32_t(2 * u + group);
+        const uint32_t slot = ia % NA;  // slots of one parity belong to one group
         if (*abort_flag || !mbar_wait(bar_aempty + 8 * slot, ((ia / NA) & 1u) ^ 1u)) {
           give_up();
           ok = false;
           break;
         }
         tc_fence_after();
-        // this row's 64 codes of sub-tile t -> 32 bf16 pairs (k order)
+        // this row's 64 codes of the sub-tile -> 32 bf16 pairs (k order)
         uint32_t a[32];
         if constexpr (BITS == 8) {
-          // source chunks 4t .. 4t+3 of the row, 16 codes each
 #pragma unroll
           for (int h = 0; h < 4; ++h) {
-            const uint4 q = *reinterpret_cast<const uint4*>(wsrc + sw128_off(row, uint32_t(4 * t + h)));
+            const uint4 q = raw[u * kChunks + h];
             const uint32_t qw[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               // bytes (c0 c1 c2 c3) -> (c0 c2 c1 c3): c0, c1 at bits 0 / 16
               const uint32_t p = __byte_perm(qw[i], 0u, 0x3120);
-              a[8 * h + 2 * i] = codes_to_bf16x2<8>(p);
-              a[8 * h + 2 * i + 1] = codes_to_bf16x2<8>(p >> 8);
+              a[8 * h + 2 * i] = codes_to_bf16x2(p);
+              a[8 * h + 2 * i + 1] = codes_to_bf16x2(p >> 8);
             }
           }
         } else {
-          // source chunks 2t, 2t+1 of the row, 32 codes each; each 32-bit
-          // word holds 8 codes: even k at bits 0,4,8,12, odd k at 16,20,24,28
+          // each 32-bit word holds 8 codes: even k at bits 0,4,8,12, odd k
+          // at 16,20,24,28
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            const uint4 q = *reinterpret_cast<const uint4*>(wsrc + sw128_off(row, uint32_t(2 * t + h)));
+            const uint4 q = raw[u * kChunks + h];
             const uint32_t qw[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
 #pragma unroll
-              for (int j = 0; j < 4; ++j) a[16 * h + 4 * i + j] = codes_to_bf16x2<4>(qw[i] >> (4 * j));
+              for (int jj = 0; jj < 4; ++jj)
+                a[16 * h + 4 * i + jj] = nibbles_to_bf16x2(qw[i] >> (4 * jj));
             }
           }
         }
@@ -388,9 +432,6 @@ __global__ void __launch_bounds__(kWoThreads, 2)
         __syncwarp();
         if (lane == 0) mbar_arrive(bar_afull + 8 * slot);
       }
-      if (!ok) break;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar_empty + 8 * st);  // this warp is done with the stage
     }
     if (cw < 4) {
       // epilogue: warp w reads TMEM lanes 32*(w%4) .. +31 = output channels
