@@ -79,11 +79,15 @@ PROFILED_TRAFFIC = {
     ("gemm", "mlp_up_4096x4096x14336"): (75.995904e6 + 83.197696e6, "abc2533ea4ecf75c"),
     ("gemm", "fp8_down_4096x14336x4096"): (258.165504e6 + 42.465280e6, "abc2533ea4ecf75c"),
     ("gemm", "fp8_tensor_4096x4096x14336"): (75.910400e6 + 82.917888e6, "abc2533ea4ecf75c"),
-    ("gemm_small", "prefill_512x4096x4096"): (18.910720e6 + 0.0, "6c9622eca20eceb1"),
+    ("gemm_small", "prefill_512x4096x4096"): (18.910720e6 + 0.0, "7eda12a8fa5cadb4"),
+    ("gemm_skinny", "decode_16x8192x28672"): (235.149568e6 + 4.384256e6, "30641829128746f8"),
+    ("gemm_wonly", "decode_w8a16_16x8192x28672"): (237.113344e6 + 3.692288e6, "c6b07cfabb7fec57"),
+    ("gemm_wonly", "decode_w4a16_16x8192x28672"): (119.396608e6 + 3.782912e6, "c6b07cfabb7fec57"),
     ("quant", "mlp_up_4096x4096x14336"): (33.647872e6 + 0.004352e6, "e5dd1a242fc0384b"),
     ("quant", "fp8_down_4096x14336x4096"): (117.741312e6 + 30.062080e6, "e5dd1a242fc0384b"),
     ("quant", "fp8_tensor_4096x4096x14336"): (33.577984e6 + 0.005632e6, "e5dd1a242fc0384b"),
     ("quant", "prefill_512x4096x4096"): (4.287744e6 + 0.0, "e5dd1a242fc0384b"),
+    ("quant", "decode_16x8192x28672"): (0.362240e6 + 0.0, "e5dd1a242fc0384b"),
 }
 KERNEL_SOURCES = {"gemm": ("sq_gemm.cu", "sq_common.cuh"),
                   "gemm_wonly": ("sq_gemm_wonly.cu", "sq_common.cuh"),

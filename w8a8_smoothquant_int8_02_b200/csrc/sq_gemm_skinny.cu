@@ -16,21 +16,23 @@
 // tensor-core instruction and the (up to) 16 token rows of Xq the N = 16
 // operand, so the accumulator holds D[n][m] = acc[m][n] in 128 lanes x 16
 // columns of tensor memory. One CTA per 128 output channels streams its
-// weight rows over all of K through a 6-stage ring of 16 KB weight slices
-// (+ 2 KB of token codes); two CTAs fit on an SM, so 224 CTAs at N = 28672
-// cover every SM with no split of K and no workspace.
-//   warp 0    : TMA producer (Wq slice [128 rows x 128 B] + Xq slice
-//               [16 rows x 128 B], 128-byte swizzle; token rows beyond M read
-//               as zero)
-//   warps 1, 6-8: warp 1 allocates 128 tensor-memory columns (eight
-//               accumulators of 16 columns); one thread of each warp issues
-//               the MMAs of every fourth k-block (K = 32 per instruction)
+// weight rows over all of K through a 3-stage ring; each stage holds 256
+// contiguous bytes of K from each of the 128 weight rows (two 128-byte TMA
+// boxes: 32 KB) and the matching token codes (4 KB). Two CTAs fit on an SM,
+// so 224 CTAs at N = 28672 cover every SM with no split of K and no
+// workspace. Reading 256 rather than 128 bytes of each row per stage cut the
+// time by about 6 % (fewer, longer DRAM bursts per row).
+//   warp 0    : TMA producer (Wq [128 rows x 2 x 128 B] + Xq [16 rows x
+//               2 x 128 B], 128-byte swizzle; token rows beyond M and k
+//               beyond K read as zero)
+//   warps 1, 6: warp 1 allocates 64 tensor-memory columns (four accumulators
+//               of 16 columns); one thread of each warp issues the MMAs of
+//               alternate stages (K = 32 per instruction, eight per stage)
 //               into its own two accumulators in turn, and frees ring slots
-//               with tcgen05.commit. An MMA of 128 x 16 x 32 is short, and a
-//               single thread's stream of them is slow once commits are
-//               interleaved (on the order of a hundred nanoseconds or more
-//               per instruction, measured on B200), while the streams of
-//               different warps overlap: four issuers keep up with HBM.
+//               with tcgen05.commit. A single thread's stream of these short
+//               MMAs is slow once commits are interleaved (about 200 ns per
+//               instruction, measured on B200); the streams of different
+//               warps overlap.
 //   warps 2-5 : epilogue -- warp w reads lanes 32*(w%4)..+31 (its output
 //               channels) x 16 columns (the tokens) of each accumulator, adds
 //               them (int32, exact; E4M3 binary32 in a fixed order),
@@ -50,14 +52,15 @@
 
 namespace sqk {
 
-constexpr int kSkBK = 128;       // bytes of K per stage
+constexpr int kSkBK = 128;       // bytes of K per TMA box (one 128-byte swizzle row)
+constexpr int kSkBoxes = 2;      // boxes per row per stage: 256 contiguous bytes of each weight row
 constexpr int kSkMP = 16;        // token columns (N of the instruction)
-constexpr int kSkStages = 6;
-constexpr int kSkIssuers = 4;    // MMA-issuing threads: warp 1, then warps 6 ..
+constexpr int kSkStages = 3;
+constexpr int kSkIssuers = 2;    // MMA-issuing threads: warps 1 and 6
 constexpr int kSkMmaWarpB = 6;   // warp of the second issuer
 constexpr int kSkThreads = 32 * (kSkMmaWarpB + kSkIssuers - 1);  // producer, MMA, 4 epilogue, MMA
-constexpr uint32_t kSkABytes = 128 * kSkBK;     // weight slice
-constexpr uint32_t kSkBBytes = kSkMP * kSkBK;   // token slice
+constexpr uint32_t kSkABytes = 128 * kSkBK * kSkBoxes;     // weight slice
+constexpr uint32_t kSkBBytes = kSkMP * kSkBK * kSkBoxes;   // token slice
 constexpr uint32_t kSkStageBytes = kSkABytes + kSkBBytes;
 constexpr uint32_t kSkBarOff = kSkStages * kSkStageBytes;
 // barriers: full[S], empty[S], tfull, drain; then the TMEM slot and abort flag
@@ -65,7 +68,13 @@ constexpr uint32_t kSkMiscOff = kSkBarOff + (2 * kSkStages + 2) * 8;
 constexpr uint32_t kSkDynamic = kSkMiscOff + 16 + 1024;  // slack for 1024-B alignment
 constexpr int kSkNAcc = 2 * kSkIssuers;                  // two accumulators per issuer
 constexpr uint32_t kSkTmemCols = kSkNAcc * 16;          // 16 columns each
+static_assert(kSkTmemCols >= 32 && (kSkTmemCols & (kSkTmemCols - 1)) == 0,
+              "tensor memory is allocated in powers of two of at least 32 columns");
 static_assert(kSkStageBytes % 1024 == 0, "stages must keep 1024-byte alignment");
+// an issuer waits for the release of a stage's previous use before waiting
+// for it to fill; that bounds the barrier to one phase behind only while the
+// issuer's own previous k-block (kb - kSkIssuers) is no older than that use
+static_assert(kSkStages >= kSkIssuers, "an issuer must not skip a whole ring of stages");
 static_assert(kSkDynamic * 2 + 2048 <= 233472, "two CTAs per SM must fit");
 
 // 32 lanes x 16 consecutive 32-bit columns of tensor memory -> registers,
@@ -100,7 +109,7 @@ __global__ void __launch_bounds__(kSkThreads, 2)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kSkMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kSkMiscOff + 4);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nk = (K + kSkBK - 1) / kSkBK;
+  const int nk = (K + kSkBK * kSkBoxes - 1) / (kSkBK * kSkBoxes);
   const int n_active = nk < kSkIssuers ? nk : kSkIssuers;  // issuers with k-blocks
 
   if (threadIdx.x == 0) {
@@ -148,8 +157,12 @@ __global__ void __launch_bounds__(kSkThreads, 2)
         const uint32_t dst = s_base + st * kSkStageBytes;
         const int kbe = kb + kb_rot < nk ? kb + kb_rot : kb + kb_rot - nk;
         mbar_arrive_expect_tx(bar_full + 8 * st, kSkStageBytes);
-        tma_load_2d(dst, &tm_w, bar_full + 8 * st, kbe * kSkBK, n0);
-        tma_load_2d(dst + kSkABytes, &tm_x, bar_full + 8 * st, kbe * kSkBK, 0);
+#pragma unroll
+        for (int b = 0; b < kSkBoxes; ++b) {
+          const int kx = (kbe * kSkBoxes + b) * kSkBK;
+          tma_load_2d(dst + b * 128 * kSkBK, &tm_w, bar_full + 8 * st, kx, n0);
+          tma_load_2d(dst + kSkABytes + b * kSkMP * kSkBK, &tm_x, bar_full + 8 * st, kx, 0);
+        }
         ++issued;
       }
       // no copy may still be writing shared memory when the CTA exits: wait
@@ -192,9 +205,9 @@ __global__ void __launch_bounds__(kSkThreads, 2)
         const uint32_t b_addr = a_addr + kSkABytes;
         // this thread's MMA j accumulates into accumulator 2 * q + j % 2
 #pragma unroll
-        for (int kk = 0; kk < kSkBK / 32; ++kk, ++j) {
-          const uint64_t ad = sw128_desc(a_addr + kk * 32);
-          const uint64_t bd = sw128_desc(b_addr + kk * 32);
+        for (int kk = 0; kk < kSkBoxes * kSkBK / 32; ++kk, ++j) {
+          const uint64_t ad = sw128_desc(a_addr + (kk / 4) * 128 * kSkBK + (kk % 4) * 32);
+          const uint64_t bd = sw128_desc(b_addr + (kk / 4) * kSkMP * kSkBK + (kk % 4) * 32);
           const uint32_t d = tmem_base + (2u * uint32_t(q) + j % 2u) * 16u;
           const uint32_t accum = j >= 2u ? 1u : 0u;
           if constexpr (E4M3) mma_f8(d, ad, bd, idesc, accum);

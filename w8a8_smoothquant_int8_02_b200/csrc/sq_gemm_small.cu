@@ -53,6 +53,10 @@ constexpr uint32_t kSmMiscOff = kSmBarOff + (2 * kSmStages + 2) * 8;
 constexpr uint32_t kSmDynamic = kSmMiscOff + 16 + 1024;   // slack for 1024-B alignment
 constexpr uint32_t kSmTmemCols = 512;                      // four 128-column accumulators
 static_assert(kSmStageBytes % 1024 == 0, "stages must keep 1024-byte alignment");
+// an issuer waits for the release of a stage's previous use before waiting
+// for it to fill; that bounds the barrier to one phase behind only while the
+// issuer's own previous k-block (kb - kSmIssuers) is no older than that use
+static_assert(kSmStages >= kSmIssuers, "an issuer must not skip a whole ring of stages");
 static_assert(kSmDynamic + 1024 > 233472 / 2, "one CTA per SM (it holds all tensor memory)");
 static_assert(kSmDynamic <= 232448, "shared memory budget exceeded");
 

@@ -95,6 +95,12 @@ struct WoCfg {
   static_assert(2 * (kDynamic + 1024) <= 233472, "two CTAs per SM must fit");
   static_assert(SUBS % 2 == 0 && kWoNA % 2 == 0,
                 "each A slot must be filled by one widening group only");
+  // an issuer's consecutive token stages are kWoIssuers / SUBS apart (1 when
+  // it has a sub-tile in every stage); the wait for the previous use of a
+  // slot bounds the barrier to one phase behind only if that gap is no
+  // larger than the ring
+  static_assert(SUBS >= kWoIssuers || kWoIssuers / SUBS <= SX,
+                "an issuer must not skip a whole ring of token stages");
 };
 static_assert(kWoAColBase + kWoNA * 32 <= kWoTmemCols, "A ring must fit the allocation");
 static_assert(kWoNA >= kWoIssuers, "every issuer needs an A slot of its own in flight");
