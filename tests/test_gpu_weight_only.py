@@ -36,7 +36,8 @@ def test_quantize_weight_int4(dtype, K, N):
 
 
 SHAPES = [(1, 8, 32), (5, 136, 1056), (16, 1000, 256), (16, 4096, 8192), (3, 28672, 256),
-          (17, 256, 512), (40, 384, 4096), (16, 128, 16384)]
+          (17, 256, 512), (40, 384, 4096), (16, 128, 16384), (16, 2048, 8192),
+          (9, 2056, 8256), (16, 28672, 1024)]   # 8256: a partial last stage
 
 
 @pytest.mark.parametrize("bits", [8, 4])
