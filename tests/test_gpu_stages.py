@@ -204,6 +204,47 @@ def test_gemm_every_tile_shape(tile, M, N, K, qtype, split, monkeypatch):
         np.testing.assert_array_equal(host(yb), oracle.f32_to_bf16(host(yf)))
 
 
+@pytest.mark.parametrize("M,N,K", [(512, 4096, 1024), (300, 1000, 1040), (129, 8192, 2048),
+                                   (1024, 2048, 1024)])
+@pytest.mark.parametrize("qtype", ["i8", "e4m3"])
+def test_gemm_one_wave(M, N, K, qtype):
+    """The one-wave GEMM (every 128 x 128 output tile on its own SM, four
+    MMA-issuing threads per tile, each with its own accumulator, added in a
+    fixed order): ragged M, N and K, full-range E4M3 codes."""
+    if qtype == "i8":
+        xq = synth.random_matrix((M, K), np.int8, seed=M * 7 + K)
+        wq = synth.random_matrix((N, K), np.int8, seed=N * 11 + K)
+    else:
+        g = np.random.default_rng(M + 2 * N + K)
+        xq = g.choice(E4M3_FINITE, size=(M, K)).astype(np.uint8)
+        wq = g.choice(E4M3_FINITE, size=(N, K)).astype(np.uint8)
+    sx = synth.random_floats(M, seed=61, lo=1e-6, hi=1e-3)
+    sw = synth.random_floats(N, seed=62, lo=1e-6, hi=1e-3)
+    bias = synth.to_bf16_bits(synth.random_floats(N, seed=63, std=0.1))
+    d = [dev(a) for a in (xq, sx, wq, sw)]
+    if qtype == "i8":
+        acc = torch.empty((M, N), dtype=torch.int32, device="cuda")
+        yf = ops.gemm_w8a8(*d, bias=dev(bias), out_dtype=torch.float32, acc=acc)
+        yb = ops.gemm_w8a8(*d, bias=dev(bias))
+    else:
+        yf = ops.gemm_fp8(*d, bias=dev(bias), out_dtype=torch.float32)
+        yb = ops.gemm_fp8(*d, bias=dev(bias))
+    assert ops.device_status() == ops.SQ_OK
+    if qtype == "i8":
+        acc_ref = oracle.gemm_i8(xq, wq)
+        yf_ref, yb_ref = oracle.epilogue(acc_ref, sx, sw, bias)
+        np.testing.assert_array_equal(host(acc), acc_ref)
+        np.testing.assert_array_equal(host(yf), yf_ref)
+        np.testing.assert_array_equal(host(yb), yb_ref)
+    else:
+        yf_ref, _ = oracle.epilogue(oracle.gemm_e4m3(xq, wq), sx, sw, bias)
+        rows, cols = np.divmod(np.arange(M * N, dtype=np.int64), N)
+        e = fp8_normalized_error(host(yf).reshape(-1), yf_ref.reshape(-1), xq, wq, sx, sw, bias,
+                                 rows, cols)
+        assert e.max() <= 1e-3, e.max()
+        np.testing.assert_array_equal(host(yb), oracle.f32_to_bf16(host(yf)))
+
+
 def test_split_tiles_leave_workspace_clean_and_match_whole_tiles(monkeypatch):
     """Stream-K split tiles give the same bits as whole tiles (INT8 partial
     sums are exact) and the workspace counters are zero again afterwards."""
