@@ -71,6 +71,8 @@ def _load():
             lib.sqo_quantize_weight.argtypes = [P, I, I64, I64, P, I, P, P]
             lib.sqo_quantize_act.argtypes = [P, I, I64, I64, P, I, P, P]
             lib.sqo_quantize_act_tensor.argtypes = [P, I, I64, I64, P, I, P, P, P, P]
+            lib.sqo_rmsnorm_quantize_act.argtypes = [P, I64, I64, P, ctypes.c_float, I, P, P,
+                                                     P, P]
             lib.sqo_gemm_i8.argtypes = [P, P, I64, I64, I64, P]
             lib.sqo_gemm_e4m3.argtypes = [P, P, I64, I64, I64, P]
             lib.sqo_dequant.argtypes = [ctypes.c_float, ctypes.c_float,
@@ -226,6 +228,26 @@ def quantize_act(x: np.ndarray, s, qtype: int = INT8):
     _load().sqo_quantize_act(_ptr(x), _dtype_code(x), M, K, _ptr(s), qtype,
                              _ptr(xq), _ptr(sx))
     return xq, sx
+
+
+def rmsnorm_quantize_act(x_bf16: np.ndarray, g, eps: float, qtype: int = INT8):
+    """The producer of X with the smoothing folded in: RMS normalization of
+    each row of x (bf16 bits [M,K]) with gain g [K] (= gamma / s), then
+    per-token quantization. The sum of squares is exact over the elements
+    whose bf16 exponent is within 48 of the row's largest (the rest are below
+    2^-94 of the largest square), rounded once to binary64; 1/sqrt(ss/K +
+    eps) in binary64 steps, rounded to binary32; xn = (x * r) * g in binary32.
+    Returns (xq [M,K] codes, sx [M], r [M] float32, xn [M,K] float32)."""
+    x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
+    M, K = x.shape
+    g = _c(g, np.float32)
+    xq = np.empty((M, K), np.uint8 if qtype == E4M3 else np.int8)
+    sx = np.empty(M, np.float32)
+    r = np.empty(M, np.float32)
+    xn = np.empty((M, K), np.float32)
+    _load().sqo_rmsnorm_quantize_act(_ptr(x), M, K, _ptr(g), float(eps), qtype, _ptr(xq),
+                                     _ptr(sx), _ptr(r), _ptr(xn))
+    return xq, sx, r, xn
 
 
 def quantize_act_tensor(x: np.ndarray, s, qtype: int = INT8, scale=None):

@@ -165,6 +165,85 @@ void sqo_fold_smoothing(const void* p, int dtype, int64_t rows, int64_t cols,
                                          per_column ? s[c] : s[r]);
 }
 
+/* ------------------------------------------------------------------------ */
+/* The producer of X with the smoothing folded in ([LES] §2: the transform   */
+/* is applied offline, no runtime overhead; [WAQ] §3 "Step 1": X~ = X        */
+/* diag(1/s) prepared before inference). The pages name no producer; the     */
+/* transformer models they quantize (Llama) feed each linear layer from an   */
+/* RMS normalization, so that is the producer taken: xn = x / rms(x) * g,    */
+/* g = gamma / s folded offline, then per-token quantization of xn.          */
+/* ------------------------------------------------------------------------ */
+
+/* bf16 magnitude bits h (sign cleared, h != 0) as N * 2^(e - 7): N = 1.f in
+ * 8 bits for normal numbers (128..255), 0.f for subnormals (1..127). */
+static void bf16_int_exp(uint16_t h, int* N, int* e) {
+    const int be = (h >> 7) & 0xFF, f = h & 0x7F;
+    if (be == 0) { *N = f; *e = -126; }
+    else { *N = 128 + f; *e = be - 127; }
+}
+
+/* one normalized element: the bf16 value times 1/rms, then times the gain,
+ * each product a rounded binary32 operation */
+static float rms_apply(uint16_t xk, float r, float gk) {
+    const float a = sqo_bf16_to_f32(xk) * r;
+    return a * gk;
+}
+
+void sqo_rmsnorm_quantize_act(const uint16_t* x, int64_t M, int64_t K, const float* g,
+                              float eps, int qtype, void* xq, float* sx, float* rinv,
+                              float* xn) {
+    const float qmax = (qtype == 1) ? 448.0f : 127.0f;
+    #pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m) {
+        const uint16_t* row = x + m * K;
+        /* the exact sum of squares: each x^2 = N^2 * 2^(2e - 14) is an
+         * integer multiple of 2^(2 e_max - 110) when e >= e_max - 48 */
+        int emax = -1000;
+        for (int64_t k = 0; k < K; ++k) {
+            const uint16_t h = row[k] & 0x7FFF;
+            if (h == 0) continue;
+            int N, e;
+            bf16_int_exp(h, &N, &e);
+            if (e > emax) emax = e;
+        }
+        unsigned __int128 S = 0;
+        if (emax > -1000) {
+            for (int64_t k = 0; k < K; ++k) {
+                const uint16_t h = row[k] & 0x7FFF;
+                if (h == 0) continue;
+                int N, e;
+                bf16_int_exp(h, &N, &e);
+                if (e < emax - 48) continue;
+                S += (unsigned __int128)(uint32_t)(N * N) << (2 * (e - emax) + 96);
+            }
+        }
+        const double ss = (emax > -1000) ? ldexp((double)S, 2 * emax - 110) : 0.0;
+        const double mean = ss / (double)K;
+        const double v = mean + (double)eps;
+        const double t = sqrt(v);
+        const float r = (float)(1.0 / t);
+        if (rinv) rinv[m] = r;
+        /* xn_k = (x_k * r) * g_k, then the row's scale and codes */
+        float amax = 0.0f;
+        for (int64_t k = 0; k < K; ++k) {
+            const float y = rms_apply(row[k], r, g[k]);
+            if (xn) xn[m * K + k] = y;
+            const float ay = fabsf(y);
+            if (ay > amax) amax = ay;
+        }
+        const float row_scale = amax / qmax;
+        sx[m] = row_scale;
+        for (int64_t k = 0; k < K; ++k) {
+            const float y = rms_apply(row[k], r, g[k]);
+            if (qtype == 1)
+                ((uint8_t*)xq)[m * K + k] =
+                    (row_scale == 0.0f) ? 0 : sqo_e4m3_encode_rn_sat(y / row_scale);
+            else
+                ((int8_t*)xq)[m * K + k] = (row_scale == 0.0f) ? 0 : quant_i8(y, row_scale);
+        }
+    }
+}
+
 int sqo_num_threads(void) {
 #ifdef _OPENMP
     return omp_get_max_threads();

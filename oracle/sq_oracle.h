@@ -129,6 +129,21 @@ void sqo_gemm_weight_only(const uint16_t* x, const void* wq, int bits, const flo
                           const uint16_t* bias, int64_t M, int64_t N, int64_t K,
                           double* y);
 
+/* RMS normalization of each row of x (bf16 bits [M,K]) with the per-channel
+ * gain g [K] (binary32; the smoothing factors folded in: g = gamma / s),
+ * fused with per-token quantization (qtype 0 INT8, 1 E4M3). Per row:
+ *   ss  = sum of x_k^2 over the k with e_k >= e_max - 48 (e: the bf16
+ *         exponent of x_k, e_max the largest in the row), exactly, then
+ *         rounded once to binary64;
+ *   r   = binary32( binary64( 1 / sqrt( ss / K + eps ) ) ), each binary64
+ *         operation rounded once (eps > 0, as binary64);
+ *   xn_k = (x_k * r) * g_k in binary32, each product rounded once;
+ *   then sqo_quantize_act of xn without smoothing.
+ * rinv [M] (r) and xn [M,K] are written when non-NULL. */
+void sqo_rmsnorm_quantize_act(const uint16_t* x, int64_t M, int64_t K, const float* g,
+                              float eps, int qtype, void* xq, float* sx, float* rinv,
+                              float* xn);
+
 /* Threads OpenMP will use (1 when built without OpenMP). */
 int sqo_num_threads(void);
 

@@ -152,6 +152,16 @@ MUTANTS = [
      "q = unpack_code((const uint8_t*)wq + n * (K / 2), k ^ 1);"),
     ("weight_only_wrong_channel_scale",
      "double w_deq = (double)q * (double)sw[n];", "double w_deq = (double)q * (double)sw[m % N];"),
+    ("rms_drops_eps", "const double v = mean + (double)eps;", "const double v = mean;"),
+    ("rms_divides_by_k_minus_one", "const double mean = ss / (double)K;",
+     "const double mean = ss / (double)(K - 1);"),
+    ("rms_square_window_off_by_one", "<< (2 * (e - emax) + 96);", "<< (2 * (e - emax) + 95);"),
+    ("rms_no_square_root", "const double t = sqrt(v);", "const double t = v;"),
+    ("rms_no_reciprocal", "const float r = (float)(1.0 / t);", "const float r = (float)t;"),
+    ("rms_gain_before_the_norm", "const float a = sqo_bf16_to_f32(xk) * r;\n    return a * gk;",
+     "const float a = sqo_bf16_to_f32(xk) * gk;\n    return a * r;"),
+    ("rms_binary32_root", "const float r = (float)(1.0 / t);",
+     "const float r = 1.0f / sqrtf((float)v);"),
 ]
 
 

@@ -746,3 +746,124 @@ def test_weight_only_on_integer_activations_is_the_int8_gemm_scaled():
     y = oracle.gemm_weight_only(synth.to_bf16_bits(xi.astype(np.float32)), wq, sw, None, 8)
     acc = oracle.gemm_i8(xi, wq).astype(np.float64)
     np.testing.assert_array_equal(y, acc * sw.astype(np.float64)[None, :])
+
+
+# ---------------------------------------------------------------------------
+# The producer of X with the smoothing folded in: RMS normalization, then
+# per-token quantization ("Weight-Activation Quantization" §3 "Step 1" and the
+# grasp.study lesson §2: the smoothing is applied offline, with no runtime
+# overhead). Pinned against exact rational arithmetic, closed forms, exact
+# scalings and the per-token quantization already pinned above.
+# ---------------------------------------------------------------------------
+
+def _rms_reference(xb, g, eps):
+    """r and xn from the definition, the sum of squares in exact rational
+    arithmetic (every element here is within 48 binades of the row's
+    largest), then the binary64 steps in Python floats (IEEE, rounded once
+    each) and the binary32 products in numpy float32."""
+    from fractions import Fraction
+    xf = oracle.bf16_to_f32_array(xb)
+    M, K = xb.shape
+    r = np.empty(M, np.float32)
+    for m in range(M):
+        ss = sum((Fraction(float(v)) ** 2 for v in xf[m]), Fraction(0))
+        mean = float(ss) / float(K)              # float(Fraction) is correctly rounded
+        t = math.sqrt(mean + float(np.float32(eps)))
+        r[m] = np.float32(1.0 / t)
+    xn = (xf * r[:, None]).astype(np.float32) * g.astype(np.float32)[None, :]
+    return r, xn.astype(np.float32)
+
+
+@pytest.mark.parametrize("K", [64, 384, 1024])
+def test_rmsnorm_matches_exact_rational_sum_of_squares(K):
+    x = synth.random_floats((6, K), seed=70 + K, std=1.0)
+    x[:, 5] *= 80.0                                    # an outlier channel
+    x[2] *= 1e-3                                       # a small row
+    xb = synth.to_bf16_bits(x)
+    g = synth.random_floats(K, seed=71, lo=0.25, hi=3.0)
+    for eps in (1e-6, 1e-2):
+        xq, sx, r, xn = oracle.rmsnorm_quantize_act(xb, g, eps)
+        r_ref, xn_ref = _rms_reference(xb, g, eps)
+        np.testing.assert_array_equal(r.view(np.uint32), r_ref.view(np.uint32))
+        np.testing.assert_array_equal(xn.view(np.uint32), xn_ref.view(np.uint32))
+        # then exactly the per-token quantization of xn, without smoothing
+        for qt in (oracle.INT8, oracle.E4M3):
+            q2, s2 = oracle.quantize_act(xn_ref, None, qt)
+            q1, s1, _, _ = oracle.rmsnorm_quantize_act(xb, g, eps, qt)
+            np.testing.assert_array_equal(q1.view(np.uint8), q2.view(np.uint8))
+            np.testing.assert_array_equal(s1, s2)
+
+
+def test_rmsnorm_single_value_closed_form():
+    """One nonzero x = 2 in a row of 64: mean square 4/64 = 1/16, 1/rms = 4,
+    so xn = 2 * 4 * g exactly (eps far below the binary64 resolution of 1/16)."""
+    K = 64
+    x = np.zeros((1, K), np.float32)
+    x[0, 9] = 2.0
+    g = synth.random_floats(K, seed=72, lo=0.5, hi=2.0)
+    xq, sx, r, xn = oracle.rmsnorm_quantize_act(synth.to_bf16_bits(x), g, 1e-38)
+    assert r[0] == np.float32(4.0)
+    expect = np.zeros(K, np.float32)
+    expect[9] = np.float32(8.0) * g[9]
+    np.testing.assert_array_equal(xn[0], expect)
+    assert xq[0, 9] == 127 and not xq[0, np.arange(K) != 9].any()
+
+
+def test_rmsnorm_is_exactly_homogeneous_under_powers_of_two():
+    """Scaling a row by 2^j (exact in bf16) scales 1/rms by 2^-j and leaves
+    xn and the codes bit for bit unchanged (eps negligible)."""
+    x = synth.random_floats((4, 256), seed=73, std=1.0)
+    g = synth.random_floats(256, seed=74, lo=0.5, hi=2.0)
+    q0, s0, r0, xn0 = oracle.rmsnorm_quantize_act(synth.to_bf16_bits(x), g, 1e-38)
+    for j in (-9, 7):
+        q1, s1, r1, xn1 = oracle.rmsnorm_quantize_act(synth.to_bf16_bits(x * 2.0 ** j), g, 1e-38)
+        np.testing.assert_array_equal(r1, r0 * np.float32(2.0 ** -j))
+        np.testing.assert_array_equal(xn1, xn0)
+        np.testing.assert_array_equal(q1, q0)
+
+
+def test_rmsnorm_zero_row_and_eps():
+    """An all-zero row: 1/rms = 1/sqrt(eps) (binary64, then binary32), zero
+    codes and scale 0."""
+    x = np.zeros((2, 32), np.float32)
+    x[1, 3] = 1.0
+    eps = np.float32(1e-2)
+    xq, sx, r, xn = oracle.rmsnorm_quantize_act(synth.to_bf16_bits(x), np.ones(32, np.float32), eps)
+    assert r[0] == np.float32(1.0 / math.sqrt(float(eps)))
+    assert sx[0] == 0.0 and not xq[0].any()
+    assert r[1] == np.float32(1.0 / math.sqrt(1.0 / 32.0 + float(eps)))
+
+
+@pytest.mark.parametrize("qt", [oracle.INT8, oracle.E4M3])
+def test_rmsnorm_with_folded_gain_equals_smoothing_after_the_norm(qt):
+    """With power-of-two smoothing factors, the norm with the folded gain
+    gamma / s gives the codes and scales of the per-token quantization of the
+    norm's output (gain gamma) smoothed by s at run time: the fold moves the
+    division, exactly."""
+    K = 128
+    x = synth.random_floats((5, K), seed=75, std=1.0)
+    x[:, 17] *= 50.0
+    xb = synth.to_bf16_bits(x)
+    gamma = synth.random_floats(K, seed=76, lo=0.5, hi=2.0)
+    s = (2.0 ** np.random.default_rng(77).integers(-6, 7, K)).astype(np.float32)
+    g_folded = oracle.fold_smoothing(gamma, s)[0]
+    q1, s1, _, _ = oracle.rmsnorm_quantize_act(xb, g_folded, 1e-6, qt)
+    _, _, _, xn_gamma = oracle.rmsnorm_quantize_act(xb, gamma, 1e-6, qt)
+    q2, s2 = oracle.quantize_act(xn_gamma, s, qt)
+    np.testing.assert_array_equal(q1.view(np.uint8), q2.view(np.uint8))
+    np.testing.assert_array_equal(s1, s2)
+
+
+def test_rmsnorm_drops_only_terms_far_below_the_row_maximum():
+    """Elements more than 48 binades below the row's largest do not enter the
+    sum of squares (each is below 2^-94 of the largest square); elements
+    within that range do, exactly."""
+    K = 64
+    x = np.zeros((3, K), np.float32)
+    x[:, 0] = 2.0 ** 20
+    x[1, 1:] = 2.0 ** -40          # 60 binades below: dropped
+    x[2, 1:4] = 2.0 ** 10          # 10 binades below: kept
+    xq, sx, r, xn = oracle.rmsnorm_quantize_act(synth.to_bf16_bits(x), np.ones(K, np.float32), 1e-38)
+    assert r[1] == r[0]
+    ss = 2.0 ** 40 + 3 * 2.0 ** 20
+    assert r[2] == np.float32(1.0 / math.sqrt(ss / K))
