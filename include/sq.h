@@ -53,7 +53,7 @@
 extern "C" {
 #endif
 
-#define SQ_ABI_VERSION 6
+#define SQ_ABI_VERSION 7
 
 typedef enum {
     SQ_OK = 0,
@@ -227,6 +227,32 @@ sq_status sq_quantize_act_tensor(const void* x, sq_dtype xt, int64_t M, int64_t 
  */
 sq_status sq_fold_smoothing(const void* p, sq_dtype pt, int64_t rows, int64_t cols,
                             const float* s, sq_axis axis, float* out, void* stream);
+
+/*
+ * The producer of X with the smoothing folded in: RMS normalization fused with
+ * per-token quantization. Source: "Weight-Activation Quantization"
+ * (infra.bea.ai) §3 "Step 1" (X_tilde = X diag(1/s) prepared before
+ * inference) and the grasp.study lesson on W8A16 vs W8A8, §2 (the transform
+ * is applied offline, with no runtime overhead). The pages name no producer
+ * of X; the models they quantize feed each linear layer from an RMS
+ * normalization with a per-channel gain, and g = gamma / s (from
+ * sq_fold_smoothing) makes it emit X_tilde itself, so this call replaces the
+ * normalization and sq_quantize_act(.., s = NULL, ..) with one pass.
+ *   x   : [M,K] bf16, the normalization's input (16-byte aligned)
+ *   g   : [K] binary32 gain with 1/s folded in (16-byte aligned)
+ *   eps : > 0, finite
+ *   qt  : SQ_I8 or SQ_E4M3;  xq : [M,K] codes (16-byte aligned);  sx : [M]
+ * Per row: ss = the sum of x_k^2 over the k whose bf16 exponent is within 48
+ * of the row's largest, exactly, rounded once to binary64 (the others are
+ * below 2^-94 of the largest square); r = binary32(1 / sqrt(ss / K + eps))
+ * with each of the four binary64 operations rounded once; xn_k = (x_k * r) *
+ * g_k in binary32; then sx and the codes of xn exactly as sq_quantize_act
+ * with s = NULL. K a multiple of 8, at most 16384 (SQ_ERR_UNSUPPORTED
+ * beyond). xq and sx may overlap neither each other nor x or g
+ * (SQ_ERR_INVALID_ARG). M == 0 is a no-op that accepts NULL pointers.
+ */
+sq_status sq_rmsnorm_quantize_act(const void* x, const float* g, float eps, int64_t M,
+                                  int64_t K, sq_dtype qt, void* xq, float* sx, void* stream);
 
 /*
  * Size in bytes of the GEMM workspace for the current device (its SM count

@@ -53,7 +53,7 @@ def test_exported_symbols_are_visible_to_the_dynamic_linker():
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.sq_abi_version() == 6
+    assert lib.sq_abi_version() == 7
     for st in range(7):
         assert ops.status_string(st).startswith("SQ_")
     assert "TIMEOUT" in ops.status_string(ops.SQ_ERR_TIMEOUT)
@@ -252,3 +252,39 @@ def test_abi_from_plain_c(tmp_path):
     out = subprocess.run([str(exe)], capture_output=True, text=True)
     assert out.returncode == 0, out.stderr
     assert out.stdout.strip() == "ok"
+
+
+def test_rmsnorm_quantize_validation(lib):
+    f = lib.sq_rmsnorm_quantize_act
+    ok = dict(x=A, g=A + 0x100000, eps=1e-6, M=4, K=64, qt=ops.SQ_I8, xq=A + 0x200000,
+              sx=A + 0x300000)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return f(c(a["x"]), c(a["g"]), a["eps"], a["M"], a["K"], a["qt"], c(a["xq"]),
+                 c(a["sx"]), None)
+
+    assert call(x=NUL) == ops.SQ_ERR_INVALID_ARG
+    assert call(g=NUL) == ops.SQ_ERR_INVALID_ARG
+    assert call(xq=NUL) == ops.SQ_ERR_INVALID_ARG
+    assert call(sx=NUL) == ops.SQ_ERR_INVALID_ARG
+    assert call(qt=ops.SQ_BF16) == ops.SQ_ERR_INVALID_ARG
+    assert call(qt=ops.SQ_I4) == ops.SQ_ERR_INVALID_ARG
+    assert call(K=60) == ops.SQ_ERR_INVALID_ARG             # not a multiple of 8
+    assert call(K=0) == ops.SQ_ERR_INVALID_ARG
+    assert call(M=-1) == ops.SQ_ERR_INVALID_ARG
+    assert call(eps=0.0) == ops.SQ_ERR_INVALID_ARG
+    assert call(eps=-1e-6) == ops.SQ_ERR_INVALID_ARG
+    assert call(eps=float("inf")) == ops.SQ_ERR_INVALID_ARG
+    assert call(eps=float("nan")) == ops.SQ_ERR_INVALID_ARG
+    assert call(K=16384 + 8) == ops.SQ_ERR_UNSUPPORTED      # the row no longer fits on chip
+    assert call(xq=A) == ops.SQ_ERR_INVALID_ARG             # codes over the input
+    assert call(xq=A + 2 * 4 * 64 - 16) == ops.SQ_ERR_INVALID_ARG   # partial overlap
+    assert call(sx=A + 0x100000 + 16) == ops.SQ_ERR_INVALID_ARG     # scales over the gain
+    assert call(sx=A + 0x200000 + 64) == ops.SQ_ERR_INVALID_ARG     # scales over the codes
+    assert call(x=A + 8) == ops.SQ_ERR_MISALIGNED
+    assert call(g=A + 0x100000 + 4) == ops.SQ_ERR_MISALIGNED
+    assert call(xq=A + 0x200000 + 8) == ops.SQ_ERR_MISALIGNED
+    assert call(sx=A + 0x300000 + 2) == ops.SQ_ERR_MISALIGNED
+    # empty batch: a no-op that accepts NULL pointers
+    assert call(M=0, x=NUL, g=NUL, xq=NUL, sx=NUL) == ops.SQ_OK

@@ -1,0 +1,92 @@
+"""The producer of X with the smoothing folded in: RMS normalization fused with
+per-token quantization (sq_rmsnorm_quantize_act), against the CPU oracle.
+
+Bar: codes and per-token scales bit for bit ("Weight-Activation Quantization"
+§3 "Step 1" and the grasp.study lesson §2: the smoothing moves offline into
+the producer; the normalization's sum of squares is exact, so nothing is left
+to rounding order).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from w8a8_smoothquant_int8_02_b200 import ops, synth
+
+from _gpu_util import dev, host
+
+pytestmark = pytest.mark.gpu
+
+
+def _rows(M, K, seed):
+    x = synth.random_floats((M, K), seed=seed, std=1.0)
+    g = np.random.default_rng(seed)
+    if K > 16:
+        x[:, g.choice(K, size=max(1, K // 100), replace=False)] *= 60.0   # outlier channels
+    if M > 3:
+        x[1] = 0.0                                     # an all-zero row
+        x[2] *= 2.0 ** -120                            # bf16 subnormals and tiny normals
+        x[3, :] = 2.0 ** -60                           # far below the row's largest ...
+        x[3, 0] = 2.0 ** 20                            # ... so those squares drop out
+    if M > 5:
+        x[4] *= 2.0 ** 100                             # large magnitudes
+        x[5, ::7] = -0.0                               # signed zeros
+    return synth.to_bf16_bits(x)
+
+
+@pytest.mark.parametrize("M,K", [(1, 8), (7, 64), (37, 4096), (300, 1000), (64, 16384),
+                                 (2049, 512)])
+@pytest.mark.parametrize("qt", ["i8", "e4m3"])
+@pytest.mark.parametrize("eps", [1e-6, 1e-2])
+def test_rmsnorm_quantize_matches_oracle(M, K, qt, eps):
+    xb = _rows(M, K, seed=M + K)
+    gamma = synth.random_floats(K, seed=K, lo=0.3, hi=2.5)
+    gamma[::5] *= -1.0                                 # negative gains too
+    q_ref, s_ref, _, _ = oracle.rmsnorm_quantize_act(
+        xb, gamma, eps, oracle.INT8 if qt == "i8" else oracle.E4M3)
+    xq, sx = ops.rmsnorm_quantize_act(dev(xb), dev(gamma), eps, qt)
+    assert ops.device_status() == ops.SQ_OK
+    np.testing.assert_array_equal(host(sx), s_ref)
+    np.testing.assert_array_equal(host(xq).view(np.uint8), q_ref.view(np.uint8))
+
+
+@pytest.mark.parametrize("qt", ["i8", "e4m3"])
+def test_folded_producer_feeds_the_layer(qt):
+    """Offline: calibrate, smoothing factors, fold 1/s into the norm's gain (all
+    on the GPU); runtime: the fused norm + quantization, then the 8-bit GEMM --
+    codes, scales and the GEMM output equal the oracle's chain."""
+    M, K, N = 256, 1024, 512
+    xb = _rows(M, K, seed=91)
+    gamma = synth.random_floats(K, seed=92, lo=0.5, hi=2.0)
+    w = synth.random_floats((K, N), seed=93, std=0.02)
+    qcode = oracle.INT8 if qt == "i8" else oracle.E4M3
+    _, _, _, xn_cal = oracle.rmsnorm_quantize_act(xb, gamma, 1e-6)   # the norm's output
+    ax, aw = oracle.amax(xn_cal, True), oracle.amax(w, False)
+    s = oracle.smooth_factors(ax, aw, 0.5)
+    g_ref = oracle.fold_smoothing(gamma, s)[0]
+    wq_ref, sw_ref = oracle.quantize_weight(w, s, qcode)
+    q_ref, sx_ref, _, _ = oracle.rmsnorm_quantize_act(xb, g_ref, 1e-6, qcode)
+    g_d = ops.fold_smoothing(dev(gamma), dev(s))
+    np.testing.assert_array_equal(host(g_d), g_ref)
+    xq, sx = ops.rmsnorm_quantize_act(dev(xb), g_d, 1e-6, qt)
+    np.testing.assert_array_equal(host(sx), sx_ref)
+    np.testing.assert_array_equal(host(xq).view(np.uint8), q_ref.view(np.uint8))
+    if qt == "i8":
+        y = ops.gemm_w8a8(xq, sx, dev(wq_ref), dev(sw_ref), out_dtype=torch.float32)
+        y_ref, _ = oracle.epilogue(oracle.gemm_i8(q_ref, wq_ref), sx_ref, sw_ref, None)
+        np.testing.assert_array_equal(host(y), y_ref)
+    assert ops.device_status() == ops.SQ_OK
+
+
+def test_rmsnorm_quantize_validation():
+    x = torch.zeros((4, 64), dtype=torch.bfloat16, device="cuda")
+    g = torch.ones(64, dtype=torch.float32, device="cuda")
+    with pytest.raises(ops.SQError):
+        ops.rmsnorm_quantize_act(x, g, 0.0)                      # eps must be > 0
+    with pytest.raises(ops.SQError):
+        ops.rmsnorm_quantize_act(x[:, :60].contiguous(), g[:60].contiguous(), 1e-6)  # K % 8
+    big = torch.zeros((1, 16392), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(ops.SQError):
+        ops.rmsnorm_quantize_act(big, torch.ones(16392, device="cuda"), 1e-6)   # K > 16384
+    xq, sx = ops.rmsnorm_quantize_act(x[:0], g, 1e-6)             # empty batch
+    assert xq.shape == (0, 64) and sx.shape == (0,)

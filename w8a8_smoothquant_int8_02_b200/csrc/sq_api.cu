@@ -3,6 +3,7 @@
 // Argument validation happens here, synchronously, before anything is
 // launched; the launchers in sq_quant.cu / sq_gemm.cu assume valid input.
 #include <atomic>
+#include <cmath>
 #include <cstdint>
 #include <cuda_runtime.h>
 
@@ -47,6 +48,11 @@ __global__ void probe_wait_kernel(int64_t timeout_ns, int* status) {
 }
 
 inline bool al(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+// Byte ranges [a, a+na) and [b, b+nb) share an address.
+inline bool overlap(const void* a, uint64_t na, const void* b, uint64_t nb) {
+  const uintptr_t pa = reinterpret_cast<uintptr_t>(a), pb = reinterpret_cast<uintptr_t>(b);
+  return pa < pb + nb && pb < pa + na;
+}
 inline cudaStream_t S(void* st) { return static_cast<cudaStream_t>(st); }
 inline sq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? SQ_OK : SQ_ERR_CUDA; }
 
@@ -327,6 +333,25 @@ sq_status sq_gemm_weight_only(const void* x, const void* wq, sq_dtype wqt, const
   return from_cuda(sqh::launch_gemm_weight_only(
       wqt == SQ_I4 ? 4 : 8, static_cast<const uint16_t*>(x), wq, sw, bias, M, N, K, y,
       yt == SQ_BF16 ? sqh::OutKind::BF16 : sqh::OutKind::F32, S(stream)));
+}
+
+sq_status sq_rmsnorm_quantize_act(const void* x, const float* g, float eps, int64_t M,
+                                  int64_t K, sq_dtype qt, void* xq, float* sx, void* stream) {
+  if (qt != SQ_I8 && qt != SQ_E4M3) return SQ_ERR_INVALID_ARG;
+  if (M < 0 || K <= 0 || K % 8 != 0 || M > INT32_MAX) return SQ_ERR_INVALID_ARG;
+  if (!(eps > 0.0f) || !std::isfinite(eps)) return SQ_ERR_INVALID_ARG;
+  if (K > sqh::rmsnorm_quant_max_k()) return SQ_ERR_UNSUPPORTED;
+  if (M == 0) return SQ_OK;  // empty batch: pointers may be NULL
+  if (!x || !g || !xq || !sx) return SQ_ERR_INVALID_ARG;
+  // Other rows' CTAs may still be reading x while this one writes: no output may alias an input.
+  const uint64_t xb = uint64_t(M) * uint64_t(K) * 2, qb = uint64_t(M) * uint64_t(K);
+  if (overlap(xq, qb, x, xb) || overlap(xq, qb, g, uint64_t(K) * 4) ||
+      overlap(sx, uint64_t(M) * 4, x, xb) || overlap(sx, uint64_t(M) * 4, g, uint64_t(K) * 4) ||
+      overlap(sx, uint64_t(M) * 4, xq, qb))
+    return SQ_ERR_INVALID_ARG;
+  if (!al(x, 16) || !al(g, 16) || !al(xq, 16) || !al(sx, 4)) return SQ_ERR_MISALIGNED;
+  return from_cuda(sqh::launch_rmsnorm_quant(static_cast<const uint16_t*>(x), g, eps, M, K,
+                                             qt == SQ_E4M3, xq, sx, S(stream)));
 }
 
 sq_status sq_selftest_fast_division(int64_t* mismatches, void* stream) {

@@ -29,6 +29,11 @@ cudaError_t launch_quantize_act_tensor(const void* x, bool bf16, int64_t M, int6
                                        const float* s, const float* s_inv, bool e4m3,
                                        const float* amax_prev, uint8_t* xq, float* sx,
                                        float* amax_out, cudaStream_t st);
+// RMS normalization of x with gain g (1/s folded in) fused with per-token
+// quantization; K <= rmsnorm_quant_max_k(), a multiple of 8
+int rmsnorm_quant_max_k();
+cudaError_t launch_rmsnorm_quant(const uint16_t* x, const float* g, float eps, int64_t M,
+                                 int64_t K, bool e4m3, void* xq, float* sx, cudaStream_t st);
 // offline fold of 1/s into the producer of X
 cudaError_t launch_fold_smoothing(const void* p, bool bf16, int64_t rows, int64_t cols,
                                   const float* s, bool per_column, float* out, cudaStream_t st);

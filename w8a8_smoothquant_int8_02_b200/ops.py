@@ -28,7 +28,7 @@ EXPORTED = (
     "sq_smooth_factors", "sq_quantize_weight", "sq_quantize_act", "sq_gemm_w8a8",
     "sq_gemm_fp8", "sq_linear", "sq_probe_wait_timeout", "sq_selftest_fast_division",
     "sq_gemm_workspace_bytes", "sq_gemm_w8a8_noalloc", "sq_quantize_act_tensor",
-    "sq_fold_smoothing", "sq_gemm_weight_only",
+    "sq_fold_smoothing", "sq_gemm_weight_only", "sq_rmsnorm_quantize_act",
 )
 
 _lock = threading.Lock()
@@ -72,6 +72,7 @@ def load(build_if_needed: bool = True) -> ctypes.CDLL:
             lib.sq_linear.argtypes = [P, I, P, P, P, P, P, I, I64, I64, I64, P, P, P, I, P, SZ, P]
             lib.sq_gemm_w8a8_noalloc.argtypes = [P, P, P, P, P, I64, I64, I64, P, I, P]
             lib.sq_gemm_weight_only.argtypes = [P, P, I, P, P, I64, I64, I64, P, I, P]
+            lib.sq_rmsnorm_quantize_act.argtypes = [P, P, ctypes.c_float, I64, I64, I, P, P, P]
             lib.sq_gemm_workspace_bytes.argtypes = []
             lib.sq_gemm_workspace_bytes.restype = SZ
             lib.sq_probe_wait_timeout.argtypes = [I64, P]
@@ -331,6 +332,25 @@ def gemm_weight_only(x, wq, sw, bias=None, bits=8, out_dtype=torch.bfloat16, out
                                       _p(bias), M, N, K, _p(out), _fdtype(out),
                                       _stream(x.device)), "sq_gemm_weight_only")
     return out
+
+
+def rmsnorm_quantize_act(x, g, eps, qtype="i8", xq=None, sx=None):
+    """The producer of X with the smoothing folded in: RMS normalization of the
+    bf16 rows of x [M,K] with gain g [K] (gamma / s, see fold_smoothing), fused
+    with per-token quantization. Returns (xq [M,K] codes, sx [M])."""
+    _cuda(x, g, xq, sx)
+    if x.dtype != torch.bfloat16 or g.dtype != torch.float32:
+        raise TypeError("x must be bfloat16 and g float32")
+    M, K = x.shape
+    qt = SQ_I8 if qtype == "i8" else SQ_E4M3
+    if xq is None:
+        xq = torch.empty((M, K), dtype=torch.int8 if qt == SQ_I8 else torch.uint8,
+                         device=x.device)
+    if sx is None:
+        sx = torch.empty(M, dtype=torch.float32, device=x.device)
+    _check(load().sq_rmsnorm_quantize_act(_p(x), _p(g), float(eps), M, K, qt, _p(xq), _p(sx),
+                                          _stream(x.device)), "sq_rmsnorm_quantize_act")
+    return xq, sx
 
 
 def linear(x, s, wq, sw, bias=None, qtype="i8", out_dtype=torch.bfloat16, out=None,
