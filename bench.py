@@ -49,6 +49,9 @@ def weight_bits(case):
 
 
 def metric_for(case):
+    if case.norm_eps:
+        return (f"W8A8 RMSNorm+quant+GEMM TOPS and % of INT8 TC peak at "
+                f"M{case.M} K{case.K} N{case.N}")
     if case.name.startswith("mlp_up"):
         return METRIC
     if weight_bits(case):
@@ -93,7 +96,8 @@ KERNEL_SOURCES = {"gemm": ("sq_gemm.cu", "sq_common.cuh"),
                   "gemm_wonly": ("sq_gemm_wonly.cu", "sq_common.cuh"),
                   "gemm_small": ("sq_gemm_small.cu", "sq_common.cuh"),
                   "gemm_skinny": ("sq_gemm_skinny.cu", "sq_common.cuh"),
-                  "quant": ("sq_quant.cu", "sq_common.cuh")}
+                  "quant": ("sq_quant.cu", "sq_common.cuh"),
+                  "norm": ("sq_norm.cu", "sq_common.cuh")}
 
 
 def profiled_traffic(kind, workload):
@@ -157,6 +161,8 @@ def quant_kernel_name(case):
     sms = 148
     if weight_bits(case):
         return None
+    if case.norm_eps:
+        return "rmsnorm_quant_kernel"
     if case.act_scaling == "tensor":
         return "quant_act_tensor_kernel"
     if case.x_dtype != "bf16" or case.K // 8 > 256 * 8:
@@ -167,6 +173,8 @@ def quant_kernel_name(case):
 
 
 def path_desc(case):
+    if case.norm_eps:
+        return "fused RMS normalization + act quant, 8-bit GEMM + epilogue"
     return ("weight-only GEMM on bf16 activations + epilogue" if weight_bits(case)
             else "act quant + 8-bit GEMM + epilogue")
 
@@ -290,7 +298,8 @@ def run_reference(args):
         "config": {"workload": case.name, "M": case.M, "K": case.K, "N": case.N,
                    "alpha": case.alpha if case.smooth else None,
                    "act_scaling": ("per-tensor, delayed" if case.act_scaling == "tensor"
-                                   else "per-token"),
+                                   else "per-token, from the fused RMS normalization"
+                                   if case.norm_eps else "per-token"),
                    "bias": bias is not None, "out": "bf16"},
         "cpu_baseline": {"value": val, "unit": UNIT, "cores": oracle.num_threads(),
                          "kind": "oracle",
@@ -312,6 +321,14 @@ def _oracle_prep(case, d):
         wq, sw = oracle.quantize_weight_i4(d["w"])
         return None, wq, sw, None
     qt = oracle.E4M3 if case.qtype == "e4m3" else oracle.INT8
+    if case.norm_eps:
+        # calibration on the normalization's output; the returned "s" is the
+        # gain with 1/s folded in, the runtime path's only per-channel input
+        xn_cal = oracle.rmsnorm_quantize_act(d["x_cal"], d["gamma"], case.norm_eps)[3]
+        s = oracle.smooth_factors(oracle.amax(xn_cal, True), oracle.amax(d["w"], False),
+                                  case.alpha)
+        wq, sw = oracle.quantize_weight(d["w"], s, qt)
+        return oracle.fold_smoothing(d["gamma"], s)[0], wq, sw, None
     s = None
     if case.smooth:
         s = oracle.smooth_factors(oracle.amax(d["x_cal"], True), oracle.amax(d["w"], False),
@@ -330,6 +347,10 @@ def _oracle_runtime(case, xs, s, wq, sw, bias, scale):
     if weight_bits(case):
         return oracle.gemm_weight_only(xs, wq, sw, bias, weight_bits(case))
     qt = oracle.E4M3 if case.qtype == "e4m3" else oracle.INT8
+    if case.norm_eps:     # s is the folded gain here
+        xq, sx, _, _ = oracle.rmsnorm_quantize_act(xs, s, case.norm_eps, qt)
+        acc = oracle.gemm_e4m3(xq, wq) if qt == oracle.E4M3 else oracle.gemm_i8(xq, wq)
+        return oracle.epilogue(acc, sx, sw, bias)
     if scale is None:
         return oracle.linear(xs, s, wq, sw, bias, qt)
     xq, sc, _ = oracle.quantize_act_tensor(xs, s, qt, scale=scale)
@@ -397,9 +418,15 @@ def run_ours(args):
     # ---- offline preparation (untimed) ----
     w = to_dev(d["w"])
     wbits = weight_bits(case)
+    g_fold = None
     if wbits:
         s = s_inv = None
         wq0, sw = ops.quantize_weight(w, None, "i8" if wbits == 8 else "i4")
+    elif case.norm_eps:
+        p = ops.prepare_rmsnorm(w, to_dev(d["x_cal"]), to_dev(d["gamma"]), case.norm_eps,
+                                alpha=case.alpha, qtype=qt)
+        s = s_inv = None
+        g_fold, wq0, sw = p["g"], p["wq"], p["sw"]
     elif case.smooth:
         p = ops.prepare(w, to_dev(d["x_cal"]), alpha=case.alpha, qtype=qt)
         s, s_inv, wq0, sw = p["s"], p["s_inv"], p["wq"], p["sw"]
@@ -433,6 +460,8 @@ def run_ours(args):
         if tensor:
             ops.quantize_act_tensor(xs[r], s, qt, amax_prev=amax_b[i % 2:i % 2 + 1], xq=xq, sx=sx,
                                     amax_out=amax_b[(i + 1) % 2:(i + 1) % 2 + 1], s_inv=s_inv)
+        elif g_fold is not None:
+            ops.rmsnorm_quantize_act(xs[r], g_fold, case.norm_eps, qt, xq=xq, sx=sx)
         else:
             ops.quantize_act(xs[r], s, qt, xq=xq, sx=sx, s_inv=s_inv)
 
@@ -603,6 +632,9 @@ def run_ours(args):
                 ops.quantize_act_tensor(xd, s, qt, amax_prev=amax_b[0:1], xq=xq, sx=sx,
                                         amax_out=amax_b[1:2], s_inv=s_inv)
                 gemm(xq, sx, wq0, sw, bias, out=yd, split=split)
+            elif g_fold is not None:
+                ops.rmsnorm_quantize_act(xd, g_fold, case.norm_eps, qt, xq=xq, sx=sx)
+                gemm(xq, sx, wq0, sw, bias, out=yd, split=split)
             else:
                 ops.linear(xd, s, wq0, sw, bias, qt, out=yd, xq_buf=xq, sx_buf=sx, s_inv=s_inv,
                            split=split)
@@ -658,7 +690,7 @@ def run_ours(args):
         int8_peak_sus = 2.0 * pk["bf16_sus"]
         gemm_tops = case.ops / (t_gemm * 1e-3) / 1e12
         value = ws * case.ops * K_steps / (elapsed_ms * 1e-3) / 1e12
-        # read X (bf16) + s, write Xq + sx (per-tensor: + the scale, + the max)
+        # read X (bf16) + s (or the folded gain), write Xq + sx (per-tensor: + the scale, + the max)
         q_bytes = M * K * 2 + M * K + M * 4 + (K * 4 if case.smooth else 0)
         g_bytes = M * K + N * K + M * N * 2 + 4 * (M + N) + (2 * N if bias is not None else 0)
         if wbits:
@@ -675,7 +707,9 @@ def run_ours(args):
             "config": {"workload": case.name, "M": M, "K": K, "N": N,
                        "alpha": case.alpha if case.smooth else None,
                        "act_scaling": ("none (weight-only)" if wbits else
-                                       "per-tensor, delayed" if tensor else "per-token"),
+                                       "per-tensor, delayed" if tensor else
+                                       "per-token, from the fused RMS normalization"
+                                       if case.norm_eps else "per-token"),
                        "bias": bias is not None, "out": "bf16",
                        "l2": (f"{ROTATE} rotating input sets (X + Wq, "
                               f"{ROTATE * (M * K * 2 + w_set) / 2 ** 20:.0f} MiB) > 126 MiB L2"),
@@ -698,7 +732,8 @@ def run_ours(args):
                 "bound": "hbm", "kernel": quant_kernel_name(case),
                 "achieved": q_bytes / (t_quant * 1e-3) / 1e9, "peak": pk["hbm"],
                 "unit": "GB/s", "frac": q_bytes / (t_quant * 1e-3) / 1e9 / pk["hbm"],
-                "traffic": profiled_traffic("quant", case.name), "ms_per_launch": t_quant},
+                "traffic": profiled_traffic("norm" if case.norm_eps else "quant", case.name),
+                "ms_per_launch": t_quant},
             "gpu_launches": launches_per_step(case) * K_steps,
             "clocks": clocks,
             "sustained": sustained,
@@ -781,7 +816,7 @@ def main():
     ap.add_argument("--no-graph", action="store_true",
                     help="launch the timed steps one by one instead of replaying a CUDA graph")
     ap.add_argument("--workload", default="mlp_up_4096x4096x14336",
-                    help="one of the six workloads in workloads.py (default: the MLP up-projection)")
+                    help="one of the workloads in workloads.py (default: the MLP up-projection)")
     ap.add_argument("--no-split", action="store_true",
                     help="launch the GEMM without its workspace (by default the library may split "
                          "the last partial round of tiles along K over all SMs where that pays)")

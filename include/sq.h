@@ -242,17 +242,21 @@ sq_status sq_fold_smoothing(const void* p, sq_dtype pt, int64_t rows, int64_t co
  *   g   : [K] binary32 gain with 1/s folded in (16-byte aligned)
  *   eps : > 0, finite
  *   qt  : SQ_I8 or SQ_E4M3;  xq : [M,K] codes (16-byte aligned);  sx : [M]
+ *   xn  : [M,K] binary32 or NULL (16-byte aligned): when given, the
+ *         normalization's output xn below is written too, for the offline
+ *         calibration of the smoothing factors (run it with g = gamma)
  * Per row: ss = the sum of x_k^2 over the k whose bf16 exponent is within 48
  * of the row's largest, exactly, rounded once to binary64 (the others are
  * below 2^-94 of the largest square); r = binary32(1 / sqrt(ss / K + eps))
  * with each of the four binary64 operations rounded once; xn_k = (x_k * r) *
  * g_k in binary32; then sx and the codes of xn exactly as sq_quantize_act
  * with s = NULL. K a multiple of 8, at most 16384 (SQ_ERR_UNSUPPORTED
- * beyond). xq and sx may overlap neither each other nor x or g
+ * beyond). xq, sx and xn may overlap neither each other nor x or g
  * (SQ_ERR_INVALID_ARG). M == 0 is a no-op that accepts NULL pointers.
  */
 sq_status sq_rmsnorm_quantize_act(const void* x, const float* g, float eps, int64_t M,
-                                  int64_t K, sq_dtype qt, void* xq, float* sx, void* stream);
+                                  int64_t K, sq_dtype qt, void* xq, float* sx, float* xn,
+                                  void* stream);
 
 /*
  * Size in bytes of the GEMM workspace for the current device (its SM count

@@ -56,11 +56,11 @@ int main(void) {
                SQ_ERR_INVALID_ARG, "fold: output aliasing the input");
     expect(sq_fold_smoothing(NULL, SQ_F32, 0, 40, NULL, SQ_AMAX_PER_COLUMN, NULL, NULL) == SQ_OK,
            "fold: nothing to fold");
-    expect(sq_rmsnorm_quantize_act(A, F, 1e-6f, 4, 16392, SQ_I8, (char*)A + 0x100000, F, NULL) ==
+    expect(sq_rmsnorm_quantize_act(A, F, 1e-6f, 4, 16392, SQ_I8, (char*)A + 0x100000, F, NULL, NULL) ==
                SQ_ERR_UNSUPPORTED, "norm + quantization: K beyond one row on chip");
-    expect(sq_rmsnorm_quantize_act(A, F, 0.0f, 4, 64, SQ_I8, (char*)A + 0x100000, F, NULL) ==
+    expect(sq_rmsnorm_quantize_act(A, F, 0.0f, 4, 64, SQ_I8, (char*)A + 0x100000, F, NULL, NULL) ==
                SQ_ERR_INVALID_ARG, "norm + quantization: eps must be positive");
-    expect(sq_rmsnorm_quantize_act(NULL, NULL, 1e-6f, 0, 64, SQ_E4M3, NULL, NULL, NULL) == SQ_OK,
+    expect(sq_rmsnorm_quantize_act(NULL, NULL, 1e-6f, 0, 64, SQ_E4M3, NULL, NULL, NULL, NULL) == SQ_OK,
            "norm + quantization: empty batch");
     expect(sq_probe_wait_timeout(10, NULL) == SQ_ERR_INVALID_ARG, "probe: timeout below 1 ms");
     expect(sq_selftest_fast_division(NULL, NULL) == SQ_ERR_INVALID_ARG, "self-test: NULL result");

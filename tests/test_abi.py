@@ -257,12 +257,12 @@ def test_abi_from_plain_c(tmp_path):
 def test_rmsnorm_quantize_validation(lib):
     f = lib.sq_rmsnorm_quantize_act
     ok = dict(x=A, g=A + 0x100000, eps=1e-6, M=4, K=64, qt=ops.SQ_I8, xq=A + 0x200000,
-              sx=A + 0x300000)
+              sx=A + 0x300000, xn=NUL)
 
     def call(**kw):
         a = dict(ok, **kw)
         return f(c(a["x"]), c(a["g"]), a["eps"], a["M"], a["K"], a["qt"], c(a["xq"]),
-                 c(a["sx"]), None)
+                 c(a["sx"]), c(a["xn"]), None)
 
     assert call(x=NUL) == ops.SQ_ERR_INVALID_ARG
     assert call(g=NUL) == ops.SQ_ERR_INVALID_ARG
@@ -286,5 +286,9 @@ def test_rmsnorm_quantize_validation(lib):
     assert call(g=A + 0x100000 + 4) == ops.SQ_ERR_MISALIGNED
     assert call(xq=A + 0x200000 + 8) == ops.SQ_ERR_MISALIGNED
     assert call(sx=A + 0x300000 + 2) == ops.SQ_ERR_MISALIGNED
+    assert call(xn=A + 0x400000 + 4) == ops.SQ_ERR_MISALIGNED       # float4 stores
+    assert call(xn=A + 256) == ops.SQ_ERR_INVALID_ARG               # the output over the input
+    assert call(xn=A + 0x200000 - 512) == ops.SQ_ERR_INVALID_ARG    # ... over the codes
+    assert call(xn=A + 0x300000 - 1024 + 16) == ops.SQ_ERR_INVALID_ARG   # ... over the scales
     # empty batch: a no-op that accepts NULL pointers
     assert call(M=0, x=NUL, g=NUL, xq=NUL, sx=NUL) == ops.SQ_OK

@@ -36,6 +36,7 @@ def test_metric_names(bench):
     assert "FP8" in bench.metric_for(workloads.FP8_DOWN)
     assert "per-tensor" in bench.metric_for(workloads.FP8_TENSOR)
     assert "M512 K4096 N4096" in bench.metric_for(workloads.PREFILL)
+    assert "RMSNorm" in bench.metric_for(workloads.MLP_UP_RMSNORM)
 
 
 def test_activation_kernel_per_workload(bench):
@@ -44,6 +45,7 @@ def test_activation_kernel_per_workload(bench):
     assert bench.quant_kernel_name(workloads.FP8_DOWN) == "quant_act_stream_kernel"
     assert bench.quant_kernel_name(workloads.DECODE) == "quant_act_fast_kernel"      # 16 rows
     assert bench.quant_kernel_name(workloads.FP8_TENSOR) == "quant_act_tensor_kernel"
+    assert bench.quant_kernel_name(workloads.MLP_UP_RMSNORM) == "rmsnorm_quant_kernel"
 
 
 def test_profiled_traffic_is_guarded_by_the_kernel_source(bench, tmp_path, monkeypatch):
@@ -81,6 +83,13 @@ def test_reference_arm_cpu_baseline_on_tiny(bench):
     d2 = synth.generate(small)
     out2 = bench.cpu_baseline(small, d2, budget_s=0.05)
     assert out2["value"] > 0
+    normed = workloads.MLP_UP_RMSNORM
+    small3 = synth.LinearCase(**{**normed.__dict__, "M": 8, "K": 64, "N": 32, "cal_tokens": 16,
+                                 "name": "mlp_up_rmsnorm_small"})
+    d3 = synth.generate(small3)
+    assert d3["gamma"].shape == (64,) and d3["gamma"].min() >= 0.5
+    out3 = bench.cpu_baseline(small3, d3, budget_s=0.05)
+    assert out3["value"] > 0 and "RMS normalization" in out3["sample"]
 
 
 def test_reference_arm_line(bench, capsys, monkeypatch):

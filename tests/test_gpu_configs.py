@@ -68,7 +68,22 @@ def test_workload_end_to_end(name):
     # ---- offline preparation ----
     w_d = dev(w)
     s = None
-    if case.smooth:
+    if case.norm_eps:
+        # calibration on the normalization's output, s, and the gain with 1/s
+        # folded in; the later stages take the oracle's s (stage-wise parity)
+        xn_cal = oracle.rmsnorm_quantize_act(x_cal, d["gamma"], case.norm_eps)[3]
+        ax = oracle.amax(xn_cal, True)
+        aw = oracle.amax(w, False)
+        s = oracle.smooth_factors(ax, aw, case.alpha)
+        p = ops.prepare_rmsnorm(w_d, dev(x_cal), dev(d["gamma"]), case.norm_eps,
+                                alpha=case.alpha, qtype=case.qtype)
+        np.testing.assert_array_equal(host(p["amax_x"]), ax)
+        np.testing.assert_array_equal(host(p["amax_w"]), aw)
+        assert ulp_distance(host(p["s"]), s).max() <= 2
+        g_ref = oracle.fold_smoothing(d["gamma"], s)[0]
+        g_d = ops.fold_smoothing(dev(d["gamma"]), dev(s))
+        np.testing.assert_array_equal(host(g_d), g_ref)
+    elif case.smooth:
         ax = oracle.amax(x_cal, True)
         aw = oracle.amax(w, False)
         s = oracle.smooth_factors(ax, aw, case.alpha)
@@ -97,6 +112,10 @@ def test_workload_end_to_end(name):
         xq_d, sx_d, amax_d = ops.quantize_act_tensor(dev(x), s_d, case.qtype, amax_prev=amax_cal_d,
                                                      s_inv=s_inv_d)
         assert host(amax_d)[0] == amax_x
+    elif case.norm_eps:
+        # ---- runtime: the fused normalization + per-token quantization ----
+        xq_ref, sx_ref, _, _ = oracle.rmsnorm_quantize_act(x, g_ref, case.norm_eps, qt)
+        xq_d, sx_d = ops.rmsnorm_quantize_act(dev(x), g_d, case.norm_eps, case.qtype)
     else:
         # ---- runtime: activation smoothing + per-token quantization ----
         xq_ref, sx_ref = oracle.quantize_act(x, s, qt)
@@ -130,7 +149,7 @@ def test_workload_end_to_end(name):
     del yf_ref
 
     # ---- the fused forward through one C call (same operands; per-token) ----
-    if case.act_scaling == "tensor":
+    if case.act_scaling == "tensor" or case.norm_eps:
         return
     y2 = ops.linear(dev(x), s_d, ops_w, dev(sw_ref), bias_d, case.qtype,
                     out_dtype=torch.float32, s_inv=s_inv_d, split=True)

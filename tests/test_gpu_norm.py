@@ -13,7 +13,7 @@ import torch
 import oracle
 from w8a8_smoothquant_int8_02_b200 import ops, synth
 
-from _gpu_util import dev, host
+from _gpu_util import dev, host, ulp_distance
 
 pytestmark = pytest.mark.gpu
 
@@ -42,37 +42,49 @@ def test_rmsnorm_quantize_matches_oracle(M, K, qt, eps):
     xb = _rows(M, K, seed=M + K)
     gamma = synth.random_floats(K, seed=K, lo=0.3, hi=2.5)
     gamma[::5] *= -1.0                                 # negative gains too
-    q_ref, s_ref, _, _ = oracle.rmsnorm_quantize_act(
+    q_ref, s_ref, _, xn_ref = oracle.rmsnorm_quantize_act(
         xb, gamma, eps, oracle.INT8 if qt == "i8" else oracle.E4M3)
-    xq, sx = ops.rmsnorm_quantize_act(dev(xb), dev(gamma), eps, qt)
+    want_xn = eps == 1e-6        # both forms: with and without the binary32 output
+    out = ops.rmsnorm_quantize_act(dev(xb), dev(gamma), eps, qt, want_xn=want_xn)
     assert ops.device_status() == ops.SQ_OK
-    np.testing.assert_array_equal(host(sx), s_ref)
-    np.testing.assert_array_equal(host(xq).view(np.uint8), q_ref.view(np.uint8))
+    np.testing.assert_array_equal(host(out[1]), s_ref)
+    np.testing.assert_array_equal(host(out[0]).view(np.uint8), q_ref.view(np.uint8))
+    if want_xn:                  # bit patterns: signed zeros included
+        np.testing.assert_array_equal(host(out[2]).view(np.uint32), xn_ref.view(np.uint32))
 
 
 @pytest.mark.parametrize("qt", ["i8", "e4m3"])
 def test_folded_producer_feeds_the_layer(qt):
-    """Offline: calibrate, smoothing factors, fold 1/s into the norm's gain (all
-    on the GPU); runtime: the fused norm + quantization, then the 8-bit GEMM --
-    codes, scales and the GEMM output equal the oracle's chain."""
+    """Offline, all on the GPU: the normalization's output of the calibration
+    tokens, its per-channel max, s, the quantized weights, 1/s folded into the
+    gain; at runtime the fused normalization + quantization, then the 8-bit
+    GEMM. Every stage equals the oracle's chain bit for bit (the FP8 GEMM
+    within its accumulation bound)."""
     M, K, N = 256, 1024, 512
     xb = _rows(M, K, seed=91)
+    xcal = _rows(128, K, seed=94)
     gamma = synth.random_floats(K, seed=92, lo=0.5, hi=2.0)
     w = synth.random_floats((K, N), seed=93, std=0.02)
     qcode = oracle.INT8 if qt == "i8" else oracle.E4M3
-    _, _, _, xn_cal = oracle.rmsnorm_quantize_act(xb, gamma, 1e-6)   # the norm's output
-    ax, aw = oracle.amax(xn_cal, True), oracle.amax(w, False)
-    s = oracle.smooth_factors(ax, aw, 0.5)
+    eps = 1e-5
+    p = ops.prepare_rmsnorm(dev(w), dev(xcal), dev(gamma), eps, 0.5, qt)
+    _, _, _, xn_cal = oracle.rmsnorm_quantize_act(xcal, gamma, eps)
+    ax_ref = oracle.amax(xn_cal, True)
+    np.testing.assert_array_equal(host(p["amax_x"]), ax_ref)
+    s_ref = oracle.smooth_factors(ax_ref, oracle.amax(w, False), 0.5)
+    assert ulp_distance(host(p["s"]), s_ref).max() <= 2      # pow: libm vs the GPU's
+    s = host(p["s"])       # each later stage on the same inputs (no cascade of that ulp)
     g_ref = oracle.fold_smoothing(gamma, s)[0]
     wq_ref, sw_ref = oracle.quantize_weight(w, s, qcode)
-    q_ref, sx_ref, _, _ = oracle.rmsnorm_quantize_act(xb, g_ref, 1e-6, qcode)
-    g_d = ops.fold_smoothing(dev(gamma), dev(s))
-    np.testing.assert_array_equal(host(g_d), g_ref)
-    xq, sx = ops.rmsnorm_quantize_act(dev(xb), g_d, 1e-6, qt)
+    q_ref, sx_ref, _, _ = oracle.rmsnorm_quantize_act(xb, g_ref, eps, qcode)
+    np.testing.assert_array_equal(host(p["g"]), g_ref)
+    np.testing.assert_array_equal(host(p["wq"]).view(np.uint8), wq_ref.view(np.uint8))
+    np.testing.assert_array_equal(host(p["sw"]), sw_ref)
+    xq, sx = ops.rmsnorm_quantize_act(dev(xb), p["g"], eps, qt)
     np.testing.assert_array_equal(host(sx), sx_ref)
     np.testing.assert_array_equal(host(xq).view(np.uint8), q_ref.view(np.uint8))
     if qt == "i8":
-        y = ops.gemm_w8a8(xq, sx, dev(wq_ref), dev(sw_ref), out_dtype=torch.float32)
+        y = ops.gemm_w8a8(xq, sx, p["wq"], p["sw"], out_dtype=torch.float32)
         y_ref, _ = oracle.epilogue(oracle.gemm_i8(q_ref, wq_ref), sx_ref, sw_ref, None)
         np.testing.assert_array_equal(host(y), y_ref)
     assert ops.device_status() == ops.SQ_OK

@@ -336,7 +336,8 @@ sq_status sq_gemm_weight_only(const void* x, const void* wq, sq_dtype wqt, const
 }
 
 sq_status sq_rmsnorm_quantize_act(const void* x, const float* g, float eps, int64_t M,
-                                  int64_t K, sq_dtype qt, void* xq, float* sx, void* stream) {
+                                  int64_t K, sq_dtype qt, void* xq, float* sx, float* xn,
+                                  void* stream) {
   if (qt != SQ_I8 && qt != SQ_E4M3) return SQ_ERR_INVALID_ARG;
   if (M < 0 || K <= 0 || K % 8 != 0 || M > INT32_MAX) return SQ_ERR_INVALID_ARG;
   if (!(eps > 0.0f) || !std::isfinite(eps)) return SQ_ERR_INVALID_ARG;
@@ -349,9 +350,14 @@ sq_status sq_rmsnorm_quantize_act(const void* x, const float* g, float eps, int6
       overlap(sx, uint64_t(M) * 4, x, xb) || overlap(sx, uint64_t(M) * 4, g, uint64_t(K) * 4) ||
       overlap(sx, uint64_t(M) * 4, xq, qb))
     return SQ_ERR_INVALID_ARG;
-  if (!al(x, 16) || !al(g, 16) || !al(xq, 16) || !al(sx, 4)) return SQ_ERR_MISALIGNED;
+  const uint64_t nb = uint64_t(M) * uint64_t(K) * 4;
+  if (xn && (overlap(xn, nb, x, xb) || overlap(xn, nb, g, uint64_t(K) * 4) ||
+             overlap(xn, nb, xq, qb) || overlap(xn, nb, sx, uint64_t(M) * 4)))
+    return SQ_ERR_INVALID_ARG;
+  if (!al(x, 16) || !al(g, 16) || !al(xq, 16) || !al(sx, 4) || !al(xn, 16))
+    return SQ_ERR_MISALIGNED;
   return from_cuda(sqh::launch_rmsnorm_quant(static_cast<const uint16_t*>(x), g, eps, M, K,
-                                             qt == SQ_E4M3, xq, sx, S(stream)));
+                                             qt == SQ_E4M3, xq, sx, xn, S(stream)));
 }
 
 sq_status sq_selftest_fast_division(int64_t* mismatches, void* stream) {

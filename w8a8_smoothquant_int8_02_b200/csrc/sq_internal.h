@@ -33,7 +33,8 @@ cudaError_t launch_quantize_act_tensor(const void* x, bool bf16, int64_t M, int6
 // quantization; K <= rmsnorm_quant_max_k(), a multiple of 8
 int rmsnorm_quant_max_k();
 cudaError_t launch_rmsnorm_quant(const uint16_t* x, const float* g, float eps, int64_t M,
-                                 int64_t K, bool e4m3, void* xq, float* sx, cudaStream_t st);
+                                 int64_t K, bool e4m3, void* xq, float* sx, float* xn,
+                                 cudaStream_t st);
 // offline fold of 1/s into the producer of X
 cudaError_t launch_fold_smoothing(const void* p, bool bf16, int64_t rows, int64_t cols,
                                   const float* s, bool per_column, float* out, cudaStream_t st);

@@ -21,6 +21,8 @@
 //   then the per-token quantization of xn (no smoothing): sx = max|xn| / Q,
 //   codes of xn / sx (INT8: round-half-even, clamped to +-127; E4M3:
 //   round-to-nearest-even, saturating), all-zero codes where sx is 0.
+// xn itself is written too when asked for (binary32; the calibration of the
+// smoothing factors runs on it offline).
 //
 // One CTA per row: the row is staged in shared memory, then four passes over
 // it (the largest exponent, the exact sum of squares, the largest |xn|, the
@@ -73,7 +75,7 @@ template <bool E4M3>
 __global__ void __launch_bounds__(kNormThreads)
     rmsnorm_quant_kernel(const uint16_t* __restrict__ x, const float* __restrict__ g,
                          float eps, int64_t M, int K, uint8_t* __restrict__ xq,
-                         float* __restrict__ sx) {
+                         float* __restrict__ sx, float* __restrict__ xn) {
   extern __shared__ __align__(16) uint16_t row[];  // K entries
   __shared__ int red_i[kNormThreads / 32];
   __shared__ unsigned long long red_lo[kNormThreads / 32], red_hi[kNormThreads / 32];
@@ -168,10 +170,17 @@ __global__ void __launch_bounds__(kNormThreads)
       const float4 g0 = __ldg(reinterpret_cast<const float4*>(g) + 2 * c);
       const float4 g1 = __ldg(reinterpret_cast<const float4*>(g) + 2 * c + 1);
       const float gv[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+      float y[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const float xv = (i & 1) ? bf16_hi(w[i >> 1]) : bf16_lo(w[i >> 1]);
-        amax = fmaxf(amax, fabsf(__fmul_rn(__fmul_rn(xv, r), gv[i])));
+        y[i] = __fmul_rn(__fmul_rn(xv, r), gv[i]);
+        amax = fmaxf(amax, fabsf(y[i]));
+      }
+      if (xn) {  // the normalization's output itself (offline calibration)
+        float4* o = reinterpret_cast<float4*>(xn + m * K) + 2 * c;
+        o[0] = make_float4(y[0], y[1], y[2], y[3]);
+        o[1] = make_float4(y[4], y[5], y[6], y[7]);
       }
     }
     amax = __uint_as_float(__reduce_max_sync(0xFFFFFFFFu, __float_as_uint(amax)));
@@ -231,16 +240,17 @@ using namespace sqk;
 int rmsnorm_quant_max_k() { return kNormMaxK; }
 
 cudaError_t launch_rmsnorm_quant(const uint16_t* x, const float* g, float eps, int64_t M,
-                                 int64_t K, bool e4m3, void* xq, float* sx, cudaStream_t st) {
+                                 int64_t K, bool e4m3, void* xq, float* sx, float* xn,
+                                 cudaStream_t st) {
   // one CTA per row, at most a few waves' worth resident: rows beyond the
   // grid are taken in turn
   const int64_t grid = M < 148 * 16 ? M : 148 * 16;
   const size_t smem = size_t(K) * 2;  // the staged row (at most 32 KB: no opt-in needed)
   if (e4m3)
     return launch_pdl(rmsnorm_quant_kernel<true>, unsigned(grid), kNormThreads, smem, st, x, g,
-                      eps, M, int(K), static_cast<uint8_t*>(xq), sx);
+                      eps, M, int(K), static_cast<uint8_t*>(xq), sx, xn);
   return launch_pdl(rmsnorm_quant_kernel<false>, unsigned(grid), kNormThreads, smem, st, x, g,
-                    eps, M, int(K), static_cast<uint8_t*>(xq), sx);
+                    eps, M, int(K), static_cast<uint8_t*>(xq), sx, xn);
 }
 
 }  // namespace sqh

@@ -72,7 +72,7 @@ def load(build_if_needed: bool = True) -> ctypes.CDLL:
             lib.sq_linear.argtypes = [P, I, P, P, P, P, P, I, I64, I64, I64, P, P, P, I, P, SZ, P]
             lib.sq_gemm_w8a8_noalloc.argtypes = [P, P, P, P, P, I64, I64, I64, P, I, P]
             lib.sq_gemm_weight_only.argtypes = [P, P, I, P, P, I64, I64, I64, P, I, P]
-            lib.sq_rmsnorm_quantize_act.argtypes = [P, P, ctypes.c_float, I64, I64, I, P, P, P]
+            lib.sq_rmsnorm_quantize_act.argtypes = [P, P, ctypes.c_float, I64, I64, I, P, P, P, P]
             lib.sq_gemm_workspace_bytes.argtypes = []
             lib.sq_gemm_workspace_bytes.restype = SZ
             lib.sq_probe_wait_timeout.argtypes = [I64, P]
@@ -334,11 +334,13 @@ def gemm_weight_only(x, wq, sw, bias=None, bits=8, out_dtype=torch.bfloat16, out
     return out
 
 
-def rmsnorm_quantize_act(x, g, eps, qtype="i8", xq=None, sx=None):
+def rmsnorm_quantize_act(x, g, eps, qtype="i8", xq=None, sx=None, xn=None, want_xn=False):
     """The producer of X with the smoothing folded in: RMS normalization of the
     bf16 rows of x [M,K] with gain g [K] (gamma / s, see fold_smoothing), fused
-    with per-token quantization. Returns (xq [M,K] codes, sx [M])."""
-    _cuda(x, g, xq, sx)
+    with per-token quantization. Returns (xq [M,K] codes, sx [M]); with
+    want_xn (or an xn buffer given) also the normalization's output xn [M,K]
+    float32, the input of the offline calibration."""
+    _cuda(x, g, xq, sx, xn)
     if x.dtype != torch.bfloat16 or g.dtype != torch.float32:
         raise TypeError("x must be bfloat16 and g float32")
     M, K = x.shape
@@ -348,9 +350,11 @@ def rmsnorm_quantize_act(x, g, eps, qtype="i8", xq=None, sx=None):
                          device=x.device)
     if sx is None:
         sx = torch.empty(M, dtype=torch.float32, device=x.device)
+    if xn is None and want_xn:
+        xn = torch.empty((M, K), dtype=torch.float32, device=x.device)
     _check(load().sq_rmsnorm_quantize_act(_p(x), _p(g), float(eps), M, K, qt, _p(xq), _p(sx),
-                                          _stream(x.device)), "sq_rmsnorm_quantize_act")
-    return xq, sx
+                                          _p(xn), _stream(x.device)), "sq_rmsnorm_quantize_act")
+    return (xq, sx, xn) if xn is not None else (xq, sx)
 
 
 def linear(x, s, wq, sw, bias=None, qtype="i8", out_dtype=torch.bfloat16, out=None,
@@ -438,6 +442,18 @@ def prepare(w: torch.Tensor, x_cal: torch.Tensor, alpha: float = 0.5, qtype: str
     s, s_inv = smooth_factors(ax, aw, alpha, with_inverse=True)
     wq, sw = quantize_weight(w, s, qtype)
     return dict(s=s, s_inv=s_inv, wq=wq, sw=sw, amax_x=ax, amax_w=aw)
+
+
+def prepare_rmsnorm(w: torch.Tensor, x_cal: torch.Tensor, gamma: torch.Tensor, eps: float,
+                    alpha: float = 0.5, qtype: str = "i8"):
+    """Offline preparation of a layer fed by an RMS normalization: the
+    calibration runs on the normalization's output (gain gamma), then s, the
+    quantized weights, and the gain with 1/s folded in (g = gamma / s) for
+    rmsnorm_quantize_act at runtime."""
+    _, _, xn = rmsnorm_quantize_act(x_cal, gamma, eps, qtype, want_xn=True)
+    p = prepare(w, xn, alpha, qtype)
+    p["g"] = fold_smoothing(gamma, p["s"])
+    return p
 
 
 class SmoothQuantLinear:

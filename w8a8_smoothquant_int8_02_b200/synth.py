@@ -7,9 +7,12 @@ Recipe (the pages describe transformer activations with a few outlier
 channels 10-100x larger than the rest -- "Weight-Activation Quantization" §2
 "The Problem: Activation Outliers" -- and roughly Gaussian weights):
 
-* numpy ``Generator(PCG64(SeedSequence(seed)))``; six independent child
+* numpy ``Generator(PCG64(SeedSequence(seed)))``; seven independent child
   streams, spawned in this order: outlier-channel set, outlier factors, X,
-  X_cal, W, bias.
+  X_cal, W, bias, the normalization's gain.
+* A layer fed by an RMS normalization (``norm_eps`` > 0): X and X_cal are the
+  normalization's input, drawn as above; its gain gamma ~ U(0.5, 2.0) per
+  channel in float32.
 * X, X_cal ~ N(0, 1) in float32. A fixed set of input channels (the first
   ``round(p*K)`` entries of a seeded permutation of K, or an explicit list) is
   multiplied by one factor per channel drawn from U(lo, hi); the same channels
@@ -51,6 +54,7 @@ class LinearCase:
     cal_tokens: int = 512         # 0 => calibrate on X itself
     act_scaling: str = "token"    # "token" (per-token), "tensor" (per-tensor, delayed), "none"
     smooth: bool = True           # False => no smoothing factors (plain FP8 / INT8)
+    norm_eps: float = 0.0         # > 0 => X comes from an RMS normalization (this eps)
     seed: int = 0
     note: str = field(default="")
 
@@ -68,7 +72,7 @@ def generate(case: LinearCase, M: int | None = None) -> dict:
     M = case.M if M is None else M
     K, N = case.K, case.N
     ss = np.random.SeedSequence(case.seed)
-    st_set, st_fac, st_x, st_cal, st_w, st_b = ss.spawn(6)
+    st_set, st_fac, st_x, st_cal, st_w, st_b, st_g = ss.spawn(7)
     if case.outlier_channels:
         ch = np.array(sorted(case.outlier_channels), np.int64)
         fac = np.full(ch.size, case.outlier_factor, np.float32)
@@ -98,7 +102,11 @@ def generate(case: LinearCase, M: int | None = None) -> dict:
         x = to_bf16_bits(x)
         x_cal = to_bf16_bits(x_cal) if case.cal_tokens else x
         w = to_bf16_bits(w)
-    return dict(x=x, x_cal=x_cal, w=w, bias=bias, outlier_channels=ch,
+    gamma = None
+    if case.norm_eps:
+        gamma = np.random.Generator(np.random.PCG64(st_g)).uniform(
+            0.5, 2.0, size=K).astype(np.float32)
+    return dict(x=x, x_cal=x_cal, w=w, bias=bias, gamma=gamma, outlier_channels=ch,
                 outlier_factors=fac)
 
 

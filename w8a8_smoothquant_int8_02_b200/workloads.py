@@ -1,6 +1,7 @@
 """The linear-layer workloads this library is measured on: five per-token
-SmoothQuant cases, one per-tensor FP8 case, and the two weight-only schemes
-(W8A16, W4A16) at the decode shape.
+SmoothQuant cases, one per-tensor FP8 case, the two weight-only schemes
+(W8A16, W4A16) at the decode shape, and the MLP up-projection fed by an RMS
+normalization with the smoothing folded into its gain.
 
 Shapes follow transformer linear layers: Y[M,N] = X[M,K] W[K,N], M tokens,
 K input channels, N output channels.  Prefill / MLP shapes are compute-bound
@@ -73,6 +74,19 @@ DECODE_W4A16 = LinearCase(
          "quantized; W bf16 [8192,28672] N(0,0.02) as per-channel INT4 codes packed two per "
          "byte; HBM-bound")
 
+# The MLP up-projection with its producer: X is the output of the layer's RMS
+# normalization, 1/s is folded into the normalization's gain offline, and one
+# kernel normalizes and quantizes each token row (the pages' "offline, no
+# runtime overhead" smoothing made literal).
+MLP_UP_RMSNORM = LinearCase(
+    name="mlp_up_rmsnorm_4096x4096x14336", M=4096, K=4096, N=14336, x_dtype="bf16",
+    alpha=0.5, qtype="i8", w_std=0.02, outlier_frac=0.01, outlier_lo=20.0,
+    outlier_hi=100.0, bias_std=0.01, cal_tokens=512, norm_eps=1e-5,
+    note="the MLP-up shape fed by an RMS normalization: its input X bf16 [4096,4096] with 1% "
+         "outlier channels x U(20,100), gain U(0.5,2), eps 1e-5; calibration on the "
+         "normalization's output of 512 tokens; W bf16 [4096,14336] N(0,0.02); bias bf16 "
+         "N(0,0.01)")
+
 ALL = {c.name: c for c in (TINY, PREFILL, MLP_UP, FP8_DOWN, DECODE, FP8_TENSOR, DECODE_W8A16,
-                           DECODE_W4A16)}
+                           DECODE_W4A16, MLP_UP_RMSNORM)}
 WEIGHT_ONLY_BITS = {"w8": 8, "w4": 4}   # qtype of a weight-only workload -> weight bits
