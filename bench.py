@@ -162,7 +162,7 @@ def quant_kernel_name(case):
     if weight_bits(case):
         return None
     if case.norm_eps:
-        return "rmsnorm_quant_kernel"
+        return "rmsnorm_quant_stream_kernel"
     if case.act_scaling == "tensor":
         return "quant_act_tensor_kernel"
     if case.x_dtype != "bf16" or case.K // 8 > 256 * 8:

@@ -31,6 +31,10 @@ def _rows(M, K, seed):
     if M > 5:
         x[4] *= 2.0 ** 100                             # large magnitudes
         x[5, ::7] = -0.0                               # signed zeros
+    if M > 6:
+        x[6] = g.standard_normal(K) * 2.0 ** -131      # a row of bf16 subnormals only
+    if M > 7:
+        x[7, 1::2] *= 2.0 ** -20                       # half the row 20 binades down
     return synth.to_bf16_bits(x)
 
 
@@ -44,7 +48,8 @@ def test_rmsnorm_quantize_matches_oracle(M, K, qt, eps):
     gamma[::5] *= -1.0                                 # negative gains too
     q_ref, s_ref, _, xn_ref = oracle.rmsnorm_quantize_act(
         xb, gamma, eps, oracle.INT8 if qt == "i8" else oracle.E4M3)
-    want_xn = eps == 1e-6        # both forms: with and without the binary32 output
+    # both forms: the plain one (which also writes xn) and the streaming one
+    want_xn = eps == 1e-6
     out = ops.rmsnorm_quantize_act(dev(xb), dev(gamma), eps, qt, want_xn=want_xn)
     assert ops.device_status() == ops.SQ_OK
     np.testing.assert_array_equal(host(out[1]), s_ref)

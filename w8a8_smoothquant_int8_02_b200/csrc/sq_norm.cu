@@ -24,11 +24,19 @@
 // xn itself is written too when asked for (binary32; the calibration of the
 // smoothing factors runs on it offline).
 //
-// One CTA per row: the row is staged in shared memory, then four passes over
-// it (the largest exponent, the exact sum of squares, the largest |xn|, the
-// codes), each closed by a block reduction. HBM-bound in principle (2 bytes
-// read and 1 written per element).
+// Two kernels give the same results bit for bit:
+//  * rmsnorm_quant_kernel, the plain form (and the only one that also writes
+//    xn): one CTA per row, the row staged in shared memory, four passes over
+//    it (the largest exponent, the exact sum of squares, the largest |xn|,
+//    the codes) with IEEE divisions, each closed by a block reduction;
+//  * rmsnorm_quant_stream_kernel, used otherwise: persistent CTAs with the
+//    next rows in flight (bulk copies into a shared-memory ring), each
+//    thread's part of the row in registers, three block barriers
+//    per row, packed binary32 pairs, and no division instruction on rows
+//    whose largest |xn| is in [2^-60, 2^100].
+// HBM-bound in principle: 2 bytes read and 1 written per element.
 #include <cstdint>
+#include <cuda_runtime.h>
 
 #include "sq_common.cuh"
 #include "sq_internal.h"
@@ -231,6 +239,353 @@ __global__ void __launch_bounds__(kNormThreads)
   }
 }
 
+// ----------------------------------------------------------------------------
+// The streaming form. Per row, with every thread holding its V 8-element
+// chunks c = threadIdx.x + j * blockDim.x of the row (bf16):
+//  1. the largest magnitude bit pattern (bf16 magnitudes order like their
+//     15-bit patterns, so its exponent field is e_max's) -- barrier 1, after
+//     which thread 0 refills the ring slot with the row SLOTS ahead;
+//  2. the exact sum of squares in three parts: the squares of normal
+//     elements within 16 binades of the largest (band A) and those 17 to 32
+//     binades below it (band B) as a^2 with a = n * 2^(e - e_max + 16) < 2^24
+//     (band B: n * 2^(e - e_max + 32) < 2^23), one 32 x 32 -> 64-bit
+//     multiply-add each, in two 64-bit sums (units 2^(2 e_max - 46) and
+//     2^(2 e_max - 78); at most 2^14 terms, so no overflow); the rest
+//     (smaller, subnormal; rare) go to a 128-bit shared accumulator in units
+//     of 2^(2 e_max - 110) by 64-bit shared atomics (the carry of the low
+//     word added to the high one) -- barrier 2; every warp then combines the
+//     three (2^64 and 2^32 apart) and takes r in the same binary64 steps as
+//     the plain form;
+//  3. y = (x * r) * g in packed pairs, kept in registers, and their largest
+//     magnitude -- barrier 3;
+//  4. sx = RN(amax / Q) and the codes of RN(y / sx): for amax in
+//     [2^-60, 2^100] without a division instruction -- the scale by the
+//     exact constant-divisor correction, the quotients by two corrections of
+//     the reciprocal product (P. Markstein, "IA-64 and Elementary Functions",
+//     2000), the INT8 code as the low byte of RN(q + 1.5 * 2^23), the E4M3
+//     code by cvt.rn.satfinite with the sign bit of y (quotients too small
+//     for an E4M3 subnormal keep their exact quotient's sign); other rows
+//     (all zeros, extreme magnitudes) by IEEE divisions, as the plain form.
+// The inputs must be finite (Inf and NaN give unspecified codes).
+// ----------------------------------------------------------------------------
+
+// Per-halfword unsigned max / min of two packed pairs.
+__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+__device__ __forceinline__ uint32_t min_u16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("min.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+// RN(a / Q) for Q = 127 or 448, exact for every a whose quotient and
+// residual stay normal: q0 = RN(a c) with c = RN(1/Q), one correction from
+// the exact residual a - Q q0.
+template <bool E4M3>
+__device__ __forceinline__ float norm_div_by_qmax(float a) {
+  constexpr float kQ = E4M3 ? 448.0f : 127.0f;
+  constexpr float kC = 1.0f / kQ;
+  const float q0 = __fmul_rn(a, kC);
+  return __fmaf_rn(__fmaf_rn(-kQ, q0, a), kC, q0);
+}
+
+// One square of a bf16 magnitude h != 0 outside the fast band, added to the
+// 128-bit accumulator in units of 2^(2 e_max - 110) (dropped below e_max - 48).
+__device__ __forceinline__ void norm_slow_square(uint32_t h, int emax, U128& acc) {
+  uint32_t n;
+  int e;
+  bf16_int_exp(h, n, e);
+  if (e < emax - 48) return;
+  const uint64_t v = uint64_t(n * n);
+  const int sh = 2 * (e - emax) + 96;
+  if (sh < 64) u128_add(acc, v << sh, sh ? v >> (64 - sh) : 0);
+  else u128_add(acc, 0, v << (sh - 64));
+}
+
+template <int V, bool E4M3, int SLOTS, int MAXT>
+__global__ void __launch_bounds__(MAXT, 512 / MAXT)
+    rmsnorm_quant_stream_kernel(const uint16_t* __restrict__ x, const float* __restrict__ g,
+                                float eps, int64_t M, int K, uint8_t* __restrict__ xq,
+                                float* __restrict__ sx, int* status) {
+  extern __shared__ __align__(128) uint8_t ring[];
+  __shared__ uint32_t red_mx[2][32];
+  __shared__ unsigned long long red_sum[2][2][32];
+  __shared__ uint32_t red_am[2][32];
+  __shared__ unsigned long long slow_lo[2], slow_hi[2];
+  __shared__ __align__(8) uint64_t bars[SLOTS];
+  const uint32_t row_bytes = uint32_t(K) * 2;
+  const int nchunk = K >> 3;
+  const int nthreads = blockDim.x, nwarps = nthreads >> 5;
+  const int64_t stride = gridDim.x;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  pdl_launch_dependents();
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < SLOTS; ++i) mbar_init(smem_u32(&bars[i]), 1);
+    fence_barrier_init();
+    slow_lo[0] = slow_lo[1] = slow_hi[0] = slow_hi[1] = 0ull;
+  }
+  // x and g may come from the kernel before this one, which may still read
+  // xq / sx
+  pdl_wait();
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < SLOTS; ++i) {
+      const int64_t m = blockIdx.x + i * stride;
+      if (m < M) {
+        mbar_arrive_expect_tx(smem_u32(&bars[i]), row_bytes);
+        bulk_load(smem_u32(ring + size_t(i) * row_bytes), x + m * K, row_bytes,
+                  smem_u32(&bars[i]));
+      }
+    }
+  }
+  __syncthreads();
+  int slot = 0, sel = 0;
+  uint32_t phase = 0;
+#pragma unroll 1
+  for (int64_t m = blockIdx.x; m < M; m += stride) {
+    const bool timed_out = !mbar_wait(smem_u32(&bars[slot]), phase);
+    const uint8_t* row = ring + size_t(slot) * row_bytes;
+    // 1. this thread's chunks, the largest magnitude pattern
+    uint4 raw[V];
+    uint32_t mx2 = 0, mn2 = 0xFFFFFFFFu;
+#pragma unroll
+    for (int j = 0; j < V; ++j) {
+      const int c = threadIdx.x + j * nthreads;
+      raw[j] = c < nchunk ? *reinterpret_cast<const uint4*>(row + size_t(c) * 16)
+                          : make_uint4(0u, 0u, 0u, 0u);
+      const uint32_t w[4] = {raw[j].x, raw[j].y, raw[j].z, raw[j].w};
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const uint32_t wm = w[t] & 0x7FFF7FFFu;
+        mx2 = max_u16x2(mx2, wm);
+        mn2 = min_u16x2(mn2, wm);
+      }
+    }
+    const uint32_t wmx = __reduce_max_sync(0xFFFFFFFFu, max(mx2 & 0xFFFFu, mx2 >> 16));
+    if (lane == 0) red_mx[sel][warp] = wmx;
+    if (__syncthreads_or(timed_out)) {
+      if (threadIdx.x == 0) {
+        record_status(status, kStatusTimeout);
+        // let the copies still in flight land before the CTA exits
+        for (int k = 0; k < SLOTS; ++k) {
+          if (m + k * stride < M) {
+            const int sk = (slot + k) % SLOTS;
+            (void)mbar_wait(smem_u32(&bars[sk]), phase ^ uint32_t(slot + k >= SLOTS));
+          }
+        }
+      }
+      break;
+    }
+    if (threadIdx.x == 0) {
+      // every thread has read this slot: refill it with the row SLOTS ahead,
+      // and clear the slow accumulator of the next row (its last readers,
+      // two rows back, are past barrier 3 of the previous row)
+      const int64_t mn = m + SLOTS * stride;
+      if (mn < M) {
+        fence_proxy_async_smem();
+        mbar_arrive_expect_tx(smem_u32(&bars[slot]), row_bytes);
+        bulk_load(smem_u32(ring + size_t(slot) * row_bytes), x + mn * K, row_bytes,
+                  smem_u32(&bars[slot]));
+      }
+      slow_lo[sel ^ 1] = 0ull;
+      slow_hi[sel ^ 1] = 0ull;
+    }
+    const uint32_t hmax =
+        __reduce_max_sync(0xFFFFFFFFu, red_mx[sel][lane < nwarps ? lane : 0]);
+    const int efmax = int(hmax >> 7);                 // 0 when the largest is subnormal
+    const int emax = efmax ? efmax - 127 : -126;
+    // bands A and B: normal elements with exponent field >= efmax - 32 (none
+    // when the largest is below 2^-94: the whole row takes the slow path)
+    const int lo_ef = efmax > 32 ? efmax - 32 : 256;
+    // 2. the exact sum of squares. Band A: the shift e - e_max + 16 in
+    // [0, 16], clamped at 32 (a = 0) below the band, negative offsets
+    // included; band B: 16 more, kept only when below 16 (one unsigned
+    // comparison excludes both band A and everything below band B)
+    uint64_t accA = 0, accB = 0;
+    if (efmax > 32) {
+      const uint32_t sh0 = uint32_t(16 - efmax);
+#pragma unroll
+      for (int j = 0; j < V; ++j) {
+        const uint32_t w[4] = {raw[j].x, raw[j].y, raw[j].z, raw[j].w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const uint32_t h = (i & 1) ? (w[i >> 1] >> 16) : (w[i >> 1] & 0xFFFFu);
+          const uint32_t n = 0x80u | (h & 0x7Fu);
+          const uint32_t shA = ((h >> 7) & 0xFFu) + sh0;
+          const uint32_t shB = shA + 16u;
+          const uint32_t aA = __funnelshift_lc(0u, n, shA);
+          const uint32_t aB = shB < 16u ? n << shB : 0u;
+          accA += uint64_t(aA) * aA;
+          accB += uint64_t(aB) * aB;
+        }
+      }
+    }
+    // some element of this thread below band B (zeros included: the slow
+    // loop skips them)
+    const bool slow = min(mn2 & 0xFFFFu, mn2 >> 16) < (uint32_t(lo_ef) << 7);
+    if (slow) {  // rare: this thread's small and subnormal elements (rolled
+                 // loops: the row goes through local memory here only)
+      U128 s128 = {0, 0};
+#pragma unroll 1
+      for (int j = 0; j < V; ++j) {
+        const uint32_t w[4] = {raw[j].x, raw[j].y, raw[j].z, raw[j].w};
+#pragma unroll 1
+        for (int i = 0; i < 8; ++i) {
+          const uint32_t h = ((i & 1) ? (w[i >> 1] >> 16) : w[i >> 1]) & 0x7FFFu;
+          if (h != 0u && int(h >> 7) < lo_ef) norm_slow_square(h, emax, s128);
+        }
+      }
+      const unsigned long long old = atomicAdd(&slow_lo[sel], s128.lo);
+      const unsigned long long carry = old + s128.lo < old ? 1ull : 0ull;
+      if (s128.hi + carry) atomicAdd(&slow_hi[sel], s128.hi + carry);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      accA += __shfl_xor_sync(0xFFFFFFFFu, accA, off);
+      accB += __shfl_xor_sync(0xFFFFFFFFu, accB, off);
+    }
+    if (lane == 0) {
+      red_sum[sel][0][warp] = accA;
+      red_sum[sel][1][warp] = accB;
+    }
+    __syncthreads();
+    uint64_t totA = lane < nwarps ? red_sum[sel][0][lane] : 0ull;
+    uint64_t totB = lane < nwarps ? red_sum[sel][1][lane] : 0ull;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      totA += __shfl_xor_sync(0xFFFFFFFFu, totA, off);
+      totB += __shfl_xor_sync(0xFFFFFFFFu, totB, off);
+    }
+    // in the slow part's units: band A 2^64, band B 2^32
+    U128 ss128 = {slow_lo[sel], slow_hi[sel]};
+    u128_add(ss128, totB << 32, (totB >> 32) + totA);
+    const double ss =
+        hmax ? u128_to_double_scaled(ss128, 2 * emax - 110) : 0.0;
+    const double mean = __ddiv_rn(ss, double(K));
+    const double t = __dsqrt_rn(__dadd_rn(mean, double(eps)));
+    const float r = __double2float_rn(__ddiv_rn(1.0, t));
+    // 3. y = (x * r) * g, the largest |y|
+    const uint64_t r2 = f2_make(r, r);
+    uint64_t y2[V][4];
+    float am0 = 0.0f, am1 = 0.0f;
+#pragma unroll
+    for (int j = 0; j < V; ++j) {
+      const uint32_t w[4] = {raw[j].x, raw[j].y, raw[j].z, raw[j].w};
+      // the gains from L1 (the same K floats for every row); zeros past the row
+      const int c = threadIdx.x + j * nthreads;
+      ulonglong2 ga = make_ulonglong2(0ull, 0ull), gb = ga;
+      if (c < nchunk) {
+        ga = __ldg(reinterpret_cast<const ulonglong2*>(g) + 2 * c);
+        gb = __ldg(reinterpret_cast<const ulonglong2*>(g) + 2 * c + 1);
+      }
+      const uint64_t g2[4] = {ga.x, ga.y, gb.x, gb.y};
+#pragma unroll
+      for (int t2 = 0; t2 < 4; ++t2) {
+        y2[j][t2] = f2_mul(f2_mul(f2_make(bf16_lo(w[t2]), bf16_hi(w[t2])), r2), g2[t2]);
+        float a, b;
+        f2_split(y2[j][t2], a, b);
+        if (t2 & 1) am1 = max3_nan(am1, fabsf(a), fabsf(b));
+        else am0 = max3_nan(am0, fabsf(a), fabsf(b));
+      }
+    }
+    const uint32_t wam = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(fmaxf(am0, am1)));
+    if (lane == 0) red_am[sel][warp] = wam;
+    __syncthreads();
+    const float amax = __uint_as_float(
+        __reduce_max_sync(0xFFFFFFFFu, red_am[sel][lane < nwarps ? lane : 0]));
+    uint8_t* out = xq + m * K;
+    // 4. the scale and the codes
+    if (amax >= 0x1p-60f && amax <= 0x1p100f) {
+      const float scale = norm_div_by_qmax<E4M3>(amax);
+      if (threadIdx.x == 0) sx[m] = scale;
+      const float rs = __frcp_rn(scale);
+      const uint64_t rs2 = f2_make(rs, rs), nsc2 = f2_make(-scale, -scale);
+#pragma unroll
+      for (int j = 0; j < V; ++j) {
+        const int c = threadIdx.x + j * nthreads;
+        if (c >= nchunk) continue;
+        uint64_t qq[4];
+#pragma unroll
+        for (int t2 = 0; t2 < 4; ++t2) {
+          const uint64_t a2 = y2[j][t2];
+          uint64_t q = f2_mul(a2, rs2);
+          q = f2_fma(f2_fma(nsc2, q, a2), rs2, q);
+          qq[t2] = f2_fma(f2_fma(nsc2, q, a2), rs2, q);
+        }
+        uint2 o;
+        if constexpr (E4M3) {
+          uint32_t cd[4], sg[4];
+#pragma unroll
+          for (int t2 = 0; t2 < 4; ++t2) {
+            float lo, hi;
+            f2_split(qq[t2], lo, hi);
+            cd[t2] = pack_e4m3x2(lo, hi);
+            float ylo, yhi;
+            f2_split(y2[j][t2], ylo, yhi);
+            // the signs of y, as the sign bits of two code bytes
+            sg[t2] = __byte_perm(__float_as_uint(ylo), __float_as_uint(yhi), 0x0073) & 0x8080u;
+          }
+          o.x = ((cd[0] | (cd[1] << 16)) & 0x7F7F7F7Fu) | sg[0] | (sg[1] << 16);
+          o.y = ((cd[2] | (cd[3] << 16)) & 0x7F7F7F7Fu) | sg[2] | (sg[3] << 16);
+        } else {
+          // rne(q) is the integer part of q + 1.5 * 2^23 (|q| <= 127.00001);
+          // its low byte is the two's-complement code
+          const uint64_t mg2 = f2_make(12582912.0f, 12582912.0f);
+          uint32_t tb[8];
+#pragma unroll
+          for (int t2 = 0; t2 < 4; ++t2) {
+            float lo, hi;
+            f2_split(f2_add(qq[t2], mg2), lo, hi);
+            tb[2 * t2] = __float_as_uint(lo);
+            tb[2 * t2 + 1] = __float_as_uint(hi);
+          }
+          o.x = __byte_perm(__byte_perm(tb[0], tb[1], 0x0040), __byte_perm(tb[2], tb[3], 0x0040),
+                            0x5410);
+          o.y = __byte_perm(__byte_perm(tb[4], tb[5], 0x0040), __byte_perm(tb[6], tb[7], 0x0040),
+                            0x5410);
+        }
+        *reinterpret_cast<uint2*>(out + size_t(c) * 8) = o;
+      }
+    } else {
+      const float scale = __fdiv_rn(amax, E4M3 ? 448.0f : 127.0f);
+      if (threadIdx.x == 0) sx[m] = scale;
+#pragma unroll
+      for (int j = 0; j < V; ++j) {
+        const int c = threadIdx.x + j * nthreads;
+        if (c >= nchunk) continue;
+        float q[8];
+#pragma unroll
+        for (int t2 = 0; t2 < 4; ++t2) {
+          float lo, hi;
+          f2_split(y2[j][t2], lo, hi);
+          q[2 * t2] = scale == 0.0f ? 0.0f : __fdiv_rn(lo, scale);
+          q[2 * t2 + 1] = scale == 0.0f ? 0.0f : __fdiv_rn(hi, scale);
+        }
+        uint2 o;
+        if constexpr (E4M3) {
+          o.x = pack_e4m3x2(q[0], q[1]) | (pack_e4m3x2(q[2], q[3]) << 16);
+          o.y = pack_e4m3x2(q[4], q[5]) | (pack_e4m3x2(q[6], q[7]) << 16);
+          if (scale == 0.0f) o = make_uint2(0u, 0u);
+        } else {
+          uint32_t b[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) b[i] = uint32_t(max(-127, min(127, __float2int_rn(q[i])))) & 0xFFu;
+          o.x = b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24);
+          o.y = b[4] | (b[5] << 8) | (b[6] << 16) | (b[7] << 24);
+        }
+        *reinterpret_cast<uint2*>(out + size_t(c) * 8) = o;
+      }
+    }
+    sel ^= 1;
+    if (++slot == SLOTS) {
+      slot = 0;
+      phase ^= 1u;
+    }
+  }
+}
+
 }  // namespace sqk
 
 namespace sqh {
@@ -239,11 +594,55 @@ using namespace sqk;
 
 int rmsnorm_quant_max_k() { return kNormMaxK; }
 
+static int norm_sm_count() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+// The streaming form: V = 4 chunks per thread, the CTA as wide as the row
+// needs (a multiple of 32 threads, at most MAXT), SLOTS rows in flight, as
+// many CTAs as fit on the SMs at once (no more than there are rows).
+template <int MAXT>
+static cudaError_t launch_norm_stream(const uint16_t* x, const float* g, float eps, int64_t M,
+                                      int K, bool e4m3, uint8_t* xq, float* sx,
+                                      cudaStream_t st) {
+  constexpr int V = 4, SLOTS = 4;
+  const int nchunk = K >> 3;
+  const int threads = ((nchunk + V - 1) / V + 31) / 32 * 32;
+  const size_t smem = size_t(SLOTS) * size_t(K) * 2;
+  int* status = status_ptr();
+  auto kern = e4m3 ? rmsnorm_quant_stream_kernel<V, true, SLOTS, MAXT>
+                   : rmsnorm_quant_stream_kernel<V, false, SLOTS, MAXT>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       int(smem));
+  if (e != cudaSuccess) return e;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem) !=
+          cudaSuccess || per_sm < 1)
+    per_sm = 1;
+  int64_t grid = int64_t(per_sm) * norm_sm_count();
+  if (grid > M) grid = M;
+  return launch_pdl(kern, unsigned(grid), threads, smem, st, x, g, eps, M, K, xq, sx, status);
+}
+
 cudaError_t launch_rmsnorm_quant(const uint16_t* x, const float* g, float eps, int64_t M,
                                  int64_t K, bool e4m3, void* xq, float* sx, float* xn,
                                  cudaStream_t st) {
-  // one CTA per row, at most a few waves' worth resident: rows beyond the
-  // grid are taken in turn
+  if (!xn) {
+    const int nchunk = int(K >> 3);  // <= 2048
+    uint8_t* q = static_cast<uint8_t*>(xq);
+    if (nchunk <= 4 * 128) return launch_norm_stream<128>(x, g, eps, M, int(K), e4m3, q, sx, st);
+    if (nchunk <= 4 * 256) return launch_norm_stream<256>(x, g, eps, M, int(K), e4m3, q, sx, st);
+    return launch_norm_stream<512>(x, g, eps, M, int(K), e4m3, q, sx, st);
+  }
+  // the plain form: one CTA per row, at most a few waves' worth resident:
+  // rows beyond the grid are taken in turn
   const int64_t grid = M < 148 * 16 ? M : 148 * 16;
   const size_t smem = size_t(K) * 2;  // the staged row (at most 32 KB: no opt-in needed)
   if (e4m3)
