@@ -305,6 +305,134 @@ __device__ __forceinline__ void norm_slow_square(uint32_t h, int emax, U128& acc
   else u128_add(acc, 0, v << (sh - 64));
 }
 
+// The two bands' sums of squares of one 8-element chunk (bf16 pairs in u),
+// sh0 = 16 - efmax as an unsigned offset. Band A: the shift e - e_max + 16
+// in [0, 16], clamped at 32 (a = 0) below the band, negative offsets
+// included; band B: 16 more, kept only when below 16 (one unsigned comparison
+// excludes both band A and everything below band B).
+__device__ __forceinline__ void norm_band_squares(const uint4& u, uint32_t sh0, uint64_t& accA,
+                                                  uint64_t& accB) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint32_t h = (i & 1) ? (w[i >> 1] >> 16) : (w[i >> 1] & 0xFFFFu);
+    const uint32_t n = 0x80u | (h & 0x7Fu);
+    const uint32_t shA = ((h >> 7) & 0xFFu) + sh0;
+    const uint32_t shB = shA + 16u;
+    const uint32_t aA = __funnelshift_lc(0u, n, shA);
+    const uint32_t aB = shB < 16u ? n << shB : 0u;
+    accA += uint64_t(aA) * aA;
+    accB += uint64_t(aB) * aB;
+  }
+}
+
+// The squares of one chunk's elements below both bands (nonzero, exponent
+// field < lo_ef) into the 128-bit remainder.
+__device__ __forceinline__ void norm_slow_chunk(const uint4& u, int lo_ef, int emax, U128& acc) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint32_t h = ((i & 1) ? (w[i >> 1] >> 16) : w[i >> 1]) & 0x7FFFu;
+    if (h != 0u && int(h >> 7) < lo_ef) norm_slow_square(h, emax, acc);
+  }
+}
+
+// r = binary32(1 / sqrt(ss / K + eps)) from the exact sum: the remainder in
+// units of 2^(2 e_max - 110), band A's sum 2^64 and band B's 2^32 of them.
+__device__ __forceinline__ float norm_rinv(U128 rest, uint64_t totA, uint64_t totB, uint32_t hmax,
+                                           int emax, int K, float eps) {
+  u128_add(rest, totB << 32, (totB >> 32) + totA);
+  const double ss = hmax ? u128_to_double_scaled(rest, 2 * emax - 110) : 0.0;
+  const double mean = __ddiv_rn(ss, double(K));
+  const double t = __dsqrt_rn(__dadd_rn(mean, double(eps)));
+  return __double2float_rn(__ddiv_rn(1.0, t));
+}
+
+// y = (x * r) * g for one chunk, as four packed pairs; g8 = the chunk's 8 gains.
+__device__ __forceinline__ void norm_apply(const uint4& u, uint64_t r2, const float* g8,
+                                           uint64_t (&y2)[4]) {
+  const ulonglong2 ga = __ldg(reinterpret_cast<const ulonglong2*>(g8));
+  const ulonglong2 gb = __ldg(reinterpret_cast<const ulonglong2*>(g8) + 1);
+  const uint64_t g2[4] = {ga.x, ga.y, gb.x, gb.y};
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int t = 0; t < 4; ++t)
+    y2[t] = f2_mul(f2_mul(f2_make(bf16_lo(w[t]), bf16_hi(w[t])), r2), g2[t]);
+}
+
+// The codes of one chunk for a row whose largest |y| is in [2^-60, 2^100]:
+// q = RN(y / sx) by two corrections of the reciprocal product (rs2 = RN(1/sx),
+// nsc2 = -sx, as pairs); INT8: the low byte of RN(q + 1.5 * 2^23), i.e.
+// rne(q) (|q| <= 127.00001); E4M3: cvt.rn.satfinite with the sign bit of y.
+template <bool E4M3>
+__device__ __forceinline__ uint2 norm_codes_fast(const uint64_t (&y2)[4], uint64_t rs2,
+                                                 uint64_t nsc2) {
+  uint64_t qq[4];
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    const uint64_t a2 = y2[t];
+    uint64_t q = f2_mul(a2, rs2);
+    q = f2_fma(f2_fma(nsc2, q, a2), rs2, q);
+    qq[t] = f2_fma(f2_fma(nsc2, q, a2), rs2, q);
+  }
+  uint2 o;
+  if constexpr (E4M3) {
+    uint32_t cd[4], sg[4];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      float lo, hi;
+      f2_split(qq[t], lo, hi);
+      cd[t] = pack_e4m3x2(lo, hi);
+      float ylo, yhi;
+      f2_split(y2[t], ylo, yhi);
+      // the signs of y, as the sign bits of two code bytes
+      sg[t] = __byte_perm(__float_as_uint(ylo), __float_as_uint(yhi), 0x0073) & 0x8080u;
+    }
+    o.x = ((cd[0] | (cd[1] << 16)) & 0x7F7F7F7Fu) | sg[0] | (sg[1] << 16);
+    o.y = ((cd[2] | (cd[3] << 16)) & 0x7F7F7F7Fu) | sg[2] | (sg[3] << 16);
+  } else {
+    const uint64_t mg2 = f2_make(12582912.0f, 12582912.0f);
+    uint32_t tb[8];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      float lo, hi;
+      f2_split(f2_add(qq[t], mg2), lo, hi);
+      tb[2 * t] = __float_as_uint(lo);
+      tb[2 * t + 1] = __float_as_uint(hi);
+    }
+    o.x = __byte_perm(__byte_perm(tb[0], tb[1], 0x0040), __byte_perm(tb[2], tb[3], 0x0040), 0x5410);
+    o.y = __byte_perm(__byte_perm(tb[4], tb[5], 0x0040), __byte_perm(tb[6], tb[7], 0x0040), 0x5410);
+  }
+  return o;
+}
+
+// The codes of one chunk by IEEE divisions (rows outside that window; scale
+// 0 gives zero codes), as the plain form.
+template <bool E4M3>
+__device__ __forceinline__ uint2 norm_codes_exact(const uint64_t (&y2)[4], float scale) {
+  float q[8];
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    float lo, hi;
+    f2_split(y2[t], lo, hi);
+    q[2 * t] = scale == 0.0f ? 0.0f : __fdiv_rn(lo, scale);
+    q[2 * t + 1] = scale == 0.0f ? 0.0f : __fdiv_rn(hi, scale);
+  }
+  uint2 o;
+  if constexpr (E4M3) {
+    o.x = pack_e4m3x2(q[0], q[1]) | (pack_e4m3x2(q[2], q[3]) << 16);
+    o.y = pack_e4m3x2(q[4], q[5]) | (pack_e4m3x2(q[6], q[7]) << 16);
+    if (scale == 0.0f) o = make_uint2(0u, 0u);
+  } else {
+    uint32_t b[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) b[i] = uint32_t(max(-127, min(127, __float2int_rn(q[i])))) & 0xFFu;
+    o.x = b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24);
+    o.y = b[4] | (b[5] << 8) | (b[6] << 16) | (b[7] << 24);
+  }
+  return o;
+}
+
 template <int V, bool E4M3, int SLOTS, int MAXT>
 __global__ void __launch_bounds__(MAXT, 512 / MAXT)
     rmsnorm_quant_stream_kernel(const uint16_t* __restrict__ x, const float* __restrict__ g,
@@ -407,20 +535,7 @@ __global__ void __launch_bounds__(MAXT, 512 / MAXT)
     if (efmax > 32) {
       const uint32_t sh0 = uint32_t(16 - efmax);
 #pragma unroll
-      for (int j = 0; j < V; ++j) {
-        const uint32_t w[4] = {raw[j].x, raw[j].y, raw[j].z, raw[j].w};
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const uint32_t h = (i & 1) ? (w[i >> 1] >> 16) : (w[i >> 1] & 0xFFFFu);
-          const uint32_t n = 0x80u | (h & 0x7Fu);
-          const uint32_t shA = ((h >> 7) & 0xFFu) + sh0;
-          const uint32_t shB = shA + 16u;
-          const uint32_t aA = __funnelshift_lc(0u, n, shA);
-          const uint32_t aB = shB < 16u ? n << shB : 0u;
-          accA += uint64_t(aA) * aA;
-          accB += uint64_t(aB) * aB;
-        }
-      }
+      for (int j = 0; j < V; ++j) norm_band_squares(raw[j], sh0, accA, accB);
     }
     // some element of this thread below band B (zeros included: the slow
     // loop skips them)
@@ -429,14 +544,7 @@ __global__ void __launch_bounds__(MAXT, 512 / MAXT)
                  // loops: the row goes through local memory here only)
       U128 s128 = {0, 0};
 #pragma unroll 1
-      for (int j = 0; j < V; ++j) {
-        const uint32_t w[4] = {raw[j].x, raw[j].y, raw[j].z, raw[j].w};
-#pragma unroll 1
-        for (int i = 0; i < 8; ++i) {
-          const uint32_t h = ((i & 1) ? (w[i >> 1] >> 16) : w[i >> 1]) & 0x7FFFu;
-          if (h != 0u && int(h >> 7) < lo_ef) norm_slow_square(h, emax, s128);
-        }
-      }
+      for (int j = 0; j < V; ++j) norm_slow_chunk(raw[j], lo_ef, emax, s128);
       const unsigned long long old = atomicAdd(&slow_lo[sel], s128.lo);
       const unsigned long long carry = old + s128.lo < old ? 1ull : 0ull;
       if (s128.hi + carry) atomicAdd(&slow_hi[sel], s128.hi + carry);
@@ -458,32 +566,23 @@ __global__ void __launch_bounds__(MAXT, 512 / MAXT)
       totA += __shfl_xor_sync(0xFFFFFFFFu, totA, off);
       totB += __shfl_xor_sync(0xFFFFFFFFu, totB, off);
     }
-    // in the slow part's units: band A 2^64, band B 2^32
-    U128 ss128 = {slow_lo[sel], slow_hi[sel]};
-    u128_add(ss128, totB << 32, (totB >> 32) + totA);
-    const double ss =
-        hmax ? u128_to_double_scaled(ss128, 2 * emax - 110) : 0.0;
-    const double mean = __ddiv_rn(ss, double(K));
-    const double t = __dsqrt_rn(__dadd_rn(mean, double(eps)));
-    const float r = __double2float_rn(__ddiv_rn(1.0, t));
+    const float r = norm_rinv(U128{slow_lo[sel], slow_hi[sel]}, totA, totB, hmax, emax, K, eps);
     // 3. y = (x * r) * g, the largest |y|
     const uint64_t r2 = f2_make(r, r);
     uint64_t y2[V][4];
     float am0 = 0.0f, am1 = 0.0f;
 #pragma unroll
     for (int j = 0; j < V; ++j) {
-      const uint32_t w[4] = {raw[j].x, raw[j].y, raw[j].z, raw[j].w};
-      // the gains from L1 (the same K floats for every row); zeros past the row
       const int c = threadIdx.x + j * nthreads;
-      ulonglong2 ga = make_ulonglong2(0ull, 0ull), gb = ga;
+      // the gains from L1 (the same K floats for every row); none past the row
       if (c < nchunk) {
-        ga = __ldg(reinterpret_cast<const ulonglong2*>(g) + 2 * c);
-        gb = __ldg(reinterpret_cast<const ulonglong2*>(g) + 2 * c + 1);
+        norm_apply(raw[j], r2, g + size_t(c) * 8, y2[j]);
+      } else {
+#pragma unroll
+        for (int t2 = 0; t2 < 4; ++t2) y2[j][t2] = 0ull;
       }
-      const uint64_t g2[4] = {ga.x, ga.y, gb.x, gb.y};
 #pragma unroll
       for (int t2 = 0; t2 < 4; ++t2) {
-        y2[j][t2] = f2_mul(f2_mul(f2_make(bf16_lo(w[t2]), bf16_hi(w[t2])), r2), g2[t2]);
         float a, b;
         f2_split(y2[j][t2], a, b);
         if (t2 & 1) am1 = max3_nan(am1, fabsf(a), fabsf(b));
@@ -505,48 +604,8 @@ __global__ void __launch_bounds__(MAXT, 512 / MAXT)
 #pragma unroll
       for (int j = 0; j < V; ++j) {
         const int c = threadIdx.x + j * nthreads;
-        if (c >= nchunk) continue;
-        uint64_t qq[4];
-#pragma unroll
-        for (int t2 = 0; t2 < 4; ++t2) {
-          const uint64_t a2 = y2[j][t2];
-          uint64_t q = f2_mul(a2, rs2);
-          q = f2_fma(f2_fma(nsc2, q, a2), rs2, q);
-          qq[t2] = f2_fma(f2_fma(nsc2, q, a2), rs2, q);
-        }
-        uint2 o;
-        if constexpr (E4M3) {
-          uint32_t cd[4], sg[4];
-#pragma unroll
-          for (int t2 = 0; t2 < 4; ++t2) {
-            float lo, hi;
-            f2_split(qq[t2], lo, hi);
-            cd[t2] = pack_e4m3x2(lo, hi);
-            float ylo, yhi;
-            f2_split(y2[j][t2], ylo, yhi);
-            // the signs of y, as the sign bits of two code bytes
-            sg[t2] = __byte_perm(__float_as_uint(ylo), __float_as_uint(yhi), 0x0073) & 0x8080u;
-          }
-          o.x = ((cd[0] | (cd[1] << 16)) & 0x7F7F7F7Fu) | sg[0] | (sg[1] << 16);
-          o.y = ((cd[2] | (cd[3] << 16)) & 0x7F7F7F7Fu) | sg[2] | (sg[3] << 16);
-        } else {
-          // rne(q) is the integer part of q + 1.5 * 2^23 (|q| <= 127.00001);
-          // its low byte is the two's-complement code
-          const uint64_t mg2 = f2_make(12582912.0f, 12582912.0f);
-          uint32_t tb[8];
-#pragma unroll
-          for (int t2 = 0; t2 < 4; ++t2) {
-            float lo, hi;
-            f2_split(f2_add(qq[t2], mg2), lo, hi);
-            tb[2 * t2] = __float_as_uint(lo);
-            tb[2 * t2 + 1] = __float_as_uint(hi);
-          }
-          o.x = __byte_perm(__byte_perm(tb[0], tb[1], 0x0040), __byte_perm(tb[2], tb[3], 0x0040),
-                            0x5410);
-          o.y = __byte_perm(__byte_perm(tb[4], tb[5], 0x0040), __byte_perm(tb[6], tb[7], 0x0040),
-                            0x5410);
-        }
-        *reinterpret_cast<uint2*>(out + size_t(c) * 8) = o;
+        if (c < nchunk)
+          *reinterpret_cast<uint2*>(out + size_t(c) * 8) = norm_codes_fast<E4M3>(y2[j], rs2, nsc2);
       }
     } else {
       const float scale = __fdiv_rn(amax, E4M3 ? 448.0f : 127.0f);
@@ -554,31 +613,177 @@ __global__ void __launch_bounds__(MAXT, 512 / MAXT)
 #pragma unroll
       for (int j = 0; j < V; ++j) {
         const int c = threadIdx.x + j * nthreads;
-        if (c >= nchunk) continue;
-        float q[8];
-#pragma unroll
-        for (int t2 = 0; t2 < 4; ++t2) {
-          float lo, hi;
-          f2_split(y2[j][t2], lo, hi);
-          q[2 * t2] = scale == 0.0f ? 0.0f : __fdiv_rn(lo, scale);
-          q[2 * t2 + 1] = scale == 0.0f ? 0.0f : __fdiv_rn(hi, scale);
-        }
-        uint2 o;
-        if constexpr (E4M3) {
-          o.x = pack_e4m3x2(q[0], q[1]) | (pack_e4m3x2(q[2], q[3]) << 16);
-          o.y = pack_e4m3x2(q[4], q[5]) | (pack_e4m3x2(q[6], q[7]) << 16);
-          if (scale == 0.0f) o = make_uint2(0u, 0u);
-        } else {
-          uint32_t b[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) b[i] = uint32_t(max(-127, min(127, __float2int_rn(q[i])))) & 0xFFu;
-          o.x = b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24);
-          o.y = b[4] | (b[5] << 8) | (b[6] << 16) | (b[7] << 24);
-        }
-        *reinterpret_cast<uint2*>(out + size_t(c) * 8) = o;
+        if (c < nchunk)
+          *reinterpret_cast<uint2*>(out + size_t(c) * 8) = norm_codes_exact<E4M3>(y2[j], scale);
       }
     }
     sel ^= 1;
+    if (++slot == SLOTS) {
+      slot = 0;
+      phase ^= 1u;
+    }
+  }
+}
+
+// ----------------------------------------------------------------------------
+// The warp form (many rows of at most 8192 elements): every warp normalizes
+// and quantizes whole rows by itself -- rows w, w + W, ... for the grid's W
+// warps -- with its own SLOTS-row ring of bulk copies in shared memory and
+// its own barriers, so no block barrier and no cross-warp reduction is on a
+// row's path. Each lane takes the chunks c = lane + 32 j and re-reads them
+// from shared memory in every pass; the arithmetic is that of the streaming
+// form, chunk by chunk (the 128-bit remainder reduced by shuffles instead of
+// shared atomics).
+// ----------------------------------------------------------------------------
+constexpr int kNormWarpMaxK = 8192;
+constexpr int kNormWarpSlots = 1;
+
+template <bool E4M3>
+__global__ void __launch_bounds__(256)
+    rmsnorm_quant_warp_kernel(const uint16_t* __restrict__ x, const float* __restrict__ g,
+                              float eps, int64_t M, int K, uint8_t* __restrict__ xq,
+                              float* __restrict__ sx, int* status) {
+  constexpr int SLOTS = kNormWarpSlots;
+  extern __shared__ __align__(128) uint8_t ring[];  // [warps][SLOTS][K] bf16
+  __shared__ __align__(8) uint64_t bars[8][SLOTS];
+  const uint32_t row_bytes = uint32_t(K) * 2;
+  const int nchunk = K >> 3;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t nw = blockDim.x >> 5;
+  const int64_t w0 = int64_t(blockIdx.x) * nw + warp, stride = int64_t(gridDim.x) * nw;
+  uint8_t* my_ring = ring + size_t(warp) * SLOTS * row_bytes;
+  pdl_launch_dependents();
+  if (lane == 0) {
+    for (int i = 0; i < SLOTS; ++i) mbar_init(smem_u32(&bars[warp][i]), 1);
+    fence_barrier_init();
+  }
+  __syncwarp();
+  // x and g may come from the kernel before this one, which may still read
+  // xq / sx
+  pdl_wait();
+  if (lane == 0) {
+    for (int i = 0; i < SLOTS; ++i) {
+      const int64_t m = w0 + i * stride;
+      if (m < M) {
+        mbar_arrive_expect_tx(smem_u32(&bars[warp][i]), row_bytes);
+        bulk_load(smem_u32(my_ring + size_t(i) * row_bytes), x + m * K, row_bytes,
+                  smem_u32(&bars[warp][i]));
+      }
+    }
+  }
+  int slot = 0;
+  uint32_t phase = 0;
+#pragma unroll 1
+  for (int64_t m = w0; m < M; m += stride) {
+    if (__any_sync(0xFFFFFFFFu, !mbar_wait(smem_u32(&bars[warp][slot]), phase))) {
+      if (lane == 0) {
+        record_status(status, kStatusTimeout);
+        // let the copies still in flight land before the warp leaves
+        for (int k = 0; k < SLOTS; ++k) {
+          if (m + k * stride < M) {
+            const int sk = (slot + k) % SLOTS;
+            (void)mbar_wait(smem_u32(&bars[warp][sk]), phase ^ uint32_t(slot + k >= SLOTS));
+          }
+        }
+      }
+      __syncwarp();
+      break;
+    }
+    const uint4* row = reinterpret_cast<const uint4*>(my_ring + size_t(slot) * row_bytes);
+    // 1. the largest and smallest magnitude patterns
+    uint32_t mx2 = 0, mn2 = 0xFFFFFFFFu;
+#pragma unroll 4
+    for (int c = lane; c < nchunk; c += 32) {
+      const uint4 u = row[c];
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const uint32_t wm = w[t] & 0x7FFF7FFFu;
+        mx2 = max_u16x2(mx2, wm);
+        mn2 = min_u16x2(mn2, wm);
+      }
+    }
+    const uint32_t hmax = __reduce_max_sync(0xFFFFFFFFu, max(mx2 & 0xFFFFu, mx2 >> 16));
+    const int efmax = int(hmax >> 7);
+    const int emax = efmax ? efmax - 127 : -126;
+    const int lo_ef = efmax > 32 ? efmax - 32 : 256;
+    // 2. the exact sum of squares
+    uint64_t accA = 0, accB = 0;
+    if (efmax > 32) {
+      const uint32_t sh0 = uint32_t(16 - efmax);
+#pragma unroll 4
+      for (int c = lane; c < nchunk; c += 32) norm_band_squares(row[c], sh0, accA, accB);
+    }
+    U128 rest = {0, 0};
+    if (min(mn2 & 0xFFFFu, mn2 >> 16) < (uint32_t(lo_ef) << 7)) {
+#pragma unroll 1
+      for (int c = lane; c < nchunk; c += 32) norm_slow_chunk(row[c], lo_ef, emax, rest);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      accA += __shfl_xor_sync(0xFFFFFFFFu, accA, off);
+      accB += __shfl_xor_sync(0xFFFFFFFFu, accB, off);
+    }
+    if (__any_sync(0xFFFFFFFFu, (rest.lo | rest.hi) != 0ull)) {
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        const uint64_t lo = __shfl_xor_sync(0xFFFFFFFFu, rest.lo, off);
+        const uint64_t hi = __shfl_xor_sync(0xFFFFFFFFu, rest.hi, off);
+        u128_add(rest, lo, hi);
+      }
+    }
+    const float r = norm_rinv(rest, accA, accB, hmax, emax, K, eps);
+    const uint64_t r2 = f2_make(r, r);
+    // 3. the largest |y|, y = (x * r) * g
+    float am0 = 0.0f, am1 = 0.0f;
+#pragma unroll 4
+    for (int c = lane; c < nchunk; c += 32) {
+      uint64_t y2[4];
+      norm_apply(row[c], r2, g + size_t(c) * 8, y2);
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        float a, b;
+        f2_split(y2[t], a, b);
+        if (t & 1) am1 = max3_nan(am1, fabsf(a), fabsf(b));
+        else am0 = max3_nan(am0, fabsf(a), fabsf(b));
+      }
+    }
+    const float amax =
+        __uint_as_float(__reduce_max_sync(0xFFFFFFFFu, __float_as_uint(fmaxf(am0, am1))));
+    // 4. the scale and the codes (y recomputed, bit for bit the same)
+    uint2* out = reinterpret_cast<uint2*>(xq + m * K);
+    if (amax >= 0x1p-60f && amax <= 0x1p100f) {
+      const float scale = norm_div_by_qmax<E4M3>(amax);
+      if (lane == 0) sx[m] = scale;
+      const float rs = __frcp_rn(scale);
+      const uint64_t rs2 = f2_make(rs, rs), nsc2 = f2_make(-scale, -scale);
+#pragma unroll 4
+      for (int c = lane; c < nchunk; c += 32) {
+        uint64_t y2[4];
+        norm_apply(row[c], r2, g + size_t(c) * 8, y2);
+        out[c] = norm_codes_fast<E4M3>(y2, rs2, nsc2);
+      }
+    } else {
+      const float scale = __fdiv_rn(amax, E4M3 ? 448.0f : 127.0f);
+      if (lane == 0) sx[m] = scale;
+#pragma unroll 1
+      for (int c = lane; c < nchunk; c += 32) {
+        uint64_t y2[4];
+        norm_apply(row[c], r2, g + size_t(c) * 8, y2);
+        out[c] = norm_codes_exact<E4M3>(y2, scale);
+      }
+    }
+    // every lane has read this slot: refill it with the row SLOTS ahead
+    __syncwarp();
+    if (lane == 0) {
+      const int64_t mn = m + SLOTS * stride;
+      if (mn < M) {
+        fence_proxy_async_smem();
+        mbar_arrive_expect_tx(smem_u32(&bars[warp][slot]), row_bytes);
+        bulk_load(smem_u32(my_ring + size_t(slot) * row_bytes), x + mn * K, row_bytes,
+                  smem_u32(&bars[warp][slot]));
+      }
+    }
     if (++slot == SLOTS) {
       slot = 0;
       phase ^= 1u;
@@ -634,6 +839,26 @@ static cudaError_t launch_norm_stream(const uint16_t* x, const float* g, float e
 cudaError_t launch_rmsnorm_quant(const uint16_t* x, const float* g, float eps, int64_t M,
                                  int64_t K, bool e4m3, void* xq, float* sx, float* xn,
                                  cudaStream_t st) {
+  if (!xn && K <= kNormWarpMaxK && M >= 4LL * norm_sm_count()) {
+    // the warp form: up to 8 warps per CTA, each with SLOTS rows in flight,
+    // about 96 KB of ring per CTA; as many CTAs as fit, no more than the rows
+    // need
+    const int per_row = int(K) * 2 * kNormWarpSlots;
+    const int warps = max(1, min(8, 98304 / per_row));
+    const size_t smem = size_t(warps) * per_row;
+    auto kern = e4m3 ? rmsnorm_quant_warp_kernel<true> : rmsnorm_quant_warp_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         int(smem));
+    if (e != cudaSuccess) return e;
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, warps * 32, smem) !=
+            cudaSuccess || per_sm < 1)
+      per_sm = 1;
+    int64_t grid = int64_t(per_sm) * norm_sm_count();
+    grid = min(grid, (M + warps - 1) / warps);
+    return launch_pdl(kern, unsigned(grid), warps * 32, smem, st, x, g, eps, M, int(K),
+                      static_cast<uint8_t*>(xq), sx, status_ptr());
+  }
   if (!xn) {
     const int nchunk = int(K >> 3);  // <= 2048
     uint8_t* q = static_cast<uint8_t*>(xq);
