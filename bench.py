@@ -91,6 +91,7 @@ PROFILED_TRAFFIC = {
     ("quant", "fp8_tensor_4096x4096x14336"): (33.577984e6 + 0.005632e6, "e5dd1a242fc0384b"),
     ("quant", "prefill_512x4096x4096"): (4.287744e6 + 0.0, "e5dd1a242fc0384b"),
     ("quant", "decode_16x8192x28672"): (0.362240e6 + 0.0, "e5dd1a242fc0384b"),
+    ("norm", "mlp_up_rmsnorm_4096x4096x14336"): (33.620480e6 + 0.036608e6, "48f492482ffe3662"),
 }
 KERNEL_SOURCES = {"gemm": ("sq_gemm.cu", "sq_common.cuh"),
                   "gemm_wonly": ("sq_gemm_wonly.cu", "sq_common.cuh"),
@@ -162,7 +163,10 @@ def quant_kernel_name(case):
     if weight_bits(case):
         return None
     if case.norm_eps:
-        return "rmsnorm_quant_stream_kernel"
+        # one warp per row for many rows of at most 8192 elements, else the
+        # block-per-row streaming form
+        return ("rmsnorm_quant_warp_kernel" if case.K <= 8192 and case.M >= 4 * sms
+                else "rmsnorm_quant_stream_kernel")
     if case.act_scaling == "tensor":
         return "quant_act_tensor_kernel"
     if case.x_dtype != "bf16" or case.K // 8 > 256 * 8:

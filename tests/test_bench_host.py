@@ -45,7 +45,7 @@ def test_activation_kernel_per_workload(bench):
     assert bench.quant_kernel_name(workloads.FP8_DOWN) == "quant_act_stream_kernel"
     assert bench.quant_kernel_name(workloads.DECODE) == "quant_act_fast_kernel"      # 16 rows
     assert bench.quant_kernel_name(workloads.FP8_TENSOR) == "quant_act_tensor_kernel"
-    assert bench.quant_kernel_name(workloads.MLP_UP_RMSNORM) == "rmsnorm_quant_stream_kernel"
+    assert bench.quant_kernel_name(workloads.MLP_UP_RMSNORM) == "rmsnorm_quant_warp_kernel"
 
 
 def test_profiled_traffic_is_guarded_by_the_kernel_source(bench, tmp_path, monkeypatch):
