@@ -82,6 +82,7 @@ PROFILED_TRAFFIC = {
     ("gemm", "mlp_up_4096x4096x14336"): (75.995904e6 + 83.197696e6, "abc2533ea4ecf75c"),
     ("gemm", "fp8_down_4096x14336x4096"): (258.165504e6 + 42.465280e6, "abc2533ea4ecf75c"),
     ("gemm", "fp8_tensor_4096x4096x14336"): (75.910400e6 + 82.917888e6, "abc2533ea4ecf75c"),
+    ("gemm", "mlp_up_rmsnorm_4096x4096x14336"): (75.824128e6 + 82.939136e6, "abc2533ea4ecf75c"),
     ("gemm_small", "prefill_512x4096x4096"): (18.910720e6 + 0.0, "7eda12a8fa5cadb4"),
     ("gemm_skinny", "decode_16x8192x28672"): (235.149568e6 + 4.384256e6, "30641829128746f8"),
     ("gemm_wonly", "decode_w8a16_16x8192x28672"): (237.113344e6 + 3.692288e6, "c6b07cfabb7fec57"),
