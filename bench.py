@@ -459,16 +459,26 @@ def run_ours(args):
     sx = torch.empty(M, dtype=torch.float32, device=dev)
     y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream()
+    # consecutive steps are independent batches: with two code buffers the
+    # activation pass of step i+1 may run in the SMs that step i's GEMM leaves
+    # idle in its last round of tiles (SQ_OVERLAP_PREVIOUS); it completes only
+    # after that GEMM, so the steps still finish in order
+    overlap = not (wbits or tensor or args.no_overlap)
+    nbuf = 2 if overlap else 1
+    xqs = [xq] + [torch.empty_like(xq) for _ in range(nbuf - 1)]
+    sxs = [sx] + [torch.empty_like(sx) for _ in range(nbuf - 1)]
 
-    def quantize(i):
-        r = i % ROTATE
+    def quantize(i, ov=False):
+        r, b = i % ROTATE, i % nbuf
         if tensor:
-            ops.quantize_act_tensor(xs[r], s, qt, amax_prev=amax_b[i % 2:i % 2 + 1], xq=xq, sx=sx,
-                                    amax_out=amax_b[(i + 1) % 2:(i + 1) % 2 + 1], s_inv=s_inv)
+            ops.quantize_act_tensor(xs[r], s, qt, amax_prev=amax_b[i % 2:i % 2 + 1], xq=xqs[b],
+                                    sx=sxs[b], amax_out=amax_b[(i + 1) % 2:(i + 1) % 2 + 1],
+                                    s_inv=s_inv)
         elif g_fold is not None:
-            ops.rmsnorm_quantize_act(xs[r], g_fold, case.norm_eps, qt, xq=xq, sx=sx)
+            ops.rmsnorm_quantize_act(xs[r], g_fold, case.norm_eps, qt, xq=xqs[b], sx=sxs[b],
+                                     overlap=ov)
         else:
-            ops.quantize_act(xs[r], s, qt, xq=xq, sx=sx, s_inv=s_inv)
+            ops.quantize_act(xs[r], s, qt, xq=xqs[b], sx=sxs[b], s_inv=s_inv, overlap=ov)
 
     split = not args.no_split
 
@@ -476,8 +486,8 @@ def run_ours(args):
         if wbits:
             gemm(xs[i % ROTATE], None, wqs[i % ROTATE], sw, bias, out=y)
             return
-        quantize(i)
-        gemm(xq, sx, wqs[i % ROTATE], sw, bias, out=y, split=split)
+        quantize(i, overlap)
+        gemm(xqs[i % nbuf], sxs[i % nbuf], wqs[i % ROTATE], sw, bias, out=y, split=split)
 
     for i in range(max(3, args.warmup)):
         step(i)
@@ -501,7 +511,8 @@ def run_ours(args):
         if not wbits:
             quantize(i)
         ev[i][1].record(stream)
-        gemm(xs[r] if wbits else xq, sx, wqs[r], sw, bias, out=y, split=split)
+        gemm(xs[r] if wbits else xqs[i % nbuf], sxs[i % nbuf], wqs[r], sw, bias, out=y,
+             split=split)
         ev[i][2].record(stream)
     torch.cuda.synchronize()
     t_quant = float(np.mean([e[0].elapsed_time(e[1]) for e in ev]))
@@ -723,7 +734,10 @@ def run_ours(args):
                                    + (f", then one of {tail_steps}" if tail_steps else ""))
                                   if graph is not None else "one launch per kernel"),
                        "gemm_workspace": ("passed: the last partial round of tiles is split where that pays" if split else "not passed"),
-                       "gemm_tile": os.environ.get("SQ_GEMM_TILE", "auto")},
+                       "gemm_tile": os.environ.get("SQ_GEMM_TILE", "auto"),
+                       "overlap": ("the activation pass of step i+1 may run in the SMs step i's "
+                                   "GEMM leaves idle (two code buffers, SQ_OVERLAP_PREVIOUS)"
+                                   if overlap else "none")},
             "frac_of_int8_peak": None if wbits else value / ws / int8_peak,
             "frac_of_datasheet": None if wbits else value / ws / DATASHEET_8BIT_TOPS,
             "int8_peak_tops": int8_peak,
@@ -822,6 +836,10 @@ def main():
                     help="launch the timed steps one by one instead of replaying a CUDA graph")
     ap.add_argument("--workload", default="mlp_up_4096x4096x14336",
                     help="one of the workloads in workloads.py (default: the MLP up-projection)")
+    ap.add_argument("--no-overlap", action="store_true",
+                    help="keep each step's activation pass from starting before the previous "
+                         "step's GEMM has completed (by default it may use the SMs that GEMM "
+                         "leaves idle in its last round of tiles)")
     ap.add_argument("--no-split", action="store_true",
                     help="launch the GEMM without its workspace (by default the library may split "
                          "the last partial round of tiles along K over all SMs where that pays)")

@@ -53,7 +53,25 @@
 extern "C" {
 #endif
 
-#define SQ_ABI_VERSION 7
+#define SQ_ABI_VERSION 8
+
+/*
+ * Flags of the activation passes (sq_quantize_act, sq_rmsnorm_quantize_act).
+ *
+ * SQ_OVERLAP_PREVIOUS: the caller guarantees that no kernel still running when
+ * the pass starts writes x (and s, s_inv, g) or reads or writes xq, sx -- in
+ * practice that the kernel issued just before it on the stream does not, e.g.
+ * the previous batch's GEMM with xq / sx in a second buffer. The pass may then
+ * run while that kernel finishes, in the SMs it leaves idle; it still
+ * completes only after that kernel has completed, so everything issued after
+ * the pass sees the same stream order as without the flag. This library's
+ * GEMMs let the next kernel start only once their own inputs are complete, so
+ * with one of them just before the pass, every kernel before that GEMM has
+ * completed when the pass starts. Results are the same with or without the
+ * flag; the library may ignore it (forms launched without programmatic
+ * dependence always start after the previous kernel).
+ */
+#define SQ_OVERLAP_PREVIOUS 1u
 
 typedef enum {
     SQ_OK = 0,
@@ -171,10 +189,11 @@ sq_status sq_quantize_weight(const void* w, sq_dtype wt, int64_t K, int64_t N,
  *           by a reciprocal product with one exact correction step and falls
  *           back to the IEEE division wherever that is not provably exact).
  *           Results are undefined if s_inv does not come from s.
+ *   flags : 0 or SQ_OVERLAP_PREVIOUS (other bits: SQ_ERR_INVALID_ARG)
  */
 sq_status sq_quantize_act(const void* x, sq_dtype xt, int64_t M, int64_t K,
                           const float* s, const float* s_inv, sq_dtype qt,
-                          void* xq, float* sx, void* stream);
+                          void* xq, float* sx, uint32_t flags, void* stream);
 
 /*
  * Activation smoothing + PER-TENSOR quantization: one scale for the whole
@@ -245,6 +264,7 @@ sq_status sq_fold_smoothing(const void* p, sq_dtype pt, int64_t rows, int64_t co
  *   xn  : [M,K] binary32 or NULL (16-byte aligned): when given, the
  *         normalization's output xn below is written too, for the offline
  *         calibration of the smoothing factors (run it with g = gamma)
+ *   flags : 0 or SQ_OVERLAP_PREVIOUS (other bits: SQ_ERR_INVALID_ARG)
  * Per row: ss = the sum of x_k^2 over the k whose bf16 exponent is within 48
  * of the row's largest, exactly, rounded once to binary64 (the others are
  * below 2^-94 of the largest square); r = binary32(1 / sqrt(ss / K + eps))
@@ -256,7 +276,7 @@ sq_status sq_fold_smoothing(const void* p, sq_dtype pt, int64_t rows, int64_t co
  */
 sq_status sq_rmsnorm_quantize_act(const void* x, const float* g, float eps, int64_t M,
                                   int64_t K, sq_dtype qt, void* xq, float* sx, float* xn,
-                                  void* stream);
+                                  uint32_t flags, void* stream);
 
 /*
  * Size in bytes of the GEMM workspace for the current device (its SM count

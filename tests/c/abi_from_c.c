@@ -37,9 +37,9 @@ int main(void) {
            "smooth factors: alpha outside [0,1]");
     expect(sq_quantize_weight(A, SQ_BF16, 40, 64, NULL, SQ_I8, A, F, NULL) == SQ_ERR_INVALID_ARG,
            "quantize weight: K not a multiple of 16");
-    expect(sq_quantize_act(A, SQ_BF16, 4, 64, NULL, NULL, SQ_I8, (char*)A + 1, F, NULL) ==
+    expect(sq_quantize_act(A, SQ_BF16, 4, 64, NULL, NULL, SQ_I8, (char*)A + 1, F, 0u, NULL) ==
                SQ_ERR_MISALIGNED, "quantize act: misaligned codes");
-    expect(sq_quantize_act(NULL, SQ_BF16, 0, 64, NULL, NULL, SQ_I8, NULL, NULL, NULL) == SQ_OK,
+    expect(sq_quantize_act(NULL, SQ_BF16, 0, 64, NULL, NULL, SQ_I8, NULL, NULL, SQ_OVERLAP_PREVIOUS, NULL) == SQ_OK,
            "quantize act: empty batch is a no-op");
     expect(sq_quantize_act_tensor(A, SQ_BF16, 4, 64, NULL, NULL, SQ_E4M3, NULL, A, F, NULL, NULL) ==
                SQ_ERR_INVALID_ARG, "per-tensor: the tensor max output is required");
@@ -56,12 +56,14 @@ int main(void) {
                SQ_ERR_INVALID_ARG, "fold: output aliasing the input");
     expect(sq_fold_smoothing(NULL, SQ_F32, 0, 40, NULL, SQ_AMAX_PER_COLUMN, NULL, NULL) == SQ_OK,
            "fold: nothing to fold");
-    expect(sq_rmsnorm_quantize_act(A, F, 1e-6f, 4, 16392, SQ_I8, (char*)A + 0x100000, F, NULL, NULL) ==
+    expect(sq_rmsnorm_quantize_act(A, F, 1e-6f, 4, 16392, SQ_I8, (char*)A + 0x100000, F, NULL, 0u, NULL) ==
                SQ_ERR_UNSUPPORTED, "norm + quantization: K beyond one row on chip");
-    expect(sq_rmsnorm_quantize_act(A, F, 0.0f, 4, 64, SQ_I8, (char*)A + 0x100000, F, NULL, NULL) ==
+    expect(sq_rmsnorm_quantize_act(A, F, 0.0f, 4, 64, SQ_I8, (char*)A + 0x100000, F, NULL, 0u, NULL) ==
                SQ_ERR_INVALID_ARG, "norm + quantization: eps must be positive");
-    expect(sq_rmsnorm_quantize_act(NULL, NULL, 1e-6f, 0, 64, SQ_E4M3, NULL, NULL, NULL, NULL) == SQ_OK,
+    expect(sq_rmsnorm_quantize_act(NULL, NULL, 1e-6f, 0, 64, SQ_E4M3, NULL, NULL, NULL, 0u, NULL) == SQ_OK,
            "norm + quantization: empty batch");
+    expect(sq_quantize_act(A, SQ_BF16, 4, 64, NULL, NULL, SQ_I8, (char*)A + 0x100000, F, 2u, NULL) ==
+               SQ_ERR_INVALID_ARG, "quantize act: unknown flag bit");
     expect(sq_probe_wait_timeout(10, NULL) == SQ_ERR_INVALID_ARG, "probe: timeout below 1 ms");
     expect(sq_selftest_fast_division(NULL, NULL) == SQ_ERR_INVALID_ARG, "self-test: NULL result");
     (void)sq_gemm_workspace_bytes;  /* links; the size depends on the GPU */

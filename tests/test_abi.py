@@ -53,7 +53,7 @@ def test_exported_symbols_are_visible_to_the_dynamic_linker():
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.sq_abi_version() == 7
+    assert lib.sq_abi_version() == 8
     for st in range(7):
         assert ops.status_string(st).startswith("SQ_")
     assert "TIMEOUT" in ops.status_string(ops.SQ_ERR_TIMEOUT)
@@ -70,7 +70,7 @@ def test_quantize_act_validation(lib):
     def call(**kw):
         a = dict(ok, **kw)
         return f(c(a["x"]), a["xt"], a["M"], a["K"], c(a["s"]), c(a.get("s_inv")), a["qt"], c(a["xq"]),
-                 c(a["sx"]), None)
+                 c(a["sx"]), a.get("flags", 0), None)
 
     assert call(x=NUL) == ops.SQ_ERR_INVALID_ARG
     assert call(xq=NUL) == ops.SQ_ERR_INVALID_ARG
@@ -85,7 +85,10 @@ def test_quantize_act_validation(lib):
     assert call(xq=A + 8) == ops.SQ_ERR_MISALIGNED
     assert call(s=A + 4) == ops.SQ_ERR_MISALIGNED
     assert call(s_inv=A + 4) == ops.SQ_ERR_MISALIGNED
+    assert call(flags=2) == ops.SQ_ERR_INVALID_ARG     # unknown flag bit
+    assert call(flags=0x80000001) == ops.SQ_ERR_INVALID_ARG
     assert call(M=0) == ops.SQ_OK                      # empty input: no-op
+    assert call(M=0, flags=ops.SQ_OVERLAP_PREVIOUS) == ops.SQ_OK
 
 
 def test_quantize_act_tensor_validation(lib):
@@ -262,7 +265,7 @@ def test_rmsnorm_quantize_validation(lib):
     def call(**kw):
         a = dict(ok, **kw)
         return f(c(a["x"]), c(a["g"]), a["eps"], a["M"], a["K"], a["qt"], c(a["xq"]),
-                 c(a["sx"]), c(a["xn"]), None)
+                 c(a["sx"]), c(a["xn"]), a.get("flags", 0), None)
 
     assert call(x=NUL) == ops.SQ_ERR_INVALID_ARG
     assert call(g=NUL) == ops.SQ_ERR_INVALID_ARG
@@ -290,5 +293,6 @@ def test_rmsnorm_quantize_validation(lib):
     assert call(xn=A + 256) == ops.SQ_ERR_INVALID_ARG               # the output over the input
     assert call(xn=A + 0x200000 - 512) == ops.SQ_ERR_INVALID_ARG    # ... over the codes
     assert call(xn=A + 0x300000 - 1024 + 16) == ops.SQ_ERR_INVALID_ARG   # ... over the scales
+    assert call(flags=4) == ops.SQ_ERR_INVALID_ARG                   # unknown flag bit
     # empty batch: a no-op that accepts NULL pointers
     assert call(M=0, x=NUL, g=NUL, xq=NUL, sx=NUL) == ops.SQ_OK

@@ -198,7 +198,9 @@ sq_status sq_quantize_weight(const void* w, sq_dtype wt, int64_t K, int64_t N, c
 }
 
 sq_status sq_quantize_act(const void* x, sq_dtype xt, int64_t M, int64_t K, const float* s,
-                          const float* s_inv, sq_dtype qt, void* xq, float* sx, void* stream) {
+                          const float* s_inv, sq_dtype qt, void* xq, float* sx, uint32_t flags,
+                          void* stream) {
+  if (flags & ~uint32_t(SQ_OVERLAP_PREVIOUS)) return SQ_ERR_INVALID_ARG;
   if (xt != SQ_F32 && xt != SQ_BF16) return SQ_ERR_INVALID_ARG;
   if (qt != SQ_I8 && qt != SQ_E4M3) return SQ_ERR_INVALID_ARG;
   if (M < 0 || K <= 0 || K % 16 != 0 || K > 65536 || M > INT32_MAX) return SQ_ERR_INVALID_ARG;
@@ -209,7 +211,7 @@ sq_status sq_quantize_act(const void* x, sq_dtype xt, int64_t M, int64_t K, cons
   if (s_inv && !al(s_inv, 16)) return SQ_ERR_MISALIGNED;
   return from_cuda(sqh::launch_quantize_act(x, xt == SQ_BF16, M, K, s, s ? s_inv : nullptr,
                                             qt == SQ_E4M3, static_cast<uint8_t*>(xq), sx,
-                                            S(stream)));
+                                            (flags & SQ_OVERLAP_PREVIOUS) != 0, S(stream)));
 }
 
 sq_status sq_quantize_act_tensor(const void* x, sq_dtype xt, int64_t M, int64_t K,
@@ -282,7 +284,7 @@ sq_status sq_linear(const void* x, sq_dtype xt, const float* s, const float* s_i
   if (qt != SQ_I8 && qt != SQ_E4M3) return SQ_ERR_INVALID_ARG;
   sq_status c = check_gemm(xq_buf, sx_buf, wq, sw, bias, M, N, K, y, yt, nullptr);
   if (c != SQ_OK || M == 0) return c;
-  c = sq_quantize_act(x, xt, M, K, s, s_inv, qt, xq_buf, sx_buf, stream);
+  c = sq_quantize_act(x, xt, M, K, s, s_inv, qt, xq_buf, sx_buf, 0u, stream);
   if (c != SQ_OK) return c;
   if (qt == SQ_I8)
     return sq_gemm_w8a8(static_cast<const int8_t*>(xq_buf), sx_buf, static_cast<const int8_t*>(wq),
@@ -337,7 +339,8 @@ sq_status sq_gemm_weight_only(const void* x, const void* wq, sq_dtype wqt, const
 
 sq_status sq_rmsnorm_quantize_act(const void* x, const float* g, float eps, int64_t M,
                                   int64_t K, sq_dtype qt, void* xq, float* sx, float* xn,
-                                  void* stream) {
+                                  uint32_t flags, void* stream) {
+  if (flags & ~uint32_t(SQ_OVERLAP_PREVIOUS)) return SQ_ERR_INVALID_ARG;
   if (qt != SQ_I8 && qt != SQ_E4M3) return SQ_ERR_INVALID_ARG;
   if (M < 0 || K <= 0 || K % 8 != 0 || M > INT32_MAX) return SQ_ERR_INVALID_ARG;
   if (!(eps > 0.0f) || !std::isfinite(eps)) return SQ_ERR_INVALID_ARG;
@@ -357,7 +360,8 @@ sq_status sq_rmsnorm_quantize_act(const void* x, const float* g, float eps, int6
   if (!al(x, 16) || !al(g, 16) || !al(xq, 16) || !al(sx, 4) || !al(xn, 16))
     return SQ_ERR_MISALIGNED;
   return from_cuda(sqh::launch_rmsnorm_quant(static_cast<const uint16_t*>(x), g, eps, M, K,
-                                             qt == SQ_E4M3, xq, sx, xn, S(stream)));
+                                             qt == SQ_E4M3, xq, sx, xn,
+                                             (flags & SQ_OVERLAP_PREVIOUS) != 0, S(stream)));
 }
 
 sq_status sq_selftest_fast_division(int64_t* mismatches, void* stream) {

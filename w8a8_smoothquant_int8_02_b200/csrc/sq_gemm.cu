@@ -217,11 +217,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   if constexpr (CG == 2) cluster_sync_all(); else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  // the next kernel waits for this grid to complete before touching memory;
-  // everything above overlapped the previous kernel's tail, everything below
-  // reads its results
-  pdl_launch_dependents();
+  // set-up above overlaps the previous kernel; its results are read below.
+  // The next kernel may start only after that wait: by then every kernel
+  // before this one has completed, which lets an activation pass that
+  // overlaps this grid (SQ_OVERLAP_PREVIOUS) reuse the buffers of the GEMM
+  // before this one
   pdl_wait();
+  pdl_launch_dependents();
 
   const int num_mt = (M + C::kTileM - 1) / C::kTileM;
   const int num_nt = (N + BN - 1) / BN;

@@ -242,9 +242,13 @@ __global__ void __launch_bounds__(kWoThreads, 2)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  // set-up above overlaps the previous kernel; its results are read below
-  pdl_launch_dependents();
+  // set-up above overlaps the previous kernel; its results are read below.
+  // The next kernel may start only after that wait: by then every kernel
+  // before this one has completed, which lets an activation pass that
+  // overlaps this grid (SQ_OVERLAP_PREVIOUS) reuse the buffers of the GEMM
+  // before this one
   pdl_wait();
+  pdl_launch_dependents();
 
   const int n0 = int(blockIdx.x) * 128;
   const int m0 = int(blockIdx.y) * kWoTokens;

@@ -22,9 +22,12 @@ cudaError_t launch_smooth_factors(const float* ax, const float* aw, int64_t K, d
 cudaError_t launch_quantize_weight(const void* w, bool bf16, int64_t K, int64_t N, const float* s,
                                    bool e4m3, uint8_t* wq, float* sw, cudaStream_t st);
 // a5
+// overlap: the caller rules out any access of the previous kernel in the stream
+// to x, s, s_inv (writes) and xq, sx; the pass may then run while that kernel
+// finishes and completes after it
 cudaError_t launch_quantize_act(const void* x, bool bf16, int64_t M, int64_t K, const float* s,
                                 const float* s_inv, bool e4m3, uint8_t* xq, float* sx,
-                                cudaStream_t st);
+                                bool overlap, cudaStream_t st);
 cudaError_t launch_quantize_act_tensor(const void* x, bool bf16, int64_t M, int64_t K,
                                        const float* s, const float* s_inv, bool e4m3,
                                        const float* amax_prev, uint8_t* xq, float* sx,
@@ -34,7 +37,7 @@ cudaError_t launch_quantize_act_tensor(const void* x, bool bf16, int64_t M, int6
 int rmsnorm_quant_max_k();
 cudaError_t launch_rmsnorm_quant(const uint16_t* x, const float* g, float eps, int64_t M,
                                  int64_t K, bool e4m3, void* xq, float* sx, float* xn,
-                                 cudaStream_t st);
+                                 bool overlap, cudaStream_t st);
 // offline fold of 1/s into the producer of X
 cudaError_t launch_fold_smoothing(const void* p, bool bf16, int64_t rows, int64_t cols,
                                   const float* s, bool per_column, float* out, cudaStream_t st);

@@ -83,7 +83,7 @@ template <bool E4M3>
 __global__ void __launch_bounds__(kNormThreads)
     rmsnorm_quant_kernel(const uint16_t* __restrict__ x, const float* __restrict__ g,
                          float eps, int64_t M, int K, uint8_t* __restrict__ xq,
-                         float* __restrict__ sx, float* __restrict__ xn) {
+                         float* __restrict__ sx, float* __restrict__ xn, int late_wait) {
   extern __shared__ __align__(16) uint16_t row[];  // K entries
   __shared__ int red_i[kNormThreads / 32];
   __shared__ unsigned long long red_lo[kNormThreads / 32], red_hi[kNormThreads / 32];
@@ -92,9 +92,10 @@ __global__ void __launch_bounds__(kNormThreads)
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   constexpr int W = kNormThreads / 32;
   const int nchunk = K >> 3;
-  // the row may come from the kernel before this one
+  // the row may come from the kernel before this one, unless the caller has
+  // ruled that out (late_wait: then this grid only completes after it)
   pdl_launch_dependents();
-  pdl_wait();
+  if (!late_wait) pdl_wait();
 #pragma unroll 1
   for (int64_t m = blockIdx.x; m < M; m += gridDim.x) {
     const uint16_t* xr = x + m * K;
@@ -237,6 +238,7 @@ __global__ void __launch_bounds__(kNormThreads)
     // the staged row and the reduction slots are reused by the next row
     __syncthreads();
   }
+  if (late_wait) pdl_wait();
 }
 
 // ----------------------------------------------------------------------------
@@ -437,7 +439,7 @@ template <int V, bool E4M3, int SLOTS, int MAXT>
 __global__ void __launch_bounds__(MAXT, 512 / MAXT)
     rmsnorm_quant_stream_kernel(const uint16_t* __restrict__ x, const float* __restrict__ g,
                                 float eps, int64_t M, int K, uint8_t* __restrict__ xq,
-                                float* __restrict__ sx, int* status) {
+                                float* __restrict__ sx, int* status, int late_wait) {
   extern __shared__ __align__(128) uint8_t ring[];
   __shared__ uint32_t red_mx[2][32];
   __shared__ unsigned long long red_sum[2][2][32];
@@ -456,8 +458,9 @@ __global__ void __launch_bounds__(MAXT, 512 / MAXT)
     slow_lo[0] = slow_lo[1] = slow_hi[0] = slow_hi[1] = 0ull;
   }
   // x and g may come from the kernel before this one, which may still read
-  // xq / sx
-  pdl_wait();
+  // xq / sx -- unless the caller has ruled both out (late_wait: then this
+  // grid waits for that kernel only at its end)
+  if (!late_wait) pdl_wait();
   if (threadIdx.x == 0) {
     for (int i = 0; i < SLOTS; ++i) {
       const int64_t m = blockIdx.x + i * stride;
@@ -623,6 +626,7 @@ __global__ void __launch_bounds__(MAXT, 512 / MAXT)
       phase ^= 1u;
     }
   }
+  if (late_wait) pdl_wait();
 }
 
 // ----------------------------------------------------------------------------
@@ -642,7 +646,7 @@ template <bool E4M3>
 __global__ void __launch_bounds__(256)
     rmsnorm_quant_warp_kernel(const uint16_t* __restrict__ x, const float* __restrict__ g,
                               float eps, int64_t M, int K, uint8_t* __restrict__ xq,
-                              float* __restrict__ sx, int* status) {
+                              float* __restrict__ sx, int* status, int late_wait) {
   constexpr int SLOTS = kNormWarpSlots;
   extern __shared__ __align__(128) uint8_t ring[];  // [warps][SLOTS][K] bf16
   __shared__ __align__(8) uint64_t bars[8][SLOTS];
@@ -659,8 +663,8 @@ __global__ void __launch_bounds__(256)
   }
   __syncwarp();
   // x and g may come from the kernel before this one, which may still read
-  // xq / sx
-  pdl_wait();
+  // xq / sx -- unless the caller has ruled both out (late_wait)
+  if (!late_wait) pdl_wait();
   if (lane == 0) {
     for (int i = 0; i < SLOTS; ++i) {
       const int64_t m = w0 + i * stride;
@@ -789,6 +793,7 @@ __global__ void __launch_bounds__(256)
       phase ^= 1u;
     }
   }
+  if (late_wait) pdl_wait();
 }
 
 }  // namespace sqk
@@ -815,7 +820,7 @@ static int norm_sm_count() {
 // many CTAs as fit on the SMs at once (no more than there are rows).
 template <int MAXT>
 static cudaError_t launch_norm_stream(const uint16_t* x, const float* g, float eps, int64_t M,
-                                      int K, bool e4m3, uint8_t* xq, float* sx,
+                                      int K, bool e4m3, uint8_t* xq, float* sx, bool overlap,
                                       cudaStream_t st) {
   constexpr int V = 4, SLOTS = 4;
   const int nchunk = K >> 3;
@@ -833,12 +838,13 @@ static cudaError_t launch_norm_stream(const uint16_t* x, const float* g, float e
     per_sm = 1;
   int64_t grid = int64_t(per_sm) * norm_sm_count();
   if (grid > M) grid = M;
-  return launch_pdl(kern, unsigned(grid), threads, smem, st, x, g, eps, M, K, xq, sx, status);
+  return launch_pdl(kern, unsigned(grid), threads, smem, st, x, g, eps, M, K, xq, sx, status,
+                    int(overlap));
 }
 
 cudaError_t launch_rmsnorm_quant(const uint16_t* x, const float* g, float eps, int64_t M,
                                  int64_t K, bool e4m3, void* xq, float* sx, float* xn,
-                                 cudaStream_t st) {
+                                 bool overlap, cudaStream_t st) {
   if (!xn && K <= kNormWarpMaxK && M >= 4LL * norm_sm_count()) {
     // the warp form: up to 8 warps per CTA, each with SLOTS rows in flight,
     // about 96 KB of ring per CTA; as many CTAs as fit, no more than the rows
@@ -857,14 +863,16 @@ cudaError_t launch_rmsnorm_quant(const uint16_t* x, const float* g, float eps, i
     int64_t grid = int64_t(per_sm) * norm_sm_count();
     grid = min(grid, (M + warps - 1) / warps);
     return launch_pdl(kern, unsigned(grid), warps * 32, smem, st, x, g, eps, M, int(K),
-                      static_cast<uint8_t*>(xq), sx, status_ptr());
+                      static_cast<uint8_t*>(xq), sx, status_ptr(), int(overlap));
   }
   if (!xn) {
     const int nchunk = int(K >> 3);  // <= 2048
     uint8_t* q = static_cast<uint8_t*>(xq);
-    if (nchunk <= 4 * 128) return launch_norm_stream<128>(x, g, eps, M, int(K), e4m3, q, sx, st);
-    if (nchunk <= 4 * 256) return launch_norm_stream<256>(x, g, eps, M, int(K), e4m3, q, sx, st);
-    return launch_norm_stream<512>(x, g, eps, M, int(K), e4m3, q, sx, st);
+    if (nchunk <= 4 * 128)
+      return launch_norm_stream<128>(x, g, eps, M, int(K), e4m3, q, sx, overlap, st);
+    if (nchunk <= 4 * 256)
+      return launch_norm_stream<256>(x, g, eps, M, int(K), e4m3, q, sx, overlap, st);
+    return launch_norm_stream<512>(x, g, eps, M, int(K), e4m3, q, sx, overlap, st);
   }
   // the plain form: one CTA per row, at most a few waves' worth resident:
   // rows beyond the grid are taken in turn
@@ -872,9 +880,9 @@ cudaError_t launch_rmsnorm_quant(const uint16_t* x, const float* g, float eps, i
   const size_t smem = size_t(K) * 2;  // the staged row (at most 32 KB: no opt-in needed)
   if (e4m3)
     return launch_pdl(rmsnorm_quant_kernel<true>, unsigned(grid), kNormThreads, smem, st, x, g,
-                      eps, M, int(K), static_cast<uint8_t*>(xq), sx, xn);
+                      eps, M, int(K), static_cast<uint8_t*>(xq), sx, xn, int(overlap));
   return launch_pdl(rmsnorm_quant_kernel<false>, unsigned(grid), kNormThreads, smem, st, x, g,
-                    eps, M, int(K), static_cast<uint8_t*>(xq), sx, xn);
+                    eps, M, int(K), static_cast<uint8_t*>(xq), sx, xn, int(overlap));
 }
 
 }  // namespace sqh

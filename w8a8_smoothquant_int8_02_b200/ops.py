@@ -22,6 +22,7 @@ from . import build as _build
  SQ_ERR_SCRATCH_TOO_SMALL) = range(7)
 SQ_F32, SQ_BF16, SQ_I8, SQ_E4M3, SQ_I32, SQ_I4 = range(6)
 SQ_AMAX_PER_COLUMN, SQ_AMAX_PER_ROW = 0, 1
+SQ_OVERLAP_PREVIOUS = 1
 
 EXPORTED = (
     "sq_status_string", "sq_abi_version", "sq_get_device_status", "sq_calibrate_amax",
@@ -57,6 +58,7 @@ def load(build_if_needed: bool = True) -> ctypes.CDLL:
                                    "`python -m w8a8_smoothquant_int8_02_b200.build`")
             lib = ctypes.CDLL(_build.LIB)
             P, I64, I, D = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_double
+            U32 = ctypes.c_uint32
             lib.sq_status_string.argtypes = [I]
             lib.sq_status_string.restype = ctypes.c_char_p
             lib.sq_abi_version.restype = I
@@ -64,7 +66,7 @@ def load(build_if_needed: bool = True) -> ctypes.CDLL:
             lib.sq_calibrate_amax.argtypes = [P, I, I64, I64, I, P, I, P]
             lib.sq_smooth_factors.argtypes = [P, P, I64, D, P, P, P]
             lib.sq_quantize_weight.argtypes = [P, I, I64, I64, P, I, P, P, P]
-            lib.sq_quantize_act.argtypes = [P, I, I64, I64, P, P, I, P, P, P]
+            lib.sq_quantize_act.argtypes = [P, I, I64, I64, P, P, I, P, P, U32, P]
             lib.sq_fold_smoothing.argtypes = [P, I, I64, I64, P, I, P, P]
             SZ = ctypes.c_size_t
             lib.sq_gemm_w8a8.argtypes = [P, P, P, P, P, I64, I64, I64, P, I, P, P, SZ, P]
@@ -72,7 +74,7 @@ def load(build_if_needed: bool = True) -> ctypes.CDLL:
             lib.sq_linear.argtypes = [P, I, P, P, P, P, P, I, I64, I64, I64, P, P, P, I, P, SZ, P]
             lib.sq_gemm_w8a8_noalloc.argtypes = [P, P, P, P, P, I64, I64, I64, P, I, P]
             lib.sq_gemm_weight_only.argtypes = [P, P, I, P, P, I64, I64, I64, P, I, P]
-            lib.sq_rmsnorm_quantize_act.argtypes = [P, P, ctypes.c_float, I64, I64, I, P, P, P, P]
+            lib.sq_rmsnorm_quantize_act.argtypes = [P, P, ctypes.c_float, I64, I64, I, P, P, P, U32, P]
             lib.sq_gemm_workspace_bytes.argtypes = []
             lib.sq_gemm_workspace_bytes.restype = SZ
             lib.sq_probe_wait_timeout.argtypes = [I64, P]
@@ -206,9 +208,13 @@ def quantize_weight(w: torch.Tensor, s: torch.Tensor | None, qtype: str = "i8"):
 
 
 def quantize_act(x: torch.Tensor, s: torch.Tensor | None, qtype: str = "i8", xq=None, sx=None,
-                 s_inv: torch.Tensor | None = None):
+                 s_inv: torch.Tensor | None = None, overlap: bool = False):
     """a5: fused smoothing + per-token quantization; returns (xq [M,K], sx [M]).
-    s_inv (from smooth_factors(..., with_inverse=True)) only makes it faster."""
+    s_inv (from smooth_factors(..., with_inverse=True)) only makes it faster.
+    overlap=True passes SQ_OVERLAP_PREVIOUS: the caller guarantees that the
+    kernel before it on the stream neither writes x, s, s_inv nor touches xq,
+    sx (e.g. the previous batch's GEMM reading another xq buffer); the pass may
+    then run in the SMs that kernel leaves idle."""
     _cuda(x, s, xq, sx, s_inv)
     M, K = x.shape
     qt = _qtype(qtype)
@@ -217,7 +223,8 @@ def quantize_act(x: torch.Tensor, s: torch.Tensor | None, qtype: str = "i8", xq=
     if sx is None:
         sx = torch.empty(M, dtype=torch.float32, device=x.device)
     _check(load().sq_quantize_act(_p(x), _fdtype(x), M, K, _p(s), _p(s_inv), qt, _p(xq), _p(sx),
-                                  _stream(x.device)), "sq_quantize_act")
+                                  SQ_OVERLAP_PREVIOUS if overlap else 0, _stream(x.device)),
+           "sq_quantize_act")
     return xq, sx
 
 
@@ -334,12 +341,13 @@ def gemm_weight_only(x, wq, sw, bias=None, bits=8, out_dtype=torch.bfloat16, out
     return out
 
 
-def rmsnorm_quantize_act(x, g, eps, qtype="i8", xq=None, sx=None, xn=None, want_xn=False):
+def rmsnorm_quantize_act(x, g, eps, qtype="i8", xq=None, sx=None, xn=None, want_xn=False,
+                         overlap=False):
     """The producer of X with the smoothing folded in: RMS normalization of the
     bf16 rows of x [M,K] with gain g [K] (gamma / s, see fold_smoothing), fused
     with per-token quantization. Returns (xq [M,K] codes, sx [M]); with
     want_xn (or an xn buffer given) also the normalization's output xn [M,K]
-    float32, the input of the offline calibration."""
+    float32, the input of the offline calibration. overlap: as quantize_act."""
     _cuda(x, g, xq, sx, xn)
     if x.dtype != torch.bfloat16 or g.dtype != torch.float32:
         raise TypeError("x must be bfloat16 and g float32")
@@ -353,7 +361,8 @@ def rmsnorm_quantize_act(x, g, eps, qtype="i8", xq=None, sx=None, xn=None, want_
     if xn is None and want_xn:
         xn = torch.empty((M, K), dtype=torch.float32, device=x.device)
     _check(load().sq_rmsnorm_quantize_act(_p(x), _p(g), float(eps), M, K, qt, _p(xq), _p(sx),
-                                          _p(xn), _stream(x.device)), "sq_rmsnorm_quantize_act")
+                                          _p(xn), SQ_OVERLAP_PREVIOUS if overlap else 0,
+                                          _stream(x.device)), "sq_rmsnorm_quantize_act")
     return (xq, sx, xn) if xn is not None else (xq, sx)
 
 
