@@ -75,24 +75,25 @@ def rotate_count(case):
 
 
 # DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from
-# one ncu --set full capture of bench.py's own command per workload (the
-# summaries under profiles/), keyed by the sha256 prefix of the kernel's
-# sources at capture time: a kernel changed since reports null.
+# one ncu capture of those two counters on bench.py's own command per
+# workload (profiles/dram_bytes_per_launch_all_workloads.md), keyed by the
+# sha256 prefix of the kernel's sources at capture time: a kernel changed
+# since reports null.
 PROFILED_TRAFFIC = {
-    ("gemm", "mlp_up_4096x4096x14336"): (75.995904e6 + 83.197696e6, "abc2533ea4ecf75c"),
-    ("gemm", "fp8_down_4096x14336x4096"): (258.165504e6 + 42.465280e6, "abc2533ea4ecf75c"),
-    ("gemm", "fp8_tensor_4096x4096x14336"): (75.910400e6 + 82.917888e6, "abc2533ea4ecf75c"),
-    ("gemm", "mlp_up_rmsnorm_4096x4096x14336"): (75.824128e6 + 82.939136e6, "abc2533ea4ecf75c"),
-    ("gemm_small", "prefill_512x4096x4096"): (18.910720e6 + 0.0, "7eda12a8fa5cadb4"),
-    ("gemm_skinny", "decode_16x8192x28672"): (235.149568e6 + 4.384256e6, "30641829128746f8"),
-    ("gemm_wonly", "decode_w8a16_16x8192x28672"): (237.113344e6 + 3.692288e6, "c6b07cfabb7fec57"),
-    ("gemm_wonly", "decode_w4a16_16x8192x28672"): (119.396608e6 + 3.782912e6, "c6b07cfabb7fec57"),
-    ("quant", "mlp_up_4096x4096x14336"): (33.647872e6 + 0.004352e6, "e5dd1a242fc0384b"),
-    ("quant", "fp8_down_4096x14336x4096"): (117.741312e6 + 30.062080e6, "e5dd1a242fc0384b"),
-    ("quant", "fp8_tensor_4096x4096x14336"): (33.577984e6 + 0.005632e6, "e5dd1a242fc0384b"),
-    ("quant", "prefill_512x4096x4096"): (4.287744e6 + 0.0, "e5dd1a242fc0384b"),
-    ("quant", "decode_16x8192x28672"): (0.362240e6 + 0.0, "e5dd1a242fc0384b"),
-    ("norm", "mlp_up_rmsnorm_4096x4096x14336"): (33.620480e6 + 0.036608e6, "48f492482ffe3662"),
+    ("quant", "mlp_up_4096x4096x14336"): (33.648896e6 + 0.000768e6, "a01687d33b9f4575"),
+    ("gemm", "mlp_up_4096x4096x14336"): (75.848448e6 + 80.070912e6, "634da0a9c1526fe2"),
+    ("quant", "fp8_down_4096x14336x4096"): (117.747968e6 + 28.593152e6, "a01687d33b9f4575"),
+    ("gemm", "fp8_down_4096x14336x4096"): (258.194176e6 + 38.725888e6, "634da0a9c1526fe2"),
+    ("gemm", "fp8_tensor_4096x4096x14336"): (75.751680e6 + 82.965760e6, "634da0a9c1526fe2"),
+    ("quant", "fp8_tensor_4096x4096x14336"): (33.577984e6 + 0.000000e6, "a01687d33b9f4575"),
+    ("quant", "prefill_512x4096x4096"): (4.288256e6 + 0.000000e6, "a01687d33b9f4575"),
+    ("gemm_small", "prefill_512x4096x4096"): (18.911744e6 + 0.000000e6, "2c1a43c91e6b64ee"),
+    ("quant", "decode_16x8192x28672"): (0.362496e6 + 0.000000e6, "a01687d33b9f4575"),
+    ("gemm_skinny", "decode_16x8192x28672"): (235.150336e6 + 0.074240e6, "5b049eeaf965ee9c"),
+    ("gemm_wonly", "decode_w8a16_16x8192x28672"): (237.114880e6 + 3.152640e6, "cc74ba938948939e"),
+    ("gemm_wonly", "decode_w4a16_16x8192x28672"): (119.307776e6 + 4.051968e6, "cc74ba938948939e"),
+    ("norm", "mlp_up_rmsnorm_4096x4096x14336"): (33.621504e6 + 0.000000e6, "680317c85e77264f"),
+    ("gemm", "mlp_up_rmsnorm_4096x4096x14336"): (75.831808e6 + 80.078336e6, "634da0a9c1526fe2"),
 }
 KERNEL_SOURCES = {"gemm": ("sq_gemm.cu", "sq_common.cuh"),
                   "gemm_wonly": ("sq_gemm_wonly.cu", "sq_common.cuh"),
