@@ -527,9 +527,13 @@ def test_quantize_act_streaming_rows_edge_values(qtype, K):
     s_out[min(K - 1, 40)] = 2.0 ** -30                   # outside [2^-20, 2^20]
     xb = synth.to_bf16_bits(x)
     qt = oracle.E4M3 if qtype == "e4m3" else oracle.INT8
-    for smooth in (s_in, s_out, None):
+    # with and without the caller's reciprocals (rows longer than 8192 take a
+    # different form when they are given)
+    for smooth, inv in ((s_in, None), (s_out, None), (None, None), (s_in, reciprocals(s_in)),
+                        (s_out, reciprocals(s_out))):
         xq_ref, sx_ref = oracle.quantize_act(xb, smooth, qt)
-        xq, sx = ops.quantize_act(dev(xb), None if smooth is None else dev(smooth), qtype)
+        xq, sx = ops.quantize_act(dev(xb), None if smooth is None else dev(smooth), qtype,
+                                  s_inv=None if inv is None else dev(inv))
         assert ops.device_status() == ops.SQ_OK
         np.testing.assert_array_equal(host(sx), sx_ref)
         np.testing.assert_array_equal(host(xq).view(np.uint8), xq_ref.view(np.uint8))
