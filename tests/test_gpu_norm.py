@@ -107,3 +107,24 @@ def test_rmsnorm_quantize_validation():
         ops.rmsnorm_quantize_act(big, torch.ones(16392, device="cuda"), 1e-6)   # K > 16384
     xq, sx = ops.rmsnorm_quantize_act(x[:0], g, 1e-6)             # empty batch
     assert xq.shape == (0, 64) and sx.shape == (0,)
+
+
+@pytest.mark.parametrize("force_exact", [False, True])
+@pytest.mark.parametrize("qt", ["i8", "e4m3"])
+def test_many_rows_sum_paths(force_exact, qt, monkeypatch):
+    """Many rows (the one-warp-per-row form): its binary64 sum of squares with
+    the interval check, which falls back to the exact integer sum for the
+    rows whose r it cannot settle (about one in a few thousand here), and the
+    exact sum for every row (SQ_NORM_EXACT_SUM=1); both bit-exact."""
+    if force_exact:
+        monkeypatch.setenv("SQ_NORM_EXACT_SUM", "1")
+    M, K = 20000, 256
+    xb = _rows(M, K, seed=4242)
+    gamma = synth.random_floats(K, seed=4243, lo=0.3, hi=2.5)
+    q_ref, s_ref, _, _ = oracle.rmsnorm_quantize_act(
+        xb, gamma, 1e-5, oracle.INT8 if qt == "i8" else oracle.E4M3)
+    xq, sx = ops.rmsnorm_quantize_act(dev(xb), dev(gamma), 1e-5, qt)
+    assert ops.device_status() == ops.SQ_OK
+    np.testing.assert_array_equal(host(sx), s_ref)
+    np.testing.assert_array_equal(host(xq).view(np.uint8), q_ref.view(np.uint8))
+

@@ -36,6 +36,7 @@
 //    whose largest |xn| is in [2^-60, 2^100].
 // HBM-bound in principle: 2 bytes read and 1 written per element.
 #include <cstdint>
+#include <cstdlib>
 #include <cuda_runtime.h>
 
 #include "sq_common.cuh"
@@ -337,6 +338,14 @@ __device__ __forceinline__ void norm_slow_chunk(const uint4& u, int lo_ef, int e
     const uint32_t h = ((i & 1) ? (w[i >> 1] >> 16) : w[i >> 1]) & 0x7FFFu;
     if (h != 0u && int(h >> 7) < lo_ef) norm_slow_square(h, emax, acc);
   }
+}
+
+// binary32(1 / sqrt(ss / K + eps)) with each binary64 step rounded once (the
+// chain the oracle takes from its exact sum, here from a given binary64 ss).
+__device__ __forceinline__ float norm_chain(double ss, int K, float eps) {
+  const double mean = __ddiv_rn(ss, double(K));
+  const double t = __dsqrt_rn(__dadd_rn(mean, double(eps)));
+  return __double2float_rn(__ddiv_rn(1.0, t));
 }
 
 // r = binary32(1 / sqrt(ss / K + eps)) from the exact sum: the remainder in
@@ -646,7 +655,8 @@ template <bool E4M3>
 __global__ void __launch_bounds__(256)
     rmsnorm_quant_warp_kernel(const uint16_t* __restrict__ x, const float* __restrict__ g,
                               float eps, int64_t M, int K, uint8_t* __restrict__ xq,
-                              float* __restrict__ sx, int* status, int late_wait) {
+                              float* __restrict__ sx, int* status, int late_wait,
+                              int force_exact) {
   constexpr int SLOTS = kNormWarpSlots;
   extern __shared__ __align__(128) uint8_t ring[];  // [warps][SLOTS][K] bf16
   __shared__ __align__(8) uint64_t bars[8][SLOTS];
@@ -694,6 +704,38 @@ __global__ void __launch_bounds__(256)
       break;
     }
     const uint4* row = reinterpret_cast<const uint4*>(my_ring + size_t(slot) * row_bytes);
+    // 0. the sum of squares in binary64: every square of a bf16 value is exact
+    // there, so the computed sum lies within (n - 1) * 2^-53 of the exact one
+    // (n <= 16384 terms, all non-negative; whatever the order), far inside
+    // the 2^-36 used below, and the elements the exact sum leaves out (more
+    // than 48 binades below the largest) change it by less than 2^-80. The
+    // chain to r is monotone in ss, so if both ends of [ss (1 - 2^-36),
+    // ss (1 + 2^-36)] give the same binary32 r, that is the r of the exact
+    // sum; otherwise (about one row in 2^11) the exact sum is taken below.
+    float r = 0.0f;
+    bool exact = force_exact != 0;
+    if (!exact) {
+      double acc = 0.0;
+#pragma unroll 4
+      for (int c = lane; c < nchunk; c += 32) {
+        const uint4 u = row[c];
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const double dl = double(bf16_lo(w[t])), dh = double(bf16_hi(w[t]));
+          acc = __fma_rn(dl, dl, acc);
+          acc = __fma_rn(dh, dh, acc);
+        }
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) acc = __dadd_rn(acc, __shfl_down_sync(0xFFFFFFFFu, acc, off));
+      acc = __shfl_sync(0xFFFFFFFFu, acc, 0);  // one value for every lane
+      const float r_lo = norm_chain(__dmul_ru(acc, 1.0 + 0x1p-36), K, eps);
+      const float r_hi = norm_chain(__dmul_rd(acc, 1.0 - 0x1p-36), K, eps);
+      exact = r_lo != r_hi;
+      r = r_lo;
+    }
+    if (exact) {
     // 1. the largest and smallest magnitude patterns
     uint32_t mx2 = 0, mn2 = 0xFFFFFFFFu;
 #pragma unroll 4
@@ -736,7 +778,8 @@ __global__ void __launch_bounds__(256)
         u128_add(rest, lo, hi);
       }
     }
-    const float r = norm_rinv(rest, accA, accB, hmax, emax, K, eps);
+    r = norm_rinv(rest, accA, accB, hmax, emax, K, eps);
+    }
     const uint64_t r2 = f2_make(r, r);
     // 3. the largest |y|, y = (x * r) * g
     float am0 = 0.0f, am1 = 0.0f;
@@ -862,8 +905,12 @@ cudaError_t launch_rmsnorm_quant(const uint16_t* x, const float* g, float eps, i
       per_sm = 1;
     int64_t grid = int64_t(per_sm) * norm_sm_count();
     grid = min(grid, (M + warps - 1) / warps);
+    // SQ_NORM_EXACT_SUM=1 takes the exact integer sum for every row (the path
+    // the binary64 one falls back to), so that tests can cover it at will
+    const char* fe = std::getenv("SQ_NORM_EXACT_SUM");
+    const int force_exact = fe && fe[0] == '1';
     return launch_pdl(kern, unsigned(grid), warps * 32, smem, st, x, g, eps, M, int(K),
-                      static_cast<uint8_t*>(xq), sx, status_ptr(), int(overlap));
+                      static_cast<uint8_t*>(xq), sx, status_ptr(), int(overlap), force_exact);
   }
   if (!xn) {
     const int nchunk = int(K >> 3);  // <= 2048
