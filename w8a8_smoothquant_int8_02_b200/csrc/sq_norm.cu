@@ -359,6 +359,22 @@ __device__ __forceinline__ float norm_rinv(U128 rest, uint64_t totA, uint64_t to
   return __double2float_rn(__ddiv_rn(1.0, t));
 }
 
+// The 8 gains of one chunk as four packed pairs (loads only).
+__device__ __forceinline__ void norm_gains(const float* g8, uint64_t (&g2)[4]) {
+  const ulonglong2 ga = __ldg(reinterpret_cast<const ulonglong2*>(g8));
+  const ulonglong2 gb = __ldg(reinterpret_cast<const ulonglong2*>(g8) + 1);
+  g2[0] = ga.x, g2[1] = ga.y, g2[2] = gb.x, g2[3] = gb.y;
+}
+
+// y = (x * r) * g for one chunk from its gains g2 (packed pairs).
+__device__ __forceinline__ void norm_apply_g(const uint4& u, uint64_t r2, const uint64_t (&g2)[4],
+                                             uint64_t (&y2)[4]) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int t = 0; t < 4; ++t)
+    y2[t] = f2_mul(f2_mul(f2_make(bf16_lo(w[t]), bf16_hi(w[t])), r2), g2[t]);
+}
+
 // y = (x * r) * g for one chunk, as four packed pairs; g8 = the chunk's 8 gains.
 __device__ __forceinline__ void norm_apply(const uint4& u, uint64_t r2, const float* g8,
                                            uint64_t (&y2)[4]) {
@@ -781,18 +797,27 @@ __global__ void __launch_bounds__(256)
     r = norm_rinv(rest, accA, accB, hmax, emax, K, eps);
     }
     const uint64_t r2 = f2_make(r, r);
-    // 3. the largest |y|, y = (x * r) * g
+    // 3. the largest |y|, y = (x * r) * g. Two chunks per step, every load
+    // of the step (row from shared memory, gains from L1) issued first.
     float am0 = 0.0f, am1 = 0.0f;
-#pragma unroll 4
-    for (int c = lane; c < nchunk; c += 32) {
-      uint64_t y2[4];
-      norm_apply(row[c], r2, g + size_t(c) * 8, y2);
+#pragma unroll 2
+    for (int c = lane; c < nchunk; c += 64) {
+      const bool two = c + 32 < nchunk;
+      const uint4 u0 = row[c];
+      const uint4 u1 = two ? row[c + 32] : make_uint4(0u, 0u, 0u, 0u);
+      uint64_t g0[4], g1[4] = {0ull, 0ull, 0ull, 0ull};
+      norm_gains(g + size_t(c) * 8, g0);
+      if (two) norm_gains(g + size_t(c + 32) * 8, g1);
+      uint64_t y0[4], y1[4];
+      norm_apply_g(u0, r2, g0, y0);
+      norm_apply_g(u1, r2, g1, y1);
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
-        float a, b;
-        f2_split(y2[t], a, b);
-        if (t & 1) am1 = max3_nan(am1, fabsf(a), fabsf(b));
-        else am0 = max3_nan(am0, fabsf(a), fabsf(b));
+        float a, b, a1, b1;
+        f2_split(y0[t], a, b);
+        f2_split(y1[t], a1, b1);
+        am0 = max3_nan(am0, fabsf(a), fabsf(b));
+        am1 = max3_nan(am1, fabsf(a1), fabsf(b1));
       }
     }
     const float amax =
@@ -804,11 +829,19 @@ __global__ void __launch_bounds__(256)
       if (lane == 0) sx[m] = scale;
       const float rs = __frcp_rn(scale);
       const uint64_t rs2 = f2_make(rs, rs), nsc2 = f2_make(-scale, -scale);
-#pragma unroll 4
-      for (int c = lane; c < nchunk; c += 32) {
-        uint64_t y2[4];
-        norm_apply(row[c], r2, g + size_t(c) * 8, y2);
-        out[c] = norm_codes_fast<E4M3>(y2, rs2, nsc2);
+#pragma unroll 2
+      for (int c = lane; c < nchunk; c += 64) {
+        const bool two = c + 32 < nchunk;
+        const uint4 u0 = row[c];
+        const uint4 u1 = two ? row[c + 32] : make_uint4(0u, 0u, 0u, 0u);
+        uint64_t g0[4], g1[4] = {0ull, 0ull, 0ull, 0ull};
+        norm_gains(g + size_t(c) * 8, g0);
+        if (two) norm_gains(g + size_t(c + 32) * 8, g1);
+        uint64_t y0[4], y1[4];
+        norm_apply_g(u0, r2, g0, y0);
+        norm_apply_g(u1, r2, g1, y1);
+        out[c] = norm_codes_fast<E4M3>(y0, rs2, nsc2);
+        if (two) out[c + 32] = norm_codes_fast<E4M3>(y1, rs2, nsc2);
       }
     } else {
       const float scale = __fdiv_rn(amax, E4M3 ? 448.0f : 127.0f);
