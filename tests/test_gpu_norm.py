@@ -128,3 +128,19 @@ def test_many_rows_sum_paths(force_exact, qt, monkeypatch):
     np.testing.assert_array_equal(host(sx), s_ref)
     np.testing.assert_array_equal(host(xq).view(np.uint8), q_ref.view(np.uint8))
 
+
+
+@pytest.mark.parametrize("M,K", [(37, 4096), (300, 1000), (64, 16384), (511, 8192)])
+def test_block_form_exact_sum_path(M, K, monkeypatch):
+    """The one-CTA-per-row form (fewer rows, or rows above 8192 elements) with
+    the exact integer sum forced for every row (SQ_NORM_EXACT_SUM=1), and
+    with its binary64 sum; both bit-exact against the oracle."""
+    xb = _rows(M, K, seed=M * 7 + K)
+    gamma = synth.random_floats(K, seed=K + 11, lo=0.3, hi=2.5)
+    q_ref, s_ref, _, _ = oracle.rmsnorm_quantize_act(xb, gamma, 1e-5)
+    for force in ("1", "0"):
+        monkeypatch.setenv("SQ_NORM_EXACT_SUM", force)
+        xq, sx = ops.rmsnorm_quantize_act(dev(xb), dev(gamma), 1e-5, "i8")
+        assert ops.device_status() == ops.SQ_OK
+        np.testing.assert_array_equal(host(sx), s_ref)
+        np.testing.assert_array_equal(host(xq).view(np.uint8), q_ref.view(np.uint8))

@@ -464,10 +464,12 @@ template <int V, bool E4M3, int SLOTS, int MAXT>
 __global__ void __launch_bounds__(MAXT, 512 / MAXT)
     rmsnorm_quant_stream_kernel(const uint16_t* __restrict__ x, const float* __restrict__ g,
                                 float eps, int64_t M, int K, uint8_t* __restrict__ xq,
-                                float* __restrict__ sx, int* status, int late_wait) {
+                                float* __restrict__ sx, int* status, int late_wait,
+                                int force_exact) {
   extern __shared__ __align__(128) uint8_t ring[];
   __shared__ uint32_t red_mx[2][32];
   __shared__ unsigned long long red_sum[2][2][32];
+  __shared__ double red_dbl[2][32];
   __shared__ uint32_t red_am[2][32];
   __shared__ unsigned long long slow_lo[2], slow_hi[2];
   __shared__ __align__(8) uint64_t bars[SLOTS];
@@ -552,10 +554,41 @@ __global__ void __launch_bounds__(MAXT, 512 / MAXT)
         __reduce_max_sync(0xFFFFFFFFu, red_mx[sel][lane < nwarps ? lane : 0]);
     const int efmax = int(hmax >> 7);                 // 0 when the largest is subnormal
     const int emax = efmax ? efmax - 127 : -126;
+    // 2. the sum of squares in binary64 with the interval check of the warp
+    // form (the per-warp sums added in warp order, the same order in every
+    // thread, so that all of them hold the same ss); the exact sum below only
+    // for the rows whose r that cannot settle (a block-uniform branch)
+    float r = 0.0f;
+    bool exact = force_exact != 0;
+    if (!exact) {
+      double dacc = 0.0;
+#pragma unroll
+      for (int j = 0; j < V; ++j) {
+        const uint32_t w[4] = {raw[j].x, raw[j].y, raw[j].z, raw[j].w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const double dl = double(bf16_lo(w[t])), dh = double(bf16_hi(w[t]));
+          dacc = __fma_rn(dl, dl, dacc);
+          dacc = __fma_rn(dh, dh, dacc);
+        }
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1)
+        dacc = __dadd_rn(dacc, __shfl_down_sync(0xFFFFFFFFu, dacc, off));
+      if (lane == 0) red_dbl[sel][warp] = dacc;
+      __syncthreads();
+      double ss = 0.0;
+      for (int i = 0; i < nwarps; ++i) ss = __dadd_rn(ss, red_dbl[sel][i]);
+      const float r_lo = norm_chain(__dmul_ru(ss, 1.0 + 0x1p-36), K, eps);
+      const float r_hi = norm_chain(__dmul_rd(ss, 1.0 - 0x1p-36), K, eps);
+      exact = r_lo != r_hi;
+      r = r_lo;
+    }
+    if (exact) {
     // bands A and B: normal elements with exponent field >= efmax - 32 (none
     // when the largest is below 2^-94: the whole row takes the slow path)
     const int lo_ef = efmax > 32 ? efmax - 32 : 256;
-    // 2. the exact sum of squares. Band A: the shift e - e_max + 16 in
+    // the exact sum of squares. Band A: the shift e - e_max + 16 in
     // [0, 16], clamped at 32 (a = 0) below the band, negative offsets
     // included; band B: 16 more, kept only when below 16 (one unsigned
     // comparison excludes both band A and everything below band B)
@@ -594,7 +627,8 @@ __global__ void __launch_bounds__(MAXT, 512 / MAXT)
       totA += __shfl_xor_sync(0xFFFFFFFFu, totA, off);
       totB += __shfl_xor_sync(0xFFFFFFFFu, totB, off);
     }
-    const float r = norm_rinv(U128{slow_lo[sel], slow_hi[sel]}, totA, totB, hmax, emax, K, eps);
+    r = norm_rinv(U128{slow_lo[sel], slow_hi[sel]}, totA, totB, hmax, emax, K, eps);
+    }
     // 3. y = (x * r) * g, the largest |y|
     const uint64_t r2 = f2_make(r, r);
     uint64_t y2[V][4];
@@ -880,6 +914,13 @@ using namespace sqk;
 
 int rmsnorm_quant_max_k() { return kNormMaxK; }
 
+// SQ_NORM_EXACT_SUM=1 takes the exact integer sum of squares for every row
+// (the path the binary64 sum falls back to), so that tests can cover it at will.
+static int norm_force_exact() {
+  const char* e = std::getenv("SQ_NORM_EXACT_SUM");
+  return e && e[0] == '1';
+}
+
 static int norm_sm_count() {
   static int n = 0;
   if (n == 0) {
@@ -915,7 +956,7 @@ static cudaError_t launch_norm_stream(const uint16_t* x, const float* g, float e
   int64_t grid = int64_t(per_sm) * norm_sm_count();
   if (grid > M) grid = M;
   return launch_pdl(kern, unsigned(grid), threads, smem, st, x, g, eps, M, K, xq, sx, status,
-                    int(overlap));
+                    int(overlap), norm_force_exact());
 }
 
 cudaError_t launch_rmsnorm_quant(const uint16_t* x, const float* g, float eps, int64_t M,
@@ -938,12 +979,9 @@ cudaError_t launch_rmsnorm_quant(const uint16_t* x, const float* g, float eps, i
       per_sm = 1;
     int64_t grid = int64_t(per_sm) * norm_sm_count();
     grid = min(grid, (M + warps - 1) / warps);
-    // SQ_NORM_EXACT_SUM=1 takes the exact integer sum for every row (the path
-    // the binary64 one falls back to), so that tests can cover it at will
-    const char* fe = std::getenv("SQ_NORM_EXACT_SUM");
-    const int force_exact = fe && fe[0] == '1';
     return launch_pdl(kern, unsigned(grid), warps * 32, smem, st, x, g, eps, M, int(K),
-                      static_cast<uint8_t*>(xq), sx, status_ptr(), int(overlap), force_exact);
+                      static_cast<uint8_t*>(xq), sx, status_ptr(), int(overlap),
+                      norm_force_exact());
   }
   if (!xn) {
     const int nchunk = int(K >> 3);  // <= 2048
