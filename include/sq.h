@@ -273,6 +273,11 @@ sq_status sq_fold_smoothing(const void* p, sq_dtype pt, int64_t rows, int64_t co
  * with s = NULL. K a multiple of 8, at most 16384 (SQ_ERR_UNSUPPORTED
  * beyond). xq, sx and xn may overlap neither each other nor x or g
  * (SQ_ERR_INVALID_ARG). M == 0 is a no-op that accepts NULL pointers.
+ * The kernels reach the r of the exact sum by a binary64 sum of the squares
+ * (each square exact, the sum within 2^-36 of the exact one) whenever both
+ * ends of that interval give the same binary32 r, and by the exact integer
+ * sum otherwise; setting SQ_NORM_EXACT_SUM=1 in the environment takes the
+ * exact sum for every row. Results are the same either way.
  */
 sq_status sq_rmsnorm_quantize_act(const void* x, const float* g, float eps, int64_t M,
                                   int64_t K, sq_dtype qt, void* xq, float* sx, float* xn,
