@@ -144,3 +144,19 @@ def test_block_form_exact_sum_path(M, K, monkeypatch):
         assert ops.device_status() == ops.SQ_OK
         np.testing.assert_array_equal(host(sx), s_ref)
         np.testing.assert_array_equal(host(xq).view(np.uint8), q_ref.view(np.uint8))
+
+
+@pytest.mark.parametrize("M,K", [(700, 8192), (1500, 2048), (600, 4096), (900, 24)])
+@pytest.mark.parametrize("qt", ["i8", "e4m3"])
+def test_warp_form_row_lengths(M, K, qt):
+    """The one-warp-per-row form at row lengths with the gains in shared memory
+    (up to 4096) and from L1 (above), bit-exact against the oracle."""
+    xb = _rows(M, K, seed=M + 3 * K)
+    gamma = synth.random_floats(K, seed=K + 17, lo=0.3, hi=2.5)
+    gamma[1::3] *= -1.0
+    q_ref, s_ref, _, _ = oracle.rmsnorm_quantize_act(
+        xb, gamma, 1e-5, oracle.INT8 if qt == "i8" else oracle.E4M3)
+    xq, sx = ops.rmsnorm_quantize_act(dev(xb), dev(gamma), 1e-5, qt)
+    assert ops.device_status() == ops.SQ_OK
+    np.testing.assert_array_equal(host(sx), s_ref)
+    np.testing.assert_array_equal(host(xq).view(np.uint8), q_ref.view(np.uint8))

@@ -366,6 +366,13 @@ __device__ __forceinline__ void norm_gains(const float* g8, uint64_t (&g2)[4]) {
   g2[0] = ga.x, g2[1] = ga.y, g2[2] = gb.x, g2[3] = gb.y;
 }
 
+// The same from the CTA's table of gains in shared memory.
+__device__ __forceinline__ void norm_gains_smem(const float* g8, uint64_t (&g2)[4]) {
+  const ulonglong2 ga = *reinterpret_cast<const ulonglong2*>(g8);
+  const ulonglong2 gb = *(reinterpret_cast<const ulonglong2*>(g8) + 1);
+  g2[0] = ga.x, g2[1] = ga.y, g2[2] = gb.x, g2[3] = gb.y;
+}
+
 // y = (x * r) * g for one chunk from its gains g2 (packed pairs).
 __device__ __forceinline__ void norm_apply_g(const uint4& u, uint64_t r2, const uint64_t (&g2)[4],
                                              uint64_t (&y2)[4]) {
@@ -701,14 +708,19 @@ __global__ void __launch_bounds__(MAXT, 512 / MAXT)
 constexpr int kNormWarpMaxK = 8192;
 constexpr int kNormWarpSlots = 1;
 
-template <bool E4M3>
+// GS: the gains in shared memory, loaded once per CTA (rows of up to 4096
+// elements), instead of from L1 in every pass
+template <bool E4M3, bool GS>
 __global__ void __launch_bounds__(256)
     rmsnorm_quant_warp_kernel(const uint16_t* __restrict__ x, const float* __restrict__ g,
                               float eps, int64_t M, int K, uint8_t* __restrict__ xq,
                               float* __restrict__ sx, int* status, int late_wait,
                               int force_exact) {
   constexpr int SLOTS = kNormWarpSlots;
-  extern __shared__ __align__(128) uint8_t ring[];  // [warps][SLOTS][K] bf16
+  // [K] binary32 gains (GS), then [warps][SLOTS][K] bf16 rows
+  extern __shared__ __align__(128) uint8_t smem_dyn[];
+  float* gtab = reinterpret_cast<float*>(smem_dyn);
+  uint8_t* ring = smem_dyn + (GS ? size_t(K) * 4 : 0);
   __shared__ __align__(8) uint64_t bars[8][SLOTS];
   const uint32_t row_bytes = uint32_t(K) * 2;
   const int nchunk = K >> 3;
@@ -725,6 +737,11 @@ __global__ void __launch_bounds__(256)
   // x and g may come from the kernel before this one, which may still read
   // xq / sx -- unless the caller has ruled both out (late_wait)
   if (!late_wait) pdl_wait();
+  if constexpr (GS) {
+    for (int i = threadIdx.x; i < K / 4; i += blockDim.x)
+      reinterpret_cast<float4*>(gtab)[i] = __ldg(reinterpret_cast<const float4*>(g) + i);
+    __syncthreads();
+  }
   if (lane == 0) {
     for (int i = 0; i < SLOTS; ++i) {
       const int64_t m = w0 + i * stride;
@@ -840,8 +857,13 @@ __global__ void __launch_bounds__(256)
       const uint4 u0 = row[c];
       const uint4 u1 = two ? row[c + 32] : make_uint4(0u, 0u, 0u, 0u);
       uint64_t g0[4], g1[4] = {0ull, 0ull, 0ull, 0ull};
-      norm_gains(g + size_t(c) * 8, g0);
-      if (two) norm_gains(g + size_t(c + 32) * 8, g1);
+      if constexpr (GS) {
+        norm_gains_smem(gtab + size_t(c) * 8, g0);
+        if (two) norm_gains_smem(gtab + size_t(c + 32) * 8, g1);
+      } else {
+        norm_gains(g + size_t(c) * 8, g0);
+        if (two) norm_gains(g + size_t(c + 32) * 8, g1);
+      }
       uint64_t y0[4], y1[4];
       norm_apply_g(u0, r2, g0, y0);
       norm_apply_g(u1, r2, g1, y1);
@@ -869,8 +891,13 @@ __global__ void __launch_bounds__(256)
         const uint4 u0 = row[c];
         const uint4 u1 = two ? row[c + 32] : make_uint4(0u, 0u, 0u, 0u);
         uint64_t g0[4], g1[4] = {0ull, 0ull, 0ull, 0ull};
-        norm_gains(g + size_t(c) * 8, g0);
-        if (two) norm_gains(g + size_t(c + 32) * 8, g1);
+        if constexpr (GS) {
+          norm_gains_smem(gtab + size_t(c) * 8, g0);
+          if (two) norm_gains_smem(gtab + size_t(c + 32) * 8, g1);
+        } else {
+          norm_gains(g + size_t(c) * 8, g0);
+          if (two) norm_gains(g + size_t(c + 32) * 8, g1);
+        }
         uint64_t y0[4], y1[4];
         norm_apply_g(u0, r2, g0, y0);
         norm_apply_g(u1, r2, g1, y1);
@@ -963,13 +990,20 @@ cudaError_t launch_rmsnorm_quant(const uint16_t* x, const float* g, float eps, i
                                  int64_t K, bool e4m3, void* xq, float* sx, float* xn,
                                  bool overlap, cudaStream_t st) {
   if (!xn && K <= kNormWarpMaxK && M >= 4LL * norm_sm_count()) {
-    // the warp form: up to 8 warps per CTA, each with SLOTS rows in flight,
-    // about 96 KB of ring per CTA; as many CTAs as fit, no more than the rows
-    // need
+    // the warp form: up to 8 warps per CTA, each with SLOTS rows in flight;
+    // rows of up to 4096 elements with the gains in shared memory, at most
+    // 72 KB per CTA (three CTAs per SM), longer ones with the gains from L1
+    // and about 96 KB of ring per CTA; as many CTAs as fit, no more than the
+    // rows need
+    const bool gs = K <= 4096;
     const int per_row = int(K) * 2 * kNormWarpSlots;
-    const int warps = max(1, min(8, 98304 / per_row));
-    const size_t smem = size_t(warps) * per_row;
-    auto kern = e4m3 ? rmsnorm_quant_warp_kernel<true> : rmsnorm_quant_warp_kernel<false>;
+    const int table = gs ? int(K) * 4 : 0;
+    const int warps = max(1, min(8, ((gs ? 73728 : 98304) - table) / per_row));
+    const size_t smem = size_t(table) + size_t(warps) * per_row;
+    auto kern = e4m3 ? (gs ? rmsnorm_quant_warp_kernel<true, true>
+                           : rmsnorm_quant_warp_kernel<true, false>)
+                     : (gs ? rmsnorm_quant_warp_kernel<false, true>
+                           : rmsnorm_quant_warp_kernel<false, false>);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          int(smem));
     if (e != cudaSuccess) return e;
