@@ -24,16 +24,23 @@
 // xn itself is written too when asked for (binary32; the calibration of the
 // smoothing factors runs on it offline).
 //
-// Two kernels give the same results bit for bit:
+// Three kernels give the same results bit for bit:
 //  * rmsnorm_quant_kernel, the plain form (and the only one that also writes
 //    xn): one CTA per row, the row staged in shared memory, four passes over
 //    it (the largest exponent, the exact sum of squares, the largest |xn|,
 //    the codes) with IEEE divisions, each closed by a block reduction;
-//  * rmsnorm_quant_stream_kernel, used otherwise: persistent CTAs with the
-//    next rows in flight (bulk copies into a shared-memory ring), each
-//    thread's part of the row in registers, three block barriers
-//    per row, packed binary32 pairs, and no division instruction on rows
-//    whose largest |xn| is in [2^-60, 2^100].
+//  * rmsnorm_quant_warp_kernel, for many rows of at most 8192 elements: one
+//    warp per row, with its own row slot and barrier, no block barrier on a
+//    row's path;
+//  * rmsnorm_quant_stream_kernel, for the other shapes: persistent CTAs with
+//    the next rows in flight (bulk copies into a shared-memory ring), each
+//    thread's part of the row in registers, three block barriers per row.
+// The last two sum the squares in binary64 (each square exact there) and
+// check that both ends of an interval around that sum, far wider than its
+// rounding error, give the same binary32 r -- then it is the r of the exact
+// sum; the rows where they do not take the exact integer sum. They work on
+// packed binary32 pairs and use no division instruction on rows whose
+// largest |xn| is in [2^-60, 2^100].
 // HBM-bound in principle: 2 bytes read and 1 written per element.
 #include <cstdint>
 #include <cstdlib>
