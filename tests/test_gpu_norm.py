@@ -160,3 +160,30 @@ def test_warp_form_row_lengths(M, K, qt):
     assert ops.device_status() == ops.SQ_OK
     np.testing.assert_array_equal(host(sx), s_ref)
     np.testing.assert_array_equal(host(xq).view(np.uint8), q_ref.view(np.uint8))
+
+
+def _sweep_cases(n=24, seed=77):
+    g = np.random.default_rng(seed)
+    cases = []
+    for i in range(n):
+        K = int(g.choice([8, 16, 24, 64, 200, 1000, 2048, 4096, 4104, 8192, 12288, 16384]))
+        M = int(g.integers(1, max(2, min(5000, 8_000_000 // K))))
+        cases.append((i, M, K, bool(g.integers(0, 2)), float(g.choice([1e-6, 1e-5, 0.1]))))
+    return cases
+
+
+@pytest.mark.parametrize("i,M,K,e4m3,eps", _sweep_cases())
+def test_seeded_shape_sweep(i, M, K, e4m3, eps):
+    """Seeded random shapes across every form (plain when xn is asked for,
+    one warp per row, one CTA per row) and both code types."""
+    xb = _rows(M, K, seed=1000 + i)
+    gamma = synth.random_floats(K, seed=2000 + i, lo=0.2, hi=3.0)
+    qt = "e4m3" if e4m3 else "i8"
+    q_ref, s_ref, _, xn_ref = oracle.rmsnorm_quantize_act(
+        xb, gamma, eps, oracle.E4M3 if e4m3 else oracle.INT8)
+    out = ops.rmsnorm_quantize_act(dev(xb), dev(gamma), eps, qt, want_xn=(i % 4 == 0))
+    assert ops.device_status() == ops.SQ_OK
+    np.testing.assert_array_equal(host(out[1]), s_ref)
+    np.testing.assert_array_equal(host(out[0]).view(np.uint8), q_ref.view(np.uint8))
+    if i % 4 == 0:
+        np.testing.assert_array_equal(host(out[2]).view(np.uint32), xn_ref.view(np.uint32))
