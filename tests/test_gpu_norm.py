@@ -187,3 +187,38 @@ def test_seeded_shape_sweep(i, M, K, e4m3, eps):
     np.testing.assert_array_equal(host(out[0]).view(np.uint8), q_ref.view(np.uint8))
     if i % 4 == 0:
         np.testing.assert_array_equal(host(out[2]).view(np.uint32), xn_ref.view(np.uint32))
+
+
+@pytest.mark.parametrize("qt", ["i8", "e4m3"])
+def test_rmsnorm_layer_api(qt):
+    """The layer object: its offline preparation and forward equal the oracle's
+    chain (calibration on the normalization's output, s, weight codes, the
+    folded gain, the fused normalization + quantization, the GEMM)."""
+    M, K, N = 300, 1024, 768
+    h = _rows(M, K, seed=501)
+    h_cal = _rows(256, K, seed=502)
+    gamma = synth.random_floats(K, seed=503, lo=0.5, hi=2.0)
+    w = synth.random_floats((K, N), seed=504, std=0.02)
+    bias = synth.to_bf16_bits(synth.random_floats(N, seed=505, std=0.01))
+    qcode = oracle.INT8 if qt == "i8" else oracle.E4M3
+    layer = ops.RMSNormSmoothQuantLinear(dev(w), dev(h_cal), dev(gamma), 1e-5, 0.5, qt,
+                                         bias=dev(bias))
+    s = host(layer.s)          # stage-wise: the later stages on the layer's own s
+    xn_cal = oracle.rmsnorm_quantize_act(h_cal, gamma, 1e-5)[3]
+    s_ref = oracle.smooth_factors(oracle.amax(xn_cal, True), oracle.amax(w, False), 0.5)
+    assert ulp_distance(s, s_ref).max() <= 2
+    g_ref = oracle.fold_smoothing(gamma, s)[0]
+    np.testing.assert_array_equal(host(layer.g), g_ref)
+    wq_ref, sw_ref = oracle.quantize_weight(w, s, qcode)
+    q_ref, sx_ref, _, _ = oracle.rmsnorm_quantize_act(h, g_ref, 1e-5, qcode)
+    y = layer(dev(h), out_dtype=torch.float32)
+    assert ops.device_status() == ops.SQ_OK
+    if qt == "i8":
+        y_ref, _ = oracle.epilogue(oracle.gemm_i8(q_ref, wq_ref), sx_ref, sw_ref, bias)
+        np.testing.assert_array_equal(host(y), y_ref)
+    else:
+        y_ref, _ = oracle.epilogue(oracle.gemm_e4m3(q_ref, wq_ref), sx_ref, sw_ref, bias)
+        err = np.abs(host(y).astype(np.float64) - y_ref)
+        scale = (np.abs(oracle.e4m3_decode(q_ref)).astype(np.float64) @
+                 np.abs(oracle.e4m3_decode(wq_ref)).astype(np.float64).T) * sx_ref[:, None] * sw_ref[None, :]
+        assert (err <= 1e-3 * (scale + np.abs(oracle.bf16_to_f32_array(bias))[None, :]) + 1e-30).all()

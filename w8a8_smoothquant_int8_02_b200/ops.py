@@ -525,3 +525,25 @@ class SmoothQuantLinear:
         self._cur = 1 - c
         g = gemm_w8a8 if self.qtype == "i8" else gemm_fp8
         return g(xq, sx, self.wq, self.sw, self.bias, out_dtype=out_dtype)
+
+
+class RMSNormSmoothQuantLinear:
+    """A prepared W8A8 linear layer fed by its RMS normalization:
+    y = (rmsnorm(h) * gamma) @ W (+ bias), with the smoothing folded into the
+    normalization's gain offline, so that one kernel normalizes and quantizes
+    each token row of h at run time and the 8-bit GEMM follows.
+
+    h_cal: calibration tokens of the normalization's input (bf16 [T, K]); the
+    smoothing factors are calibrated on the normalization's output."""
+
+    def __init__(self, w: torch.Tensor, h_cal: torch.Tensor, gamma: torch.Tensor, eps: float,
+                 alpha: float = 0.5, qtype: str = "i8", bias: torch.Tensor | None = None):
+        p = prepare_rmsnorm(w, h_cal, gamma, eps, alpha, qtype)
+        self.s, self.g, self.wq, self.sw = p["s"], p["g"], p["wq"], p["sw"]
+        self.eps, self.qtype, self.bias = float(eps), qtype, bias
+        self.in_features, self.out_features = w.shape
+
+    def __call__(self, h: torch.Tensor, out_dtype=torch.bfloat16) -> torch.Tensor:
+        xq, sx = rmsnorm_quantize_act(h, self.g, self.eps, self.qtype)
+        gm = gemm_w8a8 if self.qtype == "i8" else gemm_fp8
+        return gm(xq, sx, self.wq, self.sw, self.bias, out_dtype=out_dtype)
